@@ -1,0 +1,917 @@
+// Host side of the Fast-BLT local-decoder engine: weight layout, paged KV
+// pool, latent cache, per-call sequencing of decoder passes, and the C ABI of
+// bltdec.h.  Every decoder step runs in the kernels of kernels.cuh.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "bltdec.h"
+#include "kernels.cuh"
+
+using namespace bltdec;
+
+namespace {
+
+struct Mat {
+  uint4* w = nullptr;
+  int N = 0, K = 0, planes = 1;
+  size_t bytes() const { return (size_t)N * K * 2 * planes; }
+};
+
+uint16_t bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  u = u + 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+float bf16_to_f(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+}  // namespace
+
+struct blt_dec {
+  blt_dec_config cfg{};
+  cudaStream_t stream = nullptr;
+  bool own_stream = false;
+  int L = 0, d = 0, H = 0, dh = 0, F = 0, dg = 0, V = 0, planes = 1;
+  int PT = 0, max_pages = 0, n_pages = 0, CH = 0, CMAX = 0;
+  std::vector<Mat> qkv, o, w13, w2, vc, oc;
+  std::vector<float*> attn_norm, ffn_norm;
+  Mat head;
+  float* embed = nullptr;
+  float* final_norm = nullptr;
+  float *rope_cos = nullptr, *rope_sin = nullptr;
+  __nv_bfloat16* kv = nullptr;
+  int* page_table = nullptr;
+  std::vector<int> pt_host, free_pages, seq_npages;
+  float* c_lat = nullptr;
+  float *h = nullptr, *rs = nullptr, *q = nullptr, *att = nullptr, *act = nullptr, *logits = nullptr, *tmp = nullptr;
+  float2* part_ml = nullptr;
+  float* part_o = nullptr;
+  float *conf = nullptr, *gap = nullptr;
+  int* pred = nullptr;
+  RowsDev rows{};
+  int *lat_seq = nullptr, *lat_slot = nullptr, *n_lat_rows = nullptr;
+  SeqDev sd{};
+  std::vector<void*> allocs;
+  int state = 0;  // 0 ready, 1 draft waiting
+  int draft_k = 0, draft_batch = 0;
+  std::vector<int> kv_ub, nlat_ub;
+  int* mirror = nullptr;  // pinned [2*max_batch]: kv_len, n_lat
+  cudaEvent_t mirror_ev = nullptr;
+  bool mirror_pending = false;
+  std::string err;
+  unsigned long long weight_bytes_per_pass = 0, kv_bytes_per_key = 0;
+};
+
+namespace {
+
+int fail(blt_dec* h, int code, const char* fmt, ...) __attribute__((format(printf, 3, 4)));
+int fail(blt_dec* h, int code, const char* fmt, ...) {
+  if (h) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    h->err = buf;
+  }
+  return code;
+}
+
+#define CK(call)                                                                                     \
+  do {                                                                                               \
+    cudaError_t e_ = (call);                                                                         \
+    if (e_ != cudaSuccess) return fail(h, BLT_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));   \
+  } while (0)
+
+template <class T>
+int dalloc(blt_dec* h, T** p, size_t count) {
+  void* v = nullptr;
+  cudaError_t e = cudaMalloc(&v, std::max<size_t>(count, 1) * sizeof(T));
+  if (e != cudaSuccess) return fail(h, BLT_ERR_CUDA, "cudaMalloc(%zu): %s", count * sizeof(T), cudaGetErrorString(e));
+  h->allocs.push_back(v);
+  *p = static_cast<T*>(v);
+  return BLT_OK;
+}
+
+#define TRY(x)                  \
+  do {                          \
+    int r_ = (x);               \
+    if (r_ != BLT_OK) return r_; \
+  } while (0)
+
+// Pack W (rows given by src_row(tile_row) of a [*, K] fp32 matrix) into
+// m16k16 tensor-core A-fragment order: tile (mt, ks), plane p, lane l holds
+// rows g, g+8 and columns 2t, 2t+1, 2t+8, 2t+9 (g = l/4, t = l%4).
+template <class RowFn>
+int pack_matrix(blt_dec* h, Mat& m, int N, int K, int planes, RowFn src_row) {
+  m.N = N;
+  m.K = K;
+  m.planes = planes;
+  const int ntm = N / 16, nks = K / 16;
+  std::vector<uint16_t> buf((size_t)N * K * planes);
+  for (int mt = 0; mt < ntm; ++mt) {
+    const float* ra[8];
+    const float* rb[8];
+    for (int g = 0; g < 8; ++g) {
+      ra[g] = src_row(mt * 16 + g);
+      rb[g] = src_row(mt * 16 + g + 8);
+    }
+    for (int ks = 0; ks < nks; ++ks) {
+      uint16_t* tile = buf.data() + ((size_t)mt * nks + ks) * planes * 256;
+      for (int lane = 0; lane < 32; ++lane) {
+        const int g = lane >> 2, t = lane & 3, c = ks * 16 + 2 * t;
+        const float v[8] = {ra[g][c], ra[g][c + 1], rb[g][c], rb[g][c + 1], ra[g][c + 8], ra[g][c + 9], rb[g][c + 8], rb[g][c + 9]};
+        for (int e = 0; e < 8; ++e) {
+          const uint16_t hi = bf16_rne(v[e]);
+          tile[lane * 8 + e] = hi;
+          if (planes == 2) tile[256 + lane * 8 + e] = bf16_rne(v[e] - bf16_to_f(hi));
+        }
+      }
+    }
+  }
+  TRY(dalloc(h, &m.w, buf.size() * 2 / 16));
+  CK(cudaMemcpy(m.w, buf.data(), buf.size() * 2, cudaMemcpyHostToDevice));
+  return BLT_OK;
+}
+
+int upload(blt_dec* h, float** dst, const float* src, size_t n) {
+  TRY(dalloc(h, dst, n));
+  CK(cudaMemcpy(*dst, src, n * 4, cudaMemcpyHostToDevice));
+  return BLT_OK;
+}
+
+// ---------------------------------------------------------------------------- GEMM launch
+template <int NG, int PL, int EPI>
+constexpr int gemm_stages() {
+  return NG >= 8 ? 3 : 4;
+}
+template <int NG, int PL, int EPI>
+size_t gemm_smem() {
+  constexpr int RB = 8 * NG;
+  return (size_t)gemm_stages<NG, PL, EPI>() * RB * kXStride * 4 + RB * 4;
+}
+
+template <int NG, int PL, int EPI>
+int set_gemm_attr(blt_dec* h) {
+  CK(cudaFuncSetAttribute(k_gemm<NG, PL, EPI, gemm_stages<NG, PL, EPI>()>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          (int)gemm_smem<NG, PL, EPI>()));
+  return BLT_OK;
+}
+
+template <int EPI>
+int set_attrs_epi(blt_dec* h) {
+  TRY((set_gemm_attr<1, 1, EPI>(h)));
+  TRY((set_gemm_attr<2, 1, EPI>(h)));
+  TRY((set_gemm_attr<4, 1, EPI>(h)));
+  TRY((set_gemm_attr<8, 1, EPI>(h)));
+  TRY((set_gemm_attr<1, 2, EPI>(h)));
+  TRY((set_gemm_attr<2, 2, EPI>(h)));
+  TRY((set_gemm_attr<4, 2, EPI>(h)));
+  TRY((set_gemm_attr<8, 2, EPI>(h)));
+  return BLT_OK;
+}
+
+template <int NG, int PL, int EPI>
+void launch_ng(blt_dec* h, const GemmArgs& a, int rows_ub) {
+  constexpr int RB = 8 * NG;
+  dim3 grid(a.N / 16, (rows_ub + RB - 1) / RB);
+  k_gemm<NG, PL, EPI, gemm_stages<NG, PL, EPI>()><<<grid, kThreads, gemm_smem<NG, PL, EPI>(), h->stream>>>(a);
+}
+
+template <int EPI>
+int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
+  if (rows_ub <= 0) return BLT_OK;
+  a.w = m.w;
+  a.N = m.N;
+  a.K = m.K;
+  a.status = h->sd.status;
+  const int ng = rows_ub <= 8 ? 1 : rows_ub <= 16 ? 2 : rows_ub <= 32 ? 4 : 8;
+  if (m.planes == 1) {
+    if (ng == 1) launch_ng<1, 1, EPI>(h, a, rows_ub);
+    else if (ng == 2) launch_ng<2, 1, EPI>(h, a, rows_ub);
+    else if (ng == 4) launch_ng<4, 1, EPI>(h, a, rows_ub);
+    else launch_ng<8, 1, EPI>(h, a, rows_ub);
+  } else {
+    if (ng == 1) launch_ng<1, 2, EPI>(h, a, rows_ub);
+    else if (ng == 2) launch_ng<2, 2, EPI>(h, a, rows_ub);
+    else if (ng == 4) launch_ng<4, 2, EPI>(h, a, rows_ub);
+    else launch_ng<8, 2, EPI>(h, a, rows_ub);
+  }
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+GemmArgs base_args(blt_dec* h) {
+  GemmArgs a{};
+  a.n_rows = h->rows.n_rows;
+  a.kv = h->kv;
+  a.page_table = h->page_table;
+  a.max_pages = h->max_pages;
+  a.PT = h->PT;
+  a.L = h->L;
+  a.H = h->H;
+  a.dh = h->dh;
+  a.d = h->d;
+  a.row_seq = h->rows.seq;
+  a.row_pos = h->rows.pos;
+  a.rope_cos = h->rope_cos;
+  a.rope_sin = h->rope_sin;
+  a.max_ctx = h->cfg.max_ctx;
+  a.max_lat = h->cfg.max_latents;
+  a.status = h->sd.status;
+  return a;
+}
+
+// ---------------------------------------------------------------------------- one decoder pass
+// Runs every layer over the rows planned on the device (at most rows_ub rows,
+// keys below keys_ub, at most groups_ub attention groups).
+int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
+  const int d = h->d;
+  const float eps = h->cfg.norm_eps;
+  const int nb = std::max(1, std::min(rows_ub, 1024));
+  k_embed<<<nb, 256, 0, h->stream>>>(h->rows, h->embed, h->h, d, rows_ub);
+  const int nw_blocks = std::max(1, std::min((rows_ub + 7) / 8, 1024));
+  AttnArgs aa{};
+  aa.kv = h->kv;
+  aa.page_table = h->page_table;
+  aa.max_pages = h->max_pages;
+  aa.PT = h->PT;
+  aa.L = h->L;
+  aa.H = h->H;
+  aa.dh = h->dh;
+  aa.d = d;
+  aa.rows = h->rows;
+  aa.CH = h->CH;
+  aa.CMAX = h->CMAX;
+  aa.scale = 1.0f / std::sqrt((float)h->dh);
+  aa.q = h->q;
+  aa.part_ml = h->part_ml;
+  aa.part_o = h->part_o;
+  aa.att = h->att;
+  aa.status = h->sd.status;
+  const int nchunks = std::max(1, (keys_ub + h->CH - 1) / h->CH);
+  const size_t attn_smem = (size_t)(32 * h->dh + h->CH * h->dh + 32 * h->CH) * 4;
+  for (int l = 0; l < h->L; ++l) {
+    // B_l = D_{l-1} + W_o^c W_v^c o_lat ; rs = RMS scale of B_l
+    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, h->c_lat, h->cfg.max_latents, h->L, l, d, eps, nullptr);
+    GemmArgs a = base_args(h);
+    a.layer = l;
+    a.X = h->h;
+    a.ldx = d;
+    a.rs = h->rs;
+    a.gain = h->attn_norm[l];
+    a.q = h->q;
+    TRY(gemm<EPI_QKV>(h, h->qkv[l], a, rows_ub));
+    aa.layer = l;
+    dim3 ag(h->H, nchunks, groups_ub);
+    if (h->dh == 64) k_attn_partial<64><<<ag, 128, attn_smem, h->stream>>>(aa);
+    else if (h->dh == 32) k_attn_partial<32><<<ag, 128, attn_smem, h->stream>>>(aa);
+    else if (h->dh == 128) k_attn_partial<128><<<ag, 128, attn_smem, h->stream>>>(aa);
+    else k_attn_partial<16><<<ag, 128, attn_smem, h->stream>>>(aa);
+    k_attn_combine<<<dim3(rows_ub, h->H), h->dh, 0, h->stream>>>(aa);
+    CK(cudaGetLastError());
+    a = base_args(h);
+    a.layer = l;
+    a.X = h->att;
+    a.ldx = d;
+    a.out = h->h;
+    a.ldo = d;
+    TRY(gemm<EPI_RESID>(h, h->o[l], a, rows_ub));
+    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, nullptr, 0, 0, 0, d, eps, nullptr);
+    a = base_args(h);
+    a.layer = l;
+    a.X = h->h;
+    a.ldx = d;
+    a.rs = h->rs;
+    a.gain = h->ffn_norm[l];
+    a.out = h->act;
+    a.ldo = h->F;
+    TRY(gemm<EPI_SWIGLU>(h, h->w13[l], a, rows_ub));
+    a = base_args(h);
+    a.layer = l;
+    a.X = h->act;
+    a.ldx = h->F;
+    a.out = h->h;
+    a.ldo = d;
+    TRY(gemm<EPI_RESID>(h, h->w2[l], a, rows_ub));
+  }
+  if (want_head) {
+    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, nullptr, 0, 0, 0, d, eps, nullptr);
+    GemmArgs a = base_args(h);
+    a.X = h->h;
+    a.ldx = d;
+    a.rs = h->rs;
+    a.gain = h->final_norm;
+    a.out = h->logits;
+    a.ldo = 256;
+    TRY(gemm<EPI_STORE>(h, h->head, a, rows_ub));
+    k_head_stats<<<std::max(1, std::min((rows_ub + 7) / 8, 1024)), 256, 0, h->stream>>>(h->logits, h->rows.n_rows, h->conf,
+                                                                                          h->pred, h->gap);
+  }
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+// ---------------------------------------------------------------------------- host bookkeeping
+void refresh_bounds(blt_dec* h) {
+  if (h->mirror_pending && cudaEventQuery(h->mirror_ev) == cudaSuccess) {
+    const int B = h->cfg.max_batch;
+    for (int s = 0; s < B; ++s) {
+      h->kv_ub[s] = h->mirror[s];
+      h->nlat_ub[s] = h->mirror[B + s];
+    }
+    h->mirror_pending = false;
+  }
+}
+
+int post_mirror(blt_dec* h) {
+  const int B = h->cfg.max_batch;
+  CK(cudaMemcpyAsync(h->mirror, h->sd.kv_len, B * 4, cudaMemcpyDeviceToHost, h->stream));
+  CK(cudaMemcpyAsync(h->mirror + B, h->sd.n_lat, B * 4, cudaMemcpyDeviceToHost, h->stream));
+  CK(cudaEventRecord(h->mirror_ev, h->stream));
+  h->mirror_pending = true;
+  return BLT_OK;
+}
+
+// Make sure sequence s has KV pages for positions [0, need).
+int ensure_pages(blt_dec* h, int s, int need, PageUpd& upd) {
+  if (need > h->cfg.max_ctx) return fail(h, BLT_ERR_NO_SPACE, "sequence %d needs %d positions > max_ctx %d", s, need, h->cfg.max_ctx);
+  while (h->seq_npages[s] * h->PT < need) {
+    if (h->free_pages.empty()) return fail(h, BLT_ERR_NO_SPACE, "KV page pool exhausted");
+    const int page = h->free_pages.back();
+    h->free_pages.pop_back();
+    const int idx = s * h->max_pages + h->seq_npages[s];
+    h->pt_host[idx] = page;
+    h->seq_npages[s]++;
+    upd.idx[upd.n] = idx;
+    upd.page[upd.n] = page;
+    if (++upd.n == 64) {
+      k_page_update<<<1, 64, 0, h->stream>>>(h->page_table, upd);
+      upd.n = 0;
+    }
+  }
+  return BLT_OK;
+}
+
+int flush_pages(blt_dec* h, PageUpd& upd) {
+  if (upd.n) k_page_update<<<1, 64, 0, h->stream>>>(h->page_table, upd);
+  upd.n = 0;
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+int make_desc(blt_dec* h, int batch, const int32_t* row_off, const int32_t* lat_off, CallDesc& cd) {
+  if (batch < 1 || batch > h->cfg.max_batch || batch > kMaxCallBatch)
+    return fail(h, BLT_ERR_INVALID_ARG, "batch %d outside 1..%d", batch, std::min(h->cfg.max_batch, kMaxCallBatch));
+  cd.batch = batch;
+  for (int s = 0; s <= batch; ++s) {
+    cd.row_off[s] = row_off ? row_off[s] : 0;
+    cd.lat_off[s] = lat_off ? lat_off[s] : 0;
+    if (s > 0 && (cd.row_off[s] < cd.row_off[s - 1] || cd.lat_off[s] < cd.lat_off[s - 1]))
+      return fail(h, BLT_ERR_INVALID_ARG, "offsets must be non-decreasing");
+  }
+  if (cd.row_off[0] != 0 || cd.lat_off[0] != 0) return fail(h, BLT_ERR_INVALID_ARG, "offsets must start at 0");
+  return BLT_OK;
+}
+
+// Project new latents: c_l[slot] = W_o^c (W_v^c o) for every layer.
+int project_latents(blt_dec* h, const CallDesc& cd, const float* new_lat, bool commit) {
+  const int total = cd.lat_off[cd.batch];
+  if (total == 0) return BLT_OK;
+  if (!new_lat) return fail(h, BLT_ERR_INVALID_ARG, "new_latents is NULL but latent_offsets count %d", total);
+  const int chunk = h->cfg.max_rows;
+  for (int r0 = 0; r0 < total; r0 += chunk) {
+    const int r1 = std::min(total, r0 + chunk);
+    k_lat_plan<<<1, 256, 0, h->stream>>>(cd, h->sd, h->lat_seq, h->lat_slot, h->n_lat_rows, r0, r1, commit ? 1 : 0,
+                                         h->cfg.max_latents);
+    for (int l = 0; l < h->L; ++l) {
+      GemmArgs a = base_args(h);
+      a.n_rows = nullptr;
+      a.rows_host = r1 - r0;
+      a.layer = l;
+      a.X = new_lat + (size_t)r0 * h->dg;
+      a.ldx = h->dg;
+      a.out = h->tmp;
+      a.ldo = h->d;
+      TRY(gemm<EPI_STORE>(h, h->vc[l], a, r1 - r0));
+      a.X = h->tmp;
+      a.ldx = h->d;
+      a.out = h->c_lat;
+      a.lat_seq = h->lat_seq;
+      a.lat_slot = h->lat_slot;
+      TRY(gemm<EPI_LATC>(h, h->oc[l], a, r1 - r0));
+    }
+  }
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+PlanArgs plan_args(blt_dec* h, int mode, int k) {
+  PlanArgs p{};
+  p.mode = mode;
+  p.k = k;
+  p.max_ctx = h->cfg.max_ctx;
+  p.max_lat = h->cfg.max_latents;
+  p.mask_id = h->V - 1;
+  p.weight_bytes_per_pass = h->weight_bytes_per_pass;
+  p.kv_bytes_per_key = h->kv_bytes_per_key;
+  return p;
+}
+
+int plan(blt_dec* h, const PlanArgs& p, const CallDesc& cd) {
+  k_plan<<<1, 256, 0, h->stream>>>(p, cd, h->sd, h->rows);
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+int groups_bound(const CallDesc& cd, int per_seq_extra) {
+  int g = 0;
+  for (int s = 0; s < cd.batch; ++s) g += (cd.row_off[s + 1] - cd.row_off[s] + per_seq_extra + 31) / 32;
+  return std::max(g, 1);
+}
+
+int max_kv_ub(blt_dec* h, int batch) {
+  int m = 0;
+  for (int s = 0; s < batch; ++s) m = std::max(m, h->kv_ub[s]);
+  return m;
+}
+
+// Fill k-byte blocks (BLT-D / BLT-DV draft) with the pending rows in pass 1.
+int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, float alpha, int max_steps, float* out_logits) {
+  const int batch = cd.batch;
+  const int np_total = cd.row_off[batch];
+  const int rows1 = np_total + batch * k;
+  int npmax = 0;
+  for (int s = 0; s < batch; ++s) npmax = std::max(npmax, cd.row_off[s + 1] - cd.row_off[s]);
+  const int keys_ub = max_kv_ub(h, batch) + npmax + k;
+  PlanArgs p = plan_args(h, PL_FIRST, k);
+  p.pend_bytes = pend->bytes;
+  p.pend_lat = pend->row_latent;
+  TRY(plan(h, p, cd));
+  TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true));
+  k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits);
+  for (int st = 1; st < max_steps; ++st) {
+    PlanArgs pb = plan_args(h, PL_BLOCK, k);
+    TRY(plan(h, pb, cd));
+    TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true));
+    k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits);
+  }
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
+int check_pending(blt_dec* h, const blt_rows_in* r, bool need_rows) {
+  if (!r) return fail(h, BLT_ERR_INVALID_ARG, "rows is NULL");
+  if (need_rows && !r->row_offsets) return fail(h, BLT_ERR_INVALID_ARG, "row_offsets is NULL");
+  return BLT_OK;
+}
+
+int reserve(blt_dec* h, const CallDesc& cd, int extra_positions, bool lat_commit) {
+  PageUpd upd{};
+  for (int s = 0; s < cd.batch; ++s) {
+    const int np = cd.row_off[s + 1] - cd.row_off[s];
+    const int nl = cd.lat_off[s + 1] - cd.lat_off[s];
+    TRY(ensure_pages(h, s, h->kv_ub[s] + np + extra_positions, upd));
+    if (h->nlat_ub[s] + nl > h->cfg.max_latents)
+      return fail(h, BLT_ERR_NO_SPACE, "sequence %d latent slots %d + %d > max_latents %d", s, h->nlat_ub[s], nl,
+                  h->cfg.max_latents);
+  }
+  (void)lat_commit;
+  return flush_pages(h, upd);
+}
+
+void bump_bounds(blt_dec* h, const CallDesc& cd, int extra_kv) {
+  for (int s = 0; s < cd.batch; ++s) {
+    h->kv_ub[s] += cd.row_off[s + 1] - cd.row_off[s] + extra_kv;
+    h->nlat_ub[s] += cd.lat_off[s + 1] - cd.lat_off[s];
+  }
+}
+
+__global__ void k_count_call(unsigned long long* c) { c[4] += 1; }
+__global__ void k_snapshot_base(SeqDev sd, int batch) {
+  const int s = threadIdx.x + blockIdx.x * blockDim.x;
+  if (s < batch) sd.kv_base[s] = sd.kv_len[s];
+}
+__global__ void k_finish_prefill(SeqDev sd, CallDesc cd) {
+  const int s = threadIdx.x;
+  if (s < cd.batch) sd.kv_len[s] = sd.kv_base[s] + (cd.row_off[s + 1] - cd.row_off[s]);
+}
+__global__ void k_copy_logits(const float* src, float* dst, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) dst[i] = src[i];
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda_stream, blt_dec_t** out) {
+  if (!cfg || !w || !out) return BLT_ERR_INVALID_ARG;
+  *out = nullptr;
+  blt_dec* h = new blt_dec();
+  h->cfg = *cfg;
+  auto bad = [&](const char* msg) {
+    blt_dec_free(h);
+    return BLT_ERR_INVALID_ARG;
+  };
+  const blt_dec_config& c = *cfg;
+  if (c.n_layers < 1 || c.d_model < 128 || c.d_model % 128 || c.n_heads < 1 || c.d_model % c.n_heads ||
+      (c.d_model / c.n_heads) % 16 || c.d_model / c.n_heads > 128 || c.d_ffn % 128 || c.d_ffn < 128 || c.d_global % 128 ||
+      c.d_global < 128 || c.vocab != 257 || (c.weight_dtype != BLT_W_F32 && c.weight_dtype != BLT_W_BF16) ||
+      c.max_batch < 1 || c.max_batch > kMaxCallBatch || c.max_ctx < 2 || c.max_latents < 1 || c.max_rows < 1 ||
+      c.max_block < 1 || c.max_block > kMaxBlock || c.page_tokens < 16 || c.page_tokens % 16 || !(c.norm_eps > 0) ||
+      !(c.rope_theta > 0) || !w->embed || !w->head || !w->final_norm || !w->layer)
+    return bad("config");
+  const int dhh = c.d_model / c.n_heads;
+  if (dhh != 16 && dhh != 32 && dhh != 64 && dhh != 128) return bad("head dim");
+  h->L = c.n_layers;
+  h->d = c.d_model;
+  h->H = c.n_heads;
+  h->dh = dhh;
+  h->F = c.d_ffn;
+  h->dg = c.d_global;
+  h->V = c.vocab;
+  h->planes = c.weight_dtype == BLT_W_F32 ? 2 : 1;
+  h->PT = c.page_tokens;
+  h->max_pages = (c.max_ctx + h->PT - 1) / h->PT;
+  h->n_pages = c.kv_pages > 0 ? c.kv_pages : c.max_batch * h->max_pages;
+  h->CH = c.attn_chunk > 0 ? c.attn_chunk : 128;
+  if (h->CH > 128 || h->CH % 16) return bad("attn_chunk");
+  h->CMAX = (c.max_ctx + h->CH - 1) / h->CH;
+
+  int rc = BLT_OK;
+  auto run = [&]() -> int {
+    if (cuda_stream) {
+      h->stream = (cudaStream_t)cuda_stream;
+    } else {
+      CK(cudaStreamCreateWithFlags(&h->stream, cudaStreamNonBlocking));
+      h->own_stream = true;
+    }
+    const int d = h->d, dg = h->dg, F = h->F, L = h->L, dh = h->dh, pl = h->planes;
+    h->qkv.resize(L);
+    h->o.resize(L);
+    h->w13.resize(L);
+    h->w2.resize(L);
+    h->vc.resize(L);
+    h->oc.resize(L);
+    h->attn_norm.resize(L);
+    h->ffn_norm.resize(L);
+    for (int l = 0; l < L; ++l) {
+      const float* const* lw = w->layer + (size_t)l * BLT_LAYER_NT;
+      for (int t = 0; t < BLT_LAYER_NT; ++t)
+        if (!lw[t] && t != BLT_LAYER_WQ_C && t != BLT_LAYER_WK_C && t != BLT_LAYER_NORM_C)
+          return fail(h, BLT_ERR_INVALID_ARG, "layer %d tensor %d is NULL", l, t);
+      const float* wqkv = lw[BLT_LAYER_WQKV];
+      // q and k rows are grouped so that each 16-row tile holds 8 rotary pairs (j, j + dh/2)
+      TRY(pack_matrix(h, h->qkv[l], 3 * d, d, pl, [&](int r) -> const float* {
+        const int sec = r / d, rr = r % d;
+        if (sec == 2) return wqkv + (size_t)r * d;
+        const int tph = dh / 16;
+        const int tile = rr / 16, r16 = rr % 16;
+        const int head = tile / tph, tt = tile % tph;
+        const int j = tt * 8 + (r16 & 7) + (r16 >= 8 ? dh / 2 : 0);
+        return wqkv + ((size_t)sec * d + head * dh + j) * d;
+      }));
+      TRY(pack_matrix(h, h->o[l], d, d, pl, [&](int r) { return lw[BLT_LAYER_WO] + (size_t)r * d; }));
+      // SwiGLU: tile rows 0..7 = W1 rows j..j+7, rows 8..15 = the same rows of W3
+      TRY(pack_matrix(h, h->w13[l], 2 * F, d, pl, [&](int r) -> const float* {
+        const int tile = r / 16, r16 = r % 16;
+        const int j = tile * 8 + (r16 & 7);
+        return (r16 < 8 ? lw[BLT_LAYER_W1] : lw[BLT_LAYER_W3]) + (size_t)j * d;
+      }));
+      TRY(pack_matrix(h, h->w2[l], d, F, pl, [&](int r) { return lw[BLT_LAYER_W2] + (size_t)r * F; }));
+      TRY(pack_matrix(h, h->vc[l], d, dg, pl, [&](int r) { return lw[BLT_LAYER_WV_C] + (size_t)r * dg; }));
+      TRY(pack_matrix(h, h->oc[l], d, d, pl, [&](int r) { return lw[BLT_LAYER_WO_C] + (size_t)r * d; }));
+      TRY(upload(h, &h->attn_norm[l], lw[BLT_LAYER_ATTN_NORM], d));
+      TRY(upload(h, &h->ffn_norm[l], lw[BLT_LAYER_FFN_NORM], d));
+    }
+    TRY(pack_matrix(h, h->head, 256, d, pl, [&](int r) { return w->head + (size_t)r * d; }));
+    {
+      // the embedding is read once per row: keep it fp32, values rounded like the weights
+      std::vector<float> e((size_t)h->V * d);
+      for (size_t i = 0; i < e.size(); ++i) {
+        const float v = w->embed[i];
+        e[i] = (pl == 1) ? bf16_to_f(bf16_rne(v)) : v;
+      }
+      TRY(upload(h, &h->embed, e.data(), e.size()));
+    }
+    TRY(upload(h, &h->final_norm, w->final_norm, d));
+    {
+      const int half = dh / 2;
+      std::vector<float> cs((size_t)c.max_ctx * half), sn((size_t)c.max_ctx * half);
+      for (int p = 0; p < c.max_ctx; ++p)
+        for (int i = 0; i < half; ++i) {
+          const double ang = (double)p * std::pow((double)c.rope_theta, -2.0 * i / dh);
+          cs[(size_t)p * half + i] = (float)std::cos(ang);
+          sn[(size_t)p * half + i] = (float)std::sin(ang);
+        }
+      TRY(upload(h, &h->rope_cos, cs.data(), cs.size()));
+      TRY(upload(h, &h->rope_sin, sn.data(), sn.size()));
+    }
+    h->weight_bytes_per_pass = h->head.bytes();
+    for (int l = 0; l < L; ++l)
+      h->weight_bytes_per_pass += h->qkv[l].bytes() + h->o[l].bytes() + h->w13[l].bytes() + h->w2[l].bytes();
+    h->kv_bytes_per_key = (unsigned long long)L * 2 * d * 2;
+    // KV pool [pages][L][2][H][PT][dh] bf16
+    TRY(dalloc(h, &h->kv, (size_t)h->n_pages * L * 2 * d * h->PT));
+    TRY(dalloc(h, &h->page_table, (size_t)c.max_batch * h->max_pages));
+    CK(cudaMemset(h->page_table, 0xFF, (size_t)c.max_batch * h->max_pages * 4));
+    h->pt_host.assign((size_t)c.max_batch * h->max_pages, -1);
+    h->free_pages.resize(h->n_pages);
+    for (int i = 0; i < h->n_pages; ++i) h->free_pages[i] = h->n_pages - 1 - i;
+    h->seq_npages.assign(c.max_batch, 0);
+    TRY(dalloc(h, &h->c_lat, (size_t)c.max_batch * c.max_latents * L * d));
+    const int R = c.max_rows;
+    const int RL = std::max(R, c.max_batch * c.max_block + R);
+    TRY(dalloc(h, &h->h, (size_t)RL * d));
+    TRY(dalloc(h, &h->rs, RL));
+    TRY(dalloc(h, &h->q, (size_t)RL * d));
+    TRY(dalloc(h, &h->att, (size_t)RL * d));
+    TRY(dalloc(h, &h->act, (size_t)RL * F));
+    TRY(dalloc(h, &h->logits, (size_t)RL * 256));
+    TRY(dalloc(h, &h->tmp, (size_t)RL * d));
+    TRY(dalloc(h, &h->part_ml, (size_t)RL * h->H * h->CMAX));
+    TRY(dalloc(h, &h->part_o, (size_t)RL * h->H * h->CMAX * dh));
+    TRY(dalloc(h, &h->conf, RL));
+    TRY(dalloc(h, &h->gap, RL));
+    TRY(dalloc(h, &h->pred, RL));
+    RowsDev& rd = h->rows;
+    TRY(dalloc(h, &rd.seq, RL));
+    TRY(dalloc(h, &rd.pos, RL));
+    TRY(dalloc(h, &rd.lat, RL));
+    TRY(dalloc(h, &rd.nkeys, RL));
+    TRY(dalloc(h, &rd.byte, RL));
+    TRY(dalloc(h, &rd.n_rows, 1));
+    TRY(dalloc(h, &rd.g_seq, RL + c.max_batch));
+    TRY(dalloc(h, &rd.g_row0, RL + c.max_batch));
+    TRY(dalloc(h, &rd.g_nrows, RL + c.max_batch));
+    TRY(dalloc(h, &rd.g_kmax, RL + c.max_batch));
+    TRY(dalloc(h, &rd.n_groups, 1));
+    TRY(dalloc(h, &h->lat_seq, R));
+    TRY(dalloc(h, &h->lat_slot, R));
+    TRY(dalloc(h, &h->n_lat_rows, 1));
+    SeqDev& sd = h->sd;
+    const int B = c.max_batch;
+    TRY(dalloc(h, &sd.kv_len, B));
+    TRY(dalloc(h, &sd.kv_base, B));
+    TRY(dalloc(h, &sd.n_lat, B));
+    TRY(dalloc(h, &sd.active, B));
+    TRY(dalloc(h, &sd.steps, B));
+    TRY(dalloc(h, &sd.y_last, B));
+    TRY(dalloc(h, &sd.last_row, B));
+    TRY(dalloc(h, &sd.blk_row, (size_t)B * kMaxBlock));
+    TRY(dalloc(h, &sd.blk, (size_t)B * kMaxBlock));
+    TRY(dalloc(h, &sd.masked, (size_t)B * kMaxBlock));
+    TRY(dalloc(h, &sd.status, 1));
+    TRY(dalloc(h, &sd.counters, 8));
+    CK(cudaMemset(sd.kv_len, 0, B * 4));
+    CK(cudaMemset(sd.n_lat, 0, B * 4));
+    CK(cudaMemset(sd.active, 0, B * 4));
+    CK(cudaMemset(sd.status, 0, 4));
+    CK(cudaMemset(sd.counters, 0, 64));
+    CK(cudaMemset(sd.blk, 0, (size_t)B * kMaxBlock));
+    CK(cudaMemset(sd.masked, 0, (size_t)B * kMaxBlock));
+    CK(cudaMemset(h->c_lat, 0, (size_t)c.max_batch * c.max_latents * L * d * 4));
+    CK(cudaHostAlloc((void**)&h->mirror, 2 * B * 4, cudaHostAllocDefault));
+    CK(cudaEventCreateWithFlags(&h->mirror_ev, cudaEventDisableTiming));
+    h->kv_ub.assign(B, 0);
+    h->nlat_ub.assign(B, 0);
+    TRY(set_attrs_epi<EPI_STORE>(h));
+    TRY(set_attrs_epi<EPI_RESID>(h));
+    TRY(set_attrs_epi<EPI_SWIGLU>(h));
+    TRY(set_attrs_epi<EPI_QKV>(h));
+    TRY(set_attrs_epi<EPI_LATC>(h));
+    const size_t attn_smem = (size_t)(32 * dh + h->CH * dh + 32 * h->CH) * 4;
+    CK(cudaFuncSetAttribute(k_attn_partial<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
+    CK(cudaFuncSetAttribute(k_attn_partial<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
+    CK(cudaFuncSetAttribute(k_attn_partial<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
+    CK(cudaFuncSetAttribute(k_attn_partial<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
+    CK(cudaDeviceSynchronize());
+    return BLT_OK;
+  };
+  rc = run();
+  if (rc != BLT_OK) {
+    fprintf(stderr, "blt_dec_init: %s\n", h->err.c_str());
+    blt_dec_free(h);
+    return rc;
+  }
+  *out = h;
+  return BLT_OK;
+}
+
+int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (h->state != 0) return fail(h, BLT_ERR_STATE, "a draft is waiting for verification");
+  TRY(check_pending(h, rows, true));
+  CallDesc cd;
+  TRY(make_desc(h, batch, rows->row_offsets, rows->latent_offsets, cd));
+  const int total = cd.row_off[batch];
+  if (total > 0 && (!rows->bytes || !rows->row_latent)) return fail(h, BLT_ERR_INVALID_ARG, "bytes/row_latent NULL");
+  refresh_bounds(h);
+  TRY(reserve(h, cd, 0, true));
+  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  TRY(project_latents(h, cd, rows->new_latents, true));
+  k_snapshot_base<<<1, 256, 0, h->stream>>>(h->sd, batch);
+  int kmax = 0;
+  for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
+  const int chunk = h->cfg.max_rows;
+  for (int r0 = 0; r0 < total; r0 += chunk) {
+    const int r1 = std::min(total, r0 + chunk);
+    PlanArgs p = plan_args(h, PL_PREFILL, 0);
+    p.r0 = r0;
+    p.r1 = r1;
+    p.pend_bytes = rows->bytes;
+    p.pend_lat = rows->row_latent;
+    TRY(plan(h, p, cd));
+    TRY(run_pass(h, r1 - r0, kmax, (r1 - r0 + 31) / 32 + batch, out_logits != nullptr));
+    if (out_logits) k_copy_logits<<<256, 256, 0, h->stream>>>(h->logits, out_logits + (size_t)r0 * 256, (r1 - r0) * 256);
+  }
+  k_finish_prefill<<<1, 256, 0, h->stream>>>(h->sd, cd);
+  CK(cudaGetLastError());
+  bump_bounds(h, cd, 0);
+  return post_mirror(h);
+}
+
+int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float alpha, int max_steps,
+                          uint8_t* out_block, int32_t* out_steps, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  h->state = 0;  // a waiting draft is discarded
+  TRY(check_pending(h, pending, false));
+  if (k < 1 || k > h->cfg.max_block) return fail(h, BLT_ERR_INVALID_ARG, "k %d outside 1..%d", k, h->cfg.max_block);
+  if (!(alpha == alpha)) return fail(h, BLT_ERR_INVALID_ARG, "alpha is NaN");
+  if (!out_block) return fail(h, BLT_ERR_INVALID_ARG, "out_block is NULL");
+  if (max_steps <= 0) max_steps = k;
+  CallDesc cd;
+  TRY(make_desc(h, batch, pending->row_offsets, pending->latent_offsets, cd));
+  if (cd.row_off[batch] > 0 && (!pending->bytes || !pending->row_latent)) return fail(h, BLT_ERR_INVALID_ARG, "bytes/row_latent NULL");
+  if (cd.row_off[batch] + batch * k > h->cfg.max_rows)
+    return fail(h, BLT_ERR_NO_SPACE, "pass rows %d > max_rows %d", cd.row_off[batch] + batch * k, h->cfg.max_rows);
+  refresh_bounds(h);
+  TRY(reserve(h, cd, k, true));
+  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  TRY(project_latents(h, cd, pending->new_latents, true));
+  TRY(block_loop(h, cd, pending, k, alpha, max_steps, out_logits));
+  k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_block, out_steps);
+  CK(cudaGetLastError());
+  bump_bounds(h, cd, 0);
+  return post_mirror(h);
+}
+
+int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode, int k, float alpha, int max_steps,
+                  uint8_t* out_draft, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  h->state = 0;  // a waiting draft is discarded
+  TRY(check_pending(h, pending, true));
+  if (mode != BLT_DRAFT_AR && mode != BLT_DRAFT_DIFFUSION) return fail(h, BLT_ERR_INVALID_ARG, "mode %d", mode);
+  if (k < 1 || k > h->cfg.max_block) return fail(h, BLT_ERR_INVALID_ARG, "k %d outside 1..%d", k, h->cfg.max_block);
+  if (!out_draft) return fail(h, BLT_ERR_INVALID_ARG, "out_draft is NULL");
+  if (!(alpha == alpha)) return fail(h, BLT_ERR_INVALID_ARG, "alpha is NaN");
+  CallDesc cd;
+  TRY(make_desc(h, batch, pending->row_offsets, pending->latent_offsets, cd));
+  for (int s = 0; s < batch; ++s)
+    if (cd.row_off[s + 1] - cd.row_off[s] < 1)
+      return fail(h, BLT_ERR_INVALID_ARG, "sequence %d has no pending row (its prediction is y_l)", s);
+  if (!pending->bytes || !pending->row_latent) return fail(h, BLT_ERR_INVALID_ARG, "bytes/row_latent NULL");
+  const int rows1 = cd.row_off[batch] + (mode == BLT_DRAFT_DIFFUSION ? batch * k : 0);
+  if (rows1 > h->cfg.max_rows) return fail(h, BLT_ERR_NO_SPACE, "pass rows %d > max_rows %d", rows1, h->cfg.max_rows);
+  refresh_bounds(h);
+  TRY(reserve(h, cd, k, true));
+  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  TRY(project_latents(h, cd, pending->new_latents, true));
+  if (mode == BLT_DRAFT_AR) {
+    int npmax = 0;
+    for (int s = 0; s < batch; ++s) npmax = std::max(npmax, cd.row_off[s + 1] - cd.row_off[s]);
+    const int keys_ub = max_kv_ub(h, batch) + npmax + k;
+    PlanArgs p = plan_args(h, PL_FIRST, 0);
+    p.pend_bytes = pending->bytes;
+    p.pend_lat = pending->row_latent;
+    TRY(plan(h, p, cd));
+    TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true));
+    k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, 0, h->pred, h->logits, out_logits);
+    for (int t = 1; t < k; ++t) {
+      PlanArgs pa = plan_args(h, PL_ARDRAFT, 0);
+      pa.step = t;
+      TRY(plan(h, pa, cd));
+      TRY(run_pass(h, batch, keys_ub, batch, true));
+      k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, t, h->pred, h->logits, out_logits);
+    }
+  } else {
+    if (max_steps <= 0) max_steps = k;
+    TRY(block_loop(h, cd, pending, k, alpha, max_steps, out_logits));
+  }
+  if (mode == BLT_DRAFT_DIFFUSION) k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft, nullptr);
+  else k_copy_draft<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft);
+  CK(cudaGetLastError());
+  bump_bounds(h, cd, 0);
+  h->state = 1;
+  h->draft_k = k;
+  h->draft_batch = batch;
+  return post_mirror(h);
+}
+
+int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const float* new_latents,
+                          const int32_t* latent_offsets, int32_t* out_accepted, uint8_t* out_next, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (h->state != 1) return fail(h, BLT_ERR_STATE, "no draft is waiting for verification");
+  if (!draft_row_latent || !out_accepted || !out_next) return fail(h, BLT_ERR_INVALID_ARG, "NULL argument");
+  const int batch = h->draft_batch, k = h->draft_k;
+  if (batch * k > h->cfg.max_rows) return fail(h, BLT_ERR_NO_SPACE, "pass rows %d > max_rows %d", batch * k, h->cfg.max_rows);
+  CallDesc cd;
+  TRY(make_desc(h, batch, nullptr, latent_offsets, cd));
+  refresh_bounds(h);
+  TRY(reserve(h, cd, k, false));
+  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  TRY(project_latents(h, cd, new_latents, false));
+  PlanArgs p = plan_args(h, PL_VERIFY, k);
+  p.vlat = draft_row_latent;
+  TRY(plan(h, p, cd));
+  TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true));
+  k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
+  CK(cudaGetLastError());
+  for (int s = 0; s < batch; ++s) {
+    h->kv_ub[s] += k;
+    h->nlat_ub[s] += cd.lat_off[s + 1] - cd.lat_off[s];
+  }
+  h->state = 0;
+  return post_mirror(h);
+}
+
+int blt_dec_rewind(blt_dec_t* h, int batch, const int32_t* kv_len, const int32_t* n_latents) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (batch < 1 || batch > h->cfg.max_batch) return fail(h, BLT_ERR_INVALID_ARG, "batch %d", batch);
+  CallDesc cd{};
+  cd.batch = batch;
+  for (int s = 0; s < batch; ++s) {
+    cd.row_off[s] = kv_len ? kv_len[s] : -1;
+    cd.lat_off[s] = n_latents ? n_latents[s] : -1;
+  }
+  k_rewind<<<1, 256, 0, h->stream>>>(h->sd, cd);
+  CK(cudaGetLastError());
+  CK(cudaStreamSynchronize(h->stream));
+  const int B = h->cfg.max_batch;
+  CK(cudaMemcpy(h->mirror, h->sd.kv_len, B * 4, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(h->mirror + B, h->sd.n_lat, B * 4, cudaMemcpyDeviceToHost));
+  for (int s = 0; s < B; ++s) {
+    h->kv_ub[s] = h->mirror[s];
+    h->nlat_ub[s] = h->mirror[B + s];
+  }
+  h->mirror_pending = false;
+  h->state = 0;
+  return BLT_OK;
+}
+
+int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
+  if (!h || !out) return BLT_ERR_INVALID_ARG;
+  unsigned long long c[8];
+  CK(cudaStreamSynchronize(h->stream));
+  CK(cudaMemcpy(c, h->sd.counters, sizeof c, cudaMemcpyDeviceToHost));
+  out->passes = c[0];
+  out->rows = c[1];
+  out->prefill_rows = c[2];
+  out->latents = c[3];
+  out->calls = c[4];
+  out->weight_bytes = c[5];
+  out->kv_read_bytes = c[6];
+  return BLT_OK;
+}
+
+int blt_dec_sync(blt_dec_t* h) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  CK(cudaStreamSynchronize(h->stream));
+  int st = 0;
+  CK(cudaMemcpy(&st, h->sd.status, 4, cudaMemcpyDeviceToHost));
+  if (st != 0) {
+    CK(cudaMemset(h->sd.status, 0, 4));
+    return fail(h, st, "device status %d (%s)", st, st == BLT_ERR_STEP_LIMIT ? "step limit" : "device index check");
+  }
+  return BLT_OK;
+}
+
+const char* blt_dec_last_error(blt_dec_t* h) { return h ? h->err.c_str() : "NULL handle"; }
+
+void blt_dec_free(blt_dec_t* h) {
+  if (!h) return;
+  if (h->stream) cudaStreamSynchronize(h->stream);
+  for (void* p : h->allocs) cudaFree(p);
+  if (h->mirror) cudaFreeHost(h->mirror);
+  if (h->mirror_ev) cudaEventDestroy(h->mirror_ev);
+  if (h->own_stream && h->stream) cudaStreamDestroy(h->stream);
+  delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,845 @@
+// Kernels of one Fast-BLT local-decoder pass and its bookkeeping (sm_100a).
+//
+// Decoder layer ("계층적 BLT: 인코더, 글로벌 모델, 디코더", the layer equation of
+// the Fast-BLT summary page): the cross-attention term for a row that sees
+// exactly one latent o is W_o^c W_v^c o (softmax over one key is 1), added to
+// the residual; then pre-norm self-attention and a SwiGLU FFN.
+//
+// Canonical arithmetic of every projection y = W x (one fp32 value per output):
+//   x is split into bf16 planes x_hi + x_lo; W is one bf16 plane (or hi + lo
+//   for fp32 weights).  K is cut into k16 steps; step s belongs to lane group
+//   w = s mod 8.  Group w accumulates, in increasing s, the tensor-core products
+//   W_hi x_hi, W_hi x_lo (, W_lo x_hi) into one fp32 accumulator; the output is
+//   ((g_0 + g_1) + ...) + g_7.  The order depends on nothing but K, so a row
+//   gets bit-identical results whatever the other rows of its pass are.
+#pragma once
+
+#include "common.cuh"
+
+namespace bltdec {
+
+enum RowKind : int { ROW_CAUSAL = 0, ROW_BLOCK = 1 };
+
+// Per-pass row metadata (device arrays sized max_rows; counts are device scalars).
+struct RowsDev {
+  int* seq;     // sequence of the row
+  int* pos;     // 0-based byte position (RoPE, KV slot)
+  int* lat;     // latent slot seen by the cross-attention
+  int* nkeys;   // the row attends positions 0 .. nkeys-1 of its sequence
+  int* byte;    // input id (0..255 or [MASK])
+  int* n_rows;  // device scalar
+  // attention groups: up to 32 consecutive rows of one sequence
+  int* g_seq;
+  int* g_row0;
+  int* g_nrows;
+  int* g_kmax;
+  int* n_groups;  // device scalar
+};
+
+// ------------------------------------------------------------------------ GEMM
+enum Epi : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_LATC = 4 };
+
+struct GemmArgs {
+  const uint4* w;  // tiles [N/16][K/16][planes][32 lanes] of 16 B
+  int N, K;
+  const float* X;  // activations [rows][ldx] fp32
+  int ldx;
+  const float* rs;    // per-row RMS scale (NULL: x used as is)
+  const float* gain;  // [K] RMSNorm gain (with rs)
+  const int* n_rows;  // device row count (NULL: rows_host is exact)
+  int rows_host;
+  float* out;  // EPI_STORE / RESID / SWIGLU / LATC base
+  int ldo;
+  // EPI_QKV
+  float* q;
+  __nv_bfloat16* kv;
+  const int* page_table;
+  int max_pages, PT, layer, L, H, dh, d;
+  const int* row_seq;
+  const int* row_pos;
+  const float* rope_cos;  // [max_ctx][dh/2]
+  const float* rope_sin;
+  int max_ctx;
+  // EPI_LATC
+  const int* lat_seq;
+  const int* lat_slot;
+  int max_lat;
+  int* status;
+};
+
+__device__ __forceinline__ size_t kv_offset(const GemmArgs& a, int page, int kvsel, int h, int off, int dim) {
+  return ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * a.dh + (size_t)off * a.dh + dim;
+}
+
+template <int EPI>
+__device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16, int row, float v0, float v1) {
+  if constexpr (EPI == EPI_STORE) {
+    float* o = a.out + (size_t)row * a.ldo + mt * 16 + r16;
+    o[0] = v0;
+    o[8] = v1;
+  } else if constexpr (EPI == EPI_RESID) {
+    float* o = a.out + (size_t)row * a.ldo + mt * 16 + r16;
+    o[0] += v0;
+    o[8] += v1;
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    a.out[(size_t)row * a.ldo + mt * 8 + r16] = silu(v0) * v1;
+  } else if constexpr (EPI == EPI_LATC) {
+    const int s = a.lat_seq[row], slot = a.lat_slot[row];
+    float* o = a.out + (((size_t)s * a.max_lat + slot) * a.L + a.layer) * a.d + mt * 16 + r16;
+    o[0] = v0;
+    o[8] = v1;
+  } else {  // EPI_QKV
+    const int tiles_sec = a.d / 16;
+    const int sec = mt / tiles_sec, lt = mt % tiles_sec;
+    const int pos = a.row_pos[row];
+    if (sec < 2) {
+      const int tph = a.dh / 16;  // tiles per head
+      const int h = lt / tph, j = (lt % tph) * 8 + r16;
+      const int half = a.dh / 2;
+      const float c = a.rope_cos[(size_t)pos * half + j], s = a.rope_sin[(size_t)pos * half + j];
+      const float o0 = v0 * c - v1 * s, o1 = v1 * c + v0 * s;
+      if (sec == 0) {
+        float* q = a.q + (size_t)row * a.d + h * a.dh;
+        q[j] = o0;
+        q[j + half] = o1;
+      } else {
+        const int seq = a.row_seq[row];
+        const int pi = pos / a.PT;
+        const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+        if (page < 0) {
+          set_status(a.status, kErrDevice);
+          return;
+        }
+        __nv_bfloat16* k = a.kv + kv_offset(a, page, 0, h, pos % a.PT, 0);
+        k[j] = __float2bfloat16_rn(o0);
+        k[j + half] = __float2bfloat16_rn(o1);
+      }
+    } else {
+      const int seq = a.row_seq[row];
+      const int pi = pos / a.PT;
+      const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+      if (page < 0) {
+        set_status(a.status, kErrDevice);
+        return;
+      }
+      const int n0 = lt * 16 + r16, n1 = n0 + 8;
+      a.kv[kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh)] = __float2bfloat16_rn(v0);
+      a.kv[kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh)] = __float2bfloat16_rn(v1);
+    }
+  }
+}
+
+// One CTA: one 16-row tile of W against RB = 8*NG activation rows.
+// 8 warps; warp w owns k16 steps w, w+8, ... (the canonical split).
+template <int NG, int PL, int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
+  constexpr int RB = 8 * NG;
+  const int nrows = a.n_rows ? *a.n_rows : a.rows_host;
+  const int mt = blockIdx.x;
+  const int row0 = blockIdx.y * RB;
+  if (row0 >= nrows) return;
+  const int nr = min(RB, nrows - row0);
+
+  extern __shared__ float4 smem4[];
+  float* xs = reinterpret_cast<float*>(smem4);  // [STAGES][RB][kXStride]
+  float* rsv = xs + STAGES * RB * kXStride;     // [RB]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int nwin = a.K / kKWin;
+  const int ksteps = a.K / 16;
+
+  if (tid < RB) rsv[tid] = (a.rs && tid < nr) ? a.rs[row0 + tid] : 1.0f;
+
+  auto stage = [&](int wi, int buf) {
+    // RB rows x 128 floats = RB*32 chunks of 16 B
+    for (int c = tid; c < RB * 32; c += kThreads) {
+      const int r = c >> 5, q = c & 31;
+      const bool ok = r < nr;
+      const float* src = a.X + (size_t)(ok ? row0 + r : row0) * a.ldx + wi * kKWin + q * 4;
+      cp_async16(xs + ((size_t)buf * RB + r) * kXStride + q * 4, src, ok ? 16 : 0);
+    }
+  };
+
+  // weight tile of window wi for this warp, plane p
+  const uint4* wbase = a.w + (size_t)mt * ksteps * PL * 32 + lane;
+  auto wtile = [&](int wi, int p) -> uint4 { return ldg_stream(wbase + ((size_t)(wi * kWarps + warp) * PL + p) * 32); };
+
+  constexpr int DEPTH = 4;
+  uint4 wb[DEPTH][PL];
+#pragma unroll
+  for (int dd = 0; dd < DEPTH; ++dd)
+#pragma unroll
+    for (int p = 0; p < PL; ++p) wb[dd][p] = (dd < nwin) ? wtile(dd, p) : make_uint4(0, 0, 0, 0);
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < nwin) stage(s, s);
+    cp_async_commit();
+  }
+
+  float acc[NG][4];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+
+  __syncthreads();  // rsv
+  const bool has_gain = a.rs != nullptr;
+
+  for (int wi0 = 0; wi0 < nwin; wi0 += DEPTH) {
+#pragma unroll
+    for (int dd = 0; dd < DEPTH; ++dd) {
+      const int wi = wi0 + dd;
+      if (wi < nwin) {
+        uint4 wcur[PL];
+#pragma unroll
+        for (int p = 0; p < PL; ++p) {
+          wcur[p] = wb[dd][p];
+          if (wi + DEPTH < nwin) wb[dd][p] = wtile(wi + DEPTH, p);
+        }
+        cp_async_wait<STAGES - 2>();
+        __syncthreads();
+        // refill the stage consumed STAGES-1 windows ago
+        if (wi + STAGES - 1 < nwin) stage(wi + STAGES - 1, (wi + STAGES - 1) % STAGES);
+        cp_async_commit();
+
+        const float* xw = xs + (size_t)(wi % STAGES) * RB * kXStride;
+        const int kk = warp * 16 + 2 * t;  // column within the window
+        const int kg = wi * kKWin + kk;    // global k
+        float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
+        if (has_gain) {
+          g0 = __ldg(a.gain + kg);
+          g1 = __ldg(a.gain + kg + 1);
+          g8 = __ldg(a.gain + kg + 8);
+          g9 = __ldg(a.gain + kg + 9);
+        }
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          const int r = n * 8 + g;
+          const float* xr = xw + r * kXStride + kk;
+          const float2 p0 = *reinterpret_cast<const float2*>(xr);
+          const float2 p8 = *reinterpret_cast<const float2*>(xr + 8);
+          const float sc = rsv[r];
+          uint32_t b0h, b0l, b1h, b1l;
+          split2(p0.x * sc * g0, p0.y * sc * g1, b0h, b0l);
+          split2(p8.x * sc * g8, p8.y * sc * g9, b1h, b1l);
+          mma16816(acc[n], wcur[0], b0h, b1h);
+          mma16816(acc[n], wcur[0], b0l, b1l);
+          if constexpr (PL == 2) mma16816(acc[n], wcur[1], b0h, b1h);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // cross-warp reduction in canonical order
+  float* red = xs;  // [8][16][RB]
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    const int c = n * 8 + 2 * t;
+    red[(warp * 16 + g) * RB + c] = acc[n][0];
+    red[(warp * 16 + g) * RB + c + 1] = acc[n][1];
+    red[(warp * 16 + g + 8) * RB + c] = acc[n][2];
+    red[(warp * 16 + g + 8) * RB + c + 1] = acc[n][3];
+  }
+  __syncthreads();
+  for (int p = tid; p < 8 * RB; p += kThreads) {
+    const int r16 = p & 7, col = p >> 3;
+    if (col >= nr) continue;
+    float v0 = red[r16 * RB + col], v1 = red[(r16 + 8) * RB + col];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      v0 += red[(w * 16 + r16) * RB + col];
+      v1 += red[(w * 16 + r16 + 8) * RB + col];
+    }
+    gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1);
+  }
+}
+
+// ------------------------------------------------------------------------ row-wise kernels
+// h[row] = embed[byte[row]]
+__global__ void k_embed(const RowsDev rows, const float* __restrict__ embed, float* __restrict__ h, int d, int rows_max) {
+  const int n = *rows.n_rows;
+  for (int r = blockIdx.x; r < n; r += gridDim.x) {
+    const float* e = embed + (size_t)rows.byte[r] * d;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) h[(size_t)r * d + i] = e[i];
+  }
+}
+
+// h[row] += c_lat[seq][lat][layer] (when c_lat != NULL); rs[row] = 1/sqrt(mean(h^2) + eps).
+// One warp per row.
+__global__ void k_rownorm(const RowsDev rows, float* __restrict__ h, float* __restrict__ rs, const float* __restrict__ c_lat,
+                          int max_lat, int L, int layer, int d, float eps, const int* n_rows_override) {
+  const int n = n_rows_override ? *n_rows_override : *rows.n_rows;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int r = warp; r < n; r += nw) {
+    float* hr = h + (size_t)r * d;
+    const float* cr = c_lat ? c_lat + (((size_t)rows.seq[r] * max_lat + rows.lat[r]) * L + layer) * d : nullptr;
+    float ss = 0.f;
+    for (int i = lane * 4; i < d; i += 128) {
+      float4 v = *reinterpret_cast<float4*>(hr + i);
+      if (cr) {
+        const float4 c = *reinterpret_cast<const float4*>(cr + i);
+        v.x += c.x;
+        v.y += c.y;
+        v.z += c.z;
+        v.w += c.w;
+        *reinterpret_cast<float4*>(hr + i) = v;
+      }
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) rs[r] = 1.0f / sqrtf(ss / (float)d + eps);
+  }
+}
+
+// ------------------------------------------------------------------------ attention
+struct AttnArgs {
+  const float* q;  // [rows][d], RoPE applied
+  const __nv_bfloat16* kv;
+  const int* page_table;
+  int max_pages, PT, L, layer, H, dh, d;
+  RowsDev rows;
+  int CH, CMAX;
+  float scale;
+  float2* part_ml;  // [rows][H][CMAX]
+  float* part_o;    // [rows][H][CMAX][dh]
+  float* att;       // [rows][d]
+  int* status;
+};
+
+// grid (H, chunks, groups); 128 threads; dh == 64 or smaller power of two <= 64 handled by DH template.
+template <int DH>
+__global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
+  constexpr int MAXR = 32;
+  const int gi = blockIdx.z;
+  if (gi >= *a.rows.n_groups) return;
+  const int kmax = a.rows.g_kmax[gi];
+  const int t0 = blockIdx.y * a.CH;
+  if (t0 >= kmax) return;
+  const int h = blockIdx.x;
+  const int seq = a.rows.g_seq[gi], row0 = a.rows.g_row0[gi], nr = a.rows.g_nrows[gi];
+  const int nk = min(a.CH, kmax - t0);
+
+  extern __shared__ float4 smem4[];
+  float* qs = reinterpret_cast<float*>(smem4);  // [MAXR][DH]
+  float* vs = qs + MAXR * DH;                   // [CH][DH]
+  float* ps = vs + a.CH * DH;                   // [MAXR][CH]
+  __shared__ int lim[MAXR];
+
+  const int tid = threadIdx.x;
+  for (int i = tid; i < nr * DH; i += 128) {
+    const int r = i / DH, c = i % DH;
+    qs[r * DH + c] = a.q[(size_t)(row0 + r) * a.d + h * DH + c] * a.scale;
+  }
+  if (tid < MAXR) lim[tid] = (tid < nr) ? a.rows.nkeys[row0 + tid] - t0 : 0;
+  // V chunk -> smem (fp32)
+  for (int i = tid; i < nk * (DH / 8); i += 128) {
+    const int key = i / (DH / 8), c8 = (i % (DH / 8)) * 8;
+    const int tpos = t0 + key;
+    int page = a.page_table[seq * a.max_pages + tpos / a.PT];
+    if (page < 0) {
+      set_status(a.status, kErrDevice);
+      page = 0;
+    }
+    const __nv_bfloat16* src =
+        a.kv + ((((size_t)page * a.L + a.layer) * 2 + 1) * a.H + h) * (size_t)a.PT * DH + (size_t)(tpos % a.PT) * DH + c8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(src);
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vs[key * DH + c8 + e] = __bfloat162float(b[e]);
+  }
+  __syncthreads();
+  // scores: thread = key (CH <= 128), K row in registers
+  for (int key = tid; key < a.CH; key += 128) {
+    float kr[DH];
+    const bool valid = key < nk;
+    if (valid) {
+      const int tpos = t0 + key;
+      int page = a.page_table[seq * a.max_pages + tpos / a.PT];
+      if (page < 0) {
+        set_status(a.status, kErrDevice);
+        page = 0;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(
+          a.kv + ((((size_t)page * a.L + a.layer) * 2 + 0) * a.H + h) * (size_t)a.PT * DH + (size_t)(tpos % a.PT) * DH);
+#pragma unroll
+      for (int c = 0; c < DH / 8; ++c) {
+        const uint4 raw = src[c];
+        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kr[c * 8 + e] = __bfloat162float(b[e]);
+      }
+    }
+    for (int r = 0; r < nr; ++r) {
+      float s = -INFINITY;
+      if (valid && key < lim[r]) {
+        s = 0.f;
+#pragma unroll
+        for (int c = 0; c < DH; ++c) s = fmaf(qs[r * DH + c], kr[c], s);
+      }
+      ps[r * a.CH + key] = s;
+    }
+  }
+  __syncthreads();
+  // softmax statistics per row: warp per row
+  const int warp = tid >> 5, lane = tid & 31;
+  __shared__ float mrow[MAXR], lrow[MAXR];
+  for (int r = warp; r < nr; r += 4) {
+    float m = -INFINITY;
+    for (int k = lane; k < a.CH; k += 32) m = fmaxf(m, ps[r * a.CH + k]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int k = lane; k < a.CH; k += 32) {
+      const float s = ps[r * a.CH + k];
+      const float p = (s == -INFINITY) ? 0.f : expf(s - m);
+      ps[r * a.CH + k] = p;
+      l += p;
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      mrow[r] = m;
+      lrow[r] = l;
+    }
+  }
+  __syncthreads();
+  // o = P V: thread -> (dim, row phase)
+  for (int i = tid; i < nr * DH; i += 128) {
+    const int r = i / DH, c = i % DH;
+    float o = 0.f;
+    for (int k = 0; k < nk; ++k) o = fmaf(ps[r * a.CH + k], vs[k * DH + c], o);
+    const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + blockIdx.y;
+    a.part_o[base * DH + c] = o;
+    if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+  }
+}
+
+// att[row][h*dh + c] = combine of the row's chunks in chunk order.  grid (rows_max, H), block dh.
+__global__ void k_attn_combine(AttnArgs a) {
+  const int row = blockIdx.x;
+  if (row >= *a.rows.n_rows) return;
+  const int h = blockIdx.y, c = threadIdx.x;
+  const int nk = a.rows.nkeys[row];
+  const int nch = (nk + a.CH - 1) / a.CH;
+  const size_t base = ((size_t)row * a.H + h) * a.CMAX;
+  float m = -INFINITY;
+  for (int ch = 0; ch < nch; ++ch) {
+    const float2 ml = a.part_ml[base + ch];
+    if (ml.y > 0.f) m = fmaxf(m, ml.x);
+  }
+  float l = 0.f, o = 0.f;
+  for (int ch = 0; ch < nch; ++ch) {
+    const float2 ml = a.part_ml[base + ch];
+    if (ml.y > 0.f) {
+      const float w = expf(ml.x - m);
+      l += ml.y * w;
+      o += a.part_o[(base + ch) * a.dh + c] * w;
+    }
+  }
+  a.att[(size_t)row * a.d + h * a.dh + c] = o / l;
+}
+
+// ------------------------------------------------------------------------ byte head statistics
+// One warp per row over the 256 byte logits: confidence (largest softmax
+// probability), argmax (lowest byte on ties), gap between the two largest logits.
+__global__ void k_head_stats(const float* __restrict__ logits, const int* n_rows, float* conf, int* pred, float* gap) {
+  const int n = *n_rows;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int r = warp; r < n; r += nw) {
+    const float* z = logits + (size_t)r * 256;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = z[lane + 32 * j];
+    float b1 = -INFINITY, b2 = -INFINITY;
+    int i1 = 1 << 30;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int idx = lane + 32 * j;
+      if (v[j] > b1) {
+        b2 = b1;
+        b1 = v[j];
+        i1 = idx;
+      } else {
+        b2 = fmaxf(b2, v[j]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
+      const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
+      const int oi1 = __shfl_xor_sync(0xffffffffu, i1, o);
+      if (ob1 > b1 || (ob1 == b1 && oi1 < i1)) {
+        b2 = fmaxf(b1, ob2);
+        b1 = ob1;
+        i1 = oi1;
+      } else {
+        b2 = fmaxf(b2, ob1);
+      }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += expf(v[j] - b1);
+    s = warp_sum(s);
+    if (lane == 0) {
+      conf[r] = 1.0f / s;
+      pred[r] = i1;
+      gap[r] = b1 - b2;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ planning
+enum PlanMode : int { PL_PREFILL = 0, PL_FIRST = 1, PL_BLOCK = 2, PL_ARDRAFT = 3, PL_VERIFY = 4 };
+
+constexpr int kMaxCallBatch = 256;
+
+struct CallDesc {  // by value as a kernel parameter
+  int batch;
+  int row_off[kMaxCallBatch + 1];
+  int lat_off[kMaxCallBatch + 1];
+};
+
+struct SeqDev {
+  int* kv_len;     // cached committed positions
+  int* kv_base;    // kv_len at call start (prefill)
+  int* n_lat;      // committed latent slots
+  int* active;     // block still has masked positions
+  int* steps;      // passes used by the current block
+  int* y_last;     // greedy prediction of the last pending row (verification y_l)
+  int* last_row;   // row index of the last pending row in pass 1 (-1: none)
+  int* blk_row;    // [batch][kMaxBlock] row index of block/draft/verify row i in this pass
+  unsigned char* blk;     // [batch][kMaxBlock] block / draft bytes
+  unsigned char* masked;  // [batch][kMaxBlock]
+  int* status;
+  unsigned long long* counters;  // passes, rows, prefill_rows, latents, calls, weight_bytes, kv_bytes
+};
+
+struct PlanArgs {
+  int mode, k, step, r0, r1;
+  int max_ctx, max_lat, mask_id;
+  const unsigned char* pend_bytes;
+  const int* pend_lat;
+  const int* vlat;  // verify slots [batch][k]
+  int n_new_lat_total;
+  unsigned long long weight_bytes_per_pass;
+  unsigned long long kv_bytes_per_key;
+};
+
+// One CTA builds the rows of a pass.  Sequences' rows are contiguous, so each
+// attention group (<= 32 rows) belongs to one sequence.
+__global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd, RowsDev rd) {
+  __shared__ int cnt[kMaxCallBatch + 1];
+  __shared__ int gcnt[kMaxCallBatch + 1];
+  __shared__ int npend[kMaxCallBatch];
+  const int B = cd.batch, tid = threadIdx.x;
+  if (tid == 0) {
+    int off = 0, goff = 0;
+    for (int s = 0; s < B; ++s) {
+      int np = cd.row_off[s + 1] - cd.row_off[s];
+      int n = 0;
+      if (p.mode == PL_PREFILL) {
+        const int lo = max(cd.row_off[s], p.r0), hi = min(cd.row_off[s + 1], p.r1);
+        n = max(0, hi - lo);
+      } else if (p.mode == PL_FIRST) {
+        n = np + p.k;
+      } else if (p.mode == PL_BLOCK) {
+        n = sd.active[s] ? p.k : 0;
+      } else if (p.mode == PL_ARDRAFT) {
+        n = 1;
+      } else {
+        n = p.k;
+      }
+      npend[s] = np;
+      cnt[s] = off;
+      gcnt[s] = goff;
+      off += n;
+      goff += (n + 31) / 32;
+    }
+    cnt[B] = off;
+    gcnt[B] = goff;
+    *rd.n_rows = off;
+    *rd.n_groups = goff;
+  }
+  __syncthreads();
+  const int n_rows = cnt[B];
+  for (int r = tid; r < n_rows; r += blockDim.x) {
+    int lo = 0, hi = B;  // find s with cnt[s] <= r < cnt[s+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (cnt[mid] <= r) lo = mid;
+      else hi = mid;
+    }
+    const int s = lo, i = r - cnt[s];
+    int pos, lat, byte, nkeys, blk_i = -1;
+    const int kvl = sd.kv_len[s];
+    const int nl = sd.n_lat[s];
+    if (p.mode == PL_PREFILL) {
+      const int src = max(cd.row_off[s], p.r0) + i;
+      pos = sd.kv_base[s] + (src - cd.row_off[s]);
+      byte = p.pend_bytes[src];
+      lat = p.pend_lat[src];
+      nkeys = pos + 1;
+    } else if (p.mode == PL_FIRST) {
+      const int np = npend[s];
+      if (i < np) {
+        const int src = cd.row_off[s] + i;
+        pos = kvl + i;
+        byte = p.pend_bytes[src];
+        lat = p.pend_lat[src];
+        nkeys = pos + 1;
+        if (i == np - 1) sd.last_row[s] = r;
+      } else {
+        blk_i = i - np;
+        pos = kvl + i;
+        byte = p.mask_id;
+        lat = nl - 1;
+        nkeys = kvl + np + p.k;
+      }
+    } else if (p.mode == PL_BLOCK) {
+      blk_i = i;
+      pos = kvl + i;
+      byte = sd.masked[s * kMaxBlock + i] ? p.mask_id : sd.blk[s * kMaxBlock + i];
+      lat = nl - 1;
+      nkeys = kvl + p.k;
+    } else if (p.mode == PL_ARDRAFT) {
+      blk_i = 0;
+      pos = kvl + p.step - 1;
+      byte = sd.blk[s * kMaxBlock + p.step - 1];
+      lat = nl - 1;
+      nkeys = pos + 1;
+    } else {  // PL_VERIFY
+      blk_i = i;
+      pos = kvl + i;
+      byte = sd.blk[s * kMaxBlock + i];
+      lat = p.vlat[s * p.k + i];
+      nkeys = pos + 1;
+    }
+    const int lat_cap = nl + ((p.mode == PL_VERIFY) ? (cd.lat_off[s + 1] - cd.lat_off[s]) : 0);
+    if (pos < 0 || pos >= p.max_ctx || lat < 0 || lat >= lat_cap || lat >= p.max_lat || byte < 0 || byte > p.mask_id) {
+      set_status(sd.status, kErrDevice);
+      pos = min(max(pos, 0), p.max_ctx - 1);
+      lat = 0;
+      byte = 0;
+      nkeys = min(max(nkeys, 1), pos + 1);
+    }
+    rd.seq[r] = s;
+    rd.pos[r] = pos;
+    rd.lat[r] = lat;
+    rd.byte[r] = byte;
+    rd.nkeys[r] = nkeys;
+    if (blk_i >= 0) sd.blk_row[s * kMaxBlock + blk_i] = r;
+  }
+  // attention groups
+  for (int gi = tid; gi < gcnt[B]; gi += blockDim.x) {
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (gcnt[mid] <= gi) lo = mid;
+      else hi = mid;
+    }
+    const int s = lo, j = gi - gcnt[s];
+    const int r0 = cnt[s] + 32 * j;
+    const int n = min(32, cnt[s + 1] - r0);
+    rd.g_seq[gi] = s;
+    rd.g_row0[gi] = r0;
+    rd.g_nrows[gi] = n;
+  }
+  __syncthreads();
+  for (int gi = tid; gi < gcnt[B]; gi += blockDim.x) {
+    int km = 0;
+    for (int r = rd.g_row0[gi]; r < rd.g_row0[gi] + rd.g_nrows[gi]; ++r) km = max(km, rd.nkeys[r]);
+    rd.g_kmax[gi] = km;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (p.mode == PL_FIRST) {
+      for (int s = 0; s < B; ++s) {
+        if (npend[s] == 0) sd.last_row[s] = -1;
+        sd.kv_len[s] += npend[s];
+        if (p.k > 0) {
+          sd.active[s] = 1;
+          sd.steps[s] = 0;
+          for (int i = 0; i < p.k; ++i) sd.masked[s * kMaxBlock + i] = 1;
+        }
+      }
+    }
+    if (n_rows > 0) {
+      // algorithmic K/V bytes: each sequence's keys are read once per layer
+      unsigned long long kvk = 0;
+      for (int gi = 0; gi < gcnt[B]; ++gi) {
+        const bool first = gi == 0 || rd.g_seq[gi - 1] != rd.g_seq[gi];
+        if (first) {
+          int km = 0;
+          for (int gj = gi; gj < gcnt[B] && rd.g_seq[gj] == rd.g_seq[gi]; ++gj) km = max(km, rd.g_kmax[gj]);
+          kvk += km;
+        }
+      }
+      if (p.mode == PL_PREFILL) {
+        sd.counters[2] += n_rows;
+      } else {
+        sd.counters[0] += 1;
+        sd.counters[5] += p.weight_bytes_per_pass;
+      }
+      sd.counters[1] += n_rows;
+      sd.counters[6] += kvk * p.kv_bytes_per_key;
+    }
+  }
+}
+
+// Latent rows: new latent j of sequence s goes to slot n_lat[s] + (j - lat_off[s]).
+__global__ void k_lat_plan(CallDesc cd, SeqDev sd, int* lat_seq, int* lat_slot, int* n_lat_rows, int r0, int r1, int commit,
+                           int max_lat) {
+  const int B = cd.batch;
+  for (int j = r0 + threadIdx.x; j < r1; j += blockDim.x) {
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (cd.lat_off[mid] <= j) lo = mid;
+      else hi = mid;
+    }
+    const int slot = sd.n_lat[lo] + (j - cd.lat_off[lo]);
+    lat_seq[j - r0] = lo;
+    lat_slot[j - r0] = min(slot, max_lat - 1);
+    if (slot >= max_lat) set_status(sd.status, kErrDevice);
+  }
+  if (threadIdx.x == 0) *n_lat_rows = r1 - r0;
+  __syncthreads();
+  if (commit && threadIdx.x == 0 && r1 == cd.lat_off[B]) {
+    for (int s = 0; s < B; ++s) sd.n_lat[s] += cd.lat_off[s + 1] - cd.lat_off[s];
+    sd.counters[3] += cd.lat_off[B];
+  }
+}
+
+// ------------------------------------------------------------------------ bookkeeping
+// Confidence unmasking of every active block ("블록 언마스킹 전략").  One warp per
+// sequence, lane = block position.
+__global__ void k_unmask(SeqDev sd, int batch, int k, float alpha, int step, const float* conf, const int* pred,
+                         const float* logits, float* out_logits) {
+  const int s = blockIdx.x, lane = threadIdx.x;
+  if (s >= batch || !sd.active[s]) return;
+  if (step == 0 && lane == 0) {
+    const int lr = sd.last_row[s];
+    if (lr >= 0) sd.y_last[s] = pred[lr];
+  }
+  const bool in = lane < k;
+  const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
+  const bool m = in && sd.masked[s * kMaxBlock + lane];
+  const float c = m ? conf[row] : -1.0f;
+  const bool over = m && (c >= alpha);
+  const unsigned any_over = __ballot_sync(0xffffffffu, over);
+  bool commit = over;
+  if (!any_over) {
+    // most confident masked position, lowest position on ties
+    float best = c;
+    int bi = m ? lane : 1 << 30;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    commit = m && lane == bi;
+  }
+  if (commit) {
+    sd.blk[s * kMaxBlock + lane] = (unsigned char)pred[row];
+    sd.masked[s * kMaxBlock + lane] = 0;
+  }
+  const unsigned left = __ballot_sync(0xffffffffu, m && !commit);
+  if (out_logits && in) {
+    float* dst = out_logits + (((size_t)step * batch + s) * k + lane) * 256;
+    const float* src = logits + (size_t)row * 256;
+    for (int j = 0; j < 256; ++j) dst[j] = src[j];
+  }
+  if (lane == 0) {
+    sd.steps[s] += 1;
+    sd.active[s] = left != 0;
+  }
+}
+
+// After the block loop: copy blocks out; masked positions left -> STEP_LIMIT.
+__global__ void k_finish_block(SeqDev sd, int batch, int k, unsigned char* out_block, int* out_steps) {
+  const int s = blockIdx.x, lane = threadIdx.x;
+  if (s >= batch) return;
+  if (lane < k) out_block[s * k + lane] = sd.blk[s * kMaxBlock + lane];
+  if (lane == 0) {
+    if (out_steps) out_steps[s] = sd.steps[s];
+    if (sd.active[s]) set_status(sd.status, kErrStepLimit);
+  }
+}
+
+// AR draft: the argmax of this pass's row becomes draft byte `step`.
+__global__ void k_draft_ar(SeqDev sd, int batch, int k, int step, const int* pred, const float* logits, float* out_logits) {
+  const int s = blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= batch) return;
+  const int row = (step == 0) ? sd.last_row[s] : sd.blk_row[s * kMaxBlock];
+  const int b = pred[row];
+  sd.blk[s * kMaxBlock + step] = (unsigned char)b;
+  if (step == 0) sd.y_last[s] = b;
+  if (out_logits) {
+    float* dst = out_logits + ((size_t)step * batch + s) * 256;
+    for (int j = 0; j < 256; ++j) dst[j] = logits[(size_t)row * 256 + j];
+  }
+}
+
+__global__ void k_copy_draft(SeqDev sd, int batch, int k, unsigned char* out) {
+  const int s = blockIdx.x, lane = threadIdx.x;
+  if (s < batch && lane < k) out[s * k + lane] = sd.blk[s * kMaxBlock + lane];
+}
+
+// Greedy verification ("BLT-S와 BLT-DV"): with y_slot[i] the greedy byte for
+// draft slot i (slot 0: prediction of the last committed row; slot i > 0: of
+// draft row i-1), accept while draft[i] == y_slot[i]; the next byte is
+// y_slot[a], or the prediction of the last draft row when all k match.
+__global__ void k_accept(SeqDev sd, int batch, int k, const int* pred, const int* vlat, const float* logits, int* out_acc,
+                         unsigned char* out_next, float* out_logits) {
+  const int s = blockIdx.x, lane = threadIdx.x;
+  if (s >= batch) return;
+  const bool in = lane < k;
+  const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
+  const int y_self = in ? pred[row] : -1;
+  const int y_up = __shfl_up_sync(0xffffffffu, y_self, 1);
+  const int y_slot = (lane == 0) ? sd.y_last[s] : y_up;
+  const bool match = in && (int)sd.blk[s * kMaxBlock + lane] == y_slot;
+  const unsigned mm = __ballot_sync(0xffffffffu, !match);
+  const int a = (mm == 0u) ? k : min(__ffs(mm) - 1, k);
+  const int y_a = __shfl_sync(0xffffffffu, y_slot, a & 31);
+  const int y_k = __shfl_sync(0xffffffffu, y_self, (k - 1) & 31);
+  if (out_logits && in) {
+    float* dst = out_logits + ((size_t)s * k + lane) * 256;
+    for (int j = 0; j < 256; ++j) dst[j] = logits[(size_t)row * 256 + j];
+  }
+  if (lane == 0) {
+    const int nxt = (a == k) ? y_k : y_a;
+    out_acc[s] = a;
+    out_next[s] = (unsigned char)nxt;
+    sd.kv_len[s] += a;
+    if (a >= 1) sd.n_lat[s] = max(sd.n_lat[s], vlat[s * k + a - 1] + 1);
+  }
+}
+
+// Page table updates (entries by value).
+struct PageUpd {
+  int n;
+  int idx[64];
+  int page[64];
+};
+__global__ void k_page_update(int* pt, PageUpd u) {
+  const int i = threadIdx.x;
+  if (i < u.n) pt[u.idx[i]] = u.page[i];
+}
+
+// Set per-sequence lengths (rewind).
+__global__ void k_rewind(SeqDev sd, CallDesc cd) {
+  const int s = threadIdx.x;
+  if (s < cd.batch) {
+    if (cd.row_off[s] >= 0) sd.kv_len[s] = min(sd.kv_len[s], cd.row_off[s]);
+    if (cd.lat_off[s] >= 0) sd.n_lat[s] = min(sd.n_lat[s], cd.lat_off[s]);
+  }
+}
+
+}  // namespace bltdec
