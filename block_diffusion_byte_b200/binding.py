@@ -26,6 +26,7 @@ BLT_W_F32 = 0
 BLT_W_BF16 = 1
 BLT_DRAFT_AR = 0
 BLT_DRAFT_DIFFUSION = 1
+BLT_FLAG_TIME_PASSES = 1
 BLT_LAYER_NT = 12
 LAYER_ORDER = ("wq_c", "wk_c", "wv_c", "wo_c", "norm_c", "attn_norm", "wqkv", "wo", "ffn_norm", "w1", "w3", "w2")
 
@@ -62,6 +63,7 @@ class blt_dec_config(C.Structure):
         ("page_tokens", C.c_int32),
         ("kv_pages", C.c_int32),
         ("attn_chunk", C.c_int32),
+        ("flags", C.c_int32),
     ]
 
 
@@ -93,6 +95,9 @@ class blt_dec_counters(C.Structure):
         ("calls", C.c_uint64),
         ("weight_bytes", C.c_uint64),
         ("kv_read_bytes", C.c_uint64),
+        ("kernel_launches", C.c_uint64),
+        ("timed_passes", C.c_uint64),
+        ("pass_ns", C.c_uint64),
     ]
 
     def as_dict(self):

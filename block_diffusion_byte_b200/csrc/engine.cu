@@ -49,7 +49,8 @@ struct blt_dec {
   float* embed = nullptr;
   float* final_norm = nullptr;
   float *rope_cos = nullptr, *rope_sin = nullptr;
-  __nv_bfloat16* kv = nullptr;
+  void* kv = nullptr;  // KV pool, element type per kv_f32
+  int kv_f32 = 0;
   int* page_table = nullptr;
   std::vector<int> pt_host, free_pages, seq_npages;
   float* c_lat = nullptr;
@@ -70,6 +71,11 @@ struct blt_dec {
   bool mirror_pending = false;
   std::string err;
   unsigned long long weight_bytes_per_pass = 0, kv_bytes_per_key = 0;
+  unsigned long long launches = 0;  // kernels launched (host count)
+  // pass timing (BLT_FLAG_TIME_PASSES): event pairs recorded around passes
+  std::vector<cudaEvent_t> tev;
+  size_t tev_used = 0;
+  unsigned long long timed_passes = 0, pass_ns = 0;
 };
 
 namespace {
@@ -150,6 +156,37 @@ int upload(blt_dec* h, float** dst, const float* src, size_t n) {
   return BLT_OK;
 }
 
+// ---------------------------------------------------------------------------- pass timing
+int pass_begin(blt_dec* h) {
+  if (!(h->cfg.flags & BLT_FLAG_TIME_PASSES)) return BLT_OK;
+  if (h->tev_used + 2 > h->tev.size()) {
+    for (int i = 0; i < 64; ++i) {
+      cudaEvent_t e;
+      CK(cudaEventCreate(&e));
+      h->tev.push_back(e);
+    }
+  }
+  CK(cudaEventRecord(h->tev[h->tev_used], h->stream));
+  return BLT_OK;
+}
+int pass_end(blt_dec* h) {
+  if (!(h->cfg.flags & BLT_FLAG_TIME_PASSES)) return BLT_OK;
+  CK(cudaEventRecord(h->tev[h->tev_used + 1], h->stream));
+  h->tev_used += 2;
+  return BLT_OK;
+}
+// Fold recorded pass times into the counters (the stream must be idle).
+int drain_timing(blt_dec* h) {
+  for (size_t i = 0; i + 1 < h->tev_used; i += 2) {
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]));
+    h->pass_ns += (unsigned long long)(ms * 1e6);
+    h->timed_passes += 1;
+  }
+  h->tev_used = 0;
+  return BLT_OK;
+}
+
 // ---------------------------------------------------------------------------- GEMM launch
 template <int NG, int PL, int EPI>
 constexpr int gemm_stages() {
@@ -196,6 +233,7 @@ int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
   a.K = m.K;
   a.status = h->sd.status;
   const int ng = rows_ub <= 8 ? 1 : rows_ub <= 16 ? 2 : rows_ub <= 32 ? 4 : 8;
+  h->launches += 1;
   if (m.planes == 1) {
     if (ng == 1) launch_ng<1, 1, EPI>(h, a, rows_ub);
     else if (ng == 2) launch_ng<2, 1, EPI>(h, a, rows_ub);
@@ -215,6 +253,7 @@ GemmArgs base_args(blt_dec* h) {
   GemmArgs a{};
   a.n_rows = h->rows.n_rows;
   a.kv = h->kv;
+  a.kv_f32 = h->kv_f32;
   a.page_table = h->page_table;
   a.max_pages = h->max_pages;
   a.PT = h->PT;
@@ -232,11 +271,39 @@ GemmArgs base_args(blt_dec* h) {
   return a;
 }
 
+template <typename KVT>
+void launch_attn_t(blt_dec* h, dim3 ag, size_t smem, const AttnArgs& aa) {
+  if (h->dh == 64) k_attn_partial<64, KVT><<<ag, 128, smem, h->stream>>>(aa);
+  else if (h->dh == 32) k_attn_partial<32, KVT><<<ag, 128, smem, h->stream>>>(aa);
+  else if (h->dh == 128) k_attn_partial<128, KVT><<<ag, 128, smem, h->stream>>>(aa);
+  else k_attn_partial<16, KVT><<<ag, 128, smem, h->stream>>>(aa);
+}
+void launch_attn(blt_dec* h, dim3 ag, size_t smem, const AttnArgs& aa) {
+  if (h->kv_f32) launch_attn_t<float>(h, ag, smem, aa);
+  else launch_attn_t<__nv_bfloat16>(h, ag, smem, aa);
+}
+template <typename KVT>
+int set_attn_attrs(blt_dec* h, size_t smem) {
+  CK(cudaFuncSetAttribute(k_attn_partial<16, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<32, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<64, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<128, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  return BLT_OK;
+}
+
 // ---------------------------------------------------------------------------- one decoder pass
 // Runs every layer over the rows planned on the device (at most rows_ub rows,
 // keys below keys_ub, at most groups_ub attention groups).
+int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head);
 int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
+  TRY(pass_begin(h));
+  TRY(run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head));
+  return pass_end(h);
+}
+int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
   const int d = h->d;
+  // embed + per layer (2 row norms, attention partial + combine) + head norm and statistics; GEMMs count themselves
+  h->launches += 1 + 4 * (unsigned long long)h->L + (want_head ? 2 : 0);
   const float eps = h->cfg.norm_eps;
   const int nb = std::max(1, std::min(rows_ub, 1024));
   k_embed<<<nb, 256, 0, h->stream>>>(h->rows, h->embed, h->h, d, rows_ub);
@@ -274,10 +341,7 @@ int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head
     TRY(gemm<EPI_QKV>(h, h->qkv[l], a, rows_ub));
     aa.layer = l;
     dim3 ag(h->H, nchunks, groups_ub);
-    if (h->dh == 64) k_attn_partial<64><<<ag, 128, attn_smem, h->stream>>>(aa);
-    else if (h->dh == 32) k_attn_partial<32><<<ag, 128, attn_smem, h->stream>>>(aa);
-    else if (h->dh == 128) k_attn_partial<128><<<ag, 128, attn_smem, h->stream>>>(aa);
-    else k_attn_partial<16><<<ag, 128, attn_smem, h->stream>>>(aa);
+    launch_attn(h, ag, attn_smem, aa);
     k_attn_combine<<<dim3(rows_ub, h->H), h->dh, 0, h->stream>>>(aa);
     CK(cudaGetLastError());
     a = base_args(h);
@@ -357,6 +421,7 @@ int ensure_pages(blt_dec* h, int s, int need, PageUpd& upd) {
     upd.page[upd.n] = page;
     if (++upd.n == 64) {
       k_page_update<<<1, 64, 0, h->stream>>>(h->page_table, upd);
+      h->launches += 1;
       upd.n = 0;
     }
   }
@@ -364,7 +429,10 @@ int ensure_pages(blt_dec* h, int s, int need, PageUpd& upd) {
 }
 
 int flush_pages(blt_dec* h, PageUpd& upd) {
-  if (upd.n) k_page_update<<<1, 64, 0, h->stream>>>(h->page_table, upd);
+  if (upd.n) {
+    k_page_update<<<1, 64, 0, h->stream>>>(h->page_table, upd);
+    h->launches += 1;
+  }
   upd.n = 0;
   CK(cudaGetLastError());
   return BLT_OK;
@@ -394,6 +462,7 @@ int project_latents(blt_dec* h, const CallDesc& cd, const float* new_lat, bool c
     const int r1 = std::min(total, r0 + chunk);
     k_lat_plan<<<1, 256, 0, h->stream>>>(cd, h->sd, h->lat_seq, h->lat_slot, h->n_lat_rows, r0, r1, commit ? 1 : 0,
                                          h->cfg.max_latents);
+    h->launches += 1;
     for (int l = 0; l < h->L; ++l) {
       GemmArgs a = base_args(h);
       a.n_rows = nullptr;
@@ -429,6 +498,7 @@ PlanArgs plan_args(blt_dec* h, int mode, int k) {
 }
 
 int plan(blt_dec* h, const PlanArgs& p, const CallDesc& cd) {
+  h->launches += 1;
   k_plan<<<1, 256, 0, h->stream>>>(p, cd, h->sd, h->rows);
   CK(cudaGetLastError());
   return BLT_OK;
@@ -460,11 +530,13 @@ int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, f
   TRY(plan(h, p, cd));
   TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true));
   k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits);
+  h->launches += 1;
   for (int st = 1; st < max_steps; ++st) {
     PlanArgs pb = plan_args(h, PL_BLOCK, k);
     TRY(plan(h, pb, cd));
     TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true));
     k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits);
+    h->launches += 1;
   }
   CK(cudaGetLastError());
   return BLT_OK;
@@ -621,9 +693,14 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     h->weight_bytes_per_pass = h->head.bytes();
     for (int l = 0; l < L; ++l)
       h->weight_bytes_per_pass += h->qkv[l].bytes() + h->o[l].bytes() + h->w13[l].bytes() + h->w2[l].bytes();
-    h->kv_bytes_per_key = (unsigned long long)L * 2 * d * 2;
-    // KV pool [pages][L][2][H][PT][dh] bf16
-    TRY(dalloc(h, &h->kv, (size_t)h->n_pages * L * 2 * d * h->PT));
+    h->kv_bytes_per_key = (unsigned long long)L * 2 * d * (pl == 2 ? 4 : 2);
+    // KV pool [pages][L][2][H][PT][dh]: bf16 for bf16 weights, fp32 for fp32 weights
+    h->kv_f32 = pl == 2;
+    {
+      char* kvp = nullptr;
+      TRY(dalloc(h, &kvp, (size_t)h->n_pages * L * 2 * d * h->PT * (h->kv_f32 ? 4 : 2)));
+      h->kv = kvp;
+    }
     TRY(dalloc(h, &h->page_table, (size_t)c.max_batch * h->max_pages));
     CK(cudaMemset(h->page_table, 0xFF, (size_t)c.max_batch * h->max_pages * 4));
     h->pt_host.assign((size_t)c.max_batch * h->max_pages, -1);
@@ -692,10 +769,8 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(set_attrs_epi<EPI_QKV>(h));
     TRY(set_attrs_epi<EPI_LATC>(h));
     const size_t attn_smem = (size_t)(32 * dh + h->CH * dh + 32 * h->CH) * 4;
-    CK(cudaFuncSetAttribute(k_attn_partial<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
-    CK(cudaFuncSetAttribute(k_attn_partial<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
-    CK(cudaFuncSetAttribute(k_attn_partial<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
-    CK(cudaFuncSetAttribute(k_attn_partial<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)attn_smem));
+    TRY(set_attn_attrs<float>(h, attn_smem));
+    TRY(set_attn_attrs<__nv_bfloat16>(h, attn_smem));
     CK(cudaDeviceSynchronize());
     return BLT_OK;
   };
@@ -721,8 +796,10 @@ int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out
   refresh_bounds(h);
   TRY(reserve(h, cd, 0, true));
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  h->launches += 1;
   TRY(project_latents(h, cd, rows->new_latents, true));
   k_snapshot_base<<<1, 256, 0, h->stream>>>(h->sd, batch);
+  h->launches += 1;
   int kmax = 0;
   for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
   const int chunk = h->cfg.max_rows;
@@ -735,9 +812,13 @@ int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out
     p.pend_lat = rows->row_latent;
     TRY(plan(h, p, cd));
     TRY(run_pass(h, r1 - r0, kmax, (r1 - r0 + 31) / 32 + batch, out_logits != nullptr));
-    if (out_logits) k_copy_logits<<<256, 256, 0, h->stream>>>(h->logits, out_logits + (size_t)r0 * 256, (r1 - r0) * 256);
+    if (out_logits) {
+      k_copy_logits<<<256, 256, 0, h->stream>>>(h->logits, out_logits + (size_t)r0 * 256, (r1 - r0) * 256);
+      h->launches += 1;
+    }
   }
   k_finish_prefill<<<1, 256, 0, h->stream>>>(h->sd, cd);
+  h->launches += 1;
   CK(cudaGetLastError());
   bump_bounds(h, cd, 0);
   return post_mirror(h);
@@ -761,9 +842,11 @@ int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, i
   refresh_bounds(h);
   TRY(reserve(h, cd, k, true));
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  h->launches += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
   TRY(block_loop(h, cd, pending, k, alpha, max_steps, out_logits));
   k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_block, out_steps);
+  h->launches += 1;
   CK(cudaGetLastError());
   bump_bounds(h, cd, 0);
   return post_mirror(h);
@@ -790,6 +873,7 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
   refresh_bounds(h);
   TRY(reserve(h, cd, k, true));
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  h->launches += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
   if (mode == BLT_DRAFT_AR) {
     int npmax = 0;
@@ -801,12 +885,14 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
     TRY(plan(h, p, cd));
     TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true));
     k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, 0, h->pred, h->logits, out_logits);
+    h->launches += 1;
     for (int t = 1; t < k; ++t) {
       PlanArgs pa = plan_args(h, PL_ARDRAFT, 0);
       pa.step = t;
       TRY(plan(h, pa, cd));
       TRY(run_pass(h, batch, keys_ub, batch, true));
       k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, t, h->pred, h->logits, out_logits);
+      h->launches += 1;
     }
   } else {
     if (max_steps <= 0) max_steps = k;
@@ -814,6 +900,7 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
   }
   if (mode == BLT_DRAFT_DIFFUSION) k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft, nullptr);
   else k_copy_draft<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft);
+  h->launches += 1;
   CK(cudaGetLastError());
   bump_bounds(h, cd, 0);
   h->state = 1;
@@ -835,12 +922,14 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
   refresh_bounds(h);
   TRY(reserve(h, cd, k, false));
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  h->launches += 1;
   TRY(project_latents(h, cd, new_latents, false));
   PlanArgs p = plan_args(h, PL_VERIFY, k);
   p.vlat = draft_row_latent;
   TRY(plan(h, p, cd));
   TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true));
   k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
+  h->launches += 1;
   CK(cudaGetLastError());
   for (int s = 0; s < batch; ++s) {
     h->kv_ub[s] += k;
@@ -879,6 +968,7 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   if (!h || !out) return BLT_ERR_INVALID_ARG;
   unsigned long long c[8];
   CK(cudaStreamSynchronize(h->stream));
+  TRY(drain_timing(h));
   CK(cudaMemcpy(c, h->sd.counters, sizeof c, cudaMemcpyDeviceToHost));
   out->passes = c[0];
   out->rows = c[1];
@@ -887,6 +977,9 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->calls = c[4];
   out->weight_bytes = c[5];
   out->kv_read_bytes = c[6];
+  out->kernel_launches = h->launches;
+  out->timed_passes = h->timed_passes;
+  out->pass_ns = h->pass_ns;
   return BLT_OK;
 }
 
@@ -910,6 +1003,7 @@ void blt_dec_free(blt_dec_t* h) {
   for (void* p : h->allocs) cudaFree(p);
   if (h->mirror) cudaFreeHost(h->mirror);
   if (h->mirror_ev) cudaEventDestroy(h->mirror_ev);
+  for (cudaEvent_t e : h->tev) cudaEventDestroy(e);
   if (h->own_stream && h->stream) cudaStreamDestroy(h->stream);
   delete h;
 }

@@ -52,7 +52,8 @@ struct GemmArgs {
   int ldo;
   // EPI_QKV
   float* q;
-  __nv_bfloat16* kv;
+  void* kv;    // KV pool: bf16, or fp32 when kv_f32
+  int kv_f32;
   const int* page_table;
   int max_pages, PT, layer, L, H, dh, d;
   const int* row_seq;
@@ -110,9 +111,16 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
           set_status(a.status, kErrDevice);
           return;
         }
-        __nv_bfloat16* k = a.kv + kv_offset(a, page, 0, h, pos % a.PT, 0);
-        k[j] = __float2bfloat16_rn(o0);
-        k[j + half] = __float2bfloat16_rn(o1);
+        const size_t off = kv_offset(a, page, 0, h, pos % a.PT, 0);
+        if (a.kv_f32) {
+          float* k = static_cast<float*>(a.kv) + off;
+          k[j] = o0;
+          k[j + half] = o1;
+        } else {
+          __nv_bfloat16* k = static_cast<__nv_bfloat16*>(a.kv) + off;
+          k[j] = __float2bfloat16_rn(o0);
+          k[j + half] = __float2bfloat16_rn(o1);
+        }
       }
     } else {
       const int seq = a.row_seq[row];
@@ -123,8 +131,15 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         return;
       }
       const int n0 = lt * 16 + r16, n1 = n0 + 8;
-      a.kv[kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh)] = __float2bfloat16_rn(v0);
-      a.kv[kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh)] = __float2bfloat16_rn(v1);
+      const size_t o0 = kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh);
+      const size_t o1 = kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh);
+      if (a.kv_f32) {
+        static_cast<float*>(a.kv)[o0] = v0;
+        static_cast<float*>(a.kv)[o1] = v1;
+      } else {
+        static_cast<__nv_bfloat16*>(a.kv)[o0] = __float2bfloat16_rn(v0);
+        static_cast<__nv_bfloat16*>(a.kv)[o1] = __float2bfloat16_rn(v1);
+      }
     }
   }
 }
@@ -297,7 +312,7 @@ __global__ void k_rownorm(const RowsDev rows, float* __restrict__ h, float* __re
 // ------------------------------------------------------------------------ attention
 struct AttnArgs {
   const float* q;  // [rows][d], RoPE applied
-  const __nv_bfloat16* kv;
+  const void* kv;
   const int* page_table;
   int max_pages, PT, L, layer, H, dh, d;
   RowsDev rows;
@@ -309,8 +324,20 @@ struct AttnArgs {
   int* status;
 };
 
-// grid (H, chunks, groups); 128 threads; dh == 64 or smaller power of two <= 64 handled by DH template.
-template <int DH>
+// 8 consecutive K/V elements (16-byte aligned) widened to fp32.
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* out) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) out[e] = __bfloat162float(b[e]);
+}
+__device__ __forceinline__ void load8(const float* p, float* out) {
+  const float4 x = reinterpret_cast<const float4*>(p)[0], y = reinterpret_cast<const float4*>(p)[1];
+  out[0] = x.x, out[1] = x.y, out[2] = x.z, out[3] = x.w, out[4] = y.x, out[5] = y.y, out[6] = y.z, out[7] = y.w;
+}
+
+// grid (H, chunks, groups); 128 threads; one head of DH dims; KVT = K/V element type.
+template <int DH, typename KVT>
 __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   constexpr int MAXR = 32;
   const int gi = blockIdx.z;
@@ -343,12 +370,9 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
       set_status(a.status, kErrDevice);
       page = 0;
     }
-    const __nv_bfloat16* src =
-        a.kv + ((((size_t)page * a.L + a.layer) * 2 + 1) * a.H + h) * (size_t)a.PT * DH + (size_t)(tpos % a.PT) * DH + c8;
-    const uint4 raw = *reinterpret_cast<const uint4*>(src);
-    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) vs[key * DH + c8 + e] = __bfloat162float(b[e]);
+    const KVT* src = static_cast<const KVT*>(a.kv) + ((((size_t)page * a.L + a.layer) * 2 + 1) * a.H + h) * (size_t)a.PT * DH +
+                     (size_t)(tpos % a.PT) * DH + c8;
+    load8(src, vs + key * DH + c8);
   }
   __syncthreads();
   // scores: thread = key (CH <= 128), K row in registers
@@ -362,15 +386,10 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
         set_status(a.status, kErrDevice);
         page = 0;
       }
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.kv + ((((size_t)page * a.L + a.layer) * 2 + 0) * a.H + h) * (size_t)a.PT * DH + (size_t)(tpos % a.PT) * DH);
+      const KVT* src = static_cast<const KVT*>(a.kv) + ((((size_t)page * a.L + a.layer) * 2 + 0) * a.H + h) * (size_t)a.PT * DH +
+                       (size_t)(tpos % a.PT) * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 8; ++c) {
-        const uint4 raw = src[c];
-        const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) kr[c * 8 + e] = __bfloat162float(b[e]);
-      }
+      for (int c = 0; c < DH / 8; ++c) load8(src + c * 8, kr + c * 8);
     }
     for (int r = 0; r < nr; ++r) {
       float s = -INFINITY;

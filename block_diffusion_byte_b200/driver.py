@@ -33,7 +33,7 @@ from . import binding as B
 
 
 def engine_config(shape: ModelShape, max_batch: int, max_ctx: int, max_latents: int, max_rows: int, max_block: int,
-                  page_tokens: int = 64, kv_pages: int = 0, attn_chunk: int = 0) -> B.blt_dec_config:
+                  page_tokens: int = 64, kv_pages: int = 0, attn_chunk: int = 0, flags: int = 0) -> B.blt_dec_config:
     return B.blt_dec_config(
         n_layers=shape.n_layers,
         d_model=shape.d_model,
@@ -52,6 +52,7 @@ def engine_config(shape: ModelShape, max_batch: int, max_ctx: int, max_latents: 
         page_tokens=page_tokens,
         kv_pages=kv_pages,
         attn_chunk=attn_chunk,
+        flags=flags,
     )
 
 
@@ -60,13 +61,14 @@ class Engine:
 
     def __init__(self, shape: ModelShape, weights: WeightSet, max_batch: int, max_ctx: int, max_block: int,
                  max_rows: int = 1024, max_latents: Optional[int] = None, page_tokens: int = 64, attn_chunk: int = 0,
-                 device: str = "cuda"):
+                 device: str = "cuda", time_passes: bool = False):
         self.shape = shape
         self.max_batch, self.max_ctx, self.max_block, self.max_rows = max_batch, max_ctx, max_block, max_rows
         self.max_latents = max_latents or (max_ctx // 2 + 64)
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
-        cfg = engine_config(shape, max_batch, max_ctx, self.max_latents, max_rows, max_block, page_tokens, 0, attn_chunk)
+        cfg = engine_config(shape, max_batch, max_ctx, self.max_latents, max_rows, max_block, page_tokens, 0, attn_chunk,
+                            B.BLT_FLAG_TIME_PASSES if time_passes else 0)
         layers = []
         for l in range(shape.n_layers):
             lw = weights.layer(l)
@@ -109,6 +111,9 @@ class Engine:
         bts = np.array([b for bl in byte_lists for b in bl], dtype=np.uint8)
         sls = np.array([s for sl in slot_lists for s in sl], dtype=np.int32)
         lats = [v for vl in lat_lists for v in vl]
+        if bts.shape[0] > self.d_bytes.shape[0]:
+            self.d_bytes = torch.zeros(bts.shape[0], dtype=torch.uint8, device=self.device)
+            self.d_slots = torch.zeros(bts.shape[0], dtype=torch.int32, device=self.device)
         db = self._put(self.d_bytes, bts)
         ds = self._put(self.d_slots, sls)
         dl = None
@@ -117,6 +122,10 @@ class Engine:
                 self.d_lat = torch.zeros((len(lats), self.shape.d_global), dtype=torch.float32, device=self.device)
             dl = self._put(self.d_lat, np.stack(lats).astype(np.float32))
         return B.rows_in(db, ds, ro.tolist(), dl, lo.tolist())
+
+    def out_view(self, nb: int, k: int) -> torch.Tensor:
+        """The engine writes [batch, k] byte outputs densely."""
+        return self.d_out.view(-1)[: nb * k].view(nb, k)
 
     def close(self):
         if self.h:
@@ -213,7 +222,7 @@ def generate(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: Op
         r, keep = eng.rows([p[0] for p in pend], [p[1] for p in pend], [p[2] for p in pend])
         if wl.mode == "D":
             B.blt_dec_diffuse_block(h, nb, r, k, wl.alpha, 0, eng.d_out, eng.d_steps)
-            blk = eng._get(eng.d_out[:nb, :k])
+            blk = eng._get(eng.out_view(nb, k))
             steps = eng._get(eng.d_steps[:nb]) if record else None
             for i, s in enumerate(seqs):
                 new = [int(v) for v in blk[i]]
@@ -223,14 +232,14 @@ def generate(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: Op
                 rounds.append(dict(block=blk.copy(), steps=steps.copy()))
         elif wl.mode == "AR":
             B.blt_dec_draft(h, nb, r, B.BLT_DRAFT_AR, 1, 0.0, 0, eng.d_out)
-            d = eng._get(eng.d_out[:nb, :1])
+            d = eng._get(eng.out_view(nb, 1))
             for i, s in enumerate(seqs):
                 s.commit([int(d[i, 0])])
                 s.out.append(int(d[i, 0]))
         elif wl.mode in ("S", "DV"):
             mode = B.BLT_DRAFT_AR if wl.mode == "S" else B.BLT_DRAFT_DIFFUSION
             B.blt_dec_draft(h, nb, r, mode, k, wl.alpha, 0, eng.d_out)
-            draft = eng._get(eng.d_out[:nb, :k])
+            draft = eng._get(eng.out_view(nb, k))
             vslots = np.zeros((nb, k), dtype=np.int32)
             prov: List[List[np.ndarray]] = []
             for i, s in enumerate(seqs):

@@ -56,8 +56,8 @@ extern "C" {
 #define BLT_ERR_STEP_LIMIT (-5)  /* masked positions left after max_steps passes (device) */
 #define BLT_ERR_DEVICE (-6)      /* a device-side index check failed (device) */
 
-#define BLT_W_F32 0  /* weights kept as two bf16 planes (hi + lo) */
-#define BLT_W_BF16 1 /* weights kept as one bf16 plane (values must be bf16) */
+#define BLT_W_F32 0  /* weights kept as two bf16 planes (hi + lo); fp32 KV cache */
+#define BLT_W_BF16 1 /* weights kept as one bf16 plane (values rounded to bf16); bf16 KV cache */
 
 #define BLT_DRAFT_AR 0        /* BLT-S: k autoregressive passes */
 #define BLT_DRAFT_DIFFUSION 1 /* BLT-DV: confidence unmasking of a k-byte block */
@@ -93,7 +93,10 @@ typedef struct {
   int32_t page_tokens;  /* KV positions per page; multiple of 16 */
   int32_t kv_pages;     /* pages in the pool; 0 = enough for max_batch * max_ctx */
   int32_t attn_chunk;   /* keys per split-KV chunk; 0 = 128 */
+  int32_t flags;        /* BLT_FLAG_* */
 } blt_dec_config;
+
+#define BLT_FLAG_TIME_PASSES 1 /* bracket every decoder pass with CUDA events (counters.pass_ns) */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */
@@ -123,6 +126,9 @@ typedef struct {
   uint64_t calls;          /* C-ABI calls that ran decoder work */
   uint64_t weight_bytes;   /* weight bytes streamed by decoder passes (algorithmic) */
   uint64_t kv_read_bytes;  /* K/V bytes read by self-attention (algorithmic) */
+  uint64_t kernel_launches; /* engine kernels launched (host count) */
+  uint64_t timed_passes;   /* passes bracketed by events (BLT_FLAG_TIME_PASSES) */
+  uint64_t pass_ns;        /* their summed device time, ns */
 } blt_dec_counters;
 
 /* Create an engine.  Copies and re-lays out the weights on the device

@@ -48,10 +48,10 @@ def test_binding_covers_every_export(lib):
 def test_struct_layouts_match_header():
     from block_diffusion_byte_b200 import binding as B
 
-    assert ctypes.sizeof(B.blt_dec_config) == 17 * 4
+    assert ctypes.sizeof(B.blt_dec_config) == 18 * 4
     assert ctypes.sizeof(B.blt_dec_weights) == 4 * 8
     assert ctypes.sizeof(B.blt_rows_in) == 5 * 8
-    assert ctypes.sizeof(B.blt_dec_counters) == 7 * 8
+    assert ctypes.sizeof(B.blt_dec_counters) == 10 * 8
 
 
 def test_init_rejects_bad_config_without_touching_the_gpu(lib):

@@ -140,3 +140,34 @@ def test_batch_invariance(tiny_setup):
         finally:
             eng.close()
         assert solo == batched[s]
+
+
+@pytest.fixture(scope="module")
+def d4_setup():
+    from block_diffusion_byte_b200 import _build
+
+    _build.build()
+    wl = CONFIGS["d4_b1"]
+    ws = WeightSet(wl.shape).materialize()
+    return wl, ws, OracleModel(wl.shape, ws)
+
+
+def test_d4_b1_first_block_logits_and_bytes(d4_setup):
+    """9-layer d=1024 bf16 decoder, prefix 1024: first pass logits and the first 8 blocks."""
+    from block_diffusion_byte_b200 import binding as B
+    from block_diffusion_byte_b200.driver import Engine, generate
+
+    wl, ws, om = d4_setup
+    pre = _prefix(wl, 0)
+    G = 32
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + G + 40, max_block=16, max_rows=512)
+    try:
+        res = generate(eng, wl, [pre], G, record=True)
+    finally:
+        eng.close()
+    o = OracleSequence(om, wl, 0, pre)
+    o.prefill()
+    rec = []
+    want = o.generate(G, rec)
+    _compare_bytes(res.out[0], o, want, wl.prefix_len, "d4_b1")
+    assert [int(r["steps"][0]) for r in res.rounds] == [r["steps"] for r in rec][: len(res.rounds)] or res.out[0] != want
