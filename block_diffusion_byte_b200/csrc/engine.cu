@@ -11,6 +11,7 @@
 
 #include "bltdec.h"
 #include "kernels.cuh"
+#include "mega.cuh"
 
 using namespace bltdec;
 
@@ -76,6 +77,16 @@ struct blt_dec {
   std::vector<cudaEvent_t> tev;
   size_t tev_used = 0;
   unsigned long long timed_passes = 0, pass_ns = 0;
+  // persistent pass kernel
+  bool mega_ok = false;
+  int nsm = 0;
+  LayerW* d_layers = nullptr;
+  unsigned* flags = nullptr;
+  unsigned* attn_cnt = nullptr;
+  unsigned* dec_val = nullptr;
+  int* abort_flag = nullptr;
+  unsigned epoch = 0;
+  int f_qkv = 0, f_o = 0, f_w13 = 0, f_w2 = 0, f_head = 0, f_att = 0, f_dec = 0, mega_groups = 0;
 };
 
 namespace {
@@ -181,7 +192,6 @@ int drain_timing(blt_dec* h) {
     float ms = 0.f;
     CK(cudaEventElapsedTime(&ms, h->tev[i], h->tev[i + 1]));
     h->pass_ns += (unsigned long long)(ms * 1e6);
-    h->timed_passes += 1;
   }
   h->tev_used = 0;
   return BLT_OK;
@@ -195,7 +205,7 @@ constexpr int gemm_stages() {
 template <int NG, int PL, int EPI>
 size_t gemm_smem() {
   constexpr int RB = 8 * NG;
-  return (size_t)gemm_stages<NG, PL, EPI>() * RB * kXStride * 4 + RB * 4;
+  return (size_t)gemm_stages<NG, PL, EPI>() * RB * kXStride * 4 + 8 * RB * 4;
 }
 
 template <int NG, int PL, int EPI>
@@ -263,14 +273,42 @@ GemmArgs base_args(blt_dec* h) {
   a.d = h->d;
   a.row_seq = h->rows.seq;
   a.row_pos = h->rows.pos;
+  a.row_lat = h->rows.lat;
+  a.row_byte = h->rows.byte;
+  a.embed = h->embed;
+  a.c_lat = h->c_lat;
+  a.eps = h->cfg.norm_eps;
   a.rope_cos = h->rope_cos;
   a.rope_sin = h->rope_sin;
-  a.max_ctx = h->cfg.max_ctx;
   a.max_lat = h->cfg.max_latents;
   a.status = h->sd.status;
   return a;
 }
 
+size_t attn_smem_bytes(const blt_dec* h) {
+  return (size_t)(kAttnRows * h->dh + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * h->dh * (h->kv_f32 ? 4 : 2);
+}
+AttnArgs attn_args(blt_dec* h) {
+  AttnArgs aa{};
+  aa.kv = h->kv;
+  aa.page_table = h->page_table;
+  aa.max_pages = h->max_pages;
+  aa.PT = h->PT;
+  aa.L = h->L;
+  aa.H = h->H;
+  aa.dh = h->dh;
+  aa.d = h->d;
+  aa.rows = h->rows;
+  aa.CH = h->CH;
+  aa.CMAX = h->CMAX;
+  aa.scale = 1.0f / std::sqrt((float)h->dh);
+  aa.q = h->q;
+  aa.part_ml = h->part_ml;
+  aa.part_o = h->part_o;
+  aa.att = h->att;
+  aa.status = h->sd.status;
+  return aa;
+}
 template <typename KVT>
 void launch_attn_t(blt_dec* h, dim3 ag, size_t smem, const AttnArgs& aa) {
   if (h->dh == 64) k_attn_partial<64, KVT><<<ag, 128, smem, h->stream>>>(aa);
@@ -296,52 +334,28 @@ int set_attn_attrs(blt_dec* h, size_t smem) {
 // keys below keys_ub, at most groups_ub attention groups).
 int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head);
 int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
-  TRY(pass_begin(h));
-  TRY(run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head));
-  return pass_end(h);
+  return run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head);
 }
 int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
   const int d = h->d;
-  // embed + per layer (2 row norms, attention partial + combine) + head norm and statistics; GEMMs count themselves
-  h->launches += 1 + 4 * (unsigned long long)h->L + (want_head ? 2 : 0);
-  const float eps = h->cfg.norm_eps;
+  // embed + per layer (cross add, attention partial + combine) + head statistics; GEMMs count themselves
+  h->launches += 1 + 3 * (unsigned long long)h->L + (want_head ? 1 : 0);
   const int nb = std::max(1, std::min(rows_ub, 1024));
-  k_embed<<<nb, 256, 0, h->stream>>>(h->rows, h->embed, h->h, d, rows_ub);
-  const int nw_blocks = std::max(1, std::min((rows_ub + 7) / 8, 1024));
-  AttnArgs aa{};
-  aa.kv = h->kv;
-  aa.page_table = h->page_table;
-  aa.max_pages = h->max_pages;
-  aa.PT = h->PT;
-  aa.L = h->L;
-  aa.H = h->H;
-  aa.dh = h->dh;
-  aa.d = d;
-  aa.rows = h->rows;
-  aa.CH = h->CH;
-  aa.CMAX = h->CMAX;
-  aa.scale = 1.0f / std::sqrt((float)h->dh);
-  aa.q = h->q;
-  aa.part_ml = h->part_ml;
-  aa.part_o = h->part_o;
-  aa.att = h->att;
-  aa.status = h->sd.status;
+  k_embed<<<nb, 256, 0, h->stream>>>(h->rows, h->embed, h->h, d);
+  AttnArgs aa = attn_args(h);
   const int nchunks = std::max(1, (keys_ub + h->CH - 1) / h->CH);
-  const size_t attn_smem = (size_t)(32 * h->dh + h->CH * h->dh + 32 * h->CH) * 4;
   for (int l = 0; l < h->L; ++l) {
-    // B_l = D_{l-1} + W_o^c W_v^c o_lat ; rs = RMS scale of B_l
-    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, h->c_lat, h->cfg.max_latents, h->L, l, d, eps, nullptr);
+    // B_l = D_{l-1} + W_o^c W_v^c o_lat
+    k_cross_add<<<nb, 256, 0, h->stream>>>(h->rows, h->h, h->c_lat, h->cfg.max_latents, h->L, l, d);
     GemmArgs a = base_args(h);
     a.layer = l;
     a.X = h->h;
     a.ldx = d;
-    a.rs = h->rs;
     a.gain = h->attn_norm[l];
     a.q = h->q;
     TRY(gemm<EPI_QKV>(h, h->qkv[l], a, rows_ub));
     aa.layer = l;
-    dim3 ag(h->H, nchunks, groups_ub);
-    launch_attn(h, ag, attn_smem, aa);
+    launch_attn(h, dim3(h->H, nchunks, groups_ub), attn_smem_bytes(h), aa);
     k_attn_combine<<<dim3(rows_ub, h->H), h->dh, 0, h->stream>>>(aa);
     CK(cudaGetLastError());
     a = base_args(h);
@@ -351,12 +365,10 @@ int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want
     a.out = h->h;
     a.ldo = d;
     TRY(gemm<EPI_RESID>(h, h->o[l], a, rows_ub));
-    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, nullptr, 0, 0, 0, d, eps, nullptr);
     a = base_args(h);
     a.layer = l;
     a.X = h->h;
     a.ldx = d;
-    a.rs = h->rs;
     a.gain = h->ffn_norm[l];
     a.out = h->act;
     a.ldo = h->F;
@@ -370,11 +382,9 @@ int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want
     TRY(gemm<EPI_RESID>(h, h->w2[l], a, rows_ub));
   }
   if (want_head) {
-    k_rownorm<<<nw_blocks, 256, 0, h->stream>>>(h->rows, h->h, h->rs, nullptr, 0, 0, 0, d, eps, nullptr);
     GemmArgs a = base_args(h);
     a.X = h->h;
     a.ldx = d;
-    a.rs = h->rs;
     a.gain = h->final_norm;
     a.out = h->logits;
     a.ldo = 256;
@@ -542,6 +552,22 @@ int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, f
   return BLT_OK;
 }
 
+int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes, int rows_ub, const int* vlat, float* out_logits,
+             int* out_acc, unsigned char* out_next);
+bool use_mega(const blt_dec* h, int rows_ub, int batch);
+
+// The block loop on the persistent kernel when the pass is small enough.
+int diffuse_passes(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, float alpha, int max_steps, float* out_logits) {
+  const int batch = cd.batch;
+  const int rows1 = cd.row_off[batch] + batch * k;
+  if (!use_mega(h, rows1, batch)) return block_loop(h, cd, pend, k, alpha, max_steps, out_logits);
+  PlanArgs p = plan_args(h, PL_FIRST, k);
+  p.pend_bytes = pend->bytes;
+  p.pend_lat = pend->row_latent;
+  TRY(plan(h, p, cd));
+  return mega_run(h, MM_DIFFUSE, batch, k, alpha, max_steps, rows1, nullptr, out_logits, nullptr, nullptr);
+}
+
 int check_pending(blt_dec* h, const blt_rows_in* r, bool need_rows) {
   if (!r) return fail(h, BLT_ERR_INVALID_ARG, "rows is NULL");
   if (need_rows && !r->row_offsets) return fail(h, BLT_ERR_INVALID_ARG, "row_offsets is NULL");
@@ -580,6 +606,157 @@ __global__ void k_finish_prefill(SeqDev sd, CallDesc cd) {
 }
 __global__ void k_copy_logits(const float* src, float* dst, int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------------------- persistent pass kernel
+template <int NG, int PL, int DH, typename KVT>
+size_t mega_smem(const blt_dec* h) {
+  return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 +
+         (size_t)2 * h->CH * DH * sizeof(KVT);
+}
+
+template <int NG, int PL, int DH, typename KVT>
+int mega_prepare_t(blt_dec* h) {
+  const size_t smem = mega_smem<NG, PL, DH, KVT>(h);
+  CK(cudaFuncSetAttribute(k_mega<NG, PL, DH, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int per_sm = 0;
+  CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_mega<NG, PL, DH, KVT>, kMegaThreads, smem));
+  if (per_sm < 1) return fail(h, BLT_ERR_CUDA, "persistent pass kernel does not fit on an SM");
+  return BLT_OK;
+}
+
+template <int PL, int DH, typename KVT>
+int mega_prepare_pd(blt_dec* h) {
+  TRY((mega_prepare_t<1, PL, DH, KVT>(h)));
+  return mega_prepare_t<2, PL, DH, KVT>(h);
+}
+
+// Decide whether the persistent kernel applies to this model and set it up.
+int mega_setup(blt_dec* h) {
+  if ((h->cfg.flags & BLT_FLAG_PER_PHASE) || h->d > 1024 || (h->dh != 32 && h->dh != 64) || h->CH > 128) return BLT_OK;
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  int coop = 0;
+  CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
+  CK(cudaDeviceGetAttribute(&h->nsm, cudaDevAttrMultiProcessorCount, dev));
+  if (!coop) return BLT_OK;
+  int rc;
+  if (h->planes == 1) {
+    rc = h->kv_f32 ? (h->dh == 64 ? mega_prepare_pd<1, 64, float>(h) : mega_prepare_pd<1, 32, float>(h))
+                   : (h->dh == 64 ? mega_prepare_pd<1, 64, __nv_bfloat16>(h) : mega_prepare_pd<1, 32, __nv_bfloat16>(h));
+  } else {
+    rc = h->kv_f32 ? (h->dh == 64 ? mega_prepare_pd<2, 64, float>(h) : mega_prepare_pd<2, 32, float>(h))
+                   : (h->dh == 64 ? mega_prepare_pd<2, 64, __nv_bfloat16>(h) : mega_prepare_pd<2, 32, __nv_bfloat16>(h));
+  }
+  if (rc != BLT_OK) {
+    h->err.clear();
+    return BLT_OK;  // not available: calls use the per-phase kernels
+  }
+  std::vector<LayerW> lw(h->L);
+  for (int l = 0; l < h->L; ++l)
+    lw[l] = LayerW{h->qkv[l].w, h->o[l].w, h->w13[l].w, h->w2[l].w, h->attn_norm[l], h->ffn_norm[l]};
+  TRY(dalloc(h, &h->d_layers, h->L));
+  CK(cudaMemcpy(h->d_layers, lw.data(), sizeof(LayerW) * h->L, cudaMemcpyHostToDevice));
+  const int d = h->d, F = h->F;
+  h->mega_groups = kMegaMaxNG * 8 + 1;  // <= 16 rows: at most 16 sequences, one group each
+  h->f_qkv = 0;
+  h->f_o = h->f_qkv + 3 * d / 16;
+  h->f_w13 = h->f_o + d / 16;
+  h->f_w2 = h->f_w13 + 2 * F / 16;
+  h->f_head = h->f_w2 + d / 16;
+  h->f_att = h->f_head + 16;
+  h->f_dec = h->f_att + h->mega_groups * h->H;
+  const int nflags = h->f_dec + 1;
+  TRY(dalloc(h, &h->flags, nflags));
+  CK(cudaMemset(h->flags, 0, nflags * 4));
+  TRY(dalloc(h, &h->attn_cnt, h->mega_groups * h->H));
+  CK(cudaMemset(h->attn_cnt, 0, h->mega_groups * h->H * 4));
+  TRY(dalloc(h, &h->dec_val, 1));
+  TRY(dalloc(h, &h->abort_flag, 1));
+  CK(cudaMemset(h->abort_flag, 0, 4));
+  h->epoch = 1;
+  h->mega_ok = true;
+  return BLT_OK;
+}
+
+bool use_mega(const blt_dec* h, int rows_ub, int batch) {
+  return h->mega_ok && rows_ub <= 8 * kMegaMaxNG && batch <= 8 * kMegaMaxNG;
+}
+
+template <int NG, int PL, int DH, typename KVT>
+int mega_launch_t(blt_dec* h, MegaArgs& m) {
+  const size_t smem = mega_smem<NG, PL, DH, KVT>(h);
+  void* args[] = {&m};
+  CK(cudaLaunchCooperativeKernel((const void*)k_mega<NG, PL, DH, KVT>, dim3(h->nsm), dim3(kMegaThreads), args, smem, h->stream));
+  h->launches += 1;
+  return BLT_OK;
+}
+
+// All passes of one call in one launch (rows of pass 1 already planned).
+int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes, int rows_ub, const int* vlat, float* out_logits,
+             int* out_acc, unsigned char* out_next) {
+  MegaArgs m{};
+  m.layers = h->d_layers;
+  m.whead = h->head.w;
+  m.final_norm = h->final_norm;
+  m.L = h->L;
+  m.d = h->d;
+  m.H = h->H;
+  m.dh = h->dh;
+  m.F = h->F;
+  m.planes = h->planes;
+  m.eps = h->cfg.norm_eps;
+  m.ga = base_args(h);
+  m.ga.q = h->q;
+  m.aa = attn_args(h);
+  m.rows = h->rows;
+  m.sd = h->sd;
+  m.h = h->h;
+  m.q = h->q;
+  m.att = h->att;
+  m.act = h->act;
+  m.logits = h->logits;
+  m.conf = h->conf;
+  m.pred = h->pred;
+  m.gap = h->gap;
+  m.flags = h->flags;
+  m.f_qkv = h->f_qkv;
+  m.f_o = h->f_o;
+  m.f_w13 = h->f_w13;
+  m.f_w2 = h->f_w2;
+  m.f_head = h->f_head;
+  m.f_att = h->f_att;
+  m.f_dec = h->f_dec;
+  m.attn_cnt = h->attn_cnt;
+  m.dec_val = h->dec_val;
+  m.epoch0 = h->epoch;
+  h->epoch += (unsigned)(max_passes + 1) * (h->L + 1) + 1;
+  m.abort = h->abort_flag;
+  m.mode = mode;
+  m.batch = batch;
+  m.k = k;
+  m.max_passes = max_passes;
+  m.alpha = alpha;
+  m.vlat = vlat;
+  m.out_logits = out_logits;
+  m.out_acc = out_acc;
+  m.out_next = out_next;
+  m.plan = plan_args(h, PL_BLOCK, k);
+  const bool ng1 = rows_ub <= 8;
+  if (h->planes == 1) {
+    if (h->kv_f32) {
+      if (h->dh == 64) return ng1 ? mega_launch_t<1, 1, 64, float>(h, m) : mega_launch_t<2, 1, 64, float>(h, m);
+      return ng1 ? mega_launch_t<1, 1, 32, float>(h, m) : mega_launch_t<2, 1, 32, float>(h, m);
+    }
+    if (h->dh == 64) return ng1 ? mega_launch_t<1, 1, 64, __nv_bfloat16>(h, m) : mega_launch_t<2, 1, 64, __nv_bfloat16>(h, m);
+    return ng1 ? mega_launch_t<1, 1, 32, __nv_bfloat16>(h, m) : mega_launch_t<2, 1, 32, __nv_bfloat16>(h, m);
+  }
+  if (h->kv_f32) {
+    if (h->dh == 64) return ng1 ? mega_launch_t<1, 2, 64, float>(h, m) : mega_launch_t<2, 2, 64, float>(h, m);
+    return ng1 ? mega_launch_t<1, 2, 32, float>(h, m) : mega_launch_t<2, 2, 32, float>(h, m);
+  }
+  if (h->dh == 64) return ng1 ? mega_launch_t<1, 2, 64, __nv_bfloat16>(h, m) : mega_launch_t<2, 2, 64, __nv_bfloat16>(h, m);
+  return ng1 ? mega_launch_t<1, 2, 32, __nv_bfloat16>(h, m) : mega_launch_t<2, 2, 32, __nv_bfloat16>(h, m);
 }
 
 }  // namespace
@@ -733,6 +910,7 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(dalloc(h, &rd.g_row0, RL + c.max_batch));
     TRY(dalloc(h, &rd.g_nrows, RL + c.max_batch));
     TRY(dalloc(h, &rd.g_kmax, RL + c.max_batch));
+    TRY(dalloc(h, &rd.g_fresh, RL + c.max_batch));
     TRY(dalloc(h, &rd.n_groups, 1));
     TRY(dalloc(h, &h->lat_seq, R));
     TRY(dalloc(h, &h->lat_slot, R));
@@ -768,9 +946,9 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(set_attrs_epi<EPI_SWIGLU>(h));
     TRY(set_attrs_epi<EPI_QKV>(h));
     TRY(set_attrs_epi<EPI_LATC>(h));
-    const size_t attn_smem = (size_t)(32 * dh + h->CH * dh + 32 * h->CH) * 4;
-    TRY(set_attn_attrs<float>(h, attn_smem));
-    TRY(set_attn_attrs<__nv_bfloat16>(h, attn_smem));
+    TRY(set_attn_attrs<float>(h, attn_smem_bytes(h)));
+    TRY(set_attn_attrs<__nv_bfloat16>(h, attn_smem_bytes(h)));
+    TRY(mega_setup(h));
     CK(cudaDeviceSynchronize());
     return BLT_OK;
   };
@@ -844,7 +1022,9 @@ int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, i
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
   h->launches += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
-  TRY(block_loop(h, cd, pending, k, alpha, max_steps, out_logits));
+  TRY(pass_begin(h));
+  TRY(diffuse_passes(h, cd, pending, k, alpha, max_steps, out_logits));
+  TRY(pass_end(h));
   k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_block, out_steps);
   h->launches += 1;
   CK(cudaGetLastError());
@@ -875,7 +1055,14 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
   h->launches += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
-  if (mode == BLT_DRAFT_AR) {
+  TRY(pass_begin(h));
+  if (mode == BLT_DRAFT_AR && use_mega(h, std::max(cd.row_off[batch], batch), batch)) {
+    PlanArgs p = plan_args(h, PL_FIRST, 0);
+    p.pend_bytes = pending->bytes;
+    p.pend_lat = pending->row_latent;
+    TRY(plan(h, p, cd));
+    TRY(mega_run(h, MM_DRAFT_AR, batch, k, 0.f, k, std::max(cd.row_off[batch], batch), nullptr, out_logits, nullptr, nullptr));
+  } else if (mode == BLT_DRAFT_AR) {
     int npmax = 0;
     for (int s = 0; s < batch; ++s) npmax = std::max(npmax, cd.row_off[s + 1] - cd.row_off[s]);
     const int keys_ub = max_kv_ub(h, batch) + npmax + k;
@@ -884,20 +1071,21 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
     p.pend_lat = pending->row_latent;
     TRY(plan(h, p, cd));
     TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true));
-    k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, 0, h->pred, h->logits, out_logits);
+    k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, 0, h->pred, h->logits, out_logits);
     h->launches += 1;
     for (int t = 1; t < k; ++t) {
       PlanArgs pa = plan_args(h, PL_ARDRAFT, 0);
       pa.step = t;
       TRY(plan(h, pa, cd));
       TRY(run_pass(h, batch, keys_ub, batch, true));
-      k_draft_ar<<<(batch + 127) / 128, 128, 0, h->stream>>>(h->sd, batch, k, t, h->pred, h->logits, out_logits);
+      k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, t, h->pred, h->logits, out_logits);
       h->launches += 1;
     }
   } else {
     if (max_steps <= 0) max_steps = k;
-    TRY(block_loop(h, cd, pending, k, alpha, max_steps, out_logits));
+    TRY(diffuse_passes(h, cd, pending, k, alpha, max_steps, out_logits));
   }
+  TRY(pass_end(h));
   if (mode == BLT_DRAFT_DIFFUSION) k_finish_block<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft, nullptr);
   else k_copy_draft<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, out_draft);
   h->launches += 1;
@@ -924,12 +1112,18 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
   k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
   h->launches += 1;
   TRY(project_latents(h, cd, new_latents, false));
+  TRY(pass_begin(h));
   PlanArgs p = plan_args(h, PL_VERIFY, k);
   p.vlat = draft_row_latent;
   TRY(plan(h, p, cd));
-  TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true));
-  k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
-  h->launches += 1;
+  if (use_mega(h, batch * k, batch)) {
+    TRY(mega_run(h, MM_VERIFY, batch, k, 0.f, 1, batch * k, draft_row_latent, out_logits, out_accepted, out_next));
+  } else {
+    TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true));
+    k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
+    h->launches += 1;
+  }
+  TRY(pass_end(h));
   CK(cudaGetLastError());
   for (int s = 0; s < batch; ++s) {
     h->kv_ub[s] += k;
@@ -978,7 +1172,7 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->weight_bytes = c[5];
   out->kv_read_bytes = c[6];
   out->kernel_launches = h->launches;
-  out->timed_passes = h->timed_passes;
+  out->timed_passes = (h->cfg.flags & BLT_FLAG_TIME_PASSES) ? c[0] : 0;
   out->pass_ns = h->pass_ns;
   return BLT_OK;
 }

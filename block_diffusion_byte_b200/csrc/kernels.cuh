@@ -1,66 +1,111 @@
-// Kernels of one Fast-BLT local-decoder pass and its bookkeeping (sm_100a).
+// Kernels of the Fast-BLT local-decoder pass and its bookkeeping (sm_100a).
 //
-// Decoder layer ("계층적 BLT: 인코더, 글로벌 모델, 디코더", the layer equation of
-// the Fast-BLT summary page): the cross-attention term for a row that sees
-// exactly one latent o is W_o^c W_v^c o (softmax over one key is 1), added to
-// the residual; then pre-norm self-attention and a SwiGLU FFN.
+// Decoder layer (the layer equation of "Fast Byte Latent Transformer
+// (Fast-BLT) 연구 소개", section "계층적 BLT: 인코더, 글로벌 모델, 디코더"):
+//   B_l = D_{l-1} + W_o^c softmax(Q K^T / sqrt(d_k)) V     (cross-attention)
+//   D_l = DecoderTransformerLayer(B_l)                     (pre-norm self-attn + SwiGLU)
+// A row sees exactly one latent o (section "BLT-D의 어텐션 마스크"), so the
+// softmax is exactly 1 and the cross term is c = W_o^c W_v^c o, projected once
+// when the latent arrives and gathered per row.
 //
-// Canonical arithmetic of every projection y = W x (one fp32 value per output):
-//   x is split into bf16 planes x_hi + x_lo; W is one bf16 plane (or hi + lo
-//   for fp32 weights).  K is cut into k16 steps; step s belongs to lane group
-//   w = s mod 8.  Group w accumulates, in increasing s, the tensor-core products
-//   W_hi x_hi, W_hi x_lo (, W_lo x_hi) into one fp32 accumulator; the output is
-//   ((g_0 + g_1) + ...) + g_7.  The order depends on nothing but K, so a row
-//   gets bit-identical results whatever the other rows of its pass are.
+// Canonical arithmetic of every projection y = rs * (W (g . x)):
+//   x is the fp32 input row, g the RMSNorm gain (1 when there is no norm),
+//   g . x is split into bf16 planes hi + lo; W is one bf16 plane (two for
+//   fp32 weights).  K is cut into k16 steps; step s belongs to lane group
+//   w = s mod 8, which accumulates in increasing s the tensor-core products
+//   W_hi x_hi, W_hi x_lo (, W_lo x_hi) into one fp32 accumulator.  The output
+//   is rs * (((a_0 + a_1) + ...) + a_7).  The RMS scale rs = 1/sqrt(ss/K + eps)
+//   takes ss from the same fragments: every lane adds x^2 of its four values in
+//   k order, the four lanes of a row are summed by xor-shuffles (1 then 2) and
+//   the eight groups in order.  Nothing depends on which other rows share the
+//   pass, or on which kernel (per-phase or persistent) runs it, so a row's
+//   results are bit-identical in every pass shape.
 #pragma once
 
 #include "common.cuh"
 
 namespace bltdec {
 
-enum RowKind : int { ROW_CAUSAL = 0, ROW_BLOCK = 1 };
-
-// Per-pass row metadata (device arrays sized max_rows; counts are device scalars).
-struct RowsDev {
-  int* seq;     // sequence of the row
-  int* pos;     // 0-based byte position (RoPE, KV slot)
-  int* lat;     // latent slot seen by the cross-attention
-  int* nkeys;   // the row attends positions 0 .. nkeys-1 of its sequence
-  int* byte;    // input id (0..255 or [MASK])
-  int* n_rows;  // device scalar
-  // attention groups: up to 32 consecutive rows of one sequence
-  int* g_seq;
+// ------------------------------------------------------------------------ shared state
+struct RowsDev {  // per-pass row metadata (arrays of max_rows; counts are device scalars)
+  int* seq;       // sequence of the row
+  int* pos;       // 0-based byte position (RoPE, KV slot)
+  int* lat;       // latent slot seen by the cross-attention
+  int* nkeys;     // the row attends positions 0 .. nkeys-1 of its sequence
+  int* byte;      // input id (0..255 or [MASK])
+  int* n_rows;    // device scalar
+  int* g_seq;     // attention groups: up to 32 consecutive rows of one sequence
   int* g_row0;
   int* g_nrows;
   int* g_kmax;
+  int* g_fresh;   // first position written by this pass in the group's sequence
   int* n_groups;  // device scalar
 };
 
-// ------------------------------------------------------------------------ GEMM
-enum Epi : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_LATC = 4 };
+constexpr int kMaxCallBatch = 256;
+
+struct CallDesc {  // by value as a kernel parameter
+  int batch;
+  int row_off[kMaxCallBatch + 1];
+  int lat_off[kMaxCallBatch + 1];
+};
+
+struct SeqDev {
+  int* kv_len;      // cached committed positions
+  int* kv_base;     // kv_len at call start (prefill)
+  int* n_lat;       // committed latent slots
+  int* active;      // block still has masked positions
+  int* steps;       // passes used by the current block
+  int* y_last;      // greedy prediction of the last pending row (verification y_l)
+  int* last_row;    // row index of the last pending row in pass 1 (-1: none)
+  int* blk_row;     // [batch][kMaxBlock] row index of block/draft/verify row i in this pass
+  unsigned char* blk;     // [batch][kMaxBlock] block / draft bytes
+  unsigned char* masked;  // [batch][kMaxBlock]
+  int* status;
+  unsigned long long* counters;  // passes, rows, prefill_rows, latents, calls, weight_bytes, kv_bytes
+};
+
+enum PlanMode : int { PL_PREFILL = 0, PL_FIRST = 1, PL_BLOCK = 2, PL_ARDRAFT = 3, PL_VERIFY = 4 };
+
+struct PlanArgs {
+  int mode, k, step, r0, r1;
+  int max_ctx, max_lat, mask_id;
+  const unsigned char* pend_bytes;
+  const int* pend_lat;
+  const int* vlat;  // verify slots [batch][k]
+  unsigned long long weight_bytes_per_pass;
+  unsigned long long kv_bytes_per_key;
+};
+
+// ------------------------------------------------------------------------ GEMM pieces
+enum Epi : int { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_LATC = 4, EPI_XRESID = 5 };
 
 struct GemmArgs {
   const uint4* w;  // tiles [N/16][K/16][planes][32 lanes] of 16 B
   int N, K;
   const float* X;  // activations [rows][ldx] fp32
   int ldx;
-  const float* rs;    // per-row RMS scale (NULL: x used as is)
-  const float* gain;  // [K] RMSNorm gain (with rs)
+  const float* gain;  // [K] RMSNorm gain; NULL: no norm (rs = 1)
+  float eps;
   const int* n_rows;  // device row count (NULL: rows_host is exact)
   int rows_host;
-  float* out;  // EPI_STORE / RESID / SWIGLU / LATC base
+  float* out;  // EPI_STORE / RESID / SWIGLU / LATC / XRESID base
   int ldo;
+  // EPI_XRESID: out = (xsrc + c_lat) + v, xsrc = embed[byte] in layer 0, else out itself
+  const float* embed;
+  const float* c_lat;
   // EPI_QKV
   float* q;
-  void* kv;    // KV pool: bf16, or fp32 when kv_f32
+  void* kv;  // KV pool: bf16, or fp32 when kv_f32
   int kv_f32;
   const int* page_table;
   int max_pages, PT, layer, L, H, dh, d;
   const int* row_seq;
   const int* row_pos;
+  const int* row_lat;
+  const int* row_byte;
   const float* rope_cos;  // [max_ctx][dh/2]
   const float* rope_sin;
-  int max_ctx;
   // EPI_LATC
   const int* lat_seq;
   const int* lat_slot;
@@ -68,10 +113,43 @@ struct GemmArgs {
   int* status;
 };
 
+// Four gained values of one k16 step -> hi/lo B fragments (k = 2t, 2t+1 | 2t+8, 2t+9).
+struct XFrag {
+  uint32_t b0h, b1h, b0l, b1l;
+};
+__device__ __forceinline__ XFrag make_xfrag(float x0, float x1, float x8, float x9) {
+  XFrag f;
+  split2(x0, x1, f.b0h, f.b0l);
+  split2(x8, x9, f.b1h, f.b1l);
+  return f;
+}
+__device__ __forceinline__ float ss_add(float ss, float v0, float v1, float v8, float v9) {
+  ss = fmaf(v0, v0, ss);
+  ss = fmaf(v1, v1, ss);
+  ss = fmaf(v8, v8, ss);
+  return fmaf(v9, v9, ss);
+}
+template <int PL>
+__device__ __forceinline__ void mma_step(float (&c)[4], const uint4 (&w)[PL], const XFrag& x) {
+  mma16816(c, w[0], x.b0h, x.b1h);
+  mma16816(c, w[0], x.b0l, x.b1l);
+  if constexpr (PL == 2) mma16816(c, w[1], x.b0h, x.b1h);
+}
+
 __device__ __forceinline__ size_t kv_offset(const GemmArgs& a, int page, int kvsel, int h, int off, int dim) {
   return ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * a.dh + (size_t)off * a.dh + dim;
 }
 
+__device__ __forceinline__ const float* c_row(const float* c_lat, int max_lat, int L, int layer, int d, int seq, int lat) {
+  return c_lat + (((size_t)seq * max_lat + lat) * L + layer) * d;
+}
+
+__device__ __forceinline__ void kv_store(const GemmArgs& a, size_t off, float v) {
+  if (a.kv_f32) static_cast<float*>(a.kv)[off] = v;
+  else static_cast<__nv_bfloat16*>(a.kv)[off] = __float2bfloat16_rn(v);
+}
+
+// Output pair of tile rows (r16, r16 + 8) of tile mt for activation row `row`.
 template <int EPI>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16, int row, float v0, float v1) {
   if constexpr (EPI == EPI_STORE) {
@@ -80,21 +158,29 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
     o[8] = v1;
   } else if constexpr (EPI == EPI_RESID) {
     float* o = a.out + (size_t)row * a.ldo + mt * 16 + r16;
-    o[0] += v0;
-    o[8] += v1;
+    o[0] = __ldcg(o) + v0;
+    o[8] = __ldcg(o + 8) + v1;
+  } else if constexpr (EPI == EPI_XRESID) {
+    const int n = mt * 16 + r16;
+    const float* src = (a.layer == 0) ? a.embed + (size_t)__ldcg(a.row_byte + row) * a.d : a.out + (size_t)row * a.ldo;
+    const float* c = c_row(a.c_lat, a.max_lat, a.L, a.layer, a.d, __ldcg(a.row_seq + row), __ldcg(a.row_lat + row));
+    const float s0 = __ldcg(src + n) + __ldcg(c + n), s1 = __ldcg(src + n + 8) + __ldcg(c + n + 8);
+    float* o = a.out + (size_t)row * a.ldo + n;
+    o[0] = s0 + v0;
+    o[8] = s1 + v1;
   } else if constexpr (EPI == EPI_SWIGLU) {
     a.out[(size_t)row * a.ldo + mt * 8 + r16] = silu(v0) * v1;
   } else if constexpr (EPI == EPI_LATC) {
-    const int s = a.lat_seq[row], slot = a.lat_slot[row];
-    float* o = a.out + (((size_t)s * a.max_lat + slot) * a.L + a.layer) * a.d + mt * 16 + r16;
+    float* o = a.out + (((size_t)a.lat_seq[row] * a.max_lat + a.lat_slot[row]) * a.L + a.layer) * a.d + mt * 16 + r16;
     o[0] = v0;
     o[8] = v1;
-  } else {  // EPI_QKV
+  } else {  // EPI_QKV: q/k tiles hold rotary pairs (j, j + dh/2) in rows (r16, r16 + 8)
     const int tiles_sec = a.d / 16;
     const int sec = mt / tiles_sec, lt = mt % tiles_sec;
-    const int pos = a.row_pos[row];
-    if (sec < 2) {
-      const int tph = a.dh / 16;  // tiles per head
+    const int pos = __ldcg(a.row_pos + row);
+    const int seq = __ldcg(a.row_seq + row);
+    if (sec == 0 || sec == 1) {
+      const int tph = a.dh / 16;
       const int h = lt / tph, j = (lt % tph) * 8 + r16;
       const int half = a.dh / 2;
       const float c = a.rope_cos[(size_t)pos * half + j], s = a.rope_sin[(size_t)pos * half + j];
@@ -103,27 +189,18 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         float* q = a.q + (size_t)row * a.d + h * a.dh;
         q[j] = o0;
         q[j + half] = o1;
-      } else {
-        const int seq = a.row_seq[row];
-        const int pi = pos / a.PT;
-        const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
-        if (page < 0) {
-          set_status(a.status, kErrDevice);
-          return;
-        }
-        const size_t off = kv_offset(a, page, 0, h, pos % a.PT, 0);
-        if (a.kv_f32) {
-          float* k = static_cast<float*>(a.kv) + off;
-          k[j] = o0;
-          k[j + half] = o1;
-        } else {
-          __nv_bfloat16* k = static_cast<__nv_bfloat16*>(a.kv) + off;
-          k[j] = __float2bfloat16_rn(o0);
-          k[j + half] = __float2bfloat16_rn(o1);
-        }
+        return;
       }
+      const int pi = pos / a.PT;
+      const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+      if (page < 0) {
+        set_status(a.status, kErrDevice);
+        return;
+      }
+      const size_t off = kv_offset(a, page, 0, h, pos % a.PT, 0);
+      kv_store(a, off + j, o0);
+      kv_store(a, off + j + half, o1);
     } else {
-      const int seq = a.row_seq[row];
       const int pi = pos / a.PT;
       const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
       if (page < 0) {
@@ -131,21 +208,59 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         return;
       }
       const int n0 = lt * 16 + r16, n1 = n0 + 8;
-      const size_t o0 = kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh);
-      const size_t o1 = kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh);
-      if (a.kv_f32) {
-        static_cast<float*>(a.kv)[o0] = v0;
-        static_cast<float*>(a.kv)[o1] = v1;
-      } else {
-        static_cast<__nv_bfloat16*>(a.kv)[o0] = __float2bfloat16_rn(v0);
-        static_cast<__nv_bfloat16*>(a.kv)[o1] = __float2bfloat16_rn(v1);
-      }
+      kv_store(a, kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
+      kv_store(a, kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
     }
   }
 }
 
-// One CTA: one 16-row tile of W against RB = 8*NG activation rows.
-// 8 warps; warp w owns k16 steps w, w+8, ... (the canonical split).
+// Canonical cross-warp reduction of one tile (RB rows).  acc: each warp's
+// accumulators; ss: each warp's per-lane sum of squares for row n*8+g.
+// red: smem [8][16][RB]; ssr: smem [8][RB].  Calls epi(r16, col, v0, v1) with
+// the scaled pair for every valid column.  `sync` is a consumer-wide barrier;
+// red/ssr are free again after the call returns and the caller syncs.
+template <int NG, class Sync, class Fn>
+__device__ __forceinline__ void tile_reduce(const float (&acc)[NG][4], const float (&ss)[NG], bool want_ss, float* red,
+                                            float* ssr, int nr, int K, float eps, int tid, int nthreads, Sync sync, Fn epi) {
+  constexpr int RB = 8 * NG;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    const int c = n * 8 + 2 * t;
+    red[(warp * 16 + g) * RB + c] = acc[n][0];
+    red[(warp * 16 + g) * RB + c + 1] = acc[n][1];
+    red[(warp * 16 + g + 8) * RB + c] = acc[n][2];
+    red[(warp * 16 + g + 8) * RB + c + 1] = acc[n][3];
+    if (want_ss) {
+      float s = ss[n];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (t == 0) ssr[warp * RB + n * 8 + g] = s;
+    }
+  }
+  sync();
+  for (int p = tid; p < 8 * RB; p += nthreads) {
+    const int r16 = p & 7, col = p >> 3;
+    if (col >= nr) continue;
+    float v0 = red[r16 * RB + col], v1 = red[(r16 + 8) * RB + col];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+      v0 += red[(w * 16 + r16) * RB + col];
+      v1 += red[(w * 16 + r16 + 8) * RB + col];
+    }
+    float rs = 1.0f;
+    if (want_ss) {
+      float s = ssr[col];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) s += ssr[w * RB + col];
+      rs = 1.0f / sqrtf(s / (float)K + eps);
+    }
+    epi(r16, col, v0 * rs, v1 * rs);
+  }
+}
+
+// Per-phase GEMM kernel (passes with many rows, latent projection, prefill).
+// One CTA: one 16-row tile of W against RB = 8*NG rows.
 template <int NG, int PL, int EPI, int STAGES>
 __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   constexpr int RB = 8 * NG;
@@ -157,17 +272,15 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
 
   extern __shared__ float4 smem4[];
   float* xs = reinterpret_cast<float*>(smem4);  // [STAGES][RB][kXStride]
-  float* rsv = xs + STAGES * RB * kXStride;     // [RB]
+  float* ssr = xs + STAGES * RB * kXStride;     // [8][RB]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nwin = a.K / kKWin;
   const int ksteps = a.K / 16;
-
-  if (tid < RB) rsv[tid] = (a.rs && tid < nr) ? a.rs[row0 + tid] : 1.0f;
+  const bool norm = a.gain != nullptr;
 
   auto stage = [&](int wi, int buf) {
-    // RB rows x 128 floats = RB*32 chunks of 16 B
     for (int c = tid; c < RB * 32; c += kThreads) {
       const int r = c >> 5, q = c & 31;
       const bool ok = r < nr;
@@ -175,8 +288,6 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
       cp_async16(xs + ((size_t)buf * RB + r) * kXStride + q * 4, src, ok ? 16 : 0);
     }
   };
-
-  // weight tile of window wi for this warp, plane p
   const uint4* wbase = a.w + (size_t)mt * ksteps * PL * 32 + lane;
   auto wtile = [&](int wi, int p) -> uint4 { return ldg_stream(wbase + ((size_t)(wi * kWarps + warp) * PL + p) * 32); };
 
@@ -186,19 +297,14 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   for (int dd = 0; dd < DEPTH; ++dd)
 #pragma unroll
     for (int p = 0; p < PL; ++p) wb[dd][p] = (dd < nwin) ? wtile(dd, p) : make_uint4(0, 0, 0, 0);
-
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
     if (s < nwin) stage(s, s);
     cp_async_commit();
   }
-
-  float acc[NG][4];
+  float acc[NG][4], ss[NG];
 #pragma unroll
-  for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-
-  __syncthreads();  // rsv
-  const bool has_gain = a.rs != nullptr;
+  for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
 
   for (int wi0 = 0; wi0 < nwin; wi0 += DEPTH) {
 #pragma unroll
@@ -213,15 +319,13 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
         }
         cp_async_wait<STAGES - 2>();
         __syncthreads();
-        // refill the stage consumed STAGES-1 windows ago
         if (wi + STAGES - 1 < nwin) stage(wi + STAGES - 1, (wi + STAGES - 1) % STAGES);
         cp_async_commit();
-
         const float* xw = xs + (size_t)(wi % STAGES) * RB * kXStride;
-        const int kk = warp * 16 + 2 * t;  // column within the window
-        const int kg = wi * kKWin + kk;    // global k
+        const int kk = warp * 16 + 2 * t;
+        const int kg = wi * kKWin + kk;
         float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
-        if (has_gain) {
+        if (norm) {
           g0 = __ldg(a.gain + kg);
           g1 = __ldg(a.gain + kg + 1);
           g8 = __ldg(a.gain + kg + 8);
@@ -229,51 +333,24 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
         }
 #pragma unroll
         for (int n = 0; n < NG; ++n) {
-          const int r = n * 8 + g;
-          const float* xr = xw + r * kXStride + kk;
+          const float* xr = xw + (n * 8 + g) * kXStride + kk;
           const float2 p0 = *reinterpret_cast<const float2*>(xr);
           const float2 p8 = *reinterpret_cast<const float2*>(xr + 8);
-          const float sc = rsv[r];
-          uint32_t b0h, b0l, b1h, b1l;
-          split2(p0.x * sc * g0, p0.y * sc * g1, b0h, b0l);
-          split2(p8.x * sc * g8, p8.y * sc * g9, b1h, b1l);
-          mma16816(acc[n], wcur[0], b0h, b1h);
-          mma16816(acc[n], wcur[0], b0l, b1l);
-          if constexpr (PL == 2) mma16816(acc[n], wcur[1], b0h, b1h);
+          if (norm) ss[n] = ss_add(ss[n], p0.x, p0.y, p8.x, p8.y);
+          mma_step<PL>(acc[n], wcur, make_xfrag(p0.x * g0, p0.y * g1, p8.x * g8, p8.y * g9));
         }
       }
     }
   }
   cp_async_wait<0>();
   __syncthreads();
-
-  // cross-warp reduction in canonical order
-  float* red = xs;  // [8][16][RB]
-#pragma unroll
-  for (int n = 0; n < NG; ++n) {
-    const int c = n * 8 + 2 * t;
-    red[(warp * 16 + g) * RB + c] = acc[n][0];
-    red[(warp * 16 + g) * RB + c + 1] = acc[n][1];
-    red[(warp * 16 + g + 8) * RB + c] = acc[n][2];
-    red[(warp * 16 + g + 8) * RB + c + 1] = acc[n][3];
-  }
-  __syncthreads();
-  for (int p = tid; p < 8 * RB; p += kThreads) {
-    const int r16 = p & 7, col = p >> 3;
-    if (col >= nr) continue;
-    float v0 = red[r16 * RB + col], v1 = red[(r16 + 8) * RB + col];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) {
-      v0 += red[(w * 16 + r16) * RB + col];
-      v1 += red[(w * 16 + r16 + 8) * RB + col];
-    }
-    gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1);
-  }
+  tile_reduce<NG>(acc, ss, norm, xs, ssr, nr, a.K, a.eps, tid, kThreads, [] { __syncthreads(); },
+                  [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
 }
 
 // ------------------------------------------------------------------------ row-wise kernels
 // h[row] = embed[byte[row]]
-__global__ void k_embed(const RowsDev rows, const float* __restrict__ embed, float* __restrict__ h, int d, int rows_max) {
+__global__ void k_embed(const RowsDev rows, const float* __restrict__ embed, float* __restrict__ h, int d) {
   const int n = *rows.n_rows;
   for (int r = blockIdx.x; r < n; r += gridDim.x) {
     const float* e = embed + (size_t)rows.byte[r] * d;
@@ -281,31 +358,13 @@ __global__ void k_embed(const RowsDev rows, const float* __restrict__ embed, flo
   }
 }
 
-// h[row] += c_lat[seq][lat][layer] (when c_lat != NULL); rs[row] = 1/sqrt(mean(h^2) + eps).
-// One warp per row.
-__global__ void k_rownorm(const RowsDev rows, float* __restrict__ h, float* __restrict__ rs, const float* __restrict__ c_lat,
-                          int max_lat, int L, int layer, int d, float eps, const int* n_rows_override) {
-  const int n = n_rows_override ? *n_rows_override : *rows.n_rows;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int r = warp; r < n; r += nw) {
-    float* hr = h + (size_t)r * d;
-    const float* cr = c_lat ? c_lat + (((size_t)rows.seq[r] * max_lat + rows.lat[r]) * L + layer) * d : nullptr;
-    float ss = 0.f;
-    for (int i = lane * 4; i < d; i += 128) {
-      float4 v = *reinterpret_cast<float4*>(hr + i);
-      if (cr) {
-        const float4 c = *reinterpret_cast<const float4*>(cr + i);
-        v.x += c.x;
-        v.y += c.y;
-        v.z += c.z;
-        v.w += c.w;
-        *reinterpret_cast<float4*>(hr + i) = v;
-      }
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-    }
-    ss = warp_sum(ss);
-    if (lane == 0) rs[r] = 1.0f / sqrtf(ss / (float)d + eps);
+// h[row] += c_lat[seq][lat][layer]: the cross-attention term of the layer.
+__global__ void k_cross_add(const RowsDev rows, float* __restrict__ h, const float* __restrict__ c_lat, int max_lat, int L,
+                            int layer, int d) {
+  const int n = *rows.n_rows;
+  for (int r = blockIdx.x; r < n; r += gridDim.x) {
+    const float* c = c_row(c_lat, max_lat, L, layer, d, rows.seq[r], rows.lat[r]);
+    for (int i = threadIdx.x; i < d; i += blockDim.x) h[(size_t)r * d + i] += c[i];
   }
 }
 
@@ -324,72 +383,69 @@ struct AttnArgs {
   int* status;
 };
 
-// 8 consecutive K/V elements (16-byte aligned) widened to fp32.
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* out) {
+constexpr int kAttnRows = 32;  // rows per attention group
+
+__device__ __forceinline__ void widen8(const __nv_bfloat16* p, float* out) {
   const uint4 raw = *reinterpret_cast<const uint4*>(p);
   const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&raw);
 #pragma unroll
   for (int e = 0; e < 8; ++e) out[e] = __bfloat162float(b[e]);
 }
-__device__ __forceinline__ void load8(const float* p, float* out) {
+__device__ __forceinline__ void widen8(const float* p, float* out) {
   const float4 x = reinterpret_cast<const float4*>(p)[0], y = reinterpret_cast<const float4*>(p)[1];
   out[0] = x.x, out[1] = x.y, out[2] = x.z, out[3] = x.w, out[4] = y.x, out[5] = y.y, out[6] = y.z, out[7] = y.w;
 }
 
-// grid (H, chunks, groups); 128 threads; one head of DH dims; KVT = K/V element type.
 template <int DH, typename KVT>
-__global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
-  constexpr int MAXR = 32;
-  const int gi = blockIdx.z;
-  if (gi >= *a.rows.n_groups) return;
-  const int kmax = a.rows.g_kmax[gi];
-  const int t0 = blockIdx.y * a.CH;
-  if (t0 >= kmax) return;
-  const int h = blockIdx.x;
-  const int seq = a.rows.g_seq[gi], row0 = a.rows.g_row0[gi], nr = a.rows.g_nrows[gi];
+__device__ __forceinline__ const KVT* kv_chunk_src(const AttnArgs& a, int seq, int h, int tpos, int kvsel) {
+  int page = a.page_table[seq * a.max_pages + tpos / a.PT];
+  if (page < 0) {
+    set_status(a.status, kErrDevice);
+    page = 0;
+  }
+  return static_cast<const KVT*>(a.kv) + ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * DH +
+         (size_t)(tpos % a.PT) * DH;
+}
+
+// Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
+// ks/vs (raw KVT, [CH][DH]) with 16-byte cp.async (L2 only).
+template <int DH, typename KVT>
+__device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, int t0, int lo, int hi, KVT* ks, KVT* vs, int tid,
+                                             int nthr) {
+  constexpr int PER = 16 / sizeof(KVT);
+  constexpr int CPR = DH / PER;
+  const int n = max(0, hi - lo);
+  for (int i = tid; i < 2 * n * CPR; i += nthr) {
+    const int kvsel = i / (n * CPR), j = i % (n * CPR);
+    const int key = lo - t0 + j / CPR, c = (j % CPR) * PER;
+    const KVT* src = kv_chunk_src<DH, KVT>(a, seq, h, t0 + key, kvsel) + c;
+    KVT* dst = (kvsel ? vs : ks) + key * DH + c;
+    cp_async16(dst, src, 16);
+  }
+}
+
+// Softmax partial of one (group, head, chunk): scores of every row against
+// keys [t0, t0+nk) (masked per row by nkeys), m = max, l = sum exp(s - m),
+// o = sum exp(s - m) v.  q pre-scaled by 1/sqrt(dh).  smem: qs [32][DH] f32,
+// ps [32][CH] f32, ks/vs [CH][DH] KVT already loaded.
+template <int DH, typename KVT, class Sync>
+__device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
+                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync) {
+  const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
+  const int t0 = chunk * a.CH;
   const int nk = min(a.CH, kmax - t0);
-
-  extern __shared__ float4 smem4[];
-  float* qs = reinterpret_cast<float*>(smem4);  // [MAXR][DH]
-  float* vs = qs + MAXR * DH;                   // [CH][DH]
-  float* ps = vs + a.CH * DH;                   // [MAXR][CH]
-  __shared__ int lim[MAXR];
-
-  const int tid = threadIdx.x;
-  for (int i = tid; i < nr * DH; i += 128) {
+  for (int i = tid; i < nr * DH; i += nthr) {
     const int r = i / DH, c = i % DH;
-    qs[r * DH + c] = a.q[(size_t)(row0 + r) * a.d + h * DH + c] * a.scale;
+    qs[r * DH + c] = __ldcg(a.q + (size_t)(row0 + r) * a.d + h * DH + c) * a.scale;
   }
-  if (tid < MAXR) lim[tid] = (tid < nr) ? a.rows.nkeys[row0 + tid] - t0 : 0;
-  // V chunk -> smem (fp32)
-  for (int i = tid; i < nk * (DH / 8); i += 128) {
-    const int key = i / (DH / 8), c8 = (i % (DH / 8)) * 8;
-    const int tpos = t0 + key;
-    int page = a.page_table[seq * a.max_pages + tpos / a.PT];
-    if (page < 0) {
-      set_status(a.status, kErrDevice);
-      page = 0;
-    }
-    const KVT* src = static_cast<const KVT*>(a.kv) + ((((size_t)page * a.L + a.layer) * 2 + 1) * a.H + h) * (size_t)a.PT * DH +
-                     (size_t)(tpos % a.PT) * DH + c8;
-    load8(src, vs + key * DH + c8);
-  }
-  __syncthreads();
-  // scores: thread = key (CH <= 128), K row in registers
-  for (int key = tid; key < a.CH; key += 128) {
+  if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
+  sync();
+  for (int key = tid; key < a.CH; key += nthr) {
     float kr[DH];
     const bool valid = key < nk;
     if (valid) {
-      const int tpos = t0 + key;
-      int page = a.page_table[seq * a.max_pages + tpos / a.PT];
-      if (page < 0) {
-        set_status(a.status, kErrDevice);
-        page = 0;
-      }
-      const KVT* src = static_cast<const KVT*>(a.kv) + ((((size_t)page * a.L + a.layer) * 2 + 0) * a.H + h) * (size_t)a.PT * DH +
-                       (size_t)(tpos % a.PT) * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 8; ++c) load8(src + c * 8, kr + c * 8);
+      for (int c = 0; c < DH / 8; ++c) widen8(ks + key * DH + c * 8, kr + c * 8);
     }
     for (int r = 0; r < nr; ++r) {
       float s = -INFINITY;
@@ -401,11 +457,9 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
       ps[r * a.CH + key] = s;
     }
   }
-  __syncthreads();
-  // softmax statistics per row: warp per row
-  const int warp = tid >> 5, lane = tid & 31;
-  __shared__ float mrow[MAXR], lrow[MAXR];
-  for (int r = warp; r < nr; r += 4) {
+  sync();
+  const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
+  for (int r = warp; r < nr; r += nw) {
     float m = -INFINITY;
     for (int k = lane; k < a.CH; k += 32) m = fmaxf(m, ps[r * a.CH + k]);
     m = warp_max(m);
@@ -422,144 +476,150 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
       lrow[r] = l;
     }
   }
-  __syncthreads();
-  // o = P V: thread -> (dim, row phase)
-  for (int i = tid; i < nr * DH; i += 128) {
+  sync();
+  for (int i = tid; i < nr * DH; i += nthr) {
     const int r = i / DH, c = i % DH;
     float o = 0.f;
-    for (int k = 0; k < nk; ++k) o = fmaf(ps[r * a.CH + k], vs[k * DH + c], o);
-    const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + blockIdx.y;
+    for (int k = 0; k < nk; ++k) {
+      float v;
+      if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * DH + c]);
+      else v = vs[k * DH + c];
+      o = fmaf(ps[r * a.CH + k], v, o);
+    }
+    const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
     a.part_o[base * DH + c] = o;
     if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
   }
 }
 
-// att[row][h*dh + c] = combine of the row's chunks in chunk order.  grid (rows_max, H), block dh.
-__global__ void k_attn_combine(AttnArgs a) {
-  const int row = blockIdx.x;
-  if (row >= *a.rows.n_rows) return;
-  const int h = blockIdx.y, c = threadIdx.x;
-  const int nk = a.rows.nkeys[row];
+// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}, in chunk order.
+__device__ __forceinline__ void attn_combine_one(const AttnArgs& a, int row, int h, int c) {
+  const int nk = __ldcg(a.rows.nkeys + row);
   const int nch = (nk + a.CH - 1) / a.CH;
   const size_t base = ((size_t)row * a.H + h) * a.CMAX;
   float m = -INFINITY;
   for (int ch = 0; ch < nch; ++ch) {
-    const float2 ml = a.part_ml[base + ch];
+    const float2 ml = __ldcg(a.part_ml + base + ch);
     if (ml.y > 0.f) m = fmaxf(m, ml.x);
   }
   float l = 0.f, o = 0.f;
   for (int ch = 0; ch < nch; ++ch) {
-    const float2 ml = a.part_ml[base + ch];
+    const float2 ml = __ldcg(a.part_ml + base + ch);
     if (ml.y > 0.f) {
       const float w = expf(ml.x - m);
       l += ml.y * w;
-      o += a.part_o[(base + ch) * a.dh + c] * w;
+      o += __ldcg(a.part_o + (base + ch) * a.dh + c) * w;
     }
   }
   a.att[(size_t)row * a.d + h * a.dh + c] = o / l;
 }
 
+// grid (H, chunks, groups); 128 threads.
+template <int DH, typename KVT>
+__global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
+  const int gi = blockIdx.z;
+  if (gi >= *a.rows.n_groups) return;
+  const int kmax = a.rows.g_kmax[gi];
+  const int t0 = blockIdx.y * a.CH;
+  if (t0 >= kmax) return;
+  const int h = blockIdx.x;
+  extern __shared__ float4 smem4[];
+  float* qs = reinterpret_cast<float*>(smem4);
+  float* ps = qs + kAttnRows * DH;
+  KVT* ks = reinterpret_cast<KVT*>(ps + kAttnRows * a.CH);
+  KVT* vs = ks + a.CH * DH;
+  __shared__ float mrow[kAttnRows], lrow[kAttnRows];
+  __shared__ int lim[kAttnRows];
+  attn_load_kv<DH, KVT>(a, a.rows.g_seq[gi], h, t0, t0, min(t0 + a.CH, kmax), ks, vs, threadIdx.x, 128);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  attn_partial_compute<DH, KVT>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128, [] { __syncthreads(); });
+}
+
+// grid (rows_max, H), block dh.
+__global__ void k_attn_combine(AttnArgs a) {
+  const int row = blockIdx.x;
+  if (row >= *a.rows.n_rows) return;
+  attn_combine_one(a, row, blockIdx.y, threadIdx.x);
+}
+
 // ------------------------------------------------------------------------ byte head statistics
-// One warp per row over the 256 byte logits: confidence (largest softmax
-// probability), argmax (lowest byte on ties), gap between the two largest logits.
+// Over the 256 byte logits of a row (one warp): confidence = largest softmax
+// probability, argmax (lowest byte on ties), gap between the two largest logits.
+__device__ __forceinline__ void head_stats_row(const float* z, int lane, float& conf, int& pred, float& gap) {
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = __ldcg(z + lane + 32 * j);
+  float b1 = -INFINITY, b2 = -INFINITY;
+  int i1 = 1 << 30;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int idx = lane + 32 * j;
+    if (v[j] > b1) {
+      b2 = b1;
+      b1 = v[j];
+      i1 = idx;
+    } else {
+      b2 = fmaxf(b2, v[j]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
+    const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
+    const int oi1 = __shfl_xor_sync(0xffffffffu, i1, o);
+    if (ob1 > b1 || (ob1 == b1 && oi1 < i1)) {
+      b2 = fmaxf(b1, ob2);
+      b1 = ob1;
+      i1 = oi1;
+    } else {
+      b2 = fmaxf(b2, ob1);
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s += expf(v[j] - b1);
+  s = warp_sum(s);
+  conf = 1.0f / s;
+  pred = i1;
+  gap = b1 - b2;
+}
+
 __global__ void k_head_stats(const float* __restrict__ logits, const int* n_rows, float* conf, int* pred, float* gap) {
   const int n = *n_rows;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   for (int r = warp; r < n; r += nw) {
-    const float* z = logits + (size_t)r * 256;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = z[lane + 32 * j];
-    float b1 = -INFINITY, b2 = -INFINITY;
-    int i1 = 1 << 30;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int idx = lane + 32 * j;
-      if (v[j] > b1) {
-        b2 = b1;
-        b1 = v[j];
-        i1 = idx;
-      } else {
-        b2 = fmaxf(b2, v[j]);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
-      const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
-      const int oi1 = __shfl_xor_sync(0xffffffffu, i1, o);
-      if (ob1 > b1 || (ob1 == b1 && oi1 < i1)) {
-        b2 = fmaxf(b1, ob2);
-        b1 = ob1;
-        i1 = oi1;
-      } else {
-        b2 = fmaxf(b2, ob1);
-      }
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s += expf(v[j] - b1);
-    s = warp_sum(s);
+    float c, g;
+    int p;
+    head_stats_row(logits + (size_t)r * 256, lane, c, p, g);
     if (lane == 0) {
-      conf[r] = 1.0f / s;
-      pred[r] = i1;
-      gap[r] = b1 - b2;
+      conf[r] = c;
+      pred[r] = p;
+      gap[r] = g;
     }
   }
 }
 
 // ------------------------------------------------------------------------ planning
-enum PlanMode : int { PL_PREFILL = 0, PL_FIRST = 1, PL_BLOCK = 2, PL_ARDRAFT = 3, PL_VERIFY = 4 };
-
-constexpr int kMaxCallBatch = 256;
-
-struct CallDesc {  // by value as a kernel parameter
-  int batch;
-  int row_off[kMaxCallBatch + 1];
-  int lat_off[kMaxCallBatch + 1];
-};
-
-struct SeqDev {
-  int* kv_len;     // cached committed positions
-  int* kv_base;    // kv_len at call start (prefill)
-  int* n_lat;      // committed latent slots
-  int* active;     // block still has masked positions
-  int* steps;      // passes used by the current block
-  int* y_last;     // greedy prediction of the last pending row (verification y_l)
-  int* last_row;   // row index of the last pending row in pass 1 (-1: none)
-  int* blk_row;    // [batch][kMaxBlock] row index of block/draft/verify row i in this pass
-  unsigned char* blk;     // [batch][kMaxBlock] block / draft bytes
-  unsigned char* masked;  // [batch][kMaxBlock]
-  int* status;
-  unsigned long long* counters;  // passes, rows, prefill_rows, latents, calls, weight_bytes, kv_bytes
-};
-
-struct PlanArgs {
-  int mode, k, step, r0, r1;
-  int max_ctx, max_lat, mask_id;
-  const unsigned char* pend_bytes;
-  const int* pend_lat;
-  const int* vlat;  // verify slots [batch][k]
-  int n_new_lat_total;
-  unsigned long long weight_bytes_per_pass;
-  unsigned long long kv_bytes_per_key;
-};
-
-// One CTA builds the rows of a pass.  Sequences' rows are contiguous, so each
-// attention group (<= 32 rows) belongs to one sequence.
-__global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd, RowsDev rd) {
-  __shared__ int cnt[kMaxCallBatch + 1];
-  __shared__ int gcnt[kMaxCallBatch + 1];
-  __shared__ int npend[kMaxCallBatch];
-  const int B = cd.batch, tid = threadIdx.x;
+// Builds the rows of a pass (one CTA, nthr threads; sh: 3*(kMaxCallBatch+1)
+// ints of shared memory).  Sequences' rows are contiguous, so each attention
+// group (<= 32 rows) belongs to one sequence.  row_off / lat_off may be NULL
+// (no pending rows / latents).
+template <class Sync>
+__device__ void plan_rows(const PlanArgs& p, int B, const int* row_off, const int* lat_off, SeqDev sd, RowsDev rd, int tid,
+                          int nthr, int* sh, Sync sync) {
+  int* cnt = sh;
+  int* gcnt = sh + (kMaxCallBatch + 1);
+  int* npend = sh + 2 * (kMaxCallBatch + 1);
   if (tid == 0) {
     int off = 0, goff = 0;
     for (int s = 0; s < B; ++s) {
-      int np = cd.row_off[s + 1] - cd.row_off[s];
+      const int np = row_off ? row_off[s + 1] - row_off[s] : 0;
       int n = 0;
       if (p.mode == PL_PREFILL) {
-        const int lo = max(cd.row_off[s], p.r0), hi = min(cd.row_off[s + 1], p.r1);
+        const int lo = max(row_off[s], p.r0), hi = min(row_off[s + 1], p.r1);
         n = max(0, hi - lo);
       } else if (p.mode == PL_FIRST) {
         n = np + p.k;
@@ -574,17 +634,17 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
       cnt[s] = off;
       gcnt[s] = goff;
       off += n;
-      goff += (n + 31) / 32;
+      goff += (n + kAttnRows - 1) / kAttnRows;
     }
     cnt[B] = off;
     gcnt[B] = goff;
     *rd.n_rows = off;
     *rd.n_groups = goff;
   }
-  __syncthreads();
+  sync();
   const int n_rows = cnt[B];
-  for (int r = tid; r < n_rows; r += blockDim.x) {
-    int lo = 0, hi = B;  // find s with cnt[s] <= r < cnt[s+1]
+  for (int r = tid; r < n_rows; r += nthr) {
+    int lo = 0, hi = B;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (cnt[mid] <= r) lo = mid;
@@ -595,15 +655,15 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
     const int kvl = sd.kv_len[s];
     const int nl = sd.n_lat[s];
     if (p.mode == PL_PREFILL) {
-      const int src = max(cd.row_off[s], p.r0) + i;
-      pos = sd.kv_base[s] + (src - cd.row_off[s]);
+      const int src = max(row_off[s], p.r0) + i;
+      pos = sd.kv_base[s] + (src - row_off[s]);
       byte = p.pend_bytes[src];
       lat = p.pend_lat[src];
       nkeys = pos + 1;
     } else if (p.mode == PL_FIRST) {
       const int np = npend[s];
       if (i < np) {
-        const int src = cd.row_off[s] + i;
+        const int src = row_off[s] + i;
         pos = kvl + i;
         byte = p.pend_bytes[src];
         lat = p.pend_lat[src];
@@ -635,7 +695,7 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
       lat = p.vlat[s * p.k + i];
       nkeys = pos + 1;
     }
-    const int lat_cap = nl + ((p.mode == PL_VERIFY) ? (cd.lat_off[s + 1] - cd.lat_off[s]) : 0);
+    const int lat_cap = nl + ((p.mode == PL_VERIFY && lat_off) ? (lat_off[s + 1] - lat_off[s]) : 0);
     if (pos < 0 || pos >= p.max_ctx || lat < 0 || lat >= lat_cap || lat >= p.max_lat || byte < 0 || byte > p.mask_id) {
       set_status(sd.status, kErrDevice);
       pos = min(max(pos, 0), p.max_ctx - 1);
@@ -650,8 +710,7 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
     rd.nkeys[r] = nkeys;
     if (blk_i >= 0) sd.blk_row[s * kMaxBlock + blk_i] = r;
   }
-  // attention groups
-  for (int gi = tid; gi < gcnt[B]; gi += blockDim.x) {
+  for (int gi = tid; gi < gcnt[B]; gi += nthr) {
     int lo = 0, hi = B;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -659,19 +718,19 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
       else hi = mid;
     }
     const int s = lo, j = gi - gcnt[s];
-    const int r0 = cnt[s] + 32 * j;
-    const int n = min(32, cnt[s + 1] - r0);
+    const int r0 = cnt[s] + kAttnRows * j;
     rd.g_seq[gi] = s;
     rd.g_row0[gi] = r0;
-    rd.g_nrows[gi] = n;
+    rd.g_nrows[gi] = min(kAttnRows, cnt[s + 1] - r0);
   }
-  __syncthreads();
-  for (int gi = tid; gi < gcnt[B]; gi += blockDim.x) {
+  sync();
+  for (int gi = tid; gi < gcnt[B]; gi += nthr) {
     int km = 0;
     for (int r = rd.g_row0[gi]; r < rd.g_row0[gi] + rd.g_nrows[gi]; ++r) km = max(km, rd.nkeys[r]);
     rd.g_kmax[gi] = km;
+    rd.g_fresh[gi] = rd.pos[cnt[rd.g_seq[gi]]];  // positions this pass writes start at the sequence's first row
   }
-  __syncthreads();
+  sync();
   if (tid == 0) {
     if (p.mode == PL_FIRST) {
       for (int s = 0; s < B; ++s) {
@@ -685,11 +744,9 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
       }
     }
     if (n_rows > 0) {
-      // algorithmic K/V bytes: each sequence's keys are read once per layer
-      unsigned long long kvk = 0;
+      unsigned long long kvk = 0;  // algorithmic K/V bytes: each sequence's keys read once per layer
       for (int gi = 0; gi < gcnt[B]; ++gi) {
-        const bool first = gi == 0 || rd.g_seq[gi - 1] != rd.g_seq[gi];
-        if (first) {
+        if (gi == 0 || rd.g_seq[gi - 1] != rd.g_seq[gi]) {
           int km = 0;
           for (int gj = gi; gj < gcnt[B] && rd.g_seq[gj] == rd.g_seq[gi]; ++gj) km = max(km, rd.g_kmax[gj]);
           kvk += km;
@@ -705,6 +762,12 @@ __global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd
       sd.counters[6] += kvk * p.kv_bytes_per_key;
     }
   }
+  sync();
+}
+
+__global__ void __launch_bounds__(256) k_plan(PlanArgs p, CallDesc cd, SeqDev sd, RowsDev rd) {
+  __shared__ int sh[3 * (kMaxCallBatch + 1)];
+  plan_rows(p, cd.batch, cd.row_off, cd.lat_off, sd, rd, threadIdx.x, blockDim.x, sh, [] { __syncthreads(); });
 }
 
 // Latent rows: new latent j of sequence s goes to slot n_lat[s] + (j - lat_off[s]).
@@ -731,26 +794,24 @@ __global__ void k_lat_plan(CallDesc cd, SeqDev sd, int* lat_seq, int* lat_slot, 
   }
 }
 
-// ------------------------------------------------------------------------ bookkeeping
-// Confidence unmasking of every active block ("블록 언마스킹 전략").  One warp per
-// sequence, lane = block position.
-__global__ void k_unmask(SeqDev sd, int batch, int k, float alpha, int step, const float* conf, const int* pred,
-                         const float* logits, float* out_logits) {
-  const int s = blockIdx.x, lane = threadIdx.x;
-  if (s >= batch || !sd.active[s]) return;
+// ------------------------------------------------------------------------ bookkeeping (one warp per sequence)
+// Confidence unmasking ("블록 언마스킹 전략"): every masked position with
+// conf >= alpha is committed; if none, the most confident one (lowest position
+// on ties).  Returns whether masked positions remain.
+__device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, float alpha, int step, const float* conf,
+                                           const int* pred, const float* logits, float* out_logits, int lane) {
   if (step == 0 && lane == 0) {
     const int lr = sd.last_row[s];
-    if (lr >= 0) sd.y_last[s] = pred[lr];
+    if (lr >= 0) sd.y_last[s] = __ldcg(pred + lr);
   }
   const bool in = lane < k;
   const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
   const bool m = in && sd.masked[s * kMaxBlock + lane];
-  const float c = m ? conf[row] : -1.0f;
+  const float c = m ? __ldcg(conf + row) : -1.0f;
   const bool over = m && (c >= alpha);
   const unsigned any_over = __ballot_sync(0xffffffffu, over);
   bool commit = over;
   if (!any_over) {
-    // most confident masked position, lowest position on ties
     float best = c;
     int bi = m ? lane : 1 << 30;
 #pragma unroll
@@ -765,22 +826,85 @@ __global__ void k_unmask(SeqDev sd, int batch, int k, float alpha, int step, con
     commit = m && lane == bi;
   }
   if (commit) {
-    sd.blk[s * kMaxBlock + lane] = (unsigned char)pred[row];
+    sd.blk[s * kMaxBlock + lane] = (unsigned char)__ldcg(pred + row);
     sd.masked[s * kMaxBlock + lane] = 0;
   }
   const unsigned left = __ballot_sync(0xffffffffu, m && !commit);
   if (out_logits && in) {
     float* dst = out_logits + (((size_t)step * batch + s) * k + lane) * 256;
     const float* src = logits + (size_t)row * 256;
-    for (int j = 0; j < 256; ++j) dst[j] = src[j];
+    for (int j = 0; j < 256; ++j) dst[j] = __ldcg(src + j);
   }
   if (lane == 0) {
     sd.steps[s] += 1;
     sd.active[s] = left != 0;
   }
+  return left != 0;
 }
 
-// After the block loop: copy blocks out; masked positions left -> STEP_LIMIT.
+__global__ void k_unmask(SeqDev sd, int batch, int k, float alpha, int step, const float* conf, const int* pred,
+                         const float* logits, float* out_logits) {
+  const int s = blockIdx.x, lane = threadIdx.x;
+  if (s >= batch || !sd.active[s]) return;
+  unmask_seq(sd, s, batch, k, alpha, step, conf, pred, logits, out_logits, lane);
+}
+
+// AR draft: the argmax of this pass's row becomes draft byte `step`.
+__device__ __forceinline__ void draft_ar_seq(SeqDev sd, int s, int batch, int step, const int* pred, const float* logits,
+                                             float* out_logits, int lane) {
+  const int row = (step == 0) ? sd.last_row[s] : sd.blk_row[s * kMaxBlock];
+  if (lane == 0) {
+    const int b = __ldcg(pred + row);
+    sd.blk[s * kMaxBlock + step] = (unsigned char)b;
+    if (step == 0) sd.y_last[s] = b;
+  }
+  if (out_logits) {
+    float* dst = out_logits + ((size_t)step * batch + s) * 256;
+    for (int j = lane; j < 256; j += 32) dst[j] = __ldcg(logits + (size_t)row * 256 + j);
+  }
+}
+
+__global__ void k_draft_ar(SeqDev sd, int batch, int step, const int* pred, const float* logits, float* out_logits) {
+  const int s = blockIdx.x;
+  if (s < batch) draft_ar_seq(sd, s, batch, step, pred, logits, out_logits, threadIdx.x);
+}
+
+// Greedy verification ("BLT-S와 BLT-DV"): with y_slot[i] the greedy byte for
+// draft slot i (slot 0: prediction of the last committed row; slot i > 0: of
+// draft row i-1), accept while draft[i] == y_slot[i]; the next byte is
+// y_slot[a], or the prediction of the last draft row when all k match.
+__device__ __forceinline__ void accept_seq(SeqDev sd, int s, int k, const int* pred, const int* vlat, const float* logits,
+                                           int* out_acc, unsigned char* out_next, float* out_logits, int lane) {
+  const bool in = lane < k;
+  const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
+  const int y_self = in ? __ldcg(pred + row) : -1;
+  const int y_up = __shfl_up_sync(0xffffffffu, y_self, 1);
+  const int y_slot = (lane == 0) ? sd.y_last[s] : y_up;
+  const bool match = in && (int)sd.blk[s * kMaxBlock + lane] == y_slot;
+  const unsigned mm = __ballot_sync(0xffffffffu, !match);
+  const int a = (mm == 0u) ? k : min(__ffs(mm) - 1, k);
+  const int y_a = __shfl_sync(0xffffffffu, y_slot, a & 31);
+  const int y_k = __shfl_sync(0xffffffffu, y_self, (k - 1) & 31);
+  if (out_logits && in) {
+    float* dst = out_logits + ((size_t)s * k + lane) * 256;
+    for (int j = 0; j < 256; ++j) dst[j] = __ldcg(logits + (size_t)row * 256 + j);
+  }
+  if (lane == 0) {
+    const int nxt = (a == k) ? y_k : y_a;
+    out_acc[s] = a;
+    out_next[s] = (unsigned char)nxt;
+    sd.kv_len[s] += a;
+    if (a >= 1) sd.n_lat[s] = max(sd.n_lat[s], vlat[s * k + a - 1] + 1);
+  }
+}
+
+__global__ void k_accept(SeqDev sd, int batch, int k, const int* pred, const int* vlat, const float* logits, int* out_acc,
+                         unsigned char* out_next, float* out_logits) {
+  const int s = blockIdx.x;
+  if (s < batch) accept_seq(sd, s, k, pred, vlat, logits, out_acc, out_next, out_logits, threadIdx.x);
+}
+
+// After a block loop: copy blocks out; masked positions left -> STEP_LIMIT.
 __global__ void k_finish_block(SeqDev sd, int batch, int k, unsigned char* out_block, int* out_steps) {
   const int s = blockIdx.x, lane = threadIdx.x;
   if (s >= batch) return;
@@ -791,54 +915,9 @@ __global__ void k_finish_block(SeqDev sd, int batch, int k, unsigned char* out_b
   }
 }
 
-// AR draft: the argmax of this pass's row becomes draft byte `step`.
-__global__ void k_draft_ar(SeqDev sd, int batch, int k, int step, const int* pred, const float* logits, float* out_logits) {
-  const int s = blockIdx.x * blockDim.x + threadIdx.x;
-  if (s >= batch) return;
-  const int row = (step == 0) ? sd.last_row[s] : sd.blk_row[s * kMaxBlock];
-  const int b = pred[row];
-  sd.blk[s * kMaxBlock + step] = (unsigned char)b;
-  if (step == 0) sd.y_last[s] = b;
-  if (out_logits) {
-    float* dst = out_logits + ((size_t)step * batch + s) * 256;
-    for (int j = 0; j < 256; ++j) dst[j] = logits[(size_t)row * 256 + j];
-  }
-}
-
 __global__ void k_copy_draft(SeqDev sd, int batch, int k, unsigned char* out) {
   const int s = blockIdx.x, lane = threadIdx.x;
   if (s < batch && lane < k) out[s * k + lane] = sd.blk[s * kMaxBlock + lane];
-}
-
-// Greedy verification ("BLT-S와 BLT-DV"): with y_slot[i] the greedy byte for
-// draft slot i (slot 0: prediction of the last committed row; slot i > 0: of
-// draft row i-1), accept while draft[i] == y_slot[i]; the next byte is
-// y_slot[a], or the prediction of the last draft row when all k match.
-__global__ void k_accept(SeqDev sd, int batch, int k, const int* pred, const int* vlat, const float* logits, int* out_acc,
-                         unsigned char* out_next, float* out_logits) {
-  const int s = blockIdx.x, lane = threadIdx.x;
-  if (s >= batch) return;
-  const bool in = lane < k;
-  const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
-  const int y_self = in ? pred[row] : -1;
-  const int y_up = __shfl_up_sync(0xffffffffu, y_self, 1);
-  const int y_slot = (lane == 0) ? sd.y_last[s] : y_up;
-  const bool match = in && (int)sd.blk[s * kMaxBlock + lane] == y_slot;
-  const unsigned mm = __ballot_sync(0xffffffffu, !match);
-  const int a = (mm == 0u) ? k : min(__ffs(mm) - 1, k);
-  const int y_a = __shfl_sync(0xffffffffu, y_slot, a & 31);
-  const int y_k = __shfl_sync(0xffffffffu, y_self, (k - 1) & 31);
-  if (out_logits && in) {
-    float* dst = out_logits + ((size_t)s * k + lane) * 256;
-    for (int j = 0; j < 256; ++j) dst[j] = logits[(size_t)row * 256 + j];
-  }
-  if (lane == 0) {
-    const int nxt = (a == k) ? y_k : y_a;
-    out_acc[s] = a;
-    out_next[s] = (unsigned char)nxt;
-    sd.kv_len[s] += a;
-    if (a >= 1) sd.n_lat[s] = max(sd.n_lat[s], vlat[s * k + a - 1] + 1);
-  }
 }
 
 // Page table updates (entries by value).
@@ -852,7 +931,7 @@ __global__ void k_page_update(int* pt, PageUpd u) {
   if (i < u.n) pt[u.idx[i]] = u.page[i];
 }
 
-// Set per-sequence lengths (rewind).
+// Shrink per-sequence lengths (rewind).
 __global__ void k_rewind(SeqDev sd, CallDesc cd) {
   const int s = threadIdx.x;
   if (s < cd.batch) {

@@ -1,0 +1,680 @@
+// Persistent decoder-pass kernel: every pass of one C-ABI call (the confidence
+// unmasking loop of BLT-D, the k passes of a BLT-S draft, the BLT-DV draft
+// loop, or the verification pass) in one cooperative launch, one CTA per SM.
+//
+// Warp roles: warps 0..7 consume (tensor-core GEMV, attention, bookkeeping),
+// warp 8 produces: it streams this CTA's weight tiles for the whole pass
+// through a shared-memory ring with 1-D bulk TMA copies, so HBM keeps
+// streaming while consumers wait on data dependencies.
+//
+// Work: each projection is cut into units of 16 output rows (a tile row of
+// the fragment-ordered weights).  The units of all phases of a pass
+// (QKV, O, W13, W2 per layer, then the byte head) are dealt round-robin to
+// the CTAs, continuing across phases, so every CTA streams about the same
+// number of bytes at every point of the pass.
+//
+// Dependencies are per-unit epoch flags in global memory (release store by
+// the producing CTA, acquire poll by the consumer), not grid barriers: a
+// QKV k-step waits only for the W2 unit that wrote its 16 input columns,
+// an O-projection k-step for the attention head it reads, and so on.  Every
+// wait is bounded; a wait that runs out sets the abort word and the status,
+// and all CTAs leave.  The arithmetic of every unit, attention chunk,
+// combine and bookkeeping step is the device code the per-phase kernels use,
+// so both paths give bit-identical results.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace bltdec {
+
+constexpr int kMegaConsumers = 8;
+constexpr int kMegaThreads = (kMegaConsumers + 1) * 32;
+constexpr int kStageTiles = 32;                 // k16 tiles of one unit per ring slot
+constexpr int kRingBytes = 128 * 1024;          // weight ring
+constexpr int kMegaMaxNG = 2;                   // <= 16 rows per pass
+constexpr unsigned kSpinLimit = 1u << 26;       // polls before a wait gives up
+
+enum MegaMode : int { MM_DIFFUSE = 0, MM_DRAFT_AR = 1, MM_VERIFY = 2 };
+
+struct LayerW {
+  const uint4* qkv;
+  const uint4* o;
+  const uint4* w13;
+  const uint4* w2;
+  const float* attn_norm;
+  const float* ffn_norm;
+};
+
+struct MegaArgs {
+  const LayerW* layers;  // device [L]
+  const uint4* whead;
+  const float* final_norm;
+  int L, d, H, dh, F, planes;
+  float eps;
+  GemmArgs ga;  // epilogue context: pointers shared by all phases
+  AttnArgs aa;
+  RowsDev rows;
+  SeqDev sd;
+  float* h;
+  float* q;
+  float* att;
+  float* act;
+  float* logits;
+  float* conf;
+  int* pred;
+  float* gap;
+  unsigned* flags;  // epoch flags, see flag offsets below
+  int f_qkv, f_o, f_w13, f_w2, f_head, f_att, f_dec;
+  unsigned* attn_cnt;  // [max_groups][H] arrival counters
+  unsigned* dec_val;   // continue word written with the decision flag
+  unsigned epoch0;
+  int* abort;
+  int mode, batch, k, max_passes;
+  float alpha;
+  const int* vlat;
+  float* out_logits;
+  int* out_acc;
+  unsigned char* out_next;
+  PlanArgs plan;  // template for the device-side plans of passes >= 2
+};
+
+// ---------------------------------------------------------------------------- sync primitives
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void tma_1d(void* dst, const void* src, unsigned bytes, uint64_t* b) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(b))
+               : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+
+// Bounded waits.  Return false when the wait gave up (abort raised).
+__device__ __forceinline__ bool wait_flag(const MegaArgs& m, const unsigned* f, unsigned target) {
+  unsigned n = 0;
+  while ((int)(ld_acquire(f) - target) < 0) {
+    if (++n > 64) __nanosleep(64);
+    if ((n & 1023) == 0 && *(volatile int*)m.abort) return false;
+    if (n > kSpinLimit) {
+      atomicExch(m.abort, 1);
+      set_status(m.sd.status, kErrDevice);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ bool wait_mbar(const MegaArgs& m, uint64_t* b, unsigned parity) {
+  unsigned n = 0;
+  while (!mbar_try(b, parity)) {
+    if ((++n & 1023) == 0 && *(volatile int*)m.abort) return false;
+    if (n > kSpinLimit) {
+      atomicExch(m.abort, 1);
+      set_status(m.sd.status, kErrDevice);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------- schedule
+enum PhaseKind : int { PH_QKV = 0, PH_O = 1, PH_W13 = 2, PH_W2 = 3, PH_HEAD = 4 };
+
+struct Phase {
+  int kind, layer, units, ksteps, base;
+  const uint4* w;
+};
+
+// Phase ph of a pass: ph = 4*l + {0: QKV, 1: O, 2: W13, 3: W2}; ph = 4L: head.
+__device__ __forceinline__ Phase phase_of(const MegaArgs& m, int ph) {
+  Phase p;
+  const int L = m.L, d = m.d, F = m.F;
+  const int per_layer = 3 * d / 16 + d / 16 + 2 * F / 16 + d / 16;
+  p.layer = ph / 4;
+  p.base = p.layer * per_layer;
+  if (ph >= 4 * L) {
+    p.kind = PH_HEAD;
+    p.layer = L;
+    p.units = 256 / 16;
+    p.ksteps = d / 16;
+    p.base = L * per_layer;
+    p.w = m.whead;
+    return p;
+  }
+  const LayerW lw = m.layers[p.layer];
+  p.kind = ph % 4;
+  switch (p.kind) {
+    case PH_QKV:
+      p.units = 3 * d / 16, p.ksteps = d / 16, p.w = lw.qkv;
+      break;
+    case PH_O:
+      p.base += 3 * d / 16, p.units = d / 16, p.ksteps = d / 16, p.w = lw.o;
+      break;
+    case PH_W13:
+      p.base += 4 * d / 16, p.units = 2 * F / 16, p.ksteps = d / 16, p.w = lw.w13;
+      break;
+    default:
+      p.base += 4 * d / 16 + 2 * F / 16, p.units = d / 16, p.ksteps = F / 16, p.w = lw.w2;
+      break;
+  }
+  return p;
+}
+
+__device__ __forceinline__ int first_unit(const Phase& p, int cta, int G) {
+  return ((cta - p.base) % G + G) % G;
+}
+
+__device__ __forceinline__ unsigned epoch(const MegaArgs& m, int pass, int layer) {
+  return m.epoch0 + (unsigned)(pass * (m.L + 1) + layer + 1);
+}
+
+// ---------------------------------------------------------------------------- producer
+__device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* full, uint64_t* empty, int S, int lane) {
+  const int G = gridDim.x, cta = blockIdx.x;
+  const unsigned tile_bytes = 512u * m.planes;
+  unsigned it = 0;
+  bool ok = true;
+  for (int pass = 0; pass < m.max_passes && ok; ++pass) {
+    if (pass > 0) {
+      unsigned go = 0;
+      if (lane == 0) {
+        ok = wait_flag(m, m.flags + m.f_dec, epoch(m, pass - 1, m.L));
+        go = ok ? __ldcg(m.dec_val) : 0u;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!ok || go == 0u) break;
+    }
+    for (int ph = 0; ph <= 4 * m.L && ok; ++ph) {
+      const Phase p = phase_of(m, ph);
+      const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+      for (int u = first_unit(p, cta, G); u < p.units && ok; u += G) {
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(p.w) + (size_t)u * p.ksteps * tile_bytes;
+        for (int st = 0; st < nst; ++st, ++it) {
+          const int slot = it % S;
+          const unsigned tiles = min(kStageTiles, p.ksteps - st * kStageTiles);
+          if (lane == 0) {
+            ok = wait_mbar(m, empty + slot, ((it / S) & 1) ^ 1);
+            if (ok) {
+              mbar_expect_tx(full + slot, tiles * tile_bytes);
+              tma_1d(ring + (size_t)slot * kStageTiles * tile_bytes, src + (size_t)st * kStageTiles * tile_bytes, tiles * tile_bytes,
+                     full + slot);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+      }
+    }
+  }
+  // leave no copy in flight: every issued stage must have landed
+  if (lane == 0) {
+    const unsigned issued = it;
+    const unsigned from = issued > (unsigned)S ? issued - S : 0;
+    for (unsigned j = from; j < issued; ++j) {
+      unsigned n = 0;
+      while (!mbar_try(full + j % S, (j / S) & 1) && ++n < kSpinLimit) {
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------- consumer helpers
+struct MegaSmem {
+  unsigned char* ring;
+  uint64_t* full;
+  uint64_t* empty;
+  int S;
+  float* red;  // [8][16][16]
+  float* ssr;  // [8][16]
+  float* qs;
+  float* ps;
+  void* ks;
+  void* vs;
+  float* mrow;
+  float* lrow;
+  int* lim;
+  int* plan_sh;
+  int* misc;  // [0]: last-arrival flag, [1]: any-active
+};
+
+// Input value of row `row`, column k for a phase (before the gain).
+__device__ __forceinline__ float2 x_pair(const MegaArgs& m, const Phase& p, int row, int k) {
+  if (p.kind == PH_QKV) {
+    const int d = m.d;
+    const float* src = (p.layer == 0) ? m.ga.embed + (size_t)__ldcg(m.rows.byte + row) * d : m.h + (size_t)row * d;
+    const float* c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, p.layer, d, __ldcg(m.rows.seq + row), __ldcg(m.rows.lat + row));
+    const float2 a = __ldcg(reinterpret_cast<const float2*>(src + k));
+    const float2 b = __ldcg(reinterpret_cast<const float2*>(c + k));
+    return make_float2(a.x + b.x, a.y + b.y);
+  }
+  if (p.kind == PH_O) return __ldcg(reinterpret_cast<const float2*>(m.att + (size_t)row * m.d + k));
+  if (p.kind == PH_W2) return __ldcg(reinterpret_cast<const float2*>(m.act + (size_t)row * m.F + k));
+  return __ldcg(reinterpret_cast<const float2*>(m.h + (size_t)row * m.d + k));  // W13, head
+}
+
+// Wait until the inputs of k-step s of phase p (this pass) are written.
+__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s, int n_groups) {
+  const unsigned* f = m.flags;
+  if (p.kind == PH_QKV) {
+    if (p.layer == 0) return true;
+    return wait_flag(m, f + m.f_w2 + s, epoch(m, pass, p.layer - 1));
+  }
+  if (p.kind == PH_O) {
+    const int head = s * 16 / m.dh;
+    for (int g = 0; g < n_groups; ++g)
+      if (!wait_flag(m, f + m.f_att + g * m.H + head, epoch(m, pass, p.layer))) return false;
+    return true;
+  }
+  if (p.kind == PH_W13) return wait_flag(m, f + m.f_o + s, epoch(m, pass, p.layer));
+  if (p.kind == PH_W2)
+    return wait_flag(m, f + m.f_w13 + 2 * s, epoch(m, pass, p.layer)) && wait_flag(m, f + m.f_w13 + 2 * s + 1, epoch(m, pass, p.layer));
+  return wait_flag(m, f + m.f_w2 + s, epoch(m, pass, m.L - 1));  // head
+}
+
+__device__ __forceinline__ const float* phase_gain(const MegaArgs& m, const Phase& p) {
+  if (p.kind == PH_QKV) return m.layers[p.layer].attn_norm;
+  if (p.kind == PH_W13) return m.layers[p.layer].ffn_norm;
+  if (p.kind == PH_HEAD) return m.final_norm;
+  return nullptr;
+}
+
+template <int EPI>
+__device__ __forceinline__ void unit_epilogue(const MegaArgs& m, const Phase& p, const GemmArgs& ga, int u, int r16, int row,
+                                              float v0, float v1) {
+  gemm_epilogue<EPI>(ga, u, r16, row, v0, v1);
+}
+
+// Cached-input phase (K <= 1024: each warp owns <= 8 k-steps): the warp's
+// input fragments are built once and reused for every unit of the phase.
+template <int NG, int PL, int EPI>
+__device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
+                                 int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int u0 = first_unit(p, cta, G);
+  if (u0 >= p.units) return true;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const float* gain = phase_gain(m, p);
+  const bool norm = gain != nullptr;
+  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps of this warp (<= 8)
+  // dependency waits for this warp's k-steps
+  bool ok = true;
+  if (lane == 0) {
+    for (int j = 0; j < nkw && ok; ++j) ok = wait_inputs(m, p, pass, warp + 8 * j, n_groups);
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  XFrag xf[8][NG];
+  float ss[NG];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) ss[n] = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < nkw) {
+      const int k0 = (warp + 8 * j) * 16 + 2 * t;
+      float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
+      if (norm) {
+        g0 = __ldg(gain + k0);
+        g1 = __ldg(gain + k0 + 1);
+        g8 = __ldg(gain + k0 + 8);
+        g9 = __ldg(gain + k0 + 9);
+      }
+#pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        const int row = n * 8 + g;
+        float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+        if (ok && row < nr) {
+          a = x_pair(m, p, row, k0);
+          b = x_pair(m, p, row, k0 + 8);
+        }
+        if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
+        xf[j][n] = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
+      }
+    }
+  }
+  const unsigned tile_bytes = 512u * PL;
+  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // <= 2
+  for (int u = u0; u < p.units; u += G) {
+    float acc[NG][4];
+#pragma unroll
+    for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      if (st < nst) {
+        const int slot = it % sm.S;
+        if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
+        const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int tile = 8 * jj + warp;  // within the stage
+          const int ks = st * kStageTiles + tile;
+          if (ks < p.ksteps) {
+            uint4 w[PL];
+#pragma unroll
+            for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, xf[st * 4 + jj][n]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.empty + slot);
+        ++it;
+      }
+    }
+    tile_reduce<NG>(acc, ss, norm, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
+                    [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(ga, u, r16, col, v0, v1); });
+    consumer_sync();
+    if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
+  }
+  return ok;
+}
+
+// Streamed-input phase (W2, K = F > 1024): inputs loaded stage by stage, one
+// stage ahead.
+template <int NG, int PL>
+__device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
+                                   int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int u0 = first_unit(p, cta, G);
+  if (u0 >= p.units) return true;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const unsigned tile_bytes = 512u * PL;
+  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+  bool ok = true;
+  auto load = [&](int st, float2 (&xa)[4][NG], float2 (&xb)[4][NG]) {
+    bool good = true;
+    if (lane == 0) {
+      for (int jj = 0; jj < 4 && good; ++jj) {
+        const int ks = st * kStageTiles + 8 * jj + warp;
+        if (ks < p.ksteps) good = wait_inputs(m, p, pass, ks, n_groups);
+      }
+    }
+    good = __shfl_sync(0xffffffffu, good, 0);
+    __syncwarp();
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int ks = st * kStageTiles + 8 * jj + warp;
+#pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        const int row = n * 8 + g;
+        xa[jj][n] = xb[jj][n] = make_float2(0.f, 0.f);
+        if (good && ks < p.ksteps && row < nr) {
+          xa[jj][n] = x_pair(m, p, row, ks * 16 + 2 * t);
+          xb[jj][n] = x_pair(m, p, row, ks * 16 + 2 * t + 8);
+        }
+      }
+    }
+    return good;
+  };
+  for (int u = u0; u < p.units; u += G) {
+    float acc[NG][4], ss[NG];
+#pragma unroll
+    for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
+    float2 ca[4][NG], cb[4][NG], na[4][NG], nb[4][NG];
+    ok = load(0, ca, cb) && ok;
+    for (int st = 0; st < nst; ++st) {
+      if (st + 1 < nst) ok = load(st + 1, na, nb) && ok;
+      const int slot = it % sm.S;
+      if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
+      const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int tile = 8 * jj + warp;
+        const int ks = st * kStageTiles + tile;
+        if (ks < p.ksteps) {
+          uint4 w[PL];
+#pragma unroll
+          for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+          for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.empty + slot);
+      ++it;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          ca[jj][n] = na[jj][n];
+          cb[jj][n] = nb[jj][n];
+        }
+    }
+    tile_reduce<NG>(acc, ss, false, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
+                    [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI_RESID>(ga, u, r16, col, v0, v1); });
+    consumer_sync();
+    if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
+  }
+  return ok;
+}
+
+// Attention of layer l: items (group, head, chunk) dealt round-robin; the
+// last CTA to finish a (group, head) combines its chunks and raises the flag.
+template <int DH, typename KVT>
+__device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, int pass, int n_groups, int tid) {
+  const int G = gridDim.x, cta = blockIdx.x;
+  AttnArgs a = m.aa;
+  a.layer = layer;
+  const int tph = DH / 16;
+  const int tiles_sec = m.d / 16;
+  int total = 0;
+  for (int g = 0; g < n_groups; ++g) total += m.H * ((__ldcg(m.rows.g_kmax + g) + a.CH - 1) / a.CH);
+  bool ok = true;
+  KVT* ks = static_cast<KVT*>(sm.ks);
+  KVT* vs = static_cast<KVT*>(sm.vs);
+  for (int item = cta; item < total; item += G) {
+    int g = 0, rem = item, nch = 0;
+    for (; g < n_groups; ++g) {
+      nch = (__ldcg(m.rows.g_kmax + g) + a.CH - 1) / a.CH;
+      if (rem < m.H * nch) break;
+      rem -= m.H * nch;
+    }
+    const int h = rem / nch, c = rem % nch;
+    const int seq = __ldcg(m.rows.g_seq + g), kmax = __ldcg(m.rows.g_kmax + g), fresh = __ldcg(m.rows.g_fresh + g);
+    const int t0 = c * a.CH, t1 = min(t0 + a.CH, kmax);
+    // keys cached before this pass can be fetched before q/k/v of this pass exist
+    attn_load_kv<DH, KVT>(a, seq, h, t0, t0, min(t1, fresh), ks, vs, tid, 256);
+    cp_async_commit();
+    if (tid == 0) {
+      const unsigned e = epoch(m, pass, layer);
+      for (int sec = 0; sec < 3 && ok; ++sec)
+        for (int j = 0; j < tph && ok; ++j) ok = wait_flag(m, m.flags + m.f_qkv + sec * tiles_sec + h * tph + j, e);
+    }
+    consumer_sync();
+    attn_load_kv<DH, KVT>(a, seq, h, t0, max(t0, fresh), t1, ks, vs, tid, 256);
+    cp_async_commit();
+    cp_async_wait<0>();
+    consumer_sync();
+    attn_partial_compute<DH, KVT>(a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, tid, 256, consumer_sync);
+    consumer_sync();
+    if (tid == 0) {
+      __threadfence();
+      const unsigned old = atomicAdd(m.attn_cnt + g * m.H + h, 1u);
+      sm.misc[0] = (old == (unsigned)(nch - 1));
+      __threadfence();
+    }
+    consumer_sync();
+    if (sm.misc[0]) {
+      const int row0 = __ldcg(m.rows.g_row0 + g), nr = __ldcg(m.rows.g_nrows + g);
+      for (int i = tid; i < nr * DH; i += 256) attn_combine_one(a, row0 + i / DH, h, i % DH);
+      consumer_sync();
+      if (tid == 0) {
+        m.attn_cnt[g * m.H + h] = 0u;
+        st_release(m.flags + m.f_att + g * m.H + h, epoch(m, pass, layer));
+      }
+    }
+    consumer_sync();
+  }
+  return ok;
+}
+
+// After the head of pass `pass`: statistics, the mode's bookkeeping, the
+// decision to go on, the plan of the next pass (CTA 0 only).
+__device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass, int nr, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int u = 0; u < 16; ++u) wait_flag(m, m.flags + m.f_head + u, epoch(m, pass, m.L));
+    sm.misc[1] = 0;
+  }
+  consumer_sync();
+  for (int r = warp; r < nr; r += 8) {
+    float c, g;
+    int p;
+    head_stats_row(m.logits + (size_t)r * 256, lane, c, p, g);
+    if (lane == 0) {
+      m.conf[r] = c;
+      m.pred[r] = p;
+      m.gap[r] = g;
+    }
+  }
+  __threadfence_block();
+  consumer_sync();
+  int cont = 0;
+  if (m.mode == MM_DIFFUSE) {
+    for (int s = warp; s < m.batch; s += 8) {
+      if (m.sd.active[s]) {
+        const bool left = unmask_seq(m.sd, s, m.batch, m.k, m.alpha, pass, m.conf, m.pred, m.logits, m.out_logits, lane);
+        if (left && lane == 0) atomicOr(sm.misc + 1, 1);
+      }
+    }
+    consumer_sync();
+    cont = sm.misc[1] && pass + 1 < m.max_passes;
+  } else if (m.mode == MM_DRAFT_AR) {
+    for (int s = warp; s < m.batch; s += 8) draft_ar_seq(m.sd, s, m.batch, pass, m.pred, m.logits, m.out_logits, lane);
+    cont = pass + 1 < m.max_passes;
+  } else {
+    for (int s = warp; s < m.batch; s += 8)
+      accept_seq(m.sd, s, m.k, m.pred, m.vlat, m.logits, m.out_acc, m.out_next, m.out_logits, lane);
+  }
+  __threadfence_block();
+  consumer_sync();
+  if (cont) {
+    PlanArgs p = m.plan;
+    if (m.mode == MM_DIFFUSE) {
+      p.mode = PL_BLOCK;
+    } else {
+      p.mode = PL_ARDRAFT;
+      p.step = pass + 1;
+    }
+    plan_rows(p, m.batch, nullptr, nullptr, m.sd, m.rows, tid, 256, sm.plan_sh, consumer_sync);
+  }
+  consumer_sync();
+  if (tid == 0) {
+    *(volatile unsigned*)m.dec_val = cont ? 1u : 0u;
+    __threadfence();
+    st_release(m.flags + m.f_dec, epoch(m, pass, m.L));
+  }
+}
+
+template <int NG, int PL, int DH, typename KVT>
+__global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
+  extern __shared__ __align__(1024) unsigned char mega_smem[];
+  __shared__ uint64_t bars[2 * 16];
+  __shared__ int plan_sh[3 * (kMaxCallBatch + 1)];
+  __shared__ int misc[4];
+  __shared__ float mrow[kAttnRows], lrow[kAttnRows];
+  __shared__ int lim[kAttnRows];
+
+  const unsigned tile_bytes = 512u * PL;
+  const unsigned slot_bytes = kStageTiles * tile_bytes;
+  MegaSmem sm;
+  sm.S = min(16, (int)(kRingBytes / slot_bytes));
+  sm.ring = mega_smem;
+  unsigned char* p = mega_smem + kRingBytes;
+  sm.red = reinterpret_cast<float*>(p);
+  p += 8 * 16 * 8 * kMegaMaxNG * 4;
+  sm.ssr = reinterpret_cast<float*>(p);
+  p += 8 * 8 * kMegaMaxNG * 4;
+  sm.qs = reinterpret_cast<float*>(p);
+  p += kAttnRows * DH * 4;
+  sm.ps = reinterpret_cast<float*>(p);
+  p += kAttnRows * m.aa.CH * 4;
+  sm.ks = p;
+  p += m.aa.CH * DH * sizeof(KVT);
+  sm.vs = p;
+  sm.full = bars;
+  sm.empty = bars + 16;
+  sm.mrow = mrow;
+  sm.lrow = lrow;
+  sm.lim = lim;
+  sm.plan_sh = plan_sh;
+  sm.misc = misc;
+
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int i = 0; i < sm.S; ++i) {
+      mbar_init(sm.full + i, 1);
+      mbar_init(sm.empty + i, kMegaConsumers);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  if (tid >= 256) {  // producer warp
+    mega_producer(m, sm.ring, sm.full, sm.empty, sm.S, tid & 31);
+    return;
+  }
+  unsigned it = 0;
+  bool ok = true;
+  for (int pass = 0; pass < m.max_passes && ok; ++pass) {
+    if (pass > 0) {
+      if (tid == 0) misc[2] = wait_flag(m, m.flags + m.f_dec, epoch(m, pass - 1, m.L)) ? (int)__ldcg(m.dec_val) : -1;
+      consumer_sync();
+      const int go = misc[2];
+      consumer_sync();
+      if (go <= 0) {
+        ok = go == 0;
+        break;
+      }
+    }
+    const int nr = __ldcg(m.rows.n_rows);
+    const int n_groups = __ldcg(m.rows.n_groups);
+    for (int l = 0; l < m.L && ok; ++l) {
+      GemmArgs ga = m.ga;
+      ga.layer = l;
+      ok = run_phase_cached<NG, PL, EPI_QKV>(m, sm, phase_of(m, 4 * l), pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
+      ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
+      ga.out = m.h;
+      ga.ldo = m.d;
+      ok = run_phase_cached<NG, PL, EPI_XRESID>(m, sm, phase_of(m, 4 * l + 1), pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
+      ga.out = m.act;
+      ga.ldo = m.F;
+      ok = run_phase_cached<NG, PL, EPI_SWIGLU>(m, sm, phase_of(m, 4 * l + 2), pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
+      ga.out = m.h;
+      ga.ldo = m.d;
+      const Phase p2 = phase_of(m, 4 * l + 3);
+      if (p2.ksteps <= 64) ok = run_phase_cached<NG, PL, EPI_RESID>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
+      else ok = run_phase_streamed<NG, PL>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
+    }
+    if (!ok) break;
+    GemmArgs ga = m.ga;
+    ga.out = m.logits;
+    ga.ldo = 256;
+    ok = run_phase_cached<NG, PL, EPI_STORE>(m, sm, phase_of(m, 4 * m.L), pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
+    if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
+  }
+}
+
+}  // namespace bltdec

@@ -96,7 +96,8 @@ typedef struct {
   int32_t flags;        /* BLT_FLAG_* */
 } blt_dec_config;
 
-#define BLT_FLAG_TIME_PASSES 1 /* bracket every decoder pass with CUDA events (counters.pass_ns) */
+#define BLT_FLAG_TIME_PASSES 1 /* bracket the decoder passes of every call with CUDA events (counters.pass_ns) */
+#define BLT_FLAG_PER_PHASE 2   /* never use the persistent pass kernel (one launch per phase instead) */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */
@@ -127,8 +128,8 @@ typedef struct {
   uint64_t weight_bytes;   /* weight bytes streamed by decoder passes (algorithmic) */
   uint64_t kv_read_bytes;  /* K/V bytes read by self-attention (algorithmic) */
   uint64_t kernel_launches; /* engine kernels launched (host count) */
-  uint64_t timed_passes;   /* passes bracketed by events (BLT_FLAG_TIME_PASSES) */
-  uint64_t pass_ns;        /* their summed device time, ns */
+  uint64_t timed_passes;   /* decoder passes inside timed calls (BLT_FLAG_TIME_PASSES) */
+  uint64_t pass_ns;        /* summed device time of those calls' passes, ns (latent projection excluded) */
 } blt_dec_counters;
 
 /* Create an engine.  Copies and re-lays out the weights on the device

@@ -171,3 +171,67 @@ def test_d4_b1_first_block_logits_and_bytes(d4_setup):
     want = o.generate(G, rec)
     _compare_bytes(res.out[0], o, want, wl.prefix_len, "d4_b1")
     assert [int(r["steps"][0]) for r in res.rounds] == [r["steps"] for r in rec][: len(res.rounds)] or res.out[0] != want
+
+
+def _call_logits(wl, ws, per_phase, mode, k, alpha, G=24, batch=2):
+    """Logits of every engine call of a short generation (diffuse / draft / verify), via out_logits."""
+    import ctypes
+
+    from block_diffusion_byte_b200 import binding as B
+    from block_diffusion_byte_b200.driver import Engine, generate
+
+    eng = Engine(wl.shape, ws, max_batch=batch, max_ctx=wl.prefix_len + G + 64, max_block=16, max_rows=256, per_phase=per_phase)
+    try:
+        w = replace(wl, mode=mode, block=k, alpha=alpha)
+        res = generate(eng, w, [_prefix(wl, s) for s in range(batch)], G, record=True)
+        st = B.blt_dec_stats(eng.h)
+    finally:
+        eng.close()
+    return res, st
+
+
+@pytest.mark.parametrize("mode,k,alpha,batch", [("D", 4, 0.7, 2), ("D", 8, 0.5, 1), ("AR", 1, 0.0, 2), ("S", 6, 0.0, 2), ("DV", 4, 0.0, 2)])
+def test_persistent_kernel_matches_per_phase_bitwise(tiny_setup, mode, k, alpha, batch):
+    """The persistent pass kernel and the per-phase kernels share every arithmetic step
+    (every pass of these calls has at most 16 rows, so the persistent kernel runs them)."""
+    wl, ws, om = tiny_setup
+    a, sa = _call_logits(wl, ws, False, mode, k, alpha, batch=batch)
+    b, sb = _call_logits(wl, ws, True, mode, k, alpha, batch=batch)
+    assert a.out == b.out
+    assert sa["passes"] == sb["passes"]
+    assert sa["kernel_launches"] < sb["kernel_launches"]  # the persistent path ran
+    for ra, rb in zip(a.rounds, b.rounds):
+        for key in ra:
+            assert np.array_equal(ra[key], rb[key]), key
+
+
+def _block_logits(wl, ws, per_phase, k=4, alpha=0.7):
+    from block_diffusion_byte_b200 import binding as B
+    from block_diffusion_byte_b200.driver import Engine, SeqHost
+    from workload import Patcher
+
+    pre = _prefix(wl, 0)
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 64, max_block=16, max_rows=1024, per_phase=per_phase)
+    try:
+        s = SeqHost(Patcher(wl.patch_kind, wl.seed, wl.cfg_index, 0), wl.seed, wl.cfg_index, 0, wl.shape.d_global)
+        s.commit(pre)
+        b, sl, l = s.take_pending()
+        r, keep = eng.rows([b[:-1]], [sl[:-1]], [l])
+        B.blt_dec_prefill(eng.h, 1, r)
+        r, keep = eng.rows([b[-1:]], [sl[-1:]], [[]])
+        logits = torch.full((k, 1, k, 256), float("nan"), dtype=torch.float32, device="cuda")
+        B.blt_dec_diffuse_block(eng.h, 1, r, k, alpha, 0, eng.d_out, eng.d_steps, logits)
+        assert B.blt_dec_sync(eng.h) == 0
+        return logits.cpu().numpy(), eng._get(eng.d_steps[:1])[0]
+    finally:
+        eng.close()
+
+
+@pytest.mark.parametrize("which", ["tiny", "d4"])
+def test_persistent_block_logits_bitwise(tiny_setup, d4_setup, which):
+    wl, ws, om = tiny_setup if which == "tiny" else d4_setup
+    a, sa = _block_logits(wl, ws, False)
+    b, sb = _block_logits(wl, ws, True)
+    assert sa == sb
+    n = int(sa)
+    assert np.array_equal(a[:n], b[:n])
