@@ -219,6 +219,7 @@ def main():
     from block_diffusion_byte_b200 import binding as B
     from block_diffusion_byte_b200._build import build
     from block_diffusion_byte_b200.driver import Engine, generate
+    from block_diffusion_byte_b200.replicas import max_over_ranks, shard_ids
 
     if rank == 0:
         build()
@@ -228,7 +229,7 @@ def main():
     nb = wl.batch
     max_ctx = wl.prefix_len + wl.gen_bytes + 4 * wl.block + 16
     eng = Engine(wl.shape, ws, max_batch=nb, max_ctx=max_ctx, max_block=max(wl.block, 16), max_rows=1024, time_passes=True)
-    seq_ids = [rank * nb + i for i in range(nb)]
+    seq_ids = shard_ids(rank, world, nb)
     prefixes = [[int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, s, wl.prefix_len)] for s in seq_ids]
 
     def one_step():
@@ -258,10 +259,7 @@ def main():
     st1 = B.blt_dec_stats(eng.h)
     clocks = clk.summary()
     d = {k: st1[k] - st0[k] for k in st1}
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, "cuda")
     total_bytes = wl.gen_bytes * nb * world * args.steps
     value = total_bytes / (ms / 1000.0)
 
@@ -273,11 +271,7 @@ def main():
     for _ in range(e2e_steps):
         r = one_step()
     barrier()
-    e2e_s = (time.perf_counter() - t0) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_s], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks((time.perf_counter() - t0) / e2e_steps, "cuda")
     e2e_value = wl.gen_bytes * nb * world / e2e_s
 
     pk, pk_kind = peaks()

@@ -27,7 +27,7 @@ BLT_W_BF16 = 1
 BLT_DRAFT_AR = 0
 BLT_DRAFT_DIFFUSION = 1
 BLT_FLAG_TIME_PASSES = 1
-BLT_FLAG_PER_PHASE = 2
+BLT_FLAG_PERSISTENT = 2
 BLT_LAYER_NT = 12
 LAYER_ORDER = ("wq_c", "wk_c", "wv_c", "wo_c", "norm_c", "attn_norm", "wqkv", "wo", "ffn_norm", "w1", "w3", "w2")
 

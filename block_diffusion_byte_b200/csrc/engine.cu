@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -87,6 +88,10 @@ struct blt_dec {
   int* abort_flag = nullptr;
   unsigned epoch = 0;
   int f_qkv = 0, f_o = 0, f_w13 = 0, f_w2 = 0, f_head = 0, f_att = 0, f_dec = 0, mega_groups = 0;
+  // debug: BLTDEC_TRACE=<file> appends device timestamps of each persistent launch's first pass
+  unsigned long long* trace = nullptr;
+  std::string trace_path;
+  int trace_pending = 0;
 };
 
 namespace {
@@ -286,7 +291,8 @@ GemmArgs base_args(blt_dec* h) {
 }
 
 size_t attn_smem_bytes(const blt_dec* h) {
-  return (size_t)(kAttnRows * h->dh + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * h->dh * (h->kv_f32 ? 4 : 2);
+  const int es = h->kv_f32 ? 4 : 2;
+  return (size_t)(kAttnRows * h->dh + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * (h->dh + 16 / es) * es;
 }
 AttnArgs attn_args(blt_dec* h) {
   AttnArgs aa{};
@@ -612,7 +618,7 @@ __global__ void k_copy_logits(const float* src, float* dst, int n) {
 template <int NG, int PL, int DH, typename KVT>
 size_t mega_smem(const blt_dec* h) {
   return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 +
-         (size_t)2 * h->CH * DH * sizeof(KVT);
+         (size_t)2 * h->CH * kv_stride<DH, KVT>() * sizeof(KVT);
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -633,7 +639,7 @@ int mega_prepare_pd(blt_dec* h) {
 
 // Decide whether the persistent kernel applies to this model and set it up.
 int mega_setup(blt_dec* h) {
-  if ((h->cfg.flags & BLT_FLAG_PER_PHASE) || h->d > 1024 || (h->dh != 32 && h->dh != 64) || h->CH > 128) return BLT_OK;
+  if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || (h->dh != 32 && h->dh != 64) || h->CH > 128) return BLT_OK;
   int dev = 0;
   CK(cudaGetDevice(&dev));
   int coop = 0;
@@ -649,8 +655,9 @@ int mega_setup(blt_dec* h) {
                    : (h->dh == 64 ? mega_prepare_pd<2, 64, __nv_bfloat16>(h) : mega_prepare_pd<2, 32, __nv_bfloat16>(h));
   }
   if (rc != BLT_OK) {
+    fprintf(stderr, "bltdec: persistent pass kernel unavailable (%s); using per-phase kernels\n", h->err.c_str());
     h->err.clear();
-    return BLT_OK;  // not available: calls use the per-phase kernels
+    return BLT_OK;
   }
   std::vector<LayerW> lw(h->L);
   for (int l = 0; l < h->L; ++l)
@@ -676,6 +683,11 @@ int mega_setup(blt_dec* h) {
   CK(cudaMemset(h->abort_flag, 0, 4));
   h->epoch = 1;
   h->mega_ok = true;
+  if (const char* tp = getenv("BLTDEC_TRACE")) {
+    h->trace_path = tp;
+    TRY(dalloc(h, &h->trace, (size_t)h->nsm * kTraceEvents));
+    CK(cudaMemset(h->trace, 0, (size_t)h->nsm * kTraceEvents * 8));
+  }
   return BLT_OK;
 }
 
@@ -732,6 +744,13 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.epoch0 = h->epoch;
   h->epoch += (unsigned)(max_passes + 1) * (h->L + 1) + 1;
   m.abort = h->abort_flag;
+  m.trace = h->trace;
+  if (h->trace) {
+    h->trace_pending = 1;
+    void* tn = nullptr;
+    CK(cudaGetSymbolAddress(&tn, g_trace_n));
+    CK(cudaMemsetAsync(tn, 0, sizeof(int) * 1024, h->stream));
+  }
   m.mode = mode;
   m.batch = batch;
   m.k = k;
@@ -1180,6 +1199,17 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
 int blt_dec_sync(blt_dec_t* h) {
   if (!h) return BLT_ERR_INVALID_ARG;
   CK(cudaStreamSynchronize(h->stream));
+  if (h->trace && h->trace_pending) {
+    std::vector<unsigned long long> t((size_t)h->nsm * kTraceEvents);
+    CK(cudaMemcpy(t.data(), h->trace, t.size() * 8, cudaMemcpyDeviceToHost));
+    if (FILE* f = fopen(h->trace_path.c_str(), "ab")) {
+      const int hdr[3] = {h->nsm, kTraceEvents, h->L};
+      fwrite(hdr, sizeof hdr, 1, f);
+      fwrite(t.data(), 8, t.size(), f);
+      fclose(f);
+    }
+    h->trace_pending = 0;
+  }
   int st = 0;
   CK(cudaMemcpy(&st, h->sd.status, 4, cudaMemcpyDeviceToHost));
   if (st != 0) {

@@ -150,6 +150,7 @@ __device__ __forceinline__ void kv_store(const GemmArgs& a, size_t off, float v)
 }
 
 // Output pair of tile rows (r16, r16 + 8) of tile mt for activation row `row`.
+// Row metadata pointers may point to shared memory (persistent kernel copies).
 template <int EPI>
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16, int row, float v0, float v1) {
   if constexpr (EPI == EPI_STORE) {
@@ -162,8 +163,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
     o[8] = __ldcg(o + 8) + v1;
   } else if constexpr (EPI == EPI_XRESID) {
     const int n = mt * 16 + r16;
-    const float* src = (a.layer == 0) ? a.embed + (size_t)__ldcg(a.row_byte + row) * a.d : a.out + (size_t)row * a.ldo;
-    const float* c = c_row(a.c_lat, a.max_lat, a.L, a.layer, a.d, __ldcg(a.row_seq + row), __ldcg(a.row_lat + row));
+    const float* src = (a.layer == 0) ? a.embed + (size_t)a.row_byte[row] * a.d : a.out + (size_t)row * a.ldo;
+    const float* c = c_row(a.c_lat, a.max_lat, a.L, a.layer, a.d, a.row_seq[row], a.row_lat[row]);
     const float s0 = __ldcg(src + n) + __ldcg(c + n), s1 = __ldcg(src + n + 8) + __ldcg(c + n + 8);
     float* o = a.out + (size_t)row * a.ldo + n;
     o[0] = s0 + v0;
@@ -177,8 +178,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
   } else {  // EPI_QKV: q/k tiles hold rotary pairs (j, j + dh/2) in rows (r16, r16 + 8)
     const int tiles_sec = a.d / 16;
     const int sec = mt / tiles_sec, lt = mt % tiles_sec;
-    const int pos = __ldcg(a.row_pos + row);
-    const int seq = __ldcg(a.row_seq + row);
+    const int pos = a.row_pos[row];
+    const int seq = a.row_seq[row];
     if (sec == 0 || sec == 1) {
       const int tph = a.dh / 16;
       const int h = lt / tph, j = (lt % tph) * 8 + r16;
@@ -407,30 +408,77 @@ __device__ __forceinline__ const KVT* kv_chunk_src(const AttnArgs& a, int seq, i
          (size_t)(tpos % a.PT) * DH;
 }
 
+// Row stride (elements) of a K/V chunk in shared memory: 16 bytes of padding
+// so the 16-byte segments of consecutive keys fall in different banks.
+template <int DH, typename KVT>
+__host__ __device__ constexpr int kv_stride() {
+  return DH + 16 / (int)sizeof(KVT);
+}
+
 // Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
-// ks/vs (raw KVT, [CH][DH]) with 16-byte cp.async (L2 only).
+// ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).
 template <int DH, typename KVT>
 __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, int t0, int lo, int hi, KVT* ks, KVT* vs, int tid,
                                              int nthr) {
   constexpr int PER = 16 / sizeof(KVT);
   constexpr int CPR = DH / PER;
+  constexpr int ST = kv_stride<DH, KVT>();
   const int n = max(0, hi - lo);
   for (int i = tid; i < 2 * n * CPR; i += nthr) {
     const int kvsel = i / (n * CPR), j = i % (n * CPR);
     const int key = lo - t0 + j / CPR, c = (j % CPR) * PER;
     const KVT* src = kv_chunk_src<DH, KVT>(a, seq, h, t0 + key, kvsel) + c;
-    KVT* dst = (kvsel ? vs : ks) + key * DH + c;
+    KVT* dst = (kvsel ? vs : ks) + key * ST + c;
     cp_async16(dst, src, 16);
+  }
+}
+
+// Scores of rows 0..nr-1 (nr <= RM) against one key: s[r] = sum_c q[r][c] k[c] in c order.
+template <int DH, typename KVT, int RM>
+__device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, const KVT* ks, float* ps, const int* lim, int nr,
+                                            int nk, int tid, int nthr) {
+  constexpr int ST = kv_stride<DH, KVT>();
+  for (int key = tid; key < a.CH; key += nthr) {
+    float s[RM];
+#pragma unroll
+    for (int r = 0; r < RM; ++r) s[r] = 0.f;
+    const bool valid = key < nk;
+    if (valid) {
+#pragma unroll
+      for (int c8 = 0; c8 < DH / 8; ++c8) {
+        float k8[8];
+        widen8(ks + key * ST + c8 * 8, k8);
+#pragma unroll
+        for (int r = 0; r < RM; ++r) {
+          if (r < nr) {
+            const float4 qa = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8);
+            const float4 qb = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8 + 4);
+            s[r] = fmaf(qa.x, k8[0], s[r]);
+            s[r] = fmaf(qa.y, k8[1], s[r]);
+            s[r] = fmaf(qa.z, k8[2], s[r]);
+            s[r] = fmaf(qa.w, k8[3], s[r]);
+            s[r] = fmaf(qb.x, k8[4], s[r]);
+            s[r] = fmaf(qb.y, k8[5], s[r]);
+            s[r] = fmaf(qb.z, k8[6], s[r]);
+            s[r] = fmaf(qb.w, k8[7], s[r]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+      if (r < nr) ps[r * a.CH + key] = (valid && key < lim[r]) ? s[r] : -INFINITY;
   }
 }
 
 // Softmax partial of one (group, head, chunk): scores of every row against
 // keys [t0, t0+nk) (masked per row by nkeys), m = max, l = sum exp(s - m),
 // o = sum exp(s - m) v.  q pre-scaled by 1/sqrt(dh).  smem: qs [32][DH] f32,
-// ps [32][CH] f32, ks/vs [CH][DH] KVT already loaded.
-template <int DH, typename KVT, class Sync>
+// ps [32][CH] f32, ks/vs [CH][kv_stride] KVT already loaded.
+template <int DH, typename KVT, class Sync, int RMAX = kAttnRows>
 __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
                                      const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync) {
+  constexpr int ST = kv_stride<DH, KVT>();
   const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
   const int t0 = chunk * a.CH;
   const int nk = min(a.CH, kmax - t0);
@@ -440,23 +488,9 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   }
   if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
   sync();
-  for (int key = tid; key < a.CH; key += nthr) {
-    float kr[DH];
-    const bool valid = key < nk;
-    if (valid) {
-#pragma unroll
-      for (int c = 0; c < DH / 8; ++c) widen8(ks + key * DH + c * 8, kr + c * 8);
-    }
-    for (int r = 0; r < nr; ++r) {
-      float s = -INFINITY;
-      if (valid && key < lim[r]) {
-        s = 0.f;
-#pragma unroll
-        for (int c = 0; c < DH; ++c) s = fmaf(qs[r * DH + c], kr[c], s);
-      }
-      ps[r * a.CH + key] = s;
-    }
-  }
+  if (RMAX <= 8 || nr <= 8) attn_scores<DH, KVT, 8>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  else if (RMAX <= 16 || nr <= 16) attn_scores<DH, KVT, (RMAX < 16 ? RMAX : 16)>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  else attn_scores<DH, KVT, 32>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
   sync();
   const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
   for (int r = warp; r < nr; r += nw) {
@@ -482,8 +516,8 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
     float o = 0.f;
     for (int k = 0; k < nk; ++k) {
       float v;
-      if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * DH + c]);
-      else v = vs[k * DH + c];
+      if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * ST + c]);
+      else v = vs[k * ST + c];
       o = fmaf(ps[r * a.CH + k], v, o);
     }
     const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
@@ -492,23 +526,38 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   }
 }
 
-// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}, in chunk order.
+// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}, in chunk order
+// (loads issued eight chunks at a time).
 __device__ __forceinline__ void attn_combine_one(const AttnArgs& a, int row, int h, int c) {
   const int nk = __ldcg(a.rows.nkeys + row);
   const int nch = (nk + a.CH - 1) / a.CH;
   const size_t base = ((size_t)row * a.H + h) * a.CMAX;
   float m = -INFINITY;
-  for (int ch = 0; ch < nch; ++ch) {
-    const float2 ml = __ldcg(a.part_ml + base + ch);
-    if (ml.y > 0.f) m = fmaxf(m, ml.x);
+  for (int c0 = 0; c0 < nch; c0 += 8) {
+    float2 ml[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ml[i] = (c0 + i < nch) ? __ldcg(a.part_ml + base + c0 + i) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (ml[i].y > 0.f) m = fmaxf(m, ml[i].x);
   }
   float l = 0.f, o = 0.f;
-  for (int ch = 0; ch < nch; ++ch) {
-    const float2 ml = __ldcg(a.part_ml + base + ch);
-    if (ml.y > 0.f) {
-      const float w = expf(ml.x - m);
-      l += ml.y * w;
-      o += __ldcg(a.part_o + (base + ch) * a.dh + c) * w;
+  for (int c0 = 0; c0 < nch; c0 += 8) {
+    float2 ml[8];
+    float ov[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = c0 + i < nch;
+      ml[i] = in ? __ldcg(a.part_ml + base + c0 + i) : make_float2(0.f, 0.f);
+      ov[i] = in ? __ldcg(a.part_o + (base + c0 + i) * a.dh + c) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (ml[i].y > 0.f) {
+        const float w = expf(ml[i].x - m);
+        l += ml[i].y * w;
+        o += ov[i] * w;
+      }
     }
   }
   a.att[(size_t)row * a.d + h * a.dh + c] = o / l;
@@ -527,7 +576,7 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   float* qs = reinterpret_cast<float*>(smem4);
   float* ps = qs + kAttnRows * DH;
   KVT* ks = reinterpret_cast<KVT*>(ps + kAttnRows * a.CH);
-  KVT* vs = ks + a.CH * DH;
+  KVT* vs = ks + a.CH * kv_stride<DH, KVT>();
   __shared__ float mrow[kAttnRows], lrow[kAttnRows];
   __shared__ int lim[kAttnRows];
   attn_load_kv<DH, KVT>(a, a.rows.g_seq[gi], h, t0, t0, min(t0 + a.CH, kmax), ks, vs, threadIdx.x, 128);

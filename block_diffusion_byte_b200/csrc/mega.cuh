@@ -69,6 +69,7 @@ struct MegaArgs {
   unsigned* dec_val;   // continue word written with the decision flag
   unsigned epoch0;
   int* abort;
+  unsigned long long* trace;  // debug timestamps [cta][kTraceEvents] of pass 0 (NULL: off)
   int mode, batch, k, max_passes;
   float alpha;
   const int* vlat;
@@ -139,6 +140,57 @@ __device__ __forceinline__ bool wait_mbar(const MegaArgs& m, uint64_t* b, unsign
   }
   return true;
 }
+
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
+
+// Warp-wide wait until flag(i) >= target for every i < n: each lane polls
+// its share with relaxed loads (all in flight at once), then one acquire
+// fence orders the data reads that follow.  Bounded like wait_flag.
+template <class FlagFn>
+__device__ __forceinline__ bool warp_wait(const MegaArgs& m, int n, FlagFn flag, unsigned target) {
+  const int lane = threadIdx.x & 31;
+  unsigned spins = 0;
+  while (true) {
+    bool mine = true;
+    for (int i = lane; i < n; i += 32) mine &= (int)(ld_relaxed(flag(i)) - target) >= 0;
+    if (__all_sync(0xffffffffu, mine)) break;
+    ++spins;
+    if (spins > 8) __nanosleep(128);
+    if ((spins & 255) == 0 && *(volatile int*)m.abort) return false;
+    if (spins > (kSpinLimit >> 6)) {
+      if (lane == 0) {
+        atomicExch(m.abort, 1);
+        set_status(m.sd.status, kErrDevice);
+      }
+      return false;
+    }
+  }
+  fence_acquire();
+  __syncwarp();
+  return true;
+}
+
+// Device-side timestamps (debug): trace[cta][event] = %globaltimer.
+constexpr int kTraceEvents = 1024;
+__device__ int g_trace_n[1024];  // per-CTA event count of the traced pass (debug only)
+// Event word: code << 48 | low 48 bits of %globaltimer.  Recorded by thread 0 in pass 0.
+__device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code) {
+  if (m.trace && pass == 0 && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    const int i = g_trace_n[blockIdx.x]++;
+    if (i < kTraceEvents) m.trace[(size_t)blockIdx.x * kTraceEvents + i] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
+  }
+}
+enum TraceCode : int {
+  TR_PASS = 1, TR_PHASE_BEGIN = 2, TR_INPUTS = 3, TR_XBUILT = 4, TR_KLOOP = 5, TR_REDUCED = 6, TR_UNIT_DONE = 7,
+  TR_ATT_BEGIN = 8, TR_ATT_QKV = 9, TR_ATT_LOADED = 10, TR_ATT_COMPUTED = 11, TR_ATT_DONE = 12, TR_HEAD = 13, TR_BOOK = 14
+};
 
 // ---------------------------------------------------------------------------- schedule
 enum PhaseKind : int { PH_QKV = 0, PH_O = 1, PH_W13 = 2, PH_W2 = 3, PH_HEAD = 4 };
@@ -258,40 +310,55 @@ struct MegaSmem {
   int* lim;
   int* plan_sh;
   int* misc;  // [0]: last-arrival flag, [1]: any-active
+  int* rseq;  // this pass's row metadata, copied once per pass
+  int* rpos;
+  int* rlat;
+  int* rbyte;
 };
 
-// Input value of row `row`, column k for a phase (before the gain).
-__device__ __forceinline__ float2 x_pair(const MegaArgs& m, const Phase& p, int row, int k) {
-  if (p.kind == PH_QKV) {
-    const int d = m.d;
-    const float* src = (p.layer == 0) ? m.ga.embed + (size_t)__ldcg(m.rows.byte + row) * d : m.h + (size_t)row * d;
-    const float* c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, p.layer, d, __ldcg(m.rows.seq + row), __ldcg(m.rows.lat + row));
-    const float2 a = __ldcg(reinterpret_cast<const float2*>(src + k));
-    const float2 b = __ldcg(reinterpret_cast<const float2*>(c + k));
-    return make_float2(a.x + b.x, a.y + b.y);
-  }
-  if (p.kind == PH_O) return __ldcg(reinterpret_cast<const float2*>(m.att + (size_t)row * m.d + k));
-  if (p.kind == PH_W2) return __ldcg(reinterpret_cast<const float2*>(m.act + (size_t)row * m.F + k));
-  return __ldcg(reinterpret_cast<const float2*>(m.h + (size_t)row * m.d + k));  // W13, head
-}
+// Source rows of a phase input: value = a[k] (+ c[k] for the cross term).
+struct XSrc {
+  const float* a;
+  const float* c;
+};
 
-// Wait until the inputs of k-step s of phase p (this pass) are written.
-__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s, int n_groups) {
+// Input row of a phase (before the gain): QKV reads B_l = D_{l-1} + c_l (D_0 =
+// embedding), O reads the attention output, W13 and the head read the
+// residual stream, W2 reads the SwiGLU activations.
+__device__ __forceinline__ XSrc x_src(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int row) {
+  XSrc x{nullptr, nullptr};
+  const int d = m.d;
+  if (p.kind == PH_QKV) {
+    x.a = (p.layer == 0) ? m.ga.embed + (size_t)sm.rbyte[row] * d : m.h + (size_t)row * d;
+    x.c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, p.layer, d, sm.rseq[row], sm.rlat[row]);
+  } else if (p.kind == PH_O) {
+    x.a = m.att + (size_t)row * d;
+  } else if (p.kind == PH_W2) {
+    x.a = m.act + (size_t)row * m.F;
+  } else {
+    x.a = m.h + (size_t)row * d;
+  }
+  return x;
+}
+__device__ __forceinline__ float2 ld2(const float* p) { return __ldcg(reinterpret_cast<const float2*>(p)); }
+
+// Wait (whole warp) until the inputs of k-steps s0, s0 + 8, ... (n of them)
+// of phase p in this pass are written.
+__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s0, int n, int n_groups) {
   const unsigned* f = m.flags;
   if (p.kind == PH_QKV) {
     if (p.layer == 0) return true;
-    return wait_flag(m, f + m.f_w2 + s, epoch(m, pass, p.layer - 1));
+    return warp_wait(m, n, [&](int i) { return f + m.f_w2 + s0 + 8 * i; }, epoch(m, pass, p.layer - 1));
   }
   if (p.kind == PH_O) {
-    const int head = s * 16 / m.dh;
-    for (int g = 0; g < n_groups; ++g)
-      if (!wait_flag(m, f + m.f_att + g * m.H + head, epoch(m, pass, p.layer))) return false;
-    return true;
+    const int spk = m.dh / 16;  // k-steps per head
+    return warp_wait(m, n * n_groups, [&](int i) { return f + m.f_att + (i % n_groups) * m.H + (s0 + 8 * (i / n_groups)) / spk; },
+                     epoch(m, pass, p.layer));
   }
-  if (p.kind == PH_W13) return wait_flag(m, f + m.f_o + s, epoch(m, pass, p.layer));
+  if (p.kind == PH_W13) return warp_wait(m, n, [&](int i) { return f + m.f_o + s0 + 8 * i; }, epoch(m, pass, p.layer));
   if (p.kind == PH_W2)
-    return wait_flag(m, f + m.f_w13 + 2 * s, epoch(m, pass, p.layer)) && wait_flag(m, f + m.f_w13 + 2 * s + 1, epoch(m, pass, p.layer));
-  return wait_flag(m, f + m.f_w2 + s, epoch(m, pass, m.L - 1));  // head
+    return warp_wait(m, 2 * n, [&](int i) { return f + m.f_w13 + 2 * (s0 + 8 * (i >> 1)) + (i & 1); }, epoch(m, pass, p.layer));
+  return warp_wait(m, n, [&](int i) { return f + m.f_w2 + s0 + 8 * i; }, epoch(m, pass, m.L - 1));  // head
 }
 
 __device__ __forceinline__ const float* phase_gain(const MegaArgs& m, const Phase& p) {
@@ -319,43 +386,65 @@ __device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Ph
   const float* gain = phase_gain(m, p);
   const bool norm = gain != nullptr;
   const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps of this warp (<= 8)
-  // dependency waits for this warp's k-steps
-  bool ok = true;
-  if (lane == 0) {
-    for (int j = 0; j < nkw && ok; ++j) ok = wait_inputs(m, p, pass, warp + 8 * j, n_groups);
-  }
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
+  trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
+  bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);  // this warp's k-steps
+  trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
   XFrag xf[8][NG];
   float ss[NG];
+  XSrc src[NG];
+  bool live[NG];
 #pragma unroll
-  for (int n = 0; n < NG; ++n) ss[n] = 0.f;
+  for (int n = 0; n < NG; ++n) {
+    ss[n] = 0.f;
+    const int row = n * 8 + g;
+    live[n] = ok && row < nr;
+    src[n] = live[n] ? x_src(m, sm, p, row) : XSrc{nullptr, nullptr};
+  }
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < nkw) {
+  for (int half = 0; half < 2; ++half) {
+    float2 ra[4][NG], rb[4][NG];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = half * 4 + jj;
       const int k0 = (warp + 8 * j) * 16 + 2 * t;
-      float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
-      if (norm) {
-        g0 = __ldg(gain + k0);
-        g1 = __ldg(gain + k0 + 1);
-        g8 = __ldg(gain + k0 + 8);
-        g9 = __ldg(gain + k0 + 9);
-      }
 #pragma unroll
       for (int n = 0; n < NG; ++n) {
-        const int row = n * 8 + g;
-        float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-        if (ok && row < nr) {
-          a = x_pair(m, p, row, k0);
-          b = x_pair(m, p, row, k0 + 8);
+        ra[jj][n] = rb[jj][n] = make_float2(0.f, 0.f);
+        if (j < nkw && live[n]) {
+          ra[jj][n] = ld2(src[n].a + k0);
+          rb[jj][n] = ld2(src[n].a + k0 + 8);
+          if (src[n].c) {
+            const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
+            ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
+            rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
+          }
         }
-        if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
-        xf[j][n] = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = half * 4 + jj;
+      if (j < nkw) {
+        const int k0 = (warp + 8 * j) * 16 + 2 * t;
+        float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
+        if (norm) {
+          g0 = __ldg(gain + k0);
+          g1 = __ldg(gain + k0 + 1);
+          g8 = __ldg(gain + k0 + 8);
+          g9 = __ldg(gain + k0 + 9);
+        }
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          const float2 a = ra[jj][n], b = rb[jj][n];
+          if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
+          xf[j][n] = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
+        }
       }
     }
   }
   const unsigned tile_bytes = 512u * PL;
   const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // <= 2
+  trace_mark(m, pass, TR_XBUILT << 8 | p.kind);
   for (int u = u0; u < p.units; u += G) {
     float acc[NG][4];
 #pragma unroll
@@ -383,10 +472,13 @@ __device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Ph
         ++it;
       }
     }
+    trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
     tile_reduce<NG>(acc, ss, norm, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
                     [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(ga, u, r16, col, v0, v1); });
+    trace_mark(m, pass, TR_REDUCED << 8 | p.kind);
     consumer_sync();
     if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
+    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
   }
   return ok;
 }
@@ -403,30 +495,30 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
   const unsigned tile_bytes = 512u * PL;
   const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
   bool ok = true;
+  trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
+  ok = wait_inputs(m, p, pass, warp, (p.ksteps - warp + 7) / 8, n_groups);  // all of this warp's k-steps
+  trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
+  XSrc src[NG];
+  bool live[NG];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    live[n] = ok && n * 8 + g < nr;
+    src[n] = live[n] ? x_src(m, sm, p, n * 8 + g) : XSrc{nullptr, nullptr};
+  }
   auto load = [&](int st, float2 (&xa)[4][NG], float2 (&xb)[4][NG]) {
-    bool good = true;
-    if (lane == 0) {
-      for (int jj = 0; jj < 4 && good; ++jj) {
-        const int ks = st * kStageTiles + 8 * jj + warp;
-        if (ks < p.ksteps) good = wait_inputs(m, p, pass, ks, n_groups);
-      }
-    }
-    good = __shfl_sync(0xffffffffu, good, 0);
-    __syncwarp();
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int ks = st * kStageTiles + 8 * jj + warp;
 #pragma unroll
       for (int n = 0; n < NG; ++n) {
-        const int row = n * 8 + g;
         xa[jj][n] = xb[jj][n] = make_float2(0.f, 0.f);
-        if (good && ks < p.ksteps && row < nr) {
-          xa[jj][n] = x_pair(m, p, row, ks * 16 + 2 * t);
-          xb[jj][n] = x_pair(m, p, row, ks * 16 + 2 * t + 8);
+        if (live[n] && ks < p.ksteps) {
+          xa[jj][n] = ld2(src[n].a + ks * 16 + 2 * t);
+          xb[jj][n] = ld2(src[n].a + ks * 16 + 2 * t + 8);
         }
       }
     }
-    return good;
+    return ok;
   };
   for (int u = u0; u < p.units; u += G) {
     float acc[NG][4], ss[NG];
@@ -462,10 +554,13 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
           cb[jj][n] = nb[jj][n];
         }
     }
+    trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
     tile_reduce<NG>(acc, ss, false, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
                     [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI_RESID>(ga, u, r16, col, v0, v1); });
+    trace_mark(m, pass, TR_REDUCED << 8 | p.kind);
     consumer_sync();
     if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
+    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
   }
   return ok;
 }
@@ -494,21 +589,24 @@ __device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, 
     const int h = rem / nch, c = rem % nch;
     const int seq = __ldcg(m.rows.g_seq + g), kmax = __ldcg(m.rows.g_kmax + g), fresh = __ldcg(m.rows.g_fresh + g);
     const int t0 = c * a.CH, t1 = min(t0 + a.CH, kmax);
+    trace_mark(m, pass, TR_ATT_BEGIN << 8);
     // keys cached before this pass can be fetched before q/k/v of this pass exist
     attn_load_kv<DH, KVT>(a, seq, h, t0, t0, min(t1, fresh), ks, vs, tid, 256);
     cp_async_commit();
-    if (tid == 0) {
-      const unsigned e = epoch(m, pass, layer);
-      for (int sec = 0; sec < 3 && ok; ++sec)
-        for (int j = 0; j < tph && ok; ++j) ok = wait_flag(m, m.flags + m.f_qkv + sec * tiles_sec + h * tph + j, e);
-    }
+    if (tid < 32)
+      ok = warp_wait(m, 3 * tph, [&](int i) { return m.flags + m.f_qkv + (i / tph) * tiles_sec + h * tph + i % tph; },
+                     epoch(m, pass, layer)) && ok;
     consumer_sync();
+    trace_mark(m, pass, TR_ATT_QKV << 8);
     attn_load_kv<DH, KVT>(a, seq, h, t0, max(t0, fresh), t1, ks, vs, tid, 256);
     cp_async_commit();
     cp_async_wait<0>();
     consumer_sync();
-    attn_partial_compute<DH, KVT>(a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, tid, 256, consumer_sync);
+    trace_mark(m, pass, TR_ATT_LOADED << 8);
+    attn_partial_compute<DH, KVT, decltype(&consumer_sync), 8 * kMegaMaxNG>(a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim,
+                                                                          tid, 256, consumer_sync);
     consumer_sync();
+    trace_mark(m, pass, TR_ATT_COMPUTED << 8);
     if (tid == 0) {
       __threadfence();
       const unsigned old = atomicAdd(m.attn_cnt + g * m.H + h, 1u);
@@ -526,6 +624,7 @@ __device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, 
       }
     }
     consumer_sync();
+    trace_mark(m, pass, TR_ATT_DONE << 8 | sm.misc[0]);
   }
   return ok;
 }
@@ -534,10 +633,8 @@ __device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, 
 // decision to go on, the plan of the next pass (CTA 0 only).
 __device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass, int nr, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    for (int u = 0; u < 16; ++u) wait_flag(m, m.flags + m.f_head + u, epoch(m, pass, m.L));
-    sm.misc[1] = 0;
-  }
+  if (tid < 32) warp_wait(m, 16, [&](int u) { return m.flags + m.f_head + u; }, epoch(m, pass, m.L));
+  if (tid == 0) sm.misc[1] = 0;
   consumer_sync();
   for (int r = warp; r < nr; r += 8) {
     float c, g;
@@ -596,6 +693,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   __shared__ int misc[4];
   __shared__ float mrow[kAttnRows], lrow[kAttnRows];
   __shared__ int lim[kAttnRows];
+  __shared__ int rmeta[4][8 * kMegaMaxNG];
 
   const unsigned tile_bytes = 512u * PL;
   const unsigned slot_bytes = kStageTiles * tile_bytes;
@@ -612,7 +710,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.ps = reinterpret_cast<float*>(p);
   p += kAttnRows * m.aa.CH * 4;
   sm.ks = p;
-  p += m.aa.CH * DH * sizeof(KVT);
+  p += m.aa.CH * kv_stride<DH, KVT>() * sizeof(KVT);
   sm.vs = p;
   sm.full = bars;
   sm.empty = bars + 16;
@@ -621,6 +719,10 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.lim = lim;
   sm.plan_sh = plan_sh;
   sm.misc = misc;
+  sm.rseq = rmeta[0];
+  sm.rpos = rmeta[1];
+  sm.rlat = rmeta[2];
+  sm.rbyte = rmeta[3];
 
   const int tid = threadIdx.x;
   if (tid == 0) {
@@ -651,9 +753,21 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     }
     const int nr = __ldcg(m.rows.n_rows);
     const int n_groups = __ldcg(m.rows.n_groups);
+    if (tid < nr) {
+      sm.rseq[tid] = __ldcg(m.rows.seq + tid);
+      sm.rpos[tid] = __ldcg(m.rows.pos + tid);
+      sm.rlat[tid] = __ldcg(m.rows.lat + tid);
+      sm.rbyte[tid] = __ldcg(m.rows.byte + tid);
+    }
+    consumer_sync();
+    trace_mark(m, pass, TR_PASS << 8);
     for (int l = 0; l < m.L && ok; ++l) {
       GemmArgs ga = m.ga;
       ga.layer = l;
+      ga.row_seq = sm.rseq;
+      ga.row_pos = sm.rpos;
+      ga.row_lat = sm.rlat;
+      ga.row_byte = sm.rbyte;
       ok = run_phase_cached<NG, PL, EPI_QKV>(m, sm, phase_of(m, 4 * l), pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
       ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
       ga.out = m.h;
@@ -673,7 +787,9 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     ga.out = m.logits;
     ga.ldo = 256;
     ok = run_phase_cached<NG, PL, EPI_STORE>(m, sm, phase_of(m, 4 * m.L), pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
+    trace_mark(m, pass, TR_HEAD << 8);
     if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
+    trace_mark(m, pass, TR_BOOK << 8);
   }
 }
 

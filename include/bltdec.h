@@ -97,7 +97,7 @@ typedef struct {
 } blt_dec_config;
 
 #define BLT_FLAG_TIME_PASSES 1 /* bracket the decoder passes of every call with CUDA events (counters.pass_ns) */
-#define BLT_FLAG_PER_PHASE 2   /* never use the persistent pass kernel (one launch per phase instead) */
+#define BLT_FLAG_PERSISTENT 2  /* run small passes (<= 16 rows) in the persistent pass kernel (one launch per call) */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */

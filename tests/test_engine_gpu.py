@@ -173,14 +173,14 @@ def test_d4_b1_first_block_logits_and_bytes(d4_setup):
     assert [int(r["steps"][0]) for r in res.rounds] == [r["steps"] for r in rec][: len(res.rounds)] or res.out[0] != want
 
 
-def _call_logits(wl, ws, per_phase, mode, k, alpha, G=24, batch=2):
+def _call_logits(wl, ws, persistent, mode, k, alpha, G=24, batch=2):
     """Logits of every engine call of a short generation (diffuse / draft / verify), via out_logits."""
     import ctypes
 
     from block_diffusion_byte_b200 import binding as B
     from block_diffusion_byte_b200.driver import Engine, generate
 
-    eng = Engine(wl.shape, ws, max_batch=batch, max_ctx=wl.prefix_len + G + 64, max_block=16, max_rows=256, per_phase=per_phase)
+    eng = Engine(wl.shape, ws, max_batch=batch, max_ctx=wl.prefix_len + G + 64, max_block=16, max_rows=256, persistent=persistent)
     try:
         w = replace(wl, mode=mode, block=k, alpha=alpha)
         res = generate(eng, w, [_prefix(wl, s) for s in range(batch)], G, record=True)
@@ -195,8 +195,8 @@ def test_persistent_kernel_matches_per_phase_bitwise(tiny_setup, mode, k, alpha,
     """The persistent pass kernel and the per-phase kernels share every arithmetic step
     (every pass of these calls has at most 16 rows, so the persistent kernel runs them)."""
     wl, ws, om = tiny_setup
-    a, sa = _call_logits(wl, ws, False, mode, k, alpha, batch=batch)
-    b, sb = _call_logits(wl, ws, True, mode, k, alpha, batch=batch)
+    a, sa = _call_logits(wl, ws, True, mode, k, alpha, batch=batch)
+    b, sb = _call_logits(wl, ws, False, mode, k, alpha, batch=batch)
     assert a.out == b.out
     assert sa["passes"] == sb["passes"]
     assert sa["kernel_launches"] < sb["kernel_launches"]  # the persistent path ran
@@ -205,13 +205,13 @@ def test_persistent_kernel_matches_per_phase_bitwise(tiny_setup, mode, k, alpha,
             assert np.array_equal(ra[key], rb[key]), key
 
 
-def _block_logits(wl, ws, per_phase, k=4, alpha=0.7):
+def _block_logits(wl, ws, persistent, k=4, alpha=0.7):
     from block_diffusion_byte_b200 import binding as B
     from block_diffusion_byte_b200.driver import Engine, SeqHost
     from workload import Patcher
 
     pre = _prefix(wl, 0)
-    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 64, max_block=16, max_rows=1024, per_phase=per_phase)
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 64, max_block=16, max_rows=1024, persistent=persistent)
     try:
         s = SeqHost(Patcher(wl.patch_kind, wl.seed, wl.cfg_index, 0), wl.seed, wl.cfg_index, 0, wl.shape.d_global)
         s.commit(pre)
@@ -230,8 +230,8 @@ def _block_logits(wl, ws, per_phase, k=4, alpha=0.7):
 @pytest.mark.parametrize("which", ["tiny", "d4"])
 def test_persistent_block_logits_bitwise(tiny_setup, d4_setup, which):
     wl, ws, om = tiny_setup if which == "tiny" else d4_setup
-    a, sa = _block_logits(wl, ws, False)
-    b, sb = _block_logits(wl, ws, True)
+    a, sa = _block_logits(wl, ws, True)
+    b, sb = _block_logits(wl, ws, False)
     assert sa == sb
     n = int(sa)
     assert np.array_equal(a[:n], b[:n])
