@@ -34,6 +34,7 @@ LAYER_ORDER = ("wq_c", "wk_c", "wv_c", "wo_c", "norm_c", "attn_norm", "wqkv", "w
 EXPORTS = (
     "blt_dec_init",
     "blt_dec_prefill",
+    "blt_dec_prefill_noalloc",
     "blt_dec_diffuse_block",
     "blt_dec_draft",
     "blt_dec_verify_accept",
@@ -119,6 +120,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     P, I, F, V = C.c_void_p, C.c_int, C.c_float, None
     lib.blt_dec_init.argtypes = [C.POINTER(blt_dec_config), C.POINTER(blt_dec_weights), P, C.POINTER(P)]
     lib.blt_dec_prefill.argtypes = [P, I, C.POINTER(blt_rows_in), P]
+    lib.blt_dec_prefill_noalloc.argtypes = [P, I, C.POINTER(blt_rows_in), P]
     lib.blt_dec_diffuse_block.argtypes = [P, I, C.POINTER(blt_rows_in), I, F, I, P, P, P]
     lib.blt_dec_draft.argtypes = [P, I, C.POINTER(blt_rows_in), I, I, F, I, P, P]
     lib.blt_dec_verify_accept.argtypes = [P, P, P, C.POINTER(C.c_int32), P, P, P]
@@ -193,6 +195,10 @@ def blt_dec_init(cfg: blt_dec_config, embed, head, final_norm, layers, stream: O
 
 def blt_dec_prefill(h: int, batch: int, rows: blt_rows_in, out_logits=None) -> None:
     _check(h, load_library().blt_dec_prefill(h, batch, C.byref(rows), _ptr(out_logits)), "blt_dec_prefill")
+
+
+def blt_dec_prefill_noalloc(h: int, batch: int, rows: blt_rows_in, out_logits=None) -> None:
+    _check(h, load_library().blt_dec_prefill_noalloc(h, batch, C.byref(rows), _ptr(out_logits)), "blt_dec_prefill_noalloc")
 
 
 def blt_dec_diffuse_block(h, batch, pending, k, alpha, max_steps, out_block, out_steps=None, out_logits=None) -> None:

@@ -2,6 +2,7 @@
 // pool, latent cache, per-call sequencing of decoder passes, and the C ABI of
 // bltdec.h.  Every decoder step runs in the kernels of kernels.cuh.
 #include <algorithm>
+#include <mutex>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -778,6 +779,145 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   return ng1 ? mega_launch_t<1, 2, 32, __nv_bfloat16>(h, m) : mega_launch_t<2, 2, 32, __nv_bfloat16>(h, m);
 }
 
+// Body of blt_dec_prefill after argument checks (cd made, bounds refreshed).
+int prefill_impl(blt_dec* h, int batch, const blt_rows_in* rows, float* out_logits, const CallDesc& cd) {
+  const int total = cd.row_off[batch];
+  TRY(reserve(h, cd, 0, true));
+  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
+  h->launches += 1;
+  TRY(project_latents(h, cd, rows->new_latents, true));
+  k_snapshot_base<<<1, 256, 0, h->stream>>>(h->sd, batch);
+  h->launches += 1;
+  int kmax = 0;
+  for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
+  const int chunk = h->cfg.max_rows;
+  for (int r0 = 0; r0 < total; r0 += chunk) {
+    const int r1 = std::min(total, r0 + chunk);
+    PlanArgs p = plan_args(h, PL_PREFILL, 0);
+    p.r0 = r0;
+    p.r1 = r1;
+    p.pend_bytes = rows->bytes;
+    p.pend_lat = rows->row_latent;
+    TRY(plan(h, p, cd));
+    TRY(run_pass(h, r1 - r0, kmax, (r1 - r0 + 31) / 32 + batch, out_logits != nullptr));
+    if (out_logits) {
+      k_copy_logits<<<256, 256, 0, h->stream>>>(h->logits, out_logits + (size_t)r0 * 256, (r1 - r0) * 256);
+      h->launches += 1;
+    }
+  }
+  k_finish_prefill<<<1, 256, 0, h->stream>>>(h->sd, cd);
+  h->launches += 1;
+  CK(cudaGetLastError());
+  bump_bounds(h, cd, 0);
+  return post_mirror(h);
+}
+
+}  // namespace
+
+
+// ============================================================================ prefill without allocation
+// One file-scope device arena holds the per-call scratch of blt_dec_prefill_noalloc:
+// activations, attention partials, logits, the row plan and the latent temporary
+// for chunks of at most kNaRows rows over at most kNaKeys key positions.
+namespace {
+constexpr int kNaRows = 32;
+constexpr int kNaKeys = 4096;
+constexpr int kNaMaxD = 1024, kNaMaxF = 4096, kNaMaxH = 16, kNaMaxDh = 64, kNaChunk = 128;
+constexpr int kNaCMax = kNaKeys / kNaChunk;
+constexpr int kNaGroups = kNaRows / kAttnRows + kMaxCallBatch + 1;
+constexpr size_t na_align(size_t x) { return (x + 255) & ~(size_t)255; }
+constexpr size_t kNaArenaBytes =
+    na_align(4ull * kNaRows * kNaMaxD * 4) * 1 + na_align((size_t)kNaRows * kNaMaxF * 4) + na_align((size_t)kNaRows * 256 * 4) +
+    na_align((size_t)kNaRows * kNaMaxH * kNaCMax * 8) + na_align((size_t)kNaRows * kNaMaxH * kNaCMax * kNaMaxDh * 4) +
+    3 * na_align(kNaRows * 4) + 5 * na_align(kNaRows * 4 + 4) + 5 * na_align(kNaGroups * 4 + 4) + 3 * na_align(kNaRows * 4 + 4) + 16 * 256;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_arena[kNaArenaBytes];
+
+namespace {
+std::mutex g_na_mutex;
+void* g_na_base[256];  // device address of the arena, per device (resolved on first use)
+
+// Address of the arena on the current device; resolved once per device.
+int na_arena(blt_dec* h, unsigned char** out) {
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) return fail(h, BLT_ERR_CUDA, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_na_mutex);
+  if (!g_na_base[dev]) {
+    void* p = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_arena));
+    g_na_base[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_na_base[dev]);
+  return BLT_OK;
+}
+
+struct NaCarve {
+  unsigned char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t n) {
+    off = na_align(off);
+    T* p = reinterpret_cast<T*>(base + off);
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+// Points the handle's pass scratch at the arena for one call and restores it after.
+struct NaSwap {
+  blt_dec* h;
+  float *hh, *q, *att, *act, *logits, *tmp, *conf, *gap;
+  float2* part_ml;
+  float* part_o;
+  int* pred;
+  RowsDev rows;
+  int *lat_seq, *lat_slot, *n_lat_rows;
+  int cmax, max_rows;
+  NaSwap(blt_dec* hd, unsigned char* base) : h(hd) {
+    hh = h->h, q = h->q, att = h->att, act = h->act, logits = h->logits, tmp = h->tmp, conf = h->conf, gap = h->gap;
+    part_ml = h->part_ml, part_o = h->part_o, pred = h->pred, rows = h->rows;
+    lat_seq = h->lat_seq, lat_slot = h->lat_slot, n_lat_rows = h->n_lat_rows, cmax = h->CMAX, max_rows = h->cfg.max_rows;
+    NaCarve c{base};
+    h->h = c.take<float>((size_t)kNaRows * kNaMaxD);
+    h->q = c.take<float>((size_t)kNaRows * kNaMaxD);
+    h->att = c.take<float>((size_t)kNaRows * kNaMaxD);
+    h->tmp = c.take<float>((size_t)kNaRows * kNaMaxD);
+    h->act = c.take<float>((size_t)kNaRows * kNaMaxF);
+    h->logits = c.take<float>((size_t)kNaRows * 256);
+    h->part_ml = c.take<float2>((size_t)kNaRows * kNaMaxH * kNaCMax);
+    h->part_o = c.take<float>((size_t)kNaRows * kNaMaxH * kNaCMax * kNaMaxDh);
+    h->conf = c.take<float>(kNaRows);
+    h->gap = c.take<float>(kNaRows);
+    h->pred = c.take<int>(kNaRows);
+    RowsDev& r = h->rows;
+    r.seq = c.take<int>(kNaRows);
+    r.pos = c.take<int>(kNaRows);
+    r.lat = c.take<int>(kNaRows);
+    r.nkeys = c.take<int>(kNaRows);
+    r.byte = c.take<int>(kNaRows);
+    r.n_rows = c.take<int>(1);
+    r.g_seq = c.take<int>(kNaGroups);
+    r.g_row0 = c.take<int>(kNaGroups);
+    r.g_nrows = c.take<int>(kNaGroups);
+    r.g_kmax = c.take<int>(kNaGroups);
+    r.g_fresh = c.take<int>(kNaGroups);
+    r.n_groups = c.take<int>(1);
+    h->lat_seq = c.take<int>(kNaRows);
+    h->lat_slot = c.take<int>(kNaRows);
+    h->n_lat_rows = c.take<int>(1);
+    h->CMAX = kNaCMax;
+    h->cfg.max_rows = kNaRows;
+    used = c.off;
+  }
+  size_t used = 0;
+  ~NaSwap() {
+    h->h = hh, h->q = q, h->att = att, h->act = act, h->logits = logits, h->tmp = tmp, h->conf = conf, h->gap = gap;
+    h->part_ml = part_ml, h->part_o = part_o, h->pred = pred, h->rows = rows;
+    h->lat_seq = lat_seq, h->lat_slot = lat_slot, h->n_lat_rows = n_lat_rows, h->CMAX = cmax, h->cfg.max_rows = max_rows;
+  }
+};
 }  // namespace
 
 // ============================================================================ C ABI
@@ -991,34 +1131,31 @@ int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out
   const int total = cd.row_off[batch];
   if (total > 0 && (!rows->bytes || !rows->row_latent)) return fail(h, BLT_ERR_INVALID_ARG, "bytes/row_latent NULL");
   refresh_bounds(h);
-  TRY(reserve(h, cd, 0, true));
-  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
-  h->launches += 1;
-  TRY(project_latents(h, cd, rows->new_latents, true));
-  k_snapshot_base<<<1, 256, 0, h->stream>>>(h->sd, batch);
-  h->launches += 1;
-  int kmax = 0;
-  for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
-  const int chunk = h->cfg.max_rows;
-  for (int r0 = 0; r0 < total; r0 += chunk) {
-    const int r1 = std::min(total, r0 + chunk);
-    PlanArgs p = plan_args(h, PL_PREFILL, 0);
-    p.r0 = r0;
-    p.r1 = r1;
-    p.pend_bytes = rows->bytes;
-    p.pend_lat = rows->row_latent;
-    TRY(plan(h, p, cd));
-    TRY(run_pass(h, r1 - r0, kmax, (r1 - r0 + 31) / 32 + batch, out_logits != nullptr));
-    if (out_logits) {
-      k_copy_logits<<<256, 256, 0, h->stream>>>(h->logits, out_logits + (size_t)r0 * 256, (r1 - r0) * 256);
-      h->launches += 1;
-    }
-  }
-  k_finish_prefill<<<1, 256, 0, h->stream>>>(h->sd, cd);
-  h->launches += 1;
-  CK(cudaGetLastError());
-  bump_bounds(h, cd, 0);
-  return post_mirror(h);
+  return prefill_impl(h, batch, rows, out_logits, cd);
+}
+
+int blt_dec_prefill_noalloc(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (h->state != 0) return fail(h, BLT_ERR_STATE, "a draft is waiting for verification");
+  if (h->d > kNaMaxD || h->F > kNaMaxF || h->H > kNaMaxH || h->dh > kNaMaxDh || h->CH != kNaChunk)
+    return fail(h, BLT_ERR_INVALID_ARG, "model exceeds the static prefill arena (d <= %d, d_ffn <= %d, heads <= %d, head dim <= %d, "
+                "attn_chunk %d)", kNaMaxD, kNaMaxF, kNaMaxH, kNaMaxDh, kNaChunk);
+  TRY(check_pending(h, rows, true));
+  CallDesc cd;
+  TRY(make_desc(h, batch, rows->row_offsets, rows->latent_offsets, cd));
+  const int total = cd.row_off[batch];
+  if (total > 0 && (!rows->bytes || !rows->row_latent)) return fail(h, BLT_ERR_INVALID_ARG, "bytes/row_latent NULL");
+  refresh_bounds(h);
+  for (int s = 0; s < batch; ++s)
+    if (h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s] > kNaKeys)
+      return fail(h, BLT_ERR_INVALID_ARG, "sequence %d would reach %d positions > %d (static prefill arena)", s,
+                  h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s], kNaKeys);
+  unsigned char* base = nullptr;
+  TRY(na_arena(h, &base));
+  NaSwap swap(h, base);
+  if (swap.used > kNaArenaBytes) return fail(h, BLT_ERR_INVALID_ARG, "static prefill arena too small");
+  return prefill_impl(h, batch, rows, out_logits, cd);
 }
 
 int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float alpha, int max_steps,

@@ -147,6 +147,31 @@ int blt_dec_init(const blt_dec_config *cfg, const blt_dec_weights *w, void *cuda
  * Errors: INVALID_ARG, NO_SPACE, STATE (a draft is waiting for verification). */
 int blt_dec_prefill(blt_dec_t *h, int batch, const blt_rows_in *rows, float *out_logits);
 
+/* blt_dec_prefill, with no allocation of its own.  (The paper has no
+ * counterpart: this is an engineering entry point.)
+ *
+ * Same inputs, outputs, semantics and errors as blt_dec_prefill, but the
+ * per-call scratch of the decoder passes (activations, split-KV attention
+ * partials, logits, the row plan, the latent-projection temporary) lives in
+ * one file-scope static device arena instead of the handle's scratch, and
+ * the call makes no cudaMalloc, cudaFree or other allocating call.  Callers
+ * that cannot allocate device memory at call time use it: a serving process
+ * that sized the handle small (max_rows, the scratch blt_dec_init allocates)
+ * and runs under a device-memory budget that is already spent, or a host
+ * thread that must not allocate once set-up is over, can still prefill in
+ * 32-row chunks.
+ *
+ * Limits (else INVALID_ARG): d_model <= 1024, d_ffn <= 4096, n_heads <= 16,
+ * head dim <= 64, attn_chunk 128 (the default), and each sequence's cached
+ * length plus its rows <= 4096 positions.  The arena is about 5.2 MB and every
+ * GPU that loads the library holds it until the process exits.
+ * The first call on a device resolves the arena's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call shares the one arena, which keeps
+ * the last call's contents (nothing in it needs to start at zero): calls that
+ * overlap on the GPU -- on different streams or handles -- race. */
+int blt_dec_prefill_noalloc(blt_dec_t *h, int batch, const blt_rows_in *rows, float *out_logits);
+
 /* BLT-D: fill one masked block of k bytes per sequence ("BLT-D 추론",
  * "블록 언마스킹 전략").  The pending rows ride, causally, in the first pass
  * and are cached.  Block rows sit at the next k positions, attend the whole
