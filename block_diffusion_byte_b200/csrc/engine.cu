@@ -618,8 +618,9 @@ __global__ void k_copy_logits(const float* src, float* dst, int n) {
 // ---------------------------------------------------------------------------- persistent pass kernel
 template <int NG, int PL, int DH, typename KVT>
 size_t mega_smem(const blt_dec* h) {
-  return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 +
-         (size_t)2 * h->CH * kv_stride<DH, KVT>() * sizeof(KVT);
+  const size_t attn = (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * kv_stride<DH, KVT>() * sizeof(KVT);
+  const size_t xin = (size_t)64 * NG * 32 * 16;  // phase input fragments, K <= 1024
+  return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + 16 * 4 + std::max(attn, xin);
 }
 
 template <int NG, int PL, int DH, typename KVT>

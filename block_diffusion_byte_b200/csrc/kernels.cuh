@@ -438,7 +438,9 @@ template <int DH, typename KVT, int RM>
 __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, const KVT* ks, float* ps, const int* lim, int nr,
                                             int nk, int tid, int nthr) {
   constexpr int ST = kv_stride<DH, KVT>();
-  for (int key = tid; key < a.CH; key += nthr) {
+  const int per = max(1, nthr / a.CH);  // threads per key; thread `part` takes rows part, part + per, ...
+  for (int idx = tid; idx < a.CH * per; idx += nthr) {
+    const int key = idx % a.CH, part = idx / a.CH;
     float s[RM];
 #pragma unroll
     for (int r = 0; r < RM; ++r) s[r] = 0.f;
@@ -450,7 +452,7 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
         widen8(ks + key * ST + c8 * 8, k8);
 #pragma unroll
         for (int r = 0; r < RM; ++r) {
-          if (r < nr) {
+          if (r < nr && r % per == part) {
             const float4 qa = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8);
             const float4 qb = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8 + 4);
             s[r] = fmaf(qa.x, k8[0], s[r]);
@@ -467,7 +469,7 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
     }
 #pragma unroll
     for (int r = 0; r < RM; ++r)
-      if (r < nr) ps[r * a.CH + key] = (valid && key < lim[r]) ? s[r] : -INFINITY;
+      if (r < nr && r % per == part) ps[r * a.CH + key] = (valid && key < lim[r]) ? s[r] : -INFINITY;
   }
 }
 

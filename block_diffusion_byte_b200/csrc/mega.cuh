@@ -90,6 +90,9 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, unsigned bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* b, unsigned n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(n) : "memory");
+}
 __device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity) {
   unsigned ok;
   asm volatile(
@@ -301,6 +304,8 @@ struct MegaSmem {
   int S;
   float* red;  // [8][16][16]
   float* ssr;  // [8][16]
+  uint4* xs;   // phase input fragments [k-steps][NG][32 lanes] (shares space with the attention buffers)
+  float* rsv;  // [16] RMS scale per row
   float* qs;
   float* ps;
   void* ks;
@@ -374,22 +379,31 @@ __device__ __forceinline__ void unit_epilogue(const MegaArgs& m, const Phase& p,
   gemm_epilogue<EPI>(ga, u, r16, row, v0, v1);
 }
 
-// Cached-input phase (K <= 1024: each warp owns <= 8 k-steps): the warp's
-// input fragments are built once and reused for every unit of the phase.
+// Phase with K <= 1024.  (1) The CTA's eight warps build the phase input once
+// in shared memory as split-bf16 fragments, warp w building k-steps w, w+8,
+// ... and its share of every row's sum of squares (the canonical order).
+// (2) Each warp then runs whole units alone: it keeps one accumulator per
+// lane group (k-step mod 8), adds them in lane-group order, scales by the
+// row's RMS factor and applies the epilogue to the values it holds -- the
+// same arithmetic as the 8-warp reduction, with no block-wide step -- and
+// releases the unit's flag.
 template <int NG, int PL, int EPI>
-__device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
-                                 int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
+__device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
+                                int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
   const int G = gridDim.x, cta = blockIdx.x;
   const int u0 = first_unit(p, cta, G);
   if (u0 >= p.units) return true;
+  const int nunits = (p.units - u0 + G - 1) / G;
+  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+  const unsigned it0 = it;
+  it += (unsigned)(nunits * nst);
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const float* gain = phase_gain(m, p);
   const bool norm = gain != nullptr;
-  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps of this warp (<= 8)
+  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps this warp builds (<= 8)
   trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
-  bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);  // this warp's k-steps
+  bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);
   trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
-  XFrag xf[8][NG];
   float ss[NG];
   XSrc src[NG];
   bool live[NG];
@@ -425,7 +439,8 @@ __device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Ph
     for (int jj = 0; jj < 4; ++jj) {
       const int j = half * 4 + jj;
       if (j < nkw) {
-        const int k0 = (warp + 8 * j) * 16 + 2 * t;
+        const int s = warp + 8 * j;
+        const int k0 = s * 16 + 2 * t;
         float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
         if (norm) {
           g0 = __ldg(gain + k0);
@@ -437,49 +452,94 @@ __device__ bool run_phase_cached(const MegaArgs& m, const MegaSmem& sm, const Ph
         for (int n = 0; n < NG; ++n) {
           const float2 a = ra[jj][n], b = rb[jj][n];
           if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
-          xf[j][n] = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
+          const XFrag f = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
+          sm.xs[(s * NG + n) * 32 + lane] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
         }
       }
     }
   }
-  const unsigned tile_bytes = 512u * PL;
-  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // <= 2
+  if (norm) {
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      float v = ss[n];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if (t == 0) sm.ssr[warp * 16 + n * 8 + g] = v;
+    }
+  }
+  consumer_sync();
+  if (tid < 16) {
+    float r = 1.0f;
+    if (norm) {
+      float v = sm.ssr[tid];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) v += sm.ssr[w * 16 + tid];
+      r = 1.0f / sqrtf(v / (float)(p.ksteps * 16) + m.eps);
+    }
+    sm.rsv[tid] = r;
+  }
+  consumer_sync();
   trace_mark(m, pass, TR_XBUILT << 8 | p.kind);
-  for (int u = u0; u < p.units; u += G) {
-    float acc[NG][4];
+  const unsigned tile_bytes = 512u * PL;
+  for (int j = warp; j < nunits; j += kWarps) {
+    const int u = u0 + j * G;
+    float acc[8][NG][4];
 #pragma unroll
-    for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int st = 0; st < 2; ++st) {
-      if (st < nst) {
-        const int slot = it % sm.S;
-        if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
-        const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+      for (int n = 0; n < NG; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
+    for (int st = 0; st < nst; ++st) {
+      const unsigned itu = it0 + (unsigned)(j * nst + st);
+      const int slot = itu % sm.S;
+      if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
+      const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+      const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
+      for (int t8 = 0; t8 < ntiles; t8 += 8) {
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int tile = 8 * jj + warp;  // within the stage
-          const int ks = st * kStageTiles + tile;
-          if (ks < p.ksteps) {
+        for (int jj = 0; jj < 8; ++jj) {
+          const int tile = t8 + jj;
+          if (tile < ntiles) {
+            const int s = st * kStageTiles + tile;  // s mod 8 == jj
             uint4 w[PL];
 #pragma unroll
             for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
 #pragma unroll
-            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, xf[st * 4 + jj][n]);
+            for (int n = 0; n < NG; ++n) {
+              const uint4 xv = sm.xs[(s * NG + n) * 32 + lane];
+              const XFrag xf{xv.x, xv.y, xv.z, xv.w};
+              mma_step<PL>(acc[jj][n], w, xf);
+            }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sm.empty + slot);
-        ++it;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_n(sm.empty + slot, kMegaConsumers);
+    }
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      float v[4] = {acc[0][n][0], acc[0][n][1], acc[0][n][2], acc[0][n][3]};
+#pragma unroll
+      for (int a = 1; a < 8; ++a) {
+        v[0] += acc[a][n][0];
+        v[1] += acc[a][n][1];
+        v[2] += acc[a][n][2];
+        v[3] += acc[a][n][3];
+      }
+      const int c0 = n * 8 + 2 * t;
+      if (c0 < nr) {
+        const float r = sm.rsv[c0];
+        gemm_epilogue<EPI>(ga, u, g, c0, v[0] * r, v[2] * r);
+      }
+      if (c0 + 1 < nr) {
+        const float r = sm.rsv[c0 + 1];
+        gemm_epilogue<EPI>(ga, u, g, c0 + 1, v[1] * r, v[3] * r);
       }
     }
-    trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
-    tile_reduce<NG>(acc, ss, norm, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
-                    [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(ga, u, r16, col, v0, v1); });
-    trace_mark(m, pass, TR_REDUCED << 8 | p.kind);
-    consumer_sync();
-    if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
-    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
+    __syncwarp();
+    if (lane == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
+    if (warp == 0) trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
   }
+  consumer_sync();  // the input fragments are free again
   return ok;
 }
 
@@ -705,6 +765,9 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   p += 8 * 16 * 8 * kMegaMaxNG * 4;
   sm.ssr = reinterpret_cast<float*>(p);
   p += 8 * 8 * kMegaMaxNG * 4;
+  sm.rsv = reinterpret_cast<float*>(p);
+  p += 16 * 4;
+  sm.xs = reinterpret_cast<uint4*>(p);  // the phase input shares space with the attention buffers
   sm.qs = reinterpret_cast<float*>(p);
   p += kAttnRows * DH * 4;
   sm.ps = reinterpret_cast<float*>(p);
@@ -768,25 +831,25 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
       ga.row_pos = sm.rpos;
       ga.row_lat = sm.rlat;
       ga.row_byte = sm.rbyte;
-      ok = run_phase_cached<NG, PL, EPI_QKV>(m, sm, phase_of(m, 4 * l), pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
+      ok = run_phase_units<NG, PL, EPI_QKV>(m, sm, phase_of(m, 4 * l), pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
       ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
       ga.out = m.h;
       ga.ldo = m.d;
-      ok = run_phase_cached<NG, PL, EPI_XRESID>(m, sm, phase_of(m, 4 * l + 1), pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
+      ok = run_phase_units<NG, PL, EPI_XRESID>(m, sm, phase_of(m, 4 * l + 1), pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
       ga.out = m.act;
       ga.ldo = m.F;
-      ok = run_phase_cached<NG, PL, EPI_SWIGLU>(m, sm, phase_of(m, 4 * l + 2), pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
+      ok = run_phase_units<NG, PL, EPI_SWIGLU>(m, sm, phase_of(m, 4 * l + 2), pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
       ga.out = m.h;
       ga.ldo = m.d;
       const Phase p2 = phase_of(m, 4 * l + 3);
-      if (p2.ksteps <= 64) ok = run_phase_cached<NG, PL, EPI_RESID>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
+      if (p2.ksteps <= 64) ok = run_phase_units<NG, PL, EPI_RESID>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
       else ok = run_phase_streamed<NG, PL>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
     }
     if (!ok) break;
     GemmArgs ga = m.ga;
     ga.out = m.logits;
     ga.ldo = 256;
-    ok = run_phase_cached<NG, PL, EPI_STORE>(m, sm, phase_of(m, 4 * m.L), pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
+    ok = run_phase_units<NG, PL, EPI_STORE>(m, sm, phase_of(m, 4 * m.L), pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
     trace_mark(m, pass, TR_HEAD << 8);
     if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
     trace_mark(m, pass, TR_BOOK << 8);
