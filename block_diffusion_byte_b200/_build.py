@@ -9,7 +9,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libbltdec.so")
 SOURCES = [os.path.join(PKG, "csrc", "engine.cu")]
-DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("common.cuh", "kernels.cuh")] + [os.path.join(ROOT, "include", "bltdec.h")]
+CSRC = os.path.join(PKG, "csrc")
+DEPS = [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cu", ".cuh"))] + [os.path.join(ROOT, "include", "bltdec.h")]
 
 NVCC_FLAGS = [
     "-gencode",

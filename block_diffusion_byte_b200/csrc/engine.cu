@@ -749,9 +749,6 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.trace = h->trace;
   if (h->trace) {
     h->trace_pending = 1;
-    void* tn = nullptr;
-    CK(cudaGetSymbolAddress(&tn, g_trace_n));
-    CK(cudaMemsetAsync(tn, 0, sizeof(int) * 1024, h->stream));
   }
   m.mode = mode;
   m.batch = batch;

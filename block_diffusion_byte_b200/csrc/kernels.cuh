@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
     }
   };
   const uint4* wbase = a.w + (size_t)mt * ksteps * PL * 32 + lane;
-  auto wtile = [&](int wi, int p) -> uint4 { return ldg_stream(wbase + ((size_t)(wi * kWarps + warp) * PL + p) * 32); };
+  const uint64_t wpol = l2_evict_first();
+  auto wtile = [&](int wi, int p) -> uint4 { return ldg_stream(wbase + ((size_t)(wi * kWarps + warp) * PL + p) * 32, wpol); };
 
   constexpr int DEPTH = 4;
   uint4 wb[DEPTH][PL];
@@ -433,43 +434,42 @@ __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, 
   }
 }
 
-// Scores of rows 0..nr-1 (nr <= RM) against one key: s[r] = sum_c q[r][c] k[c] in c order.
-template <int DH, typename KVT, int RM>
+// Scores of rows 0..nr-1 against each key: s[r] = sum_c q[r][c] k[c], one
+// fmaf chain in c order.  `per` threads share a key (thread `part` takes rows
+// part, part + per, ...).  The key is widened 32 columns at a time and the
+// running sums live in ps between column blocks (an exact round trip), which
+// keeps the loop small for the instruction cache.
+template <int DH, typename KVT>
 __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, const KVT* ks, float* ps, const int* lim, int nr,
                                             int nk, int tid, int nthr) {
   constexpr int ST = kv_stride<DH, KVT>();
-  const int per = max(1, nthr / a.CH);  // threads per key; thread `part` takes rows part, part + per, ...
+  constexpr int CB = DH < 32 ? DH : 32;  // columns per block
+  const int per = max(1, nthr / a.CH);
   for (int idx = tid; idx < a.CH * per; idx += nthr) {
     const int key = idx % a.CH, part = idx / a.CH;
-    float s[RM];
+    if (key < nk) {
+      for (int c0 = 0; c0 < DH; c0 += CB) {
+        float kf[CB];
 #pragma unroll
-    for (int r = 0; r < RM; ++r) s[r] = 0.f;
-    const bool valid = key < nk;
-    if (valid) {
+        for (int c8 = 0; c8 < CB / 8; ++c8) widen8(ks + key * ST + c0 + c8 * 8, kf + c8 * 8);
+#pragma unroll 1
+        for (int r = part; r < nr; r += per) {
+          const float* q = qs + r * DH + c0;
+          float sr = (c0 == 0) ? 0.f : ps[r * a.CH + key];
 #pragma unroll
-      for (int c8 = 0; c8 < DH / 8; ++c8) {
-        float k8[8];
-        widen8(ks + key * ST + c8 * 8, k8);
-#pragma unroll
-        for (int r = 0; r < RM; ++r) {
-          if (r < nr && r % per == part) {
-            const float4 qa = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8);
-            const float4 qb = *reinterpret_cast<const float4*>(qs + r * DH + c8 * 8 + 4);
-            s[r] = fmaf(qa.x, k8[0], s[r]);
-            s[r] = fmaf(qa.y, k8[1], s[r]);
-            s[r] = fmaf(qa.z, k8[2], s[r]);
-            s[r] = fmaf(qa.w, k8[3], s[r]);
-            s[r] = fmaf(qb.x, k8[4], s[r]);
-            s[r] = fmaf(qb.y, k8[5], s[r]);
-            s[r] = fmaf(qb.z, k8[6], s[r]);
-            s[r] = fmaf(qb.w, k8[7], s[r]);
+          for (int c4 = 0; c4 < CB / 4; ++c4) {
+            const float4 qv = *reinterpret_cast<const float4*>(q + c4 * 4);
+            sr = fmaf(qv.x, kf[c4 * 4 + 0], sr);
+            sr = fmaf(qv.y, kf[c4 * 4 + 1], sr);
+            sr = fmaf(qv.z, kf[c4 * 4 + 2], sr);
+            sr = fmaf(qv.w, kf[c4 * 4 + 3], sr);
           }
+          ps[r * a.CH + key] = sr;
         }
       }
     }
-#pragma unroll
-    for (int r = 0; r < RM; ++r)
-      if (r < nr && r % per == part) ps[r * a.CH + key] = (valid && key < lim[r]) ? s[r] : -INFINITY;
+    for (int r = part; r < nr; r += per)
+      if (!(key < nk && key < lim[r])) ps[r * a.CH + key] = -INFINITY;
   }
 }
 
@@ -477,9 +477,14 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
 // keys [t0, t0+nk) (masked per row by nkeys), m = max, l = sum exp(s - m),
 // o = sum exp(s - m) v.  q pre-scaled by 1/sqrt(dh).  smem: qs [32][DH] f32,
 // ps [32][CH] f32, ks/vs [CH][kv_stride] KVT already loaded.
-template <int DH, typename KVT, class Sync, int RMAX = kAttnRows>
+struct NoMark {
+  __device__ void operator()(int) const {}
+};
+
+template <int DH, typename KVT, class Sync, class Mark = NoMark>
 __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
-                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync) {
+                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync,
+                                     Mark mark = Mark()) {
   constexpr int ST = kv_stride<DH, KVT>();
   const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
   const int t0 = chunk * a.CH;
@@ -490,10 +495,10 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   }
   if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
   sync();
-  if (RMAX <= 8 || nr <= 8) attn_scores<DH, KVT, 8>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
-  else if (RMAX <= 16 || nr <= 16) attn_scores<DH, KVT, (RMAX < 16 ? RMAX : 16)>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
-  else attn_scores<DH, KVT, 32>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  mark(1);
+  attn_scores<DH, KVT>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
   sync();
+  mark(2);
   const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
   for (int r = warp; r < nr; r += nw) {
     float m = -INFINITY;
@@ -513,6 +518,7 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
     }
   }
   sync();
+  mark(3);
   for (int i = tid; i < nr * DH; i += nthr) {
     const int r = i / DH, c = i % DH;
     float o = 0.f;

@@ -102,9 +102,10 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void tma_1d(void* dst, const void* src, unsigned bytes, uint64_t* b) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(b))
+__device__ __forceinline__ void tma_1d(void* dst, const void* src, unsigned bytes, uint64_t* b, uint64_t pol) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(b)), "l"(pol)
                : "memory");
 }
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -160,6 +161,7 @@ __device__ __forceinline__ bool warp_wait(const MegaArgs& m, int n, FlagFn flag,
   unsigned spins = 0;
   while (true) {
     bool mine = true;
+#pragma unroll 1
     for (int i = lane; i < n; i += 32) mine &= (int)(ld_relaxed(flag(i)) - target) >= 0;
     if (__all_sync(0xffffffffu, mine)) break;
     ++spins;
@@ -180,19 +182,20 @@ __device__ __forceinline__ bool warp_wait(const MegaArgs& m, int n, FlagFn flag,
 
 // Device-side timestamps (debug): trace[cta][event] = %globaltimer.
 constexpr int kTraceEvents = 1024;
-__device__ int g_trace_n[1024];  // per-CTA event count of the traced pass (debug only)
+__shared__ int s_trace_n;  // this CTA's event count of the traced pass (debug only)
 // Event word: code << 48 | low 48 bits of %globaltimer.  Recorded by thread 0 in pass 0.
 __device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code) {
   if (m.trace && pass == 0 && threadIdx.x == 0) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    const int i = g_trace_n[blockIdx.x]++;
+    const int i = s_trace_n++;
     if (i < kTraceEvents) m.trace[(size_t)blockIdx.x * kTraceEvents + i] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
   }
 }
 enum TraceCode : int {
   TR_PASS = 1, TR_PHASE_BEGIN = 2, TR_INPUTS = 3, TR_XBUILT = 4, TR_KLOOP = 5, TR_REDUCED = 6, TR_UNIT_DONE = 7,
-  TR_ATT_BEGIN = 8, TR_ATT_QKV = 9, TR_ATT_LOADED = 10, TR_ATT_COMPUTED = 11, TR_ATT_DONE = 12, TR_HEAD = 13, TR_BOOK = 14
+  TR_ATT_BEGIN = 8, TR_ATT_QKV = 9, TR_ATT_LOADED = 10, TR_ATT_COMPUTED = 11, TR_ATT_DONE = 12, TR_HEAD = 13, TR_BOOK = 14,
+  TR_XLOADED = 15, TR_ATT_STEP = 16
 };
 
 // ---------------------------------------------------------------------------- schedule
@@ -250,6 +253,7 @@ __device__ __forceinline__ unsigned epoch(const MegaArgs& m, int pass, int layer
 __device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* full, uint64_t* empty, int S, int lane) {
   const int G = gridDim.x, cta = blockIdx.x;
   const unsigned tile_bytes = 512u * m.planes;
+  const uint64_t pol = l2_evict_first();
   unsigned it = 0;
   bool ok = true;
   for (int pass = 0; pass < m.max_passes && ok; ++pass) {
@@ -276,7 +280,7 @@ __device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* 
             if (ok) {
               mbar_expect_tx(full + slot, tiles * tile_bytes);
               tma_1d(ring + (size_t)slot * kStageTiles * tile_bytes, src + (size_t)st * kStageTiles * tile_bytes, tiles * tile_bytes,
-                     full + slot);
+                     full + slot, pol);
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -347,23 +351,37 @@ __device__ __forceinline__ XSrc x_src(const MegaArgs& m, const MegaSmem& sm, con
 }
 __device__ __forceinline__ float2 ld2(const float* p) { return __ldcg(reinterpret_cast<const float2*>(p)); }
 
-// Wait (whole warp) until the inputs of k-steps s0, s0 + 8, ... (n of them)
-// of phase p in this pass are written.
-__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s0, int n, int n_groups) {
+// Flag of the i-th input that k-steps s0, s0 + 8, ... of phase p depend on:
+// QKV and the head read the residual stream (W2 units), O reads attention
+// heads (one per group), W13 the O units, W2 the W13 unit pairs.
+__device__ __forceinline__ const unsigned* input_flag(const MegaArgs& m, const Phase& p, int s0, int n_groups, int i) {
   const unsigned* f = m.flags;
-  if (p.kind == PH_QKV) {
-    if (p.layer == 0) return true;
-    return warp_wait(m, n, [&](int i) { return f + m.f_w2 + s0 + 8 * i; }, epoch(m, pass, p.layer - 1));
+  switch (p.kind) {
+    case PH_O: {
+      const int spk = m.dh / 16;  // k-steps per head
+      return f + m.f_att + (i % n_groups) * m.H + (s0 + 8 * (i / n_groups)) / spk;
+    }
+    case PH_W13:
+      return f + m.f_o + s0 + 8 * i;
+    case PH_W2:
+      return f + m.f_w13 + 2 * (s0 + 8 * (i >> 1)) + (i & 1);
+    default:  // QKV (layer > 0), head
+      return f + m.f_w2 + s0 + 8 * i;
   }
-  if (p.kind == PH_O) {
-    const int spk = m.dh / 16;  // k-steps per head
-    return warp_wait(m, n * n_groups, [&](int i) { return f + m.f_att + (i % n_groups) * m.H + (s0 + 8 * (i / n_groups)) / spk; },
-                     epoch(m, pass, p.layer));
-  }
-  if (p.kind == PH_W13) return warp_wait(m, n, [&](int i) { return f + m.f_o + s0 + 8 * i; }, epoch(m, pass, p.layer));
-  if (p.kind == PH_W2)
-    return warp_wait(m, 2 * n, [&](int i) { return f + m.f_w13 + 2 * (s0 + 8 * (i >> 1)) + (i & 1); }, epoch(m, pass, p.layer));
-  return warp_wait(m, n, [&](int i) { return f + m.f_w2 + s0 + 8 * i; }, epoch(m, pass, m.L - 1));  // head
+}
+
+// Wait (whole warp) until the inputs of k-steps s0, s0 + 8, ... (n of them)
+// of phase p in this pass are written.  One polling loop for every phase
+// kind keeps the kernel's code small.
+__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s0, int n, int n_groups) {
+  if (p.kind == PH_QKV && p.layer == 0) return true;
+  int count = n;
+  unsigned target = epoch(m, pass, p.layer);
+  if (p.kind == PH_O) count = n * n_groups;
+  else if (p.kind == PH_W2) count = 2 * n;
+  else if (p.kind == PH_QKV) target = epoch(m, pass, p.layer - 1);
+  else if (p.kind == PH_HEAD) target = epoch(m, pass, m.L - 1);
+  return warp_wait(m, count, [&](int i) { return input_flag(m, p, s0, n_groups, i); }, target);
 }
 
 __device__ __forceinline__ const float* phase_gain(const MegaArgs& m, const Phase& p) {
@@ -373,10 +391,83 @@ __device__ __forceinline__ const float* phase_gain(const MegaArgs& m, const Phas
   return nullptr;
 }
 
-template <int EPI>
-__device__ __forceinline__ void unit_epilogue(const MegaArgs& m, const Phase& p, const GemmArgs& ga, int u, int r16, int row,
-                                              float v0, float v1) {
-  gemm_epilogue<EPI>(ga, u, r16, row, v0, v1);
+// Epilogue of one output pair, dispatched at run time so that one copy of the
+// phase loop serves every projection (the kernel's code must stay small
+// enough for the SM's instruction caches).
+__device__ __forceinline__ void mega_epilogue(const GemmArgs& ga, int epi, int u, int r16, int row, float v0, float v1) {
+  switch (epi) {
+    case EPI_QKV:
+      gemm_epilogue<EPI_QKV>(ga, u, r16, row, v0, v1);
+      break;
+    case EPI_XRESID:
+      gemm_epilogue<EPI_XRESID>(ga, u, r16, row, v0, v1);
+      break;
+    case EPI_SWIGLU:
+      gemm_epilogue<EPI_SWIGLU>(ga, u, r16, row, v0, v1);
+      break;
+    case EPI_RESID:
+      gemm_epilogue<EPI_RESID>(ga, u, r16, row, v0, v1);
+      break;
+    default:
+      gemm_epilogue<EPI_STORE>(ga, u, r16, row, v0, v1);
+      break;
+  }
+}
+
+// Phase input of this warp's k-steps warp, warp + 8, ... (nkw of them) as
+// split-bf16 fragments in shared memory, and its share of every row's sum of
+// squares.  Every load is issued unconditionally (a dead row reads row 0, a
+// k-step past the warp's share re-reads its last one; neither is stored) so
+// the compiler can put them all in flight at once.  HASC: QKV input, which
+// adds the cross term c_l.
+template <int NG, bool HASC>
+__device__ __forceinline__ void build_inputs(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int nr, int nkw,
+                                             const float* gain, float (&ss)[NG], int warp, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const bool norm = gain != nullptr;
+  XSrc src[NG];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    ss[n] = 0.f;
+    const int row = n * 8 + g;
+    src[n] = x_src(m, sm, p, row < nr ? row : 0);
+  }
+#pragma unroll 1
+  for (int half = 0; half < 2 && half * 4 < nkw; ++half) {
+    float2 ra[4][NG], rb[4][NG];
+    float4 gv[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = min(half * 4 + jj, nkw - 1);
+      const int k0 = (warp + 8 * j) * 16 + 2 * t;
+#pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        ra[jj][n] = ld2(src[n].a + k0);
+        rb[jj][n] = ld2(src[n].a + k0 + 8);
+        if constexpr (HASC) {
+          const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
+          ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
+          rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
+        }
+      }
+      gv[jj] = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (norm) gv[jj] = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
+    }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = half * 4 + jj;
+      if (j < nkw) {
+        const int s = warp + 8 * j;
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          const float2 a = ra[jj][n], b = rb[jj][n];
+          if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
+          const XFrag f = make_xfrag(a.x * gv[jj].x, a.y * gv[jj].y, b.x * gv[jj].z, b.y * gv[jj].w);
+          sm.xs[(s * NG + n) * 32 + lane] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
+        }
+      }
+    }
+  }
 }
 
 // Phase with K <= 1024.  (1) The CTA's eight warps build the phase input once
@@ -387,8 +478,8 @@ __device__ __forceinline__ void unit_epilogue(const MegaArgs& m, const Phase& p,
 // row's RMS factor and applies the epilogue to the values it holds -- the
 // same arithmetic as the 8-warp reduction, with no block-wide step -- and
 // releases the unit's flag.
-template <int NG, int PL, int EPI>
-__device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
+template <int NG, int PL>
+__device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int epi, int pass, unsigned& it, int nr,
                                 int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
   const int G = gridDim.x, cta = blockIdx.x;
   const int u0 = first_unit(p, cta, G);
@@ -405,59 +496,9 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
   bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);
   trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
   float ss[NG];
-  XSrc src[NG];
-  bool live[NG];
-#pragma unroll
-  for (int n = 0; n < NG; ++n) {
-    ss[n] = 0.f;
-    const int row = n * 8 + g;
-    live[n] = ok && row < nr;
-    src[n] = live[n] ? x_src(m, sm, p, row) : XSrc{nullptr, nullptr};
-  }
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    float2 ra[4][NG], rb[4][NG];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int j = half * 4 + jj;
-      const int k0 = (warp + 8 * j) * 16 + 2 * t;
-#pragma unroll
-      for (int n = 0; n < NG; ++n) {
-        ra[jj][n] = rb[jj][n] = make_float2(0.f, 0.f);
-        if (j < nkw && live[n]) {
-          ra[jj][n] = ld2(src[n].a + k0);
-          rb[jj][n] = ld2(src[n].a + k0 + 8);
-          if (src[n].c) {
-            const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
-            ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
-            rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int j = half * 4 + jj;
-      if (j < nkw) {
-        const int s = warp + 8 * j;
-        const int k0 = s * 16 + 2 * t;
-        float g0 = 1.f, g1 = 1.f, g8 = 1.f, g9 = 1.f;
-        if (norm) {
-          g0 = __ldg(gain + k0);
-          g1 = __ldg(gain + k0 + 1);
-          g8 = __ldg(gain + k0 + 8);
-          g9 = __ldg(gain + k0 + 9);
-        }
-#pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          const float2 a = ra[jj][n], b = rb[jj][n];
-          if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
-          const XFrag f = make_xfrag(a.x * g0, a.y * g1, b.x * g8, b.y * g9);
-          sm.xs[(s * NG + n) * 32 + lane] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
-        }
-      }
-    }
-  }
+  if (p.kind == PH_QKV) build_inputs<NG, true>(m, sm, p, nr, nkw, gain, ss, warp, lane);
+  else build_inputs<NG, false>(m, sm, p, nr, nkw, gain, ss, warp, lane);
+  trace_mark(m, pass, TR_XLOADED << 8 | p.kind);
   if (norm) {
 #pragma unroll
     for (int n = 0; n < NG; ++n) {
@@ -495,19 +536,41 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
       const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
       const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
       for (int t8 = 0; t8 < ntiles; t8 += 8) {
+        if (t8 + 8 <= ntiles) {
+          // a full group of eight k-steps (one per accumulator): all fragment
+          // loads first, then the independent MMA chains
+          constexpr int GS = (NG * PL > 1) ? 4 : 8;
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int tile = t8 + jj;
-          if (tile < ntiles) {
-            const int s = st * kStageTiles + tile;  // s mod 8 == jj
-            uint4 w[PL];
+          for (int j0 = 0; j0 < 8; j0 += GS) {
+            uint4 w[GS][PL], xv[GS][NG];
 #pragma unroll
-            for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+            for (int jj = 0; jj < GS; ++jj) {
+              const int tile = t8 + j0 + jj;
 #pragma unroll
-            for (int n = 0; n < NG; ++n) {
-              const uint4 xv = sm.xs[(s * NG + n) * 32 + lane];
-              const XFrag xf{xv.x, xv.y, xv.z, xv.w};
-              mma_step<PL>(acc[jj][n], w, xf);
+              for (int q = 0; q < PL; ++q)
+                w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+              for (int n = 0; n < NG; ++n) xv[jj][n] = sm.xs[((st * kStageTiles + tile) * NG + n) * 32 + lane];
+            }
+#pragma unroll
+            for (int jj = 0; jj < GS; ++jj)
+#pragma unroll
+              for (int n = 0; n < NG; ++n) mma_step<PL>(acc[j0 + jj][n], w[jj], XFrag{xv[jj][n].x, xv[jj][n].y, xv[jj][n].z, xv[jj][n].w});
+          }
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int tile = t8 + jj;
+            if (tile < ntiles) {
+              const int s = st * kStageTiles + tile;  // s mod 8 == jj
+              uint4 w[PL];
+#pragma unroll
+              for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+              for (int n = 0; n < NG; ++n) {
+                const uint4 xv = sm.xs[(s * NG + n) * 32 + lane];
+                mma_step<PL>(acc[jj][n], w, XFrag{xv.x, xv.y, xv.z, xv.w});
+              }
             }
           }
         }
@@ -528,11 +591,11 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
       const int c0 = n * 8 + 2 * t;
       if (c0 < nr) {
         const float r = sm.rsv[c0];
-        gemm_epilogue<EPI>(ga, u, g, c0, v[0] * r, v[2] * r);
+        mega_epilogue(ga, epi, u, g, c0, v[0] * r, v[2] * r);
       }
       if (c0 + 1 < nr) {
         const float r = sm.rsv[c0 + 1];
-        gemm_epilogue<EPI>(ga, u, g, c0 + 1, v[1] * r, v[3] * r);
+        mega_epilogue(ga, epi, u, g, c0 + 1, v[1] * r, v[3] * r);
       }
     }
     __syncwarp();
@@ -559,23 +622,18 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
   ok = wait_inputs(m, p, pass, warp, (p.ksteps - warp + 7) / 8, n_groups);  // all of this warp's k-steps
   trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
   XSrc src[NG];
-  bool live[NG];
 #pragma unroll
-  for (int n = 0; n < NG; ++n) {
-    live[n] = ok && n * 8 + g < nr;
-    src[n] = live[n] ? x_src(m, sm, p, n * 8 + g) : XSrc{nullptr, nullptr};
-  }
+  for (int n = 0; n < NG; ++n) src[n] = x_src(m, sm, p, n * 8 + g < nr ? n * 8 + g : 0);
+  // unconditional loads (dead rows read row 0, k-steps past the end re-read
+  // the last one; neither reaches an output) so all of a stage's are in flight together
   auto load = [&](int st, float2 (&xa)[4][NG], float2 (&xb)[4][NG]) {
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
-      const int ks = st * kStageTiles + 8 * jj + warp;
+      const int ks = min(st * kStageTiles + 8 * jj + warp, p.ksteps - 1);
 #pragma unroll
       for (int n = 0; n < NG; ++n) {
-        xa[jj][n] = xb[jj][n] = make_float2(0.f, 0.f);
-        if (live[n] && ks < p.ksteps) {
-          xa[jj][n] = ld2(src[n].a + ks * 16 + 2 * t);
-          xb[jj][n] = ld2(src[n].a + ks * 16 + 2 * t + 8);
-        }
+        xa[jj][n] = ld2(src[n].a + ks * 16 + 2 * t);
+        xb[jj][n] = ld2(src[n].a + ks * 16 + 2 * t + 8);
       }
     }
     return ok;
@@ -591,16 +649,28 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
       const int slot = it % sm.S;
       if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
       const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+      if ((st + 1) * kStageTiles <= p.ksteps) {  // full stage: weight loads first, then the chain
+        uint4 w[4][PL];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int tile = 8 * jj + warp;
-        const int ks = st * kStageTiles + tile;
-        if (ks < p.ksteps) {
-          uint4 w[PL];
+        for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-          for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+          for (int q = 0; q < PL; ++q)
+            w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)(8 * jj + warp) * tile_bytes + q * 512 + lane * 16);
 #pragma unroll
-          for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w[jj], make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int tile = 8 * jj + warp;
+          if (st * kStageTiles + tile < p.ksteps) {
+            uint4 w[PL];
+#pragma unroll
+            for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+          }
         }
       }
       __syncwarp();
@@ -616,7 +686,7 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
     }
     trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
     tile_reduce<NG>(acc, ss, false, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
-                    [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI_RESID>(ga, u, r16, col, v0, v1); });
+                    [&](int r16, int col, float v0, float v1) { mega_epilogue(ga, EPI_RESID, u, r16, col, v0, v1); });
     trace_mark(m, pass, TR_REDUCED << 8 | p.kind);
     consumer_sync();
     if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
@@ -663,8 +733,9 @@ __device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, 
     cp_async_wait<0>();
     consumer_sync();
     trace_mark(m, pass, TR_ATT_LOADED << 8);
-    attn_partial_compute<DH, KVT, decltype(&consumer_sync), 8 * kMegaMaxNG>(a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim,
-                                                                          tid, 256, consumer_sync);
+    attn_partial_compute<DH, KVT, decltype(&consumer_sync)>(
+        a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, tid, 256, consumer_sync,
+        [&](int step) { trace_mark(m, pass, TR_ATT_STEP << 8 | step); });
     consumer_sync();
     trace_mark(m, pass, TR_ATT_COMPUTED << 8);
     if (tid == 0) {
@@ -789,6 +860,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
 
   const int tid = threadIdx.x;
   if (tid == 0) {
+    s_trace_n = 0;
     for (int i = 0; i < sm.S; ++i) {
       mbar_init(sm.full + i, 1);
       mbar_init(sm.empty + i, kMegaConsumers);
@@ -816,11 +888,12 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     }
     const int nr = __ldcg(m.rows.n_rows);
     const int n_groups = __ldcg(m.rows.n_groups);
-    if (tid < nr) {
-      sm.rseq[tid] = __ldcg(m.rows.seq + tid);
-      sm.rpos[tid] = __ldcg(m.rows.pos + tid);
-      sm.rlat[tid] = __ldcg(m.rows.lat + tid);
-      sm.rbyte[tid] = __ldcg(m.rows.byte + tid);
+    if (tid < 8 * kMegaMaxNG) {  // rows past nr get harmless in-range values (inputs are loaded unconditionally)
+      const bool live = tid < nr;
+      sm.rseq[tid] = live ? __ldcg(m.rows.seq + tid) : 0;
+      sm.rpos[tid] = live ? __ldcg(m.rows.pos + tid) : 0;
+      sm.rlat[tid] = live ? __ldcg(m.rows.lat + tid) : 0;
+      sm.rbyte[tid] = live ? __ldcg(m.rows.byte + tid) : 0;
     }
     consumer_sync();
     trace_mark(m, pass, TR_PASS << 8);
@@ -831,25 +904,25 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
       ga.row_pos = sm.rpos;
       ga.row_lat = sm.rlat;
       ga.row_byte = sm.rbyte;
-      ok = run_phase_units<NG, PL, EPI_QKV>(m, sm, phase_of(m, 4 * l), pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
+      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l), EPI_QKV, pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
       ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
       ga.out = m.h;
       ga.ldo = m.d;
-      ok = run_phase_units<NG, PL, EPI_XRESID>(m, sm, phase_of(m, 4 * l + 1), pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
+      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l + 1), EPI_XRESID, pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
       ga.out = m.act;
       ga.ldo = m.F;
-      ok = run_phase_units<NG, PL, EPI_SWIGLU>(m, sm, phase_of(m, 4 * l + 2), pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
+      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l + 2), EPI_SWIGLU, pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
       ga.out = m.h;
       ga.ldo = m.d;
       const Phase p2 = phase_of(m, 4 * l + 3);
-      if (p2.ksteps <= 64) ok = run_phase_units<NG, PL, EPI_RESID>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
+      if (p2.ksteps <= 64) ok = run_phase_units<NG, PL>(m, sm, p2, EPI_RESID, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
       else ok = run_phase_streamed<NG, PL>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
     }
     if (!ok) break;
     GemmArgs ga = m.ga;
     ga.out = m.logits;
     ga.ldo = 256;
-    ok = run_phase_units<NG, PL, EPI_STORE>(m, sm, phase_of(m, 4 * m.L), pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
+    ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * m.L), EPI_STORE, pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
     trace_mark(m, pass, TR_HEAD << 8);
     if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
     trace_mark(m, pass, TR_BOOK << 8);
