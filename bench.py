@@ -197,6 +197,8 @@ def main():
     ap.add_argument("--workload", default="d4_b1", choices=sorted(CONFIGS))
     ap.add_argument("--ref-seconds", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="persistent", choices=["persistent", "phased"],
+                    help="decoder passes in the persistent kernel (one launch per call) or as per-phase kernels")
     args = ap.parse_args()
     wl = CONFIGS[args.workload]
     if args.impl == "reference":
@@ -228,7 +230,8 @@ def main():
     ws = WeightSet(wl.shape, seed=wl.seed).materialize()
     nb = wl.batch
     max_ctx = wl.prefix_len + wl.gen_bytes + 4 * wl.block + 16
-    eng = Engine(wl.shape, ws, max_batch=nb, max_ctx=max_ctx, max_block=max(wl.block, 16), max_rows=1024, time_passes=True)
+    eng = Engine(wl.shape, ws, max_batch=nb, max_ctx=max_ctx, max_block=max(wl.block, 16), max_rows=1024, time_passes=True,
+                 persistent=args.path == "persistent")
     seq_ids = shard_ids(rank, world, nb)
     prefixes = [[int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, s, wl.prefix_len)] for s in seq_ids]
 
@@ -308,7 +311,7 @@ def main():
             "frac": achieved / peak,
             "frac_of_8tbs": achieved / 8000.0,
             "traffic": None,
-            "kernel": "decoder pass (all kernels of one pass)",
+            "kernel": "k_mega (persistent decoder pass)" if d["persistent_calls"] else "decoder pass (all kernels of one pass)",
             "alg_bytes_per_pass": alg_bytes,
             "pass_ms": pass_ms,
         },
@@ -319,6 +322,8 @@ def main():
             "weight_bytes_per_pass": weight_b,
             "kv_bytes_per_pass": kv_b,
             "launches_per_step": d["kernel_launches"] / args.steps,
+            "path": args.path,
+            "persistent_calls_per_step": d["persistent_calls"] / args.steps,
         },
         "clocks": clocks,
     }

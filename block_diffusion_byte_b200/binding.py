@@ -100,6 +100,7 @@ class blt_dec_counters(C.Structure):
         ("kernel_launches", C.c_uint64),
         ("timed_passes", C.c_uint64),
         ("pass_ns", C.c_uint64),
+        ("persistent_calls", C.c_uint64),
     ]
 
     def as_dict(self):

@@ -75,6 +75,7 @@ struct blt_dec {
   std::string err;
   unsigned long long weight_bytes_per_pass = 0, kv_bytes_per_key = 0;
   unsigned long long launches = 0;  // kernels launched (host count)
+  unsigned long long persistent_calls = 0;  // calls served by the persistent kernel
   // pass timing (BLT_FLAG_TIME_PASSES): event pairs recorded around passes
   std::vector<cudaEvent_t> tev;
   size_t tev_used = 0;
@@ -363,7 +364,11 @@ int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want
     TRY(gemm<EPI_QKV>(h, h->qkv[l], a, rows_ub));
     aa.layer = l;
     launch_attn(h, dim3(h->H, nchunks, groups_ub), attn_smem_bytes(h), aa);
-    k_attn_combine<<<dim3(rows_ub, h->H), h->dh, 0, h->stream>>>(aa);
+    const dim3 cg(rows_ub, h->H);
+    if (h->dh == 64) k_attn_combine<64><<<cg, 32, 0, h->stream>>>(aa);
+    else if (h->dh == 32) k_attn_combine<32><<<cg, 32, 0, h->stream>>>(aa);
+    else if (h->dh == 128) k_attn_combine<128><<<cg, 32, 0, h->stream>>>(aa);
+    else k_attn_combine<16><<<cg, 32, 0, h->stream>>>(aa);
     CK(cudaGetLastError());
     a = base_args(h);
     a.layer = l;
@@ -641,7 +646,9 @@ int mega_prepare_pd(blt_dec* h) {
 
 // Decide whether the persistent kernel applies to this model and set it up.
 int mega_setup(blt_dec* h) {
-  if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || (h->dh != 32 && h->dh != 64) || h->CH > 128) return BLT_OK;
+  if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || h->d % 128 != 0 || h->F % 128 != 0 || (h->dh != 32 && h->dh != 64) ||
+      h->CH > 128)
+    return BLT_OK;
   int dev = 0;
   CK(cudaGetDevice(&dev));
   int coop = 0;
@@ -703,6 +710,7 @@ int mega_launch_t(blt_dec* h, MegaArgs& m) {
   void* args[] = {&m};
   CK(cudaLaunchCooperativeKernel((const void*)k_mega<NG, PL, DH, KVT>, dim3(h->nsm), dim3(kMegaThreads), args, smem, h->stream));
   h->launches += 1;
+  h->persistent_calls += 1;
   return BLT_OK;
 }
 
@@ -1328,6 +1336,7 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->kernel_launches = h->launches;
   out->timed_passes = (h->cfg.flags & BLT_FLAG_TIME_PASSES) ? c[0] : 0;
   out->pass_ns = h->pass_ns;
+  out->persistent_calls = h->persistent_calls;
   return BLT_OK;
 }
 

@@ -417,7 +417,8 @@ __host__ __device__ constexpr int kv_stride() {
 }
 
 // Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
-// ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).
+// ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).  One
+// K or V row per iteration: a single page-table lookup per row.
 template <int DH, typename KVT>
 __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, int t0, int lo, int hi, KVT* ks, KVT* vs, int tid,
                                              int nthr) {
@@ -425,12 +426,14 @@ __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, 
   constexpr int CPR = DH / PER;
   constexpr int ST = kv_stride<DH, KVT>();
   const int n = max(0, hi - lo);
-  for (int i = tid; i < 2 * n * CPR; i += nthr) {
-    const int kvsel = i / (n * CPR), j = i % (n * CPR);
-    const int key = lo - t0 + j / CPR, c = (j % CPR) * PER;
-    const KVT* src = kv_chunk_src<DH, KVT>(a, seq, h, t0 + key, kvsel) + c;
-    KVT* dst = (kvsel ? vs : ks) + key * ST + c;
-    cp_async16(dst, src, 16);
+#pragma unroll 1
+  for (int i = tid; i < 2 * n; i += nthr) {
+    const int kvsel = i >= n;
+    const int key = lo - t0 + (kvsel ? i - n : i);
+    const KVT* src = kv_chunk_src<DH, KVT>(a, seq, h, t0 + key, kvsel);
+    KVT* dst = (kvsel ? vs : ks) + key * ST;
+#pragma unroll
+    for (int c = 0; c < CPR; ++c) cp_async16(dst + c * PER, src + c * PER, 16);
   }
 }
 
@@ -500,11 +503,14 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   sync();
   mark(2);
   const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
+#pragma unroll 1
   for (int r = warp; r < nr; r += nw) {
     float m = -INFINITY;
+#pragma unroll 1
     for (int k = lane; k < a.CH; k += 32) m = fmaxf(m, ps[r * a.CH + k]);
     m = warp_max(m);
     float l = 0.f;
+#pragma unroll 1
     for (int k = lane; k < a.CH; k += 32) {
       const float s = ps[r * a.CH + k];
       const float p = (s == -INFINITY) ? 0.f : expf(s - m);
@@ -519,56 +525,90 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   }
   sync();
   mark(3);
-  for (int i = tid; i < nr * DH; i += nthr) {
-    const int r = i / DH, c = i % DH;
-    float o = 0.f;
+  // o[r][c] = sum_k p[r][k] v[k][c], one fmaf chain in k order per output.
+  // A thread owns column c and rows r0, r0 + rs, ... four at a time, so each
+  // V element it loads feeds four chains.  (nthr is a multiple of DH.)
+  const int c = tid % DH, rs = nthr / DH;
+#pragma unroll 1
+  for (int r0 = tid / DH; r0 < nr; r0 += 4 * rs) {
+    int rr[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) rr[j] = min(r0 + j * rs, nr - 1);  // rows past nr repeat a live one, not stored
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int k = 0; k < nk; ++k) {
       float v;
       if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * ST + c]);
       else v = vs[k * ST + c];
-      o = fmaf(ps[r * a.CH + k], v, o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[j] = fmaf(ps[rr[j] * a.CH + k], v, o[j]);
     }
-    const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
-    a.part_o[base * DH + c] = o;
-    if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = r0 + j * rs;
+      if (r < nr) {
+        const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
+        a.part_o[base * DH + c] = o[j];
+        if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+      }
+    }
   }
 }
 
-// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}, in chunk order
-// (loads issued eight chunks at a time).
-__device__ __forceinline__ void attn_combine_one(const AttnArgs& a, int row, int h, int c) {
+// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}
+// for one (row, head), by one warp.  m = largest chunk maximum (chunks with
+// l > 0); lane j holds the weight of chunk j of each 32-chunk block; l is the
+// warp sum of the lanes' l_c w_c sums; o accumulates the chunks in order with
+// the weight broadcast from its lane.  Lane c (and c + 32, ...) owns column c.
+template <int DH>
+__device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int h, int lane) {
+  constexpr int DPL = DH >= 32 ? DH / 32 : 1;  // columns per lane
   const int nk = __ldcg(a.rows.nkeys + row);
   const int nch = (nk + a.CH - 1) / a.CH;
   const size_t base = ((size_t)row * a.H + h) * a.CMAX;
   float m = -INFINITY;
-  for (int c0 = 0; c0 < nch; c0 += 8) {
-    float2 ml[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ml[i] = (c0 + i < nch) ? __ldcg(a.part_ml + base + c0 + i) : make_float2(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (ml[i].y > 0.f) m = fmaxf(m, ml[i].x);
+#pragma unroll 1
+  for (int ch = lane; ch < nch; ch += 32) {
+    const float2 ml = __ldcg(a.part_ml + base + ch);
+    if (ml.y > 0.f) m = fmaxf(m, ml.x);
   }
-  float l = 0.f, o = 0.f;
-  for (int c0 = 0; c0 < nch; c0 += 8) {
-    float2 ml[8];
-    float ov[8];
+  m = warp_max(m);
+  float l = 0.f, o[DPL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool in = c0 + i < nch;
-      ml[i] = in ? __ldcg(a.part_ml + base + c0 + i) : make_float2(0.f, 0.f);
-      ov[i] = in ? __ldcg(a.part_o + (base + c0 + i) * a.dh + c) : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (ml[i].y > 0.f) {
-        const float w = expf(ml[i].x - m);
-        l += ml[i].y * w;
-        o += ov[i] * w;
+  for (int i = 0; i < DPL; ++i) o[i] = 0.f;
+  const bool col_ok = lane < DH;
+#pragma unroll 1
+  for (int cb = 0; cb < nch; cb += 32) {
+    float w = 0.f;
+    if (cb + lane < nch) {
+      const float2 ml = __ldcg(a.part_ml + base + cb + lane);
+      if (ml.y > 0.f) {
+        w = expf(ml.x - m);
+        l = fmaf(ml.y, w, l);
       }
     }
+    const int nb = min(32, nch - cb);
+#pragma unroll 1
+    for (int j0 = 0; j0 < nb; j0 += 4) {
+      float ov[4][DPL], wj[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wj[j] = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
+        const int ch = cb + min(j0 + j, nb - 1);
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) ov[j][i] = col_ok ? __ldcg(a.part_o + (base + ch) * DH + lane + 32 * i) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (j0 + j < nb)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) o[i] = fmaf(ov[j][i], wj[j], o[i]);
+    }
   }
-  a.att[(size_t)row * a.d + h * a.dh + c] = o / l;
+  l = warp_sum(l);
+  if (col_ok)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) a.att[(size_t)row * a.d + h * DH + lane + 32 * i] = o[i] / l;
 }
 
 // grid (H, chunks, groups); 128 threads.
@@ -594,11 +634,12 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   attn_partial_compute<DH, KVT>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128, [] { __syncthreads(); });
 }
 
-// grid (rows_max, H), block dh.
-__global__ void k_attn_combine(AttnArgs a) {
+// grid (rows_max, H), one warp.
+template <int DH>
+__global__ void __launch_bounds__(32) k_attn_combine(AttnArgs a) {
   const int row = blockIdx.x;
   if (row >= *a.rows.n_rows) return;
-  attn_combine_one(a, row, blockIdx.y, threadIdx.x);
+  attn_combine_row<DH>(a, row, blockIdx.y, threadIdx.x);
 }
 
 // ------------------------------------------------------------------------ byte head statistics

@@ -184,13 +184,16 @@ __device__ __forceinline__ bool warp_wait(const MegaArgs& m, int n, FlagFn flag,
 constexpr int kTraceEvents = 1024;
 __shared__ int s_trace_n;  // this CTA's event count of the traced pass (debug only)
 // Event word: code << 48 | low 48 bits of %globaltimer.  Recorded by thread 0 in pass 0.
+// Compiled in only with -DBLTDEC_MEGA_TRACE (the marks cost instruction-cache space).
 __device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code) {
+#ifdef BLTDEC_MEGA_TRACE
   if (m.trace && pass == 0 && threadIdx.x == 0) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     const int i = s_trace_n++;
     if (i < kTraceEvents) m.trace[(size_t)blockIdx.x * kTraceEvents + i] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
   }
+#endif
 }
 enum TraceCode : int {
   TR_PASS = 1, TR_PHASE_BEGIN = 2, TR_INPUTS = 3, TR_XBUILT = 4, TR_KLOOP = 5, TR_REDUCED = 6, TR_UNIT_DONE = 7,
@@ -267,11 +270,14 @@ __device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* 
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!ok || go == 0u) break;
     }
+#pragma unroll 1
     for (int ph = 0; ph <= 4 * m.L && ok; ++ph) {
       const Phase p = phase_of(m, ph);
       const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+#pragma unroll 1
       for (int u = first_unit(p, cta, G); u < p.units && ok; u += G) {
         const unsigned char* src = reinterpret_cast<const unsigned char*>(p.w) + (size_t)u * p.ksteps * tile_bytes;
+#pragma unroll 1
         for (int st = 0; st < nst; ++st, ++it) {
           const int slot = it % S;
           const unsigned tiles = min(kStageTiles, p.ksteps - st * kStageTiles);
@@ -292,6 +298,7 @@ __device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* 
   if (lane == 0) {
     const unsigned issued = it;
     const unsigned from = issued > (unsigned)S ? issued - S : 0;
+#pragma unroll 1
     for (unsigned j = from; j < issued; ++j) {
       unsigned n = 0;
       while (!mbar_try(full + j % S, (j / S) & 1) && ++n < kSpinLimit) {
@@ -535,44 +542,27 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
       if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
       const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
       const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
+      // ntiles is a multiple of 8 (the persistent path requires K % 128 == 0):
+      // groups of eight k-steps, one per accumulator, all fragment loads
+      // first, then the independent MMA chains
+      constexpr int GS = (NG * PL > 1) ? 4 : 8;
+#pragma unroll 1
       for (int t8 = 0; t8 < ntiles; t8 += 8) {
-        if (t8 + 8 <= ntiles) {
-          // a full group of eight k-steps (one per accumulator): all fragment
-          // loads first, then the independent MMA chains
-          constexpr int GS = (NG * PL > 1) ? 4 : 8;
 #pragma unroll
-          for (int j0 = 0; j0 < 8; j0 += GS) {
-            uint4 w[GS][PL], xv[GS][NG];
+        for (int j0 = 0; j0 < 8; j0 += GS) {
+          uint4 w[GS][PL], xv[GS][NG];
 #pragma unroll
-            for (int jj = 0; jj < GS; ++jj) {
-              const int tile = t8 + j0 + jj;
+          for (int jj = 0; jj < GS; ++jj) {
+            const int tile = t8 + j0 + jj;
 #pragma unroll
-              for (int q = 0; q < PL; ++q)
-                w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+            for (int q = 0; q < PL; ++q) w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
 #pragma unroll
-              for (int n = 0; n < NG; ++n) xv[jj][n] = sm.xs[((st * kStageTiles + tile) * NG + n) * 32 + lane];
-            }
-#pragma unroll
-            for (int jj = 0; jj < GS; ++jj)
-#pragma unroll
-              for (int n = 0; n < NG; ++n) mma_step<PL>(acc[j0 + jj][n], w[jj], XFrag{xv[jj][n].x, xv[jj][n].y, xv[jj][n].z, xv[jj][n].w});
+            for (int n = 0; n < NG; ++n) xv[jj][n] = sm.xs[((st * kStageTiles + tile) * NG + n) * 32 + lane];
           }
-        } else {
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int tile = t8 + jj;
-            if (tile < ntiles) {
-              const int s = st * kStageTiles + tile;  // s mod 8 == jj
-              uint4 w[PL];
+          for (int jj = 0; jj < GS; ++jj)
 #pragma unroll
-              for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
-#pragma unroll
-              for (int n = 0; n < NG; ++n) {
-                const uint4 xv = sm.xs[(s * NG + n) * 32 + lane];
-                mma_step<PL>(acc[jj][n], w, XFrag{xv.x, xv.y, xv.z, xv.w});
-              }
-            }
-          }
+            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[j0 + jj][n], w[jj], XFrag{xv[jj][n].x, xv[jj][n].y, xv[jj][n].z, xv[jj][n].w});
         }
       }
       __syncwarp();
@@ -747,7 +737,7 @@ __device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, 
     consumer_sync();
     if (sm.misc[0]) {
       const int row0 = __ldcg(m.rows.g_row0 + g), nr = __ldcg(m.rows.g_nrows + g);
-      for (int i = tid; i < nr * DH; i += 256) attn_combine_one(a, row0 + i / DH, h, i % DH);
+      for (int r = tid >> 5; r < nr; r += 8) attn_combine_row<DH>(a, row0 + r, h, tid & 31);
       consumer_sync();
       if (tid == 0) {
         m.attn_cnt[g * m.H + h] = 0u;
@@ -897,32 +887,40 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     }
     consumer_sync();
     trace_mark(m, pass, TR_PASS << 8);
-    for (int l = 0; l < m.L && ok; ++l) {
-      GemmArgs ga = m.ga;
-      ga.layer = l;
-      ga.row_seq = sm.rseq;
-      ga.row_pos = sm.rpos;
-      ga.row_lat = sm.rlat;
-      ga.row_byte = sm.rbyte;
-      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l), EPI_QKV, pass, it, nr, n_groups, ga, m.flags + m.f_qkv, tid) && ok;
-      ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
-      ga.out = m.h;
-      ga.ldo = m.d;
-      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l + 1), EPI_XRESID, pass, it, nr, n_groups, ga, m.flags + m.f_o, tid) && ok;
-      ga.out = m.act;
-      ga.ldo = m.F;
-      ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * l + 2), EPI_SWIGLU, pass, it, nr, n_groups, ga, m.flags + m.f_w13, tid) && ok;
-      ga.out = m.h;
-      ga.ldo = m.d;
-      const Phase p2 = phase_of(m, 4 * l + 3);
-      if (p2.ksteps <= 64) ok = run_phase_units<NG, PL>(m, sm, p2, EPI_RESID, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
-      else ok = run_phase_streamed<NG, PL>(m, sm, p2, pass, it, nr, n_groups, ga, m.flags + m.f_w2, tid) && ok;
+    // Steps of a pass: per layer QKV, attention, O, W13, W2; then the byte
+    // head.  One call site per routine keeps a single copy of each in the
+    // kernel, small enough for the SM's instruction caches.
+    GemmArgs ga = m.ga;
+    ga.row_seq = sm.rseq;
+    ga.row_pos = sm.rpos;
+    ga.row_lat = sm.rlat;
+    ga.row_byte = sm.rbyte;
+    for (int step = 0; step <= 5 * m.L && ok; ++step) {
+      const int l = step / 5, k = step - 5 * l;
+      if (k == 1) {
+        ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
+        continue;
+      }
+      const bool head = l == m.L;
+      const Phase p = phase_of(m, head ? 4 * m.L : 4 * l + (k == 0 ? 0 : k - 1));
+      ga.layer = head ? 0 : l;
+      int epi = EPI_STORE;
+      unsigned* fb = m.flags + m.f_head;
+      if (head) {
+        ga.out = m.logits, ga.ldo = 256;
+      } else if (k == 0) {
+        epi = EPI_QKV, fb = m.flags + m.f_qkv;
+      } else if (k == 2) {
+        epi = EPI_XRESID, fb = m.flags + m.f_o, ga.out = m.h, ga.ldo = m.d;
+      } else if (k == 3) {
+        epi = EPI_SWIGLU, fb = m.flags + m.f_w13, ga.out = m.act, ga.ldo = m.F;
+      } else {
+        epi = EPI_RESID, fb = m.flags + m.f_w2, ga.out = m.h, ga.ldo = m.d;
+      }
+      if (k == 4 && !head && p.ksteps > 64) ok = run_phase_streamed<NG, PL>(m, sm, p, pass, it, nr, n_groups, ga, fb, tid) && ok;
+      else ok = run_phase_units<NG, PL>(m, sm, p, epi, pass, it, nr, n_groups, ga, fb, tid) && ok;
     }
     if (!ok) break;
-    GemmArgs ga = m.ga;
-    ga.out = m.logits;
-    ga.ldo = 256;
-    ok = run_phase_units<NG, PL>(m, sm, phase_of(m, 4 * m.L), EPI_STORE, pass, it, nr, n_groups, ga, m.flags + m.f_head, tid) && ok;
     trace_mark(m, pass, TR_HEAD << 8);
     if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
     trace_mark(m, pass, TR_BOOK << 8);

@@ -130,6 +130,7 @@ typedef struct {
   uint64_t kernel_launches; /* engine kernels launched (host count) */
   uint64_t timed_passes;   /* decoder passes inside timed calls (BLT_FLAG_TIME_PASSES) */
   uint64_t pass_ns;        /* summed device time of those calls' passes, ns (latent projection excluded) */
+  uint64_t persistent_calls; /* calls whose decoder passes ran in the persistent kernel (BLT_FLAG_PERSISTENT) */
 } blt_dec_counters;
 
 /* Create an engine.  Copies and re-lays out the weights on the device

@@ -51,7 +51,7 @@ def test_struct_layouts_match_header():
     assert ctypes.sizeof(B.blt_dec_config) == 18 * 4
     assert ctypes.sizeof(B.blt_dec_weights) == 4 * 8
     assert ctypes.sizeof(B.blt_rows_in) == 5 * 8
-    assert ctypes.sizeof(B.blt_dec_counters) == 10 * 8
+    assert ctypes.sizeof(B.blt_dec_counters) == 11 * 8
 
 
 def test_init_rejects_bad_config_without_touching_the_gpu(lib):

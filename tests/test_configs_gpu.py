@@ -57,11 +57,22 @@ def _check(got, want, o, wl, what):
     assert near, f"{what}: differs at byte {i} without a flagged near-tie"
 
 
-def test_config2_full_job(dec9):
-    """BLT-D-4, prefix 1024, all 512 bytes: the configuration bench.py times."""
+@pytest.mark.parametrize("persistent", [True, False], ids=["persistent", "phased"])
+def test_config2_full_job(dec9, persistent):
+    """BLT-D-4, prefix 1024, all 512 bytes: the configuration bench.py times (persistent kernel by default)."""
+    from block_diffusion_byte_b200.driver import Engine, generate
+
     ws, om = dec9
     wl = CONFIGS["d4_b1"]
-    res = _engine_run(wl, ws, wl.gen_bytes, [0])
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + wl.gen_bytes + 4 * wl.block + 16, max_block=16,
+                 max_rows=1024, persistent=persistent)
+    try:
+        res = generate(eng, wl, [_prefix(wl, 0)], wl.gen_bytes, seq_ids=[0])
+        from block_diffusion_byte_b200 import binding as B
+
+        assert (B.blt_dec_stats(eng.h)["persistent_calls"] > 0) == persistent
+    finally:
+        eng.close()
     want, o = _oracle_run(wl, om, 0, wl.gen_bytes)
     _check(res.out[0], want, o, wl, "config 2")
 
@@ -80,12 +91,14 @@ def test_config3_dv16_batch8(dec9):
     assert ar.out == res.out
 
 
-def test_config4_s8_batch16(dec9):
-    """BLT-S k=8, prefix 4096, batch 16: byte-identical to AR greedy on the engine; oracle on one sequence."""
+@pytest.mark.parametrize("persistent", [False, True], ids=["phased", "persistent"])
+def test_config4_s8_batch16(dec9, persistent):
+    """BLT-S k=8, prefix 4096, batch 16: byte-identical to AR greedy on the engine; oracle on one sequence.
+    With the persistent kernel the 16-row drafting passes run in it (two row groups)."""
     ws, om = dec9
     wl = CONFIGS["s8_b16"]
     G = 48
-    res = _engine_run(wl, ws, G, list(range(16)))
+    res = _engine_run(wl, ws, G, list(range(16)), persistent=persistent)
     ar = _engine_run(replace(wl, mode="AR", block=1), ws, G, list(range(16)))
     assert res.out == ar.out
     want, o = _oracle_run(replace(wl, mode="AR", block=1), om, 3, G)
