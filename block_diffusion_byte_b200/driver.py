@@ -27,7 +27,7 @@ from typing import List, Optional, Sequence
 import numpy as np
 import torch
 
-from workload import ModelShape, Patcher, PatchState, WeightSet, Workload, latent_vector
+from workload import ModelShape, Patcher, PatchState, WeightSet, Workload, latent_vectors
 
 from . import binding as B
 
@@ -159,12 +159,14 @@ class SeqHost:
         """Latent slots of ``data`` appended after ``state`` and latents of the patches it closes."""
         per, st = self.patcher.advance(state, data)
         n = state.n_closed
-        slots, lats = [], []
+        slots, new_slots, new_fnvs = [], [], []
         for closes, fnv in per:
             if closes:
-                lats.append(latent_vector(self.seed, self.cfg_index, self.seq, n, fnv, self.d_global))
+                new_slots.append(n)
+                new_fnvs.append(fnv)
                 n += 1
             slots.append(n - 1)
+        lats = list(latent_vectors(self.seed, self.cfg_index, self.seq, new_slots, new_fnvs, self.d_global))
         return slots, lats, st
 
     def commit(self, data: Sequence[int]) -> None:

@@ -84,3 +84,27 @@ def test_prefix_uniform():
     x = prefix_bytes(0, 1, 0, 1 << 16)
     counts = np.bincount(x, minlength=256)
     assert counts.min() > 150 and counts.max() < 370
+
+
+def test_scalar_and_batched_generators_agree():
+    """The scalar SplitMix64 path (patcher, key derivation) equals the array form,
+    and latents generated together equal latents generated one at a time."""
+    from workload.gen import latent_vector, latent_vectors
+    from workload.rng import GAMMA, derive_keys, mix64, stream, stream_int
+
+    rng = np.random.default_rng(5)
+    keys = rng.integers(0, 2**63, 64, dtype=np.uint64) * np.uint64(2) + np.uint64(1)
+    for k in keys[:16]:
+        for i in (0, 1, 7, 1023, 2**40):
+            assert stream_int(int(k), i) == int(stream(int(k), i, 1)[0])
+    words = [(3, 4, 1, 9, int(s), int(f)) for s, f in zip(range(20), keys[:20])]
+    batched = derive_keys(3, 4, 1, 9, [w[4] for w in words], [w[5] for w in words])
+    for w, kb in zip(words, batched):
+        h = np.array([0], dtype=np.uint64)
+        with np.errstate(over="ignore"):
+            for x in w:
+                h = mix64((h ^ np.uint64(x & 0xFFFFFFFFFFFFFFFF)) + GAMMA)
+        assert int(h[0]) == int(kb)
+    a = latent_vectors(0, 1, 3, list(range(12)), [int(k) for k in keys[:12]], 256)
+    b = np.stack([latent_vector(0, 1, 3, i, int(k), 256) for i, k in enumerate(keys[:12])])
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))

@@ -24,4 +24,5 @@ from .gen import (  # noqa: F401
     Patcher,
     prefix_bytes,
     latent_vector,
+    latent_vectors,
 )

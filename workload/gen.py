@@ -33,7 +33,7 @@ from typing import Dict, List, Sequence, Tuple
 import numpy as np
 
 from .configs import ModelShape
-from .rng import FNV_OFFSET, derive_key, fnv1a64, normals, round_bf16, stream
+from .rng import FNV_OFFSET, derive_key, derive_keys, fnv1a64, normals, normals_many, round_bf16, stream, stream_int
 
 STREAM_WEIGHT = 1
 STREAM_PREFIX = 2
@@ -167,7 +167,7 @@ class Patcher:
 
     def _u32(self, j: int, b: int) -> int:
         k = (self.key ^ (int(b) & 0xFF)) & 0xFFFFFFFFFFFFFFFF
-        return int(stream(k, j, 1)[0] >> np.uint64(32))
+        return stream_int(k, j) >> 32
 
     def advance(self, st: PatchState, data: Sequence[int]) -> Tuple[List[Tuple[bool, int]], PatchState]:
         """Patch ``data`` appended after state ``st``.
@@ -191,5 +191,12 @@ class Patcher:
 
 def latent_vector(seed: int, cfg_index: int, seq: int, slot: int, fnv: int, d_global: int) -> np.ndarray:
     """Latent for 0-based slot ``slot`` closed with content hash ``fnv`` (float32)."""
-    key = derive_key(seed, STREAM_LATENT, cfg_index, seq, slot, fnv)
-    return normals(key, d_global).astype(np.float32)
+    return latent_vectors(seed, cfg_index, seq, [slot], [fnv], d_global)[0]
+
+
+def latent_vectors(seed: int, cfg_index: int, seq: int, slots: Sequence[int], fnvs: Sequence[int], d_global: int) -> np.ndarray:
+    """``latent_vector`` for every (slot, fnv) pair at once: float32 [n, d_global]."""
+    if len(slots) == 0:
+        return np.zeros((0, d_global), dtype=np.float32)
+    keys = derive_keys(seed, STREAM_LATENT, cfg_index, seq, list(slots), list(fnvs))
+    return normals_many(keys, d_global).astype(np.float32)

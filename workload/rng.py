@@ -33,13 +33,40 @@ def mix64(z: np.ndarray) -> np.ndarray:
     return z ^ (z >> _S31)
 
 
+_MASK = 0xFFFFFFFFFFFFFFFF
+
+
+def mix64_int(z: int) -> int:
+    """``mix64`` of one value in Python integers (exact, same result as the array form)."""
+    z &= _MASK
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK
+    return z ^ (z >> 31)
+
+
+def stream_int(key: int, i: int) -> int:
+    """Element ``i`` of the counter stream ``key`` (one value, Python integers)."""
+    return mix64_int(key + (i + 1) * 0x9E3779B97F4A7C15)
+
+
 def derive_key(*words: int) -> int:
     """Chain ``mix64`` over integer words into one 64-bit stream key."""
-    h = np.array([0], dtype=np.uint64)
+    h = 0
+    for w in words:
+        h = mix64_int(((h ^ (int(w) & _MASK)) + 0x9E3779B97F4A7C15) & _MASK)
+    return h
+
+
+def derive_keys(*columns) -> np.ndarray:
+    """``derive_key`` over rows of words: column ``j`` holds word ``j`` of every key
+    (ints broadcast).  Elementwise the same operations as ``derive_key``."""
+    n = max((len(c) for c in columns if not np.isscalar(c)), default=1)
+    h = np.zeros(n, dtype=np.uint64)
     with np.errstate(over="ignore"):
-        for w in words:
-            h = mix64((h ^ np.uint64(int(w) & 0xFFFFFFFFFFFFFFFF)) + GAMMA)
-    return int(h[0])
+        for c in columns:
+            w = np.asarray([int(v) & 0xFFFFFFFFFFFFFFFF for v in (c if not np.isscalar(c) else [c] * n)], dtype=np.uint64)
+            h = mix64((h ^ w) + GAMMA)
+    return h
 
 
 def stream(key: int, start: int, count: int) -> np.ndarray:
@@ -61,16 +88,24 @@ def normals(key: int, count: int) -> np.ndarray:
     ``r = sqrt(-2 ln(1 - u_a))``, ``t = 2 pi u_b``; element ``2p`` is
     ``r cos t`` and element ``2p+1`` is ``r sin t``.
     """
+    return normals_many(np.asarray([key], dtype=np.uint64), count)[0]
+
+
+def normals_many(keys: np.ndarray, count: int) -> np.ndarray:
+    """``normals`` of every key in ``keys`` at once: float64 [len(keys), count]."""
+    keys = np.asarray(keys, dtype=np.uint64).reshape(-1, 1)
     npair = (count + 1) // 2
-    raw = stream(key, 0, 2 * npair).reshape(npair, 2)
-    u1 = 1.0 - uniform53(raw[:, 0])  # (0, 1]
-    u2 = uniform53(raw[:, 1])
+    i = np.arange(1, 2 * npair + 1, dtype=np.uint64).reshape(1, -1)
+    with np.errstate(over="ignore"):
+        raw = mix64(keys + i * GAMMA).reshape(keys.shape[0], npair, 2)
+    u1 = 1.0 - uniform53(raw[:, :, 0])  # (0, 1]
+    u2 = uniform53(raw[:, :, 1])
     r = np.sqrt(-2.0 * np.log(u1))
     t = (2.0 * np.pi) * u2
-    out = np.empty((npair, 2), dtype=np.float64)
-    out[:, 0] = r * np.cos(t)
-    out[:, 1] = r * np.sin(t)
-    return out.reshape(-1)[:count]
+    out = np.empty((keys.shape[0], npair, 2), dtype=np.float64)
+    out[:, :, 0] = r * np.cos(t)
+    out[:, :, 1] = r * np.sin(t)
+    return out.reshape(keys.shape[0], -1)[:, :count]
 
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
