@@ -624,7 +624,7 @@ __global__ void k_copy_logits(const float* src, float* dst, int n) {
 template <int NG, int PL, int DH, typename KVT>
 size_t mega_smem(const blt_dec* h) {
   const size_t attn = (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * kv_stride<DH, KVT>() * sizeof(KVT);
-  const size_t xin = (size_t)64 * NG * 32 * 16;  // phase input fragments, K <= 1024
+  const size_t xin = (size_t)kMegaUnits * 8 * 16 * 8 * NG * 4;  // multi-unit reduction buffer
   return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + 16 * 4 + std::max(attn, xin);
 }
 
@@ -646,7 +646,8 @@ int mega_prepare_pd(blt_dec* h) {
 
 // Decide whether the persistent kernel applies to this model and set it up.
 int mega_setup(blt_dec* h) {
-  if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || h->d % 128 != 0 || h->F % 128 != 0 || (h->dh != 32 && h->dh != 64) ||
+  if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || h->d % 128 != 0 || h->F % 128 != 0 || h->F > 4096 ||
+      (h->dh != 32 && h->dh != 64) ||
       h->CH > 128)
     return BLT_OK;
   int dev = 0;

@@ -104,8 +104,10 @@ struct GemmArgs {
   const int* row_pos;
   const int* row_lat;
   const int* row_byte;
-  const float* rope_cos;  // [max_ctx][dh/2]
+  const float* rope_cos;  // [max_ctx][dh/2], or [row][dh/2] when rope_by_row
   const float* rope_sin;
+  int rope_by_row;      // rope tables indexed by activation row (per-pass copy) instead of position
+  const int* row_page;  // KV page of each row's position (-1: none); NULL: look up page_table
   // EPI_LATC
   const int* lat_seq;
   const int* lat_slot;
@@ -149,6 +151,13 @@ __device__ __forceinline__ void kv_store(const GemmArgs& a, size_t off, float v)
   else static_cast<__nv_bfloat16*>(a.kv)[off] = __float2bfloat16_rn(v);
 }
 
+// KV page holding position `pos` of `seq` (-1: not allocated).
+__device__ __forceinline__ int row_kv_page(const GemmArgs& a, int row, int seq, int pos) {
+  if (a.row_page) return a.row_page[row];
+  const int pi = pos / a.PT;
+  return (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+}
+
 // Output pair of tile rows (r16, r16 + 8) of tile mt for activation row `row`.
 // Row metadata pointers may point to shared memory (persistent kernel copies).
 template <int EPI>
@@ -184,7 +193,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
       const int tph = a.dh / 16;
       const int h = lt / tph, j = (lt % tph) * 8 + r16;
       const int half = a.dh / 2;
-      const float c = a.rope_cos[(size_t)pos * half + j], s = a.rope_sin[(size_t)pos * half + j];
+      const size_t ri = (size_t)(a.rope_by_row ? row : pos) * half + j;
+      const float c = a.rope_cos[ri], s = a.rope_sin[ri];
       const float o0 = v0 * c - v1 * s, o1 = v1 * c + v0 * s;
       if (sec == 0) {
         float* q = a.q + (size_t)row * a.d + h * a.dh;
@@ -192,8 +202,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         q[j + half] = o1;
         return;
       }
-      const int pi = pos / a.PT;
-      const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+      const int page = row_kv_page(a, row, seq, pos);
       if (page < 0) {
         set_status(a.status, kErrDevice);
         return;
@@ -202,8 +211,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
       kv_store(a, off + j, o0);
       kv_store(a, off + j + half, o1);
     } else {
-      const int pi = pos / a.PT;
-      const int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+      const int page = row_kv_page(a, row, seq, pos);
       if (page < 0) {
         set_status(a.status, kErrDevice);
         return;

@@ -151,6 +151,10 @@ __device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
   return v;
 }
 __device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
+__device__ __forceinline__ void st_relaxed(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
 
 // Warp-wide wait until flag(i) >= target for every i < n: each lane polls
 // its share with relaxed loads (all in flight at once), then one acquire
@@ -421,15 +425,15 @@ __device__ __forceinline__ void mega_epilogue(const GemmArgs& ga, int epi, int u
   }
 }
 
-// Phase input of this warp's k-steps warp, warp + 8, ... (nkw of them) as
-// split-bf16 fragments in shared memory, and its share of every row's sum of
-// squares.  Every load is issued unconditionally (a dead row reads row 0, a
-// k-step past the warp's share re-reads its last one; neither is stored) so
-// the compiler can put them all in flight at once.  HASC: QKV input, which
-// adds the cross term c_l.
+// Phase input of this warp's k-steps warp, warp + 8, ... (nkw <= 8 of them) as
+// split-bf16 B fragments in registers, and its lanes' sums of squares (the
+// canonical order: per lane, k-steps in increasing order).  Every load is
+// issued unconditionally (a dead row reads row 0, a k-step past the warp's
+// share re-reads its last one; neither reaches an output) so all are in
+// flight at once.  HASC: QKV input, which adds the cross term c_l.
 template <int NG, bool HASC>
-__device__ __forceinline__ void build_inputs(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int nr, int nkw,
-                                             const float* gain, float (&ss)[NG], int warp, int lane) {
+__device__ __forceinline__ void build_frags(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int nr, int nkw,
+                                            const float* gain, uint4 (&xf)[8][NG], float (&ss)[NG], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const bool norm = gain != nullptr;
   XSrc src[NG];
@@ -439,160 +443,167 @@ __device__ __forceinline__ void build_inputs(const MegaArgs& m, const MegaSmem& 
     const int row = n * 8 + g;
     src[n] = x_src(m, sm, p, row < nr ? row : 0);
   }
-#pragma unroll 1
-  for (int half = 0; half < 2 && half * 4 < nkw; ++half) {
-    float2 ra[4][NG], rb[4][NG];
-    float4 gv[4];
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int j = min(half * 4 + jj, nkw - 1);
-      const int k0 = (warp + 8 * j) * 16 + 2 * t;
+  for (int half = 0; half < 2; ++half) {
+    if (half * 4 < nkw) {
+      float2 ra[4][NG], rb[4][NG];
+      float4 gv[4];
 #pragma unroll
-      for (int n = 0; n < NG; ++n) {
-        ra[jj][n] = ld2(src[n].a + k0);
-        rb[jj][n] = ld2(src[n].a + k0 + 8);
-        if constexpr (HASC) {
-          const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
-          ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
-          rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = min(half * 4 + jj, nkw - 1);
+        const int k0 = (warp + 8 * j) * 16 + 2 * t;
+#pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          ra[jj][n] = ld2(src[n].a + k0);
+          rb[jj][n] = ld2(src[n].a + k0 + 8);
+          if constexpr (HASC) {
+            const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
+            ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
+            rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
+          }
         }
+        gv[jj] = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (norm) gv[jj] = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
       }
-      gv[jj] = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (norm) gv[jj] = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
-    }
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int j = half * 4 + jj;
-      if (j < nkw) {
-        const int s = warp + 8 * j;
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = half * 4 + jj;
 #pragma unroll
         for (int n = 0; n < NG; ++n) {
           const float2 a = ra[jj][n], b = rb[jj][n];
-          if (norm) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
+          if (norm && j < nkw) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
           const XFrag f = make_xfrag(a.x * gv[jj].x, a.y * gv[jj].y, b.x * gv[jj].z, b.y * gv[jj].w);
-          sm.xs[(s * NG + n) * 32 + lane] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
+          xf[j][n] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
         }
       }
     }
   }
 }
 
-// Phase with K <= 1024.  (1) The CTA's eight warps build the phase input once
-// in shared memory as split-bf16 fragments, warp w building k-steps w, w+8,
-// ... and its share of every row's sum of squares (the canonical order).
-// (2) Each warp then runs whole units alone: it keeps one accumulator per
-// lane group (k-step mod 8), adds them in lane-group order, scales by the
-// row's RMS factor and applies the epilogue to the values it holds -- the
-// same arithmetic as the 8-warp reduction, with no block-wide step -- and
-// releases the unit's flag.
+// Phase with K <= 1024 (at most two ring stages per unit).  All eight warps
+// work on every unit: warp w owns the k-steps s = w (mod 8) -- lane group w
+// of the canonical order -- so it waits only for the inputs of its own
+// k-steps and keeps their fragments in registers.  The CTA's units (up to
+// kMegaUnits at a time) run together: one accumulator per unit per warp, so
+// the units' MMA chains interleave; then one cross-warp reduction (the
+// operation order of tile_reduce: warps in order, the RMS scale from the
+// warps' sums of squares in order), one epilogue pass, one fence and the
+// units' flags.
+constexpr int kMegaUnits = 4;
+
 template <int NG, int PL>
 __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int epi, int pass, unsigned& it, int nr,
                                 int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
+  constexpr int RB = 8 * NG;
   const int G = gridDim.x, cta = blockIdx.x;
   const int u0 = first_unit(p, cta, G);
   if (u0 >= p.units) return true;
   const int nunits = (p.units - u0 + G - 1) / G;
-  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // 1 or 2
   const unsigned it0 = it;
   it += (unsigned)(nunits * nst);
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
   const float* gain = phase_gain(m, p);
   const bool norm = gain != nullptr;
-  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps this warp builds (<= 8)
+  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps of this warp (<= 8)
   trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
   bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);
   trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
+  uint4 xf[8][NG];
   float ss[NG];
-  if (p.kind == PH_QKV) build_inputs<NG, true>(m, sm, p, nr, nkw, gain, ss, warp, lane);
-  else build_inputs<NG, false>(m, sm, p, nr, nkw, gain, ss, warp, lane);
-  trace_mark(m, pass, TR_XLOADED << 8 | p.kind);
+  if (p.kind == PH_QKV) build_frags<NG, true>(m, sm, p, nr, nkw, gain, xf, ss, warp, lane);
+  else build_frags<NG, false>(m, sm, p, nr, nkw, gain, xf, ss, warp, lane);
   if (norm) {
 #pragma unroll
     for (int n = 0; n < NG; ++n) {
       float v = ss[n];
       v += __shfl_xor_sync(0xffffffffu, v, 1);
       v += __shfl_xor_sync(0xffffffffu, v, 2);
-      if (t == 0) sm.ssr[warp * 16 + n * 8 + g] = v;
+      if (t == 0) sm.ssr[warp * RB + n * 8 + g] = v;
     }
   }
-  consumer_sync();
-  if (tid < 16) {
-    float r = 1.0f;
-    if (norm) {
-      float v = sm.ssr[tid];
-#pragma unroll
-      for (int w = 1; w < kWarps; ++w) v += sm.ssr[w * 16 + tid];
-      r = 1.0f / sqrtf(v / (float)(p.ksteps * 16) + m.eps);
-    }
-    sm.rsv[tid] = r;
-  }
-  consumer_sync();
-  trace_mark(m, pass, TR_XBUILT << 8 | p.kind);
+  trace_mark(m, pass, TR_XLOADED << 8 | p.kind);
   const unsigned tile_bytes = 512u * PL;
-  for (int j = warp; j < nunits; j += kWarps) {
-    const int u = u0 + j * G;
-    float acc[8][NG][4];
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int n = 0; n < NG; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
-    for (int st = 0; st < nst; ++st) {
-      const unsigned itu = it0 + (unsigned)(j * nst + st);
-      const int slot = itu % sm.S;
-      if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
-      const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-      const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
-      // ntiles is a multiple of 8 (the persistent path requires K % 128 == 0):
-      // groups of eight k-steps, one per accumulator, all fragment loads
-      // first, then the independent MMA chains
-      constexpr int GS = (NG * PL > 1) ? 4 : 8;
+  float* red = reinterpret_cast<float*>(sm.xs);  // [unit][warp][16][RB]
 #pragma unroll 1
-      for (int t8 = 0; t8 < ntiles; t8 += 8) {
+  for (int ug = 0; ug < nunits; ug += kMegaUnits) {
+    const int nu = min(kMegaUnits, nunits - ug);
+    float acc[kMegaUnits][NG][4];
 #pragma unroll
-        for (int j0 = 0; j0 < 8; j0 += GS) {
-          uint4 w[GS][PL], xv[GS][NG];
+    for (int jv = 0; jv < kMegaUnits; ++jv)
 #pragma unroll
-          for (int jj = 0; jj < GS; ++jj) {
-            const int tile = t8 + j0 + jj;
+      for (int n = 0; n < NG; ++n) acc[jv][n][0] = acc[jv][n][1] = acc[jv][n][2] = acc[jv][n][3] = 0.f;
 #pragma unroll
-            for (int q = 0; q < PL; ++q) w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+    for (int st = 0; st < 2; ++st) {
+      if (st < nst) {
+        const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
 #pragma unroll
-            for (int n = 0; n < NG; ++n) xv[jj][n] = sm.xs[((st * kStageTiles + tile) * NG + n) * 32 + lane];
+        for (int jv = 0; jv < kMegaUnits; ++jv) {
+          if (jv < nu) {
+            const unsigned itu = it0 + (unsigned)((ug + jv) * nst + st);
+            const int slot = itu % sm.S;
+            if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
+            const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+            uint4 w[4][PL];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int pl = 0; pl < PL; ++pl)
+                w[q][pl] = *reinterpret_cast<const uint4*>(stage + (size_t)min(8 * q + warp, ntiles - 1) * tile_bytes + pl * 512 + lane * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (8 * q + warp < ntiles)
+#pragma unroll
+                for (int n = 0; n < NG; ++n)
+                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[st * 4 + q][n].x, xf[st * 4 + q][n].y, xf[st * 4 + q][n].z, xf[st * 4 + q][n].w});
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.empty + slot);
           }
-#pragma unroll
-          for (int jj = 0; jj < GS; ++jj)
-#pragma unroll
-            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[j0 + jj][n], w[jj], XFrag{xv[jj][n].x, xv[jj][n].y, xv[jj][n].z, xv[jj][n].w});
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_n(sm.empty + slot, kMegaConsumers);
     }
 #pragma unroll
-    for (int n = 0; n < NG; ++n) {
-      float v[4] = {acc[0][n][0], acc[0][n][1], acc[0][n][2], acc[0][n][3]};
+    for (int jv = 0; jv < kMegaUnits; ++jv) {
+      if (jv < nu) {
+        float* rw = red + (size_t)(jv * 8 + warp) * 16 * RB;
 #pragma unroll
-      for (int a = 1; a < 8; ++a) {
-        v[0] += acc[a][n][0];
-        v[1] += acc[a][n][1];
-        v[2] += acc[a][n][2];
-        v[3] += acc[a][n][3];
-      }
-      const int c0 = n * 8 + 2 * t;
-      if (c0 < nr) {
-        const float r = sm.rsv[c0];
-        mega_epilogue(ga, epi, u, g, c0, v[0] * r, v[2] * r);
-      }
-      if (c0 + 1 < nr) {
-        const float r = sm.rsv[c0 + 1];
-        mega_epilogue(ga, epi, u, g, c0 + 1, v[1] * r, v[3] * r);
+        for (int n = 0; n < NG; ++n) {
+          const int c = n * 8 + 2 * t;
+          rw[g * RB + c] = acc[jv][n][0];
+          rw[g * RB + c + 1] = acc[jv][n][1];
+          rw[(g + 8) * RB + c] = acc[jv][n][2];
+          rw[(g + 8) * RB + c + 1] = acc[jv][n][3];
+        }
       }
     }
-    __syncwarp();
-    if (lane == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
-    if (warp == 0) trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
+    consumer_sync();
+    for (int pi = tid; pi < nu * 8 * RB; pi += 256) {
+      const int jv = pi / (8 * RB), q = pi % (8 * RB);
+      const int r16 = q & 7, col = q >> 3;
+      if (col >= nr) continue;
+      const float* ru = red + (size_t)jv * 8 * 16 * RB;
+      float v0 = ru[r16 * RB + col], v1 = ru[(r16 + 8) * RB + col];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) {
+        v0 += ru[(w * 16 + r16) * RB + col];
+        v1 += ru[(w * 16 + r16 + 8) * RB + col];
+      }
+      float rs = 1.0f;
+      if (norm) {
+        float sv = sm.ssr[col];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) sv += sm.ssr[w * RB + col];
+        rs = 1.0f / sqrtf(sv / (float)(p.ksteps * 16) + m.eps);
+      }
+      mega_epilogue(ga, epi, u0 + (ug + jv) * G, r16, col, v0 * rs, v1 * rs);
+    }
+    consumer_sync();  // epilogue stores done, red free again
+    if (tid == 0) {
+      fence_acq_rel();
+      for (int jv = 0; jv < nu; ++jv) st_relaxed(flag_base + u0 + (ug + jv) * G, epoch(m, pass, p.layer));
+    }
+    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
   }
-  consumer_sync();  // the input fragments are free again
   return ok;
 }
 
@@ -628,51 +639,59 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
     }
     return ok;
   };
+  // inputs prefetched D stages ahead in registers (an L2 round trip is much
+  // longer than one stage's MMAs); stages run in groups of D so the register
+  // ring is indexed at compile time
+  constexpr int D = 2 / NG;
   for (int u = u0; u < p.units; u += G) {
     float acc[NG][4], ss[NG];
 #pragma unroll
     for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
-    float2 ca[4][NG], cb[4][NG], na[4][NG], nb[4][NG];
-    ok = load(0, ca, cb) && ok;
-    for (int st = 0; st < nst; ++st) {
-      if (st + 1 < nst) ok = load(st + 1, na, nb) && ok;
-      const int slot = it % sm.S;
-      if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
-      const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-      if ((st + 1) * kStageTiles <= p.ksteps) {  // full stage: weight loads first, then the chain
-        uint4 w[4][PL];
+    float2 xa[D][4][NG], xb[D][4][NG];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+    for (int d = 0; d < D; ++d)
+      if (d < nst) ok = load(d, xa[d], xb[d]) && ok;
+#pragma unroll 1
+    for (int s0 = 0; s0 < nst; s0 += D) {
 #pragma unroll
-          for (int q = 0; q < PL; ++q)
-            w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)(8 * jj + warp) * tile_bytes + q * 512 + lane * 16);
+    for (int d = 0; d < D; ++d) {
+      const int st = s0 + d;
+      if (st < nst) {
+        const int slot = it % sm.S;
+        if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
+        const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
+        float2 (&ca)[4][NG] = xa[d];
+        float2 (&cb)[4][NG] = xb[d];
+        if ((st + 1) * kStageTiles <= p.ksteps) {  // full stage: weight loads first, then the chain
+          uint4 w[4][PL];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+          for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-          for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w[jj], make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
-      } else {
+            for (int q = 0; q < PL; ++q)
+              w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)(8 * jj + warp) * tile_bytes + q * 512 + lane * 16);
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int tile = 8 * jj + warp;
-          if (st * kStageTiles + tile < p.ksteps) {
-            uint4 w[PL];
+          for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-            for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w[jj], make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+        } else {
 #pragma unroll
-            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+          for (int jj = 0; jj < 4; ++jj) {
+            const int tile = 8 * jj + warp;
+            if (st * kStageTiles + tile < p.ksteps) {
+              uint4 w[PL];
+#pragma unroll
+              for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
+#pragma unroll
+              for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
+            }
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.empty + slot);
+        ++it;
+        if (st + D < nst) ok = load(st + D, xa[d], xb[d]) && ok;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.empty + slot);
-      ++it;
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          ca[jj][n] = na[jj][n];
-          cb[jj][n] = nb[jj][n];
-        }
+    }
     }
     trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
     tile_reduce<NG>(acc, ss, false, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
@@ -815,6 +834,8 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   __shared__ float mrow[kAttnRows], lrow[kAttnRows];
   __shared__ int lim[kAttnRows];
   __shared__ int rmeta[4][8 * kMegaMaxNG];
+  __shared__ int rpage[8 * kMegaMaxNG];                       // KV page of each row's position
+  __shared__ float rope_c[8 * kMegaMaxNG * 32], rope_s[8 * kMegaMaxNG * 32];  // [row][dh/2], dh <= 64
 
   const unsigned tile_bytes = 512u * PL;
   const unsigned slot_bytes = kStageTiles * tile_bytes;
@@ -828,7 +849,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   p += 8 * 8 * kMegaMaxNG * 4;
   sm.rsv = reinterpret_cast<float*>(p);
   p += 16 * 4;
-  sm.xs = reinterpret_cast<uint4*>(p);  // the phase input shares space with the attention buffers
+  sm.xs = reinterpret_cast<uint4*>(p);  // the phases' reduction buffer shares space with the attention buffers
   sm.qs = reinterpret_cast<float*>(p);
   p += kAttnRows * DH * 4;
   sm.ps = reinterpret_cast<float*>(p);
@@ -886,6 +907,19 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
       sm.rbyte[tid] = live ? __ldcg(m.rows.byte + tid) : 0;
     }
     consumer_sync();
+    {  // this pass's rotary factors and KV pages per row (dead rows: position 0)
+      const int half = m.dh / 2;
+      for (int i = tid; i < 8 * kMegaMaxNG * half; i += 256) {
+        const size_t src = (size_t)sm.rpos[i / half] * half + i % half;
+        rope_c[i] = __ldg(m.ga.rope_cos + src);
+        rope_s[i] = __ldg(m.ga.rope_sin + src);
+      }
+      if (tid < 8 * kMegaMaxNG) {
+        const int pi = sm.rpos[tid] / m.ga.PT;
+        rpage[tid] = (pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + sm.rseq[tid] * m.ga.max_pages + pi) : -1;
+      }
+    }
+    consumer_sync();
     trace_mark(m, pass, TR_PASS << 8);
     // Steps of a pass: per layer QKV, attention, O, W13, W2; then the byte
     // head.  One call site per routine keeps a single copy of each in the
@@ -895,6 +929,10 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     ga.row_pos = sm.rpos;
     ga.row_lat = sm.rlat;
     ga.row_byte = sm.rbyte;
+    ga.rope_cos = rope_c;
+    ga.rope_sin = rope_s;
+    ga.rope_by_row = 1;
+    ga.row_page = rpage;
     for (int step = 0; step <= 5 * m.L && ok; ++step) {
       const int l = step / 5, k = step - 5 * l;
       if (k == 1) {
