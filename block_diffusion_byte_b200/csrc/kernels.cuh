@@ -484,6 +484,83 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
   }
 }
 
+// bf16 K/V on the tensor cores.  Scores: S^T (16 keys x 8 rows) = K (16 x 16
+// dims, bf16 A operand from smem) . q^T (dims x rows, split into bf16 hi and
+// lo B operands), hi then lo per 16-dim step, steps in dim order; one warp
+// per (key tile, row group).  Keys past nk or past a row's limit get -inf.
+// K rows past nk are never loaded: their scores are discarded.
+template <int DH>
+__device__ __forceinline__ void attn_scores_mma(const AttnArgs& a, const float* qs, const __nv_bfloat16* ks, float* ps, const int* lim,
+                                                int nr, int nk, int tid, int nthr) {
+  constexpr int ST = kv_stride<DH, __nv_bfloat16>();
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3, nw = nthr >> 5;
+  const int nkt = a.CH / 16, nrg = (nr + 7) / 8;
+#pragma unroll 1
+  for (int item = warp; item < nkt * nrg; item += nw) {
+    const int key0 = (item % nkt) * 16, rg = item / nkt;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (key0 < nk) {
+      const float* q = qs + min(rg * 8 + g, nr - 1) * DH;  // rows past nr: a live row's values, never stored
+#pragma unroll
+      for (int s = 0; s < DH / 16; ++s) {
+        const int c = s * 16 + 2 * t;
+        const __nv_bfloat16* k0 = ks + (key0 + g) * ST + c;
+        const __nv_bfloat16* k8 = ks + (key0 + g + 8) * ST + c;
+        const uint4 A = make_uint4(*reinterpret_cast<const uint32_t*>(k0), *reinterpret_cast<const uint32_t*>(k8),
+                                   *reinterpret_cast<const uint32_t*>(k0 + 8), *reinterpret_cast<const uint32_t*>(k8 + 8));
+        const float2 qa = *reinterpret_cast<const float2*>(q + c), qb = *reinterpret_cast<const float2*>(q + c + 8);
+        const XFrag xf = make_xfrag(qa.x, qa.y, qb.x, qb.y);
+        mma16816(acc, A, xf.b0h, xf.b1h);
+        mma16816(acc, A, xf.b0l, xf.b1l);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = key0 + g + (e >= 2 ? 8 : 0), r = rg * 8 + 2 * t + (e & 1);
+      if (r < nr) ps[r * a.CH + key] = (key < nk && key < lim[r]) ? acc[e] : -INFINITY;
+    }
+  }
+}
+
+// o^T (16 columns x 8 rows) = V^T (16 columns x 16 keys, bf16 A operand
+// gathered from smem) . p^T (keys x rows, split into bf16 hi and lo), key
+// tiles in order; one warp per (column tile, row group).  V rows from nk up
+// to the next multiple of 16 are zero (their p is 0 as well).
+template <int DH>
+__device__ __forceinline__ void attn_pv_mma(const AttnArgs& a, const float* ps, const __nv_bfloat16* vs, int nr, int nk, int row0,
+                                            int h, int chunk, const float* mrow, const float* lrow, int tid, int nthr) {
+  constexpr int ST = kv_stride<DH, __nv_bfloat16>();
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3, nw = nthr >> 5;
+  const int nkt = (nk + 15) / 16, nrg = (nr + 7) / 8;
+  const unsigned short* v16 = reinterpret_cast<const unsigned short*>(vs);
+  auto pk = [](unsigned short lo, unsigned short hi) { return (uint32_t)lo | ((uint32_t)hi << 16); };
+#pragma unroll 1
+  for (int item = warp; item < (DH / 16) * nrg; item += nw) {
+    const int c0 = (item % (DH / 16)) * 16, rg = item / (DH / 16);
+    const float* p = ps + min(rg * 8 + g, nr - 1) * a.CH;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int k0 = kt * 16 + 2 * t;
+      const unsigned short* va = v16 + k0 * ST + c0 + g;
+      const uint4 A = make_uint4(pk(va[0], va[ST]), pk(va[8], va[ST + 8]), pk(va[8 * ST], va[9 * ST]), pk(va[8 * ST + 8], va[9 * ST + 8]));
+      const float2 pa = *reinterpret_cast<const float2*>(p + k0), pb = *reinterpret_cast<const float2*>(p + k0 + 8);
+      const XFrag xf = make_xfrag(pa.x, pa.y, pb.x, pb.y);
+      mma16816(acc, A, xf.b0h, xf.b1h);
+      mma16816(acc, A, xf.b0l, xf.b1l);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c0 + g + (e >= 2 ? 8 : 0), r = rg * 8 + 2 * t + (e & 1);
+      if (r < nr) {
+        const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
+        a.part_o[base * DH + c] = acc[e];
+        if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+      }
+    }
+  }
+}
+
 // Softmax partial of one (group, head, chunk): scores of every row against
 // keys [t0, t0+nk) (masked per row by nkeys), m = max, l = sum exp(s - m),
 // o = sum exp(s - m) v.  q pre-scaled by 1/sqrt(dh).  smem: qs [32][DH] f32,
@@ -505,9 +582,15 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
     qs[r * DH + c] = __ldcg(a.q + (size_t)(row0 + r) * a.d + h * DH + c) * a.scale;
   }
   if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
+  if constexpr (sizeof(KVT) == 2) {  // zero V rows nk .. next multiple of 16 (read by the last key tile)
+    const int pad = ((nk + 15) & ~15) - nk;
+    for (int i = tid; i < pad * (DH / 8); i += nthr)
+      *reinterpret_cast<uint4*>(const_cast<KVT*>(vs) + (nk + i / (DH / 8)) * ST + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
+  }
   sync();
   mark(1);
-  attn_scores<DH, KVT>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  if constexpr (sizeof(KVT) == 2) attn_scores_mma<DH>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  else attn_scores<DH, KVT>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
   sync();
   mark(2);
   const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
@@ -533,6 +616,10 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   }
   sync();
   mark(3);
+  if constexpr (sizeof(KVT) == 2) {
+    attn_pv_mma<DH>(a, ps, vs, nr, nk, row0, h, chunk, mrow, lrow, tid, nthr);
+    return;
+  }
   // o[r][c] = sum_k p[r][k] v[k][c], one fmaf chain in k order per output.
   // A thread owns column c and rows r0, r0 + rs, ... four at a time, so each
   // V element it loads feeds four chains.  (nthr is a multiple of DH.)
