@@ -46,7 +46,9 @@ struct blt_dec {
   bool own_stream = false;
   int L = 0, d = 0, H = 0, dh = 0, F = 0, dg = 0, V = 0, planes = 1;
   int PT = 0, max_pages = 0, n_pages = 0, CH = 0, CMAX = 0;
-  std::vector<Mat> qkv, o, w13, w2, vc, oc;
+  std::vector<Mat> qkv, o, w13, w2;
+  Mat vc_all, oc_all;  // latent projections of all layers, stacked along N (layer l: tiles l*d/16 ..)
+  int proj_rows = 0;   // latents per projection chunk (tmp holds proj_rows x L*d)
   std::vector<float*> attn_norm, ffn_norm;
   Mat head;
   float* embed = nullptr;
@@ -479,29 +481,32 @@ int project_latents(blt_dec* h, const CallDesc& cd, const float* new_lat, bool c
   const int total = cd.lat_off[cd.batch];
   if (total == 0) return BLT_OK;
   if (!new_lat) return fail(h, BLT_ERR_INVALID_ARG, "new_latents is NULL but latent_offsets count %d", total);
-  const int chunk = h->cfg.max_rows;
+  const int chunk = std::min(h->proj_rows, h->cfg.max_rows);
+  const int LD = h->L * h->d;
   for (int r0 = 0; r0 < total; r0 += chunk) {
     const int r1 = std::min(total, r0 + chunk);
     k_lat_plan<<<1, 256, 0, h->stream>>>(cd, h->sd, h->lat_seq, h->lat_slot, h->n_lat_rows, r0, r1, commit ? 1 : 0,
                                          h->cfg.max_latents);
     h->launches += 1;
-    for (int l = 0; l < h->L; ++l) {
-      GemmArgs a = base_args(h);
-      a.n_rows = nullptr;
-      a.rows_host = r1 - r0;
-      a.layer = l;
-      a.X = new_lat + (size_t)r0 * h->dg;
-      a.ldx = h->dg;
-      a.out = h->tmp;
-      a.ldo = h->d;
-      TRY(gemm<EPI_STORE>(h, h->vc[l], a, r1 - r0));
-      a.X = h->tmp;
-      a.ldx = h->d;
-      a.out = h->c_lat;
-      a.lat_seq = h->lat_seq;
-      a.lat_slot = h->lat_slot;
-      TRY(gemm<EPI_LATC>(h, h->oc[l], a, r1 - r0));
-    }
+    // tmp[row][l*d + i] = (W_v^c of layer l) latent, every layer in one GEMM
+    GemmArgs a = base_args(h);
+    a.n_rows = nullptr;
+    a.rows_host = r1 - r0;
+    a.layer = 0;
+    a.X = new_lat + (size_t)r0 * h->dg;
+    a.ldx = h->dg;
+    a.out = h->tmp;
+    a.ldo = LD;
+    TRY(gemm<EPI_STORE>(h, h->vc_all, a, r1 - r0));
+    // c_lat[seq, slot, l] = (W_o^c of layer l) tmp[row][l*d ..]: tile group l reads column block l
+    a.X = h->tmp;
+    a.ldx = LD;
+    a.group_tiles = h->d / 16;
+    a.group_xoff = h->d;
+    a.out = h->c_lat;
+    a.lat_seq = h->lat_seq;
+    a.lat_slot = h->lat_slot;
+    TRY(gemm<EPI_LATC>(h, h->oc_all, a, r1 - r0));
   }
   CK(cudaGetLastError());
   return BLT_OK;
@@ -881,11 +886,12 @@ struct NaSwap {
   int* pred;
   RowsDev rows;
   int *lat_seq, *lat_slot, *n_lat_rows;
-  int cmax, max_rows;
+  int cmax, max_rows, proj_rows;
   NaSwap(blt_dec* hd, unsigned char* base) : h(hd) {
     hh = h->h, q = h->q, att = h->att, act = h->act, logits = h->logits, tmp = h->tmp, conf = h->conf, gap = h->gap;
     part_ml = h->part_ml, part_o = h->part_o, pred = h->pred, rows = h->rows;
     lat_seq = h->lat_seq, lat_slot = h->lat_slot, n_lat_rows = h->n_lat_rows, cmax = h->CMAX, max_rows = h->cfg.max_rows;
+    proj_rows = h->proj_rows;
     NaCarve c{base};
     h->h = c.take<float>((size_t)kNaRows * kNaMaxD);
     h->q = c.take<float>((size_t)kNaRows * kNaMaxD);
@@ -916,6 +922,7 @@ struct NaSwap {
     h->n_lat_rows = c.take<int>(1);
     h->CMAX = kNaCMax;
     h->cfg.max_rows = kNaRows;
+    h->proj_rows = std::max(1, (int)((size_t)kNaRows * kNaMaxD / ((size_t)h->L * h->d)));  // tmp holds rows x L*d
     used = c.off;
   }
   size_t used = 0;
@@ -923,6 +930,7 @@ struct NaSwap {
     h->h = hh, h->q = q, h->att = att, h->act = act, h->logits = logits, h->tmp = tmp, h->conf = conf, h->gap = gap;
     h->part_ml = part_ml, h->part_o = part_o, h->pred = pred, h->rows = rows;
     h->lat_seq = lat_seq, h->lat_slot = lat_slot, h->n_lat_rows = n_lat_rows, h->CMAX = cmax, h->cfg.max_rows = max_rows;
+    h->proj_rows = proj_rows;
   }
 };
 }  // namespace
@@ -977,8 +985,6 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     h->o.resize(L);
     h->w13.resize(L);
     h->w2.resize(L);
-    h->vc.resize(L);
-    h->oc.resize(L);
     h->attn_norm.resize(L);
     h->ffn_norm.resize(L);
     for (int l = 0; l < L; ++l) {
@@ -1005,11 +1011,14 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
         return (r16 < 8 ? lw[BLT_LAYER_W1] : lw[BLT_LAYER_W3]) + (size_t)j * d;
       }));
       TRY(pack_matrix(h, h->w2[l], d, F, pl, [&](int r) { return lw[BLT_LAYER_W2] + (size_t)r * F; }));
-      TRY(pack_matrix(h, h->vc[l], d, dg, pl, [&](int r) { return lw[BLT_LAYER_WV_C] + (size_t)r * dg; }));
-      TRY(pack_matrix(h, h->oc[l], d, d, pl, [&](int r) { return lw[BLT_LAYER_WO_C] + (size_t)r * d; }));
       TRY(upload(h, &h->attn_norm[l], lw[BLT_LAYER_ATTN_NORM], d));
       TRY(upload(h, &h->ffn_norm[l], lw[BLT_LAYER_FFN_NORM], d));
     }
+    // one projection GEMM per matrix kind covers every layer
+    TRY(pack_matrix(h, h->vc_all, L * d, dg, pl,
+                    [&](int r) { return w->layer[(size_t)(r / d) * BLT_LAYER_NT + BLT_LAYER_WV_C] + (size_t)(r % d) * dg; }));
+    TRY(pack_matrix(h, h->oc_all, L * d, d, pl,
+                    [&](int r) { return w->layer[(size_t)(r / d) * BLT_LAYER_NT + BLT_LAYER_WO_C] + (size_t)(r % d) * d; }));
     TRY(pack_matrix(h, h->head, 256, d, pl, [&](int r) { return w->head + (size_t)r * d; }));
     {
       // the embedding is read once per row: keep it fp32, values rounded like the weights
@@ -1059,7 +1068,8 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(dalloc(h, &h->att, (size_t)RL * d));
     TRY(dalloc(h, &h->act, (size_t)RL * F));
     TRY(dalloc(h, &h->logits, (size_t)RL * 256));
-    TRY(dalloc(h, &h->tmp, (size_t)RL * d));
+    TRY(dalloc(h, &h->tmp, (size_t)R * L * d));
+    h->proj_rows = R;
     TRY(dalloc(h, &h->part_ml, (size_t)RL * h->H * h->CMAX));
     TRY(dalloc(h, &h->part_o, (size_t)RL * h->H * h->CMAX * dh));
     TRY(dalloc(h, &h->conf, RL));

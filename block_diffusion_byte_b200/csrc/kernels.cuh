@@ -85,6 +85,7 @@ struct GemmArgs {
   int N, K;
   const float* X;  // activations [rows][ldx] fp32
   int ldx;
+  int group_tiles, group_xoff;  // if group_tiles > 0: output tile mt reads X + (mt / group_tiles) * group_xoff
   const float* gain;  // [K] RMSNorm gain; NULL: no norm (rs = 1)
   float eps;
   const int* n_rows;  // device row count (NULL: rows_host is exact)
@@ -289,11 +290,12 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   const int ksteps = a.K / 16;
   const bool norm = a.gain != nullptr;
 
+  const float* xg = a.X + (a.group_tiles ? (size_t)(mt / a.group_tiles) * a.group_xoff : 0);
   auto stage = [&](int wi, int buf) {
     for (int c = tid; c < RB * 32; c += kThreads) {
       const int r = c >> 5, q = c & 31;
       const bool ok = r < nr;
-      const float* src = a.X + (size_t)(ok ? row0 + r : row0) * a.ldx + wi * kKWin + q * 4;
+      const float* src = xg + (size_t)(ok ? row0 + r : row0) * a.ldx + wi * kKWin + q * 4;
       cp_async16(xs + ((size_t)buf * RB + r) * kXStride + q * 4, src, ok ? 16 : 0);
     }
   };
