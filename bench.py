@@ -41,6 +41,24 @@ from workload import CONFIGS, WeightSet, prefix_bytes  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
+def measured_traffic(workload: str, persistent: bool):
+    """DRAM bytes per decoder pass from the committed ncu record of the persistent
+    kernel, or None when the record is for another workload or path, or the kernel
+    sources changed since it was taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"k_mega_{workload}_dram.json")
+    if not persistent or not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for rel in rec["source_files"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return rec["dram_bytes_per_pass"] if h.hexdigest() == rec["source_sha256"] else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -310,7 +328,8 @@ def main():
             "unit": "GB/s",
             "frac": achieved / peak,
             "frac_of_8tbs": achieved / 8000.0,
-            "traffic": None,
+            "traffic": measured_traffic(wl.name, bool(d["persistent_calls"])),
+            "traffic_unit": "bytes per pass (dram__bytes_read.sum + dram__bytes_write.sum)",
             "kernel": "k_mega (persistent decoder pass)" if d["persistent_calls"] else "decoder pass (all kernels of one pass)",
             "alg_bytes_per_pass": alg_bytes,
             "pass_ms": pass_ms,
