@@ -36,6 +36,7 @@ EXPORTS = (
     "blt_dec_prefill",
     "blt_dec_prefill_noalloc",
     "blt_dec_diffuse_block",
+    "blt_dec_diffuse_block_eb",
     "blt_dec_draft",
     "blt_dec_verify_accept",
     "blt_dec_rewind",
@@ -123,6 +124,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.blt_dec_prefill.argtypes = [P, I, C.POINTER(blt_rows_in), P]
     lib.blt_dec_prefill_noalloc.argtypes = [P, I, C.POINTER(blt_rows_in), P]
     lib.blt_dec_diffuse_block.argtypes = [P, I, C.POINTER(blt_rows_in), I, F, I, P, P, P]
+    lib.blt_dec_diffuse_block_eb.argtypes = [P, I, C.POINTER(blt_rows_in), I, F, I, P, P, P]
     lib.blt_dec_draft.argtypes = [P, I, C.POINTER(blt_rows_in), I, I, F, I, P, P]
     lib.blt_dec_verify_accept.argtypes = [P, P, P, C.POINTER(C.c_int32), P, P, P]
     lib.blt_dec_rewind.argtypes = [P, I, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
@@ -207,6 +209,13 @@ def blt_dec_diffuse_block(h, batch, pending, k, alpha, max_steps, out_block, out
         h, batch, C.byref(pending), k, float(alpha), max_steps, _ptr(out_block), _ptr(out_steps), _ptr(out_logits)
     )
     _check(h, rc, "blt_dec_diffuse_block")
+
+
+def blt_dec_diffuse_block_eb(h, batch, pending, k, gamma, max_steps, out_block, out_steps=None, out_logits=None) -> None:
+    rc = load_library().blt_dec_diffuse_block_eb(
+        h, batch, C.byref(pending), k, float(gamma), max_steps, _ptr(out_block), _ptr(out_steps), _ptr(out_logits)
+    )
+    _check(h, rc, "blt_dec_diffuse_block_eb")
 
 
 def blt_dec_draft(h, batch, pending, mode, k, alpha, max_steps, out_draft, out_logits=None) -> None:

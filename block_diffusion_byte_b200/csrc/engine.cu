@@ -78,6 +78,8 @@ struct blt_dec {
   unsigned long long weight_bytes_per_pass = 0, kv_bytes_per_key = 0;
   unsigned long long launches = 0;  // kernels launched (host count)
   unsigned long long persistent_calls = 0;  // calls served by the persistent kernel
+  int eb = 0;             // the running call unmasks by EB sampling (blt_dec_diffuse_block_eb)
+  float* ent = nullptr;   // per-row entropy of the byte head
   // pass timing (BLT_FLAG_TIME_PASSES): event pairs recorded around passes
   std::vector<cudaEvent_t> tev;
   size_t tev_used = 0;
@@ -404,7 +406,7 @@ int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want
     a.ldo = 256;
     TRY(gemm<EPI_STORE>(h, h->head, a, rows_ub));
     k_head_stats<<<std::max(1, std::min((rows_ub + 7) / 8, 1024)), 256, 0, h->stream>>>(h->logits, h->rows.n_rows, h->conf,
-                                                                                          h->pred, h->gap);
+                                                                                          h->pred, h->gap, h->ent);
   }
   CK(cudaGetLastError());
   return BLT_OK;
@@ -556,13 +558,14 @@ int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, f
   p.pend_lat = pend->row_latent;
   TRY(plan(h, p, cd));
   TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true));
-  k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits);
+  k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits, h->eb ? h->ent : nullptr);
   h->launches += 1;
   for (int st = 1; st < max_steps; ++st) {
     PlanArgs pb = plan_args(h, PL_BLOCK, k);
     TRY(plan(h, pb, cd));
     TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true));
-    k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits);
+    k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits,
+                                          h->eb ? h->ent : nullptr);
     h->launches += 1;
   }
   CK(cudaGetLastError());
@@ -745,6 +748,8 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.act = h->act;
   m.logits = h->logits;
   m.conf = h->conf;
+  m.ent = h->ent;
+  m.eb = h->eb;
   m.pred = h->pred;
   m.gap = h->gap;
   m.flags = h->flags;
@@ -841,7 +846,7 @@ constexpr size_t na_align(size_t x) { return (x + 255) & ~(size_t)255; }
 constexpr size_t kNaArenaBytes =
     na_align(4ull * kNaRows * kNaMaxD * 4) * 1 + na_align((size_t)kNaRows * kNaMaxF * 4) + na_align((size_t)kNaRows * 256 * 4) +
     na_align((size_t)kNaRows * kNaMaxH * kNaCMax * 8) + na_align((size_t)kNaRows * kNaMaxH * kNaCMax * kNaMaxDh * 4) +
-    3 * na_align(kNaRows * 4) + 5 * na_align(kNaRows * 4 + 4) + 5 * na_align(kNaGroups * 4 + 4) + 3 * na_align(kNaRows * 4 + 4) + 16 * 256;
+    4 * na_align(kNaRows * 4) + 5 * na_align(kNaRows * 4 + 4) + 5 * na_align(kNaGroups * 4 + 4) + 3 * na_align(kNaRows * 4 + 4) + 16 * 256;
 }  // namespace
 
 static __device__ __align__(256) unsigned char g_noalloc_arena[kNaArenaBytes];
@@ -880,7 +885,7 @@ struct NaCarve {
 // Points the handle's pass scratch at the arena for one call and restores it after.
 struct NaSwap {
   blt_dec* h;
-  float *hh, *q, *att, *act, *logits, *tmp, *conf, *gap;
+  float *hh, *q, *att, *act, *logits, *tmp, *conf, *gap, *ent;
   float2* part_ml;
   float* part_o;
   int* pred;
@@ -888,7 +893,7 @@ struct NaSwap {
   int *lat_seq, *lat_slot, *n_lat_rows;
   int cmax, max_rows, proj_rows;
   NaSwap(blt_dec* hd, unsigned char* base) : h(hd) {
-    hh = h->h, q = h->q, att = h->att, act = h->act, logits = h->logits, tmp = h->tmp, conf = h->conf, gap = h->gap;
+    hh = h->h, q = h->q, att = h->att, act = h->act, logits = h->logits, tmp = h->tmp, conf = h->conf, gap = h->gap, ent = h->ent;
     part_ml = h->part_ml, part_o = h->part_o, pred = h->pred, rows = h->rows;
     lat_seq = h->lat_seq, lat_slot = h->lat_slot, n_lat_rows = h->n_lat_rows, cmax = h->CMAX, max_rows = h->cfg.max_rows;
     proj_rows = h->proj_rows;
@@ -903,6 +908,7 @@ struct NaSwap {
     h->part_o = c.take<float>((size_t)kNaRows * kNaMaxH * kNaCMax * kNaMaxDh);
     h->conf = c.take<float>(kNaRows);
     h->gap = c.take<float>(kNaRows);
+    h->ent = c.take<float>(kNaRows);
     h->pred = c.take<int>(kNaRows);
     RowsDev& r = h->rows;
     r.seq = c.take<int>(kNaRows);
@@ -927,7 +933,7 @@ struct NaSwap {
   }
   size_t used = 0;
   ~NaSwap() {
-    h->h = hh, h->q = q, h->att = att, h->act = act, h->logits = logits, h->tmp = tmp, h->conf = conf, h->gap = gap;
+    h->h = hh, h->q = q, h->att = att, h->act = act, h->logits = logits, h->tmp = tmp, h->conf = conf, h->gap = gap, h->ent = ent;
     h->part_ml = part_ml, h->part_o = part_o, h->pred = pred, h->rows = rows;
     h->lat_seq = lat_seq, h->lat_slot = lat_slot, h->n_lat_rows = n_lat_rows, h->CMAX = cmax, h->cfg.max_rows = max_rows;
     h->proj_rows = proj_rows;
@@ -1074,6 +1080,7 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(dalloc(h, &h->part_o, (size_t)RL * h->H * h->CMAX * dh));
     TRY(dalloc(h, &h->conf, RL));
     TRY(dalloc(h, &h->gap, RL));
+    TRY(dalloc(h, &h->ent, RL));
     TRY(dalloc(h, &h->pred, RL));
     RowsDev& rd = h->rows;
     TRY(dalloc(h, &rd.seq, RL));
@@ -1203,6 +1210,19 @@ int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, i
   CK(cudaGetLastError());
   bump_bounds(h, cd, 0);
   return post_mirror(h);
+}
+
+int blt_dec_diffuse_block_eb(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float gamma, int max_steps,
+                             uint8_t* out_block, int32_t* out_steps, float* out_logits) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  if (!(gamma >= 0.f) || gamma == INFINITY) {
+    h->err.clear();
+    return fail(h, BLT_ERR_INVALID_ARG, "gamma must be finite and >= 0");
+  }
+  h->eb = 1;
+  const int rc = blt_dec_diffuse_block(h, batch, pending, k, gamma, max_steps, out_block, out_steps, out_logits);
+  h->eb = 0;
+  return rc;
 }
 
 int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode, int k, float alpha, int max_steps,

@@ -741,8 +741,10 @@ __global__ void __launch_bounds__(32) k_attn_combine(AttnArgs a) {
 
 // ------------------------------------------------------------------------ byte head statistics
 // Over the 256 byte logits of a row (one warp): confidence = largest softmax
-// probability, argmax (lowest byte on ties), gap between the two largest logits.
-__device__ __forceinline__ void head_stats_row(const float* z, int lane, float& conf, int& pred, float& gap) {
+// probability, argmax (lowest byte on ties), gap between the two largest
+// logits, and the entropy (nats) of the softmax: with e_i = exp(z_i - max),
+// S = sum e_i and T = sum e_i (z_i - max), H = ln S - T / S.
+__device__ __forceinline__ void head_stats_row(const float* z, int lane, float& conf, int& pred, float& gap, float& ent) {
   float v[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] = __ldcg(z + lane + 32 * j);
@@ -772,27 +774,34 @@ __device__ __forceinline__ void head_stats_row(const float* z, int lane, float& 
       b2 = fmaxf(b2, ob1);
     }
   }
-  float s = 0.f;
+  float s = 0.f, tz = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) s += expf(v[j] - b1);
+  for (int j = 0; j < 8; ++j) {
+    const float e = expf(v[j] - b1);
+    s += e;
+    tz = fmaf(e, v[j] - b1, tz);
+  }
   s = warp_sum(s);
+  tz = warp_sum(tz);
   conf = 1.0f / s;
   pred = i1;
   gap = b1 - b2;
+  ent = logf(s) - tz / s;
 }
 
-__global__ void k_head_stats(const float* __restrict__ logits, const int* n_rows, float* conf, int* pred, float* gap) {
+__global__ void k_head_stats(const float* __restrict__ logits, const int* n_rows, float* conf, int* pred, float* gap, float* ent) {
   const int n = *n_rows;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   for (int r = warp; r < n; r += nw) {
-    float c, g;
+    float c, g, e;
     int p;
-    head_stats_row(logits + (size_t)r * 256, lane, c, p, g);
+    head_stats_row(logits + (size_t)r * 256, lane, c, p, g, e);
     if (lane == 0) {
       conf[r] = c;
       pred[r] = p;
       gap[r] = g;
+      ent[r] = e;
     }
   }
 }
@@ -990,11 +999,16 @@ __global__ void k_lat_plan(CallDesc cd, SeqDev sd, int* lat_seq, int* lat_slot, 
 }
 
 // ------------------------------------------------------------------------ bookkeeping (one warp per sequence)
-// Confidence unmasking ("블록 언마스킹 전략"): every masked position with
+// Block unmasking ("블록 언마스킹 전략"), one warp per sequence, lane = block
+// position.  Confidence rule (ent == NULL): every masked position with
 // conf >= alpha is committed; if none, the most confident one (lowest position
-// on ties).  Returns whether masked positions remain.
+// on ties).  EB sampling (ent != NULL, bound gamma = alpha): masked positions
+// ranked by entropy (position breaks ties), running sums of entropy taken in
+// rank order in fp32, every position whose running sum is <= gamma is
+// committed, and at least the first.  Returns whether masked positions remain.
 __device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, float alpha, int step, const float* conf,
-                                           const int* pred, const float* logits, float* out_logits, int lane) {
+                                           const int* pred, const float* logits, float* out_logits, int lane,
+                                           const float* ent = nullptr) {
   if (step == 0 && lane == 0) {
     const int lr = sd.last_row[s];
     if (lr >= 0) sd.y_last[s] = __ldcg(pred + lr);
@@ -1003,10 +1017,26 @@ __device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, f
   const int row = in ? sd.blk_row[s * kMaxBlock + lane] : 0;
   const bool m = in && sd.masked[s * kMaxBlock + lane];
   const float c = m ? __ldcg(conf + row) : -1.0f;
-  const bool over = m && (c >= alpha);
+  const bool over = !ent && m && (c >= alpha);
   const unsigned any_over = __ballot_sync(0xffffffffu, over);
   bool commit = over;
-  if (!any_over) {
+  if (ent) {
+    const float e = m ? __ldcg(ent + row) : INFINITY;
+    const unsigned mm = __ballot_sync(0xffffffffu, m);
+    int rank = 0;
+    for (int j = 0; j < 32; ++j) {
+      const float ej = __shfl_sync(0xffffffffu, e, j);
+      if (((mm >> j) & 1u) && (ej < e || (ej == e && j < lane))) ++rank;
+    }
+    float run = 0.f, cum = 0.f;
+    const int nm = __popc(mm);
+    for (int r = 0; r < nm; ++r) {
+      const int src = __ffs(__ballot_sync(0xffffffffu, m && rank == r)) - 1;
+      run += __shfl_sync(0xffffffffu, e, src);
+      if (m && rank == r) cum = run;
+    }
+    commit = m && (cum <= alpha || rank == 0);
+  } else if (!any_over) {
     float best = c;
     int bi = m ? lane : 1 << 30;
 #pragma unroll
@@ -1038,10 +1068,10 @@ __device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, f
 }
 
 __global__ void k_unmask(SeqDev sd, int batch, int k, float alpha, int step, const float* conf, const int* pred,
-                         const float* logits, float* out_logits) {
+                         const float* logits, float* out_logits, const float* ent) {
   const int s = blockIdx.x, lane = threadIdx.x;
   if (s >= batch || !sd.active[s]) return;
-  unmask_seq(sd, s, batch, k, alpha, step, conf, pred, logits, out_logits, lane);
+  unmask_seq(sd, s, batch, k, alpha, step, conf, pred, logits, out_logits, lane, ent);
 }
 
 // AR draft: the argmax of this pass's row becomes draft byte `step`.

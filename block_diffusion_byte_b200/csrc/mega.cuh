@@ -61,6 +61,8 @@ struct MegaArgs {
   float* act;
   float* logits;
   float* conf;
+  float* ent;  // per-row entropy of the byte head (EB sampling)
+  int eb;      // block unmasking by EB sampling (bound alpha) instead of confidence
   int* pred;
   float* gap;
   unsigned* flags;  // epoch flags, see flag offsets below
@@ -777,13 +779,14 @@ __device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass
   if (tid == 0) sm.misc[1] = 0;
   consumer_sync();
   for (int r = warp; r < nr; r += 8) {
-    float c, g;
+    float c, g, e;
     int p;
-    head_stats_row(m.logits + (size_t)r * 256, lane, c, p, g);
+    head_stats_row(m.logits + (size_t)r * 256, lane, c, p, g, e);
     if (lane == 0) {
       m.conf[r] = c;
       m.pred[r] = p;
       m.gap[r] = g;
+      m.ent[r] = e;
     }
   }
   __threadfence_block();
@@ -792,7 +795,8 @@ __device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass
   if (m.mode == MM_DIFFUSE) {
     for (int s = warp; s < m.batch; s += 8) {
       if (m.sd.active[s]) {
-        const bool left = unmask_seq(m.sd, s, m.batch, m.k, m.alpha, pass, m.conf, m.pred, m.logits, m.out_logits, lane);
+        const bool left =
+            unmask_seq(m.sd, s, m.batch, m.k, m.alpha, pass, m.conf, m.pred, m.logits, m.out_logits, lane, m.eb ? m.ent : nullptr);
         if (left && lane == 0) atomicOr(sm.misc + 1, 1);
       }
     }

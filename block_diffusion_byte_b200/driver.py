@@ -223,7 +223,10 @@ def generate(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: Op
         pend = [s.take_pending() for s in seqs]
         r, keep = eng.rows([p[0] for p in pend], [p[1] for p in pend], [p[2] for p in pend])
         if wl.mode == "D":
-            B.blt_dec_diffuse_block(h, nb, r, k, wl.alpha, 0, eng.d_out, eng.d_steps)
+            if wl.unmask == "entropy":
+                B.blt_dec_diffuse_block_eb(h, nb, r, k, wl.gamma, 0, eng.d_out, eng.d_steps)
+            else:
+                B.blt_dec_diffuse_block(h, nb, r, k, wl.alpha, 0, eng.d_out, eng.d_steps)
             blk = eng._get(eng.out_view(nb, k))
             steps = eng._get(eng.d_steps[:nb]) if record else None
             for i, s in enumerate(seqs):

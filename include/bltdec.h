@@ -193,6 +193,19 @@ int blt_dec_prefill_noalloc(blt_dec_t *h, int batch, const blt_rows_in *rows, fl
 int blt_dec_diffuse_block(blt_dec_t *h, int batch, const blt_rows_in *pending, int k, float alpha, int max_steps,
                           uint8_t *out_block, int32_t *out_steps, float *out_logits);
 
+/* BLT-D with entropy-bounded (EB) sampling instead of the confidence rule
+ * ("블록 언마스킹 전략", EB sampling; the wangzhan123.com page, section on the
+ * two unmasking rules).  Everything is as in blt_dec_diffuse_block except the
+ * per-pass choice: the still-masked positions are ordered by the entropy
+ * (nats) of their predicted distribution over the 256 bytes, lowest first
+ * (equal entropies: lower position first); running sums of those entropies
+ * are taken in that order (fp32) and every position whose running sum is
+ * <= gamma is committed, and always at least the first.  Committed bytes are
+ * the greedy argmax.  gamma: finite, >= 0 (else INVALID_ARG).  Same outputs,
+ * ownership and errors as blt_dec_diffuse_block. */
+int blt_dec_diffuse_block_eb(blt_dec_t *h, int batch, const blt_rows_in *pending, int k, float gamma, int max_steps,
+                             uint8_t *out_block, int32_t *out_steps, float *out_logits);
+
 /* Draft k bytes per sequence after the committed ones ("BLT-S", "BLT-DV").
  * Every sequence needs at least one pending row: the last pending row's
  * greedy prediction is y_l of the verification.

@@ -9,6 +9,12 @@ Source: "Fast Byte Latent Transformer (Fast-BLT) 연구 소개" (discuss.pytorch
 * "블록 언마스킹 전략", confidence-based unmasking: confidence is the largest
   predicted probability; every masked position whose confidence reaches the
   threshold alpha is committed; if none does, the single most confident one is.
+* "블록 언마스킹 전략", entropy-bounded (EB) sampling: the masked positions are
+  ordered by the entropy of their predicted distribution, lowest first, and
+  the largest leading set whose summed entropy stays within the bound gamma
+  is committed in one pass (the wangzhan123.com page, section on the two
+  unmasking rules, says the same: accumulate in that order, stop once the
+  running sum passes the bound).
 * "BLT-S와 BLT-DV", the shared greedy verification: one causal pass over the
   draft gives greedy next-byte predictions y; draft byte i is accepted while
   it equals y_{i-1}; the first mismatch is replaced by the model's byte and the
@@ -27,6 +33,11 @@ go to the lowest byte, fallback ties to the lowest position; committed
 positions are never re-masked; block rows and BLT-S draft rows see the newest
 closed latent; committed-but-uncached rows ride as causal rows in the next
 pass; exactly ``G`` bytes are produced, the last block or round cut at ``G``.
+EB sampling: entropy in nats over the 256 byte values (the mask id excluded,
+as for the confidence); equal entropies are ordered by position; when even
+the lowest entropy exceeds gamma, that one position is committed (so every
+pass makes progress, as with the confidence fallback); committed bytes are the
+greedy argmax.
 """
 
 from __future__ import annotations
@@ -42,6 +53,7 @@ from .model import BLOCK, CAUSAL, OracleModel, Row, SeqState, decoder_pass
 
 NEAR_TIE_GAP = 0.05  # top-2 logit gap below which an argmax is a near-tie
 NEAR_ALPHA = 0.03  # |conf - alpha| below which a threshold decision is a near-tie
+NEAR_EB = 0.05  # nats: entropy or cumulative-entropy margin below which an EB decision is a near-tie
 
 
 class StepLimit(RuntimeError):
@@ -68,6 +80,32 @@ def unmask_select(masked: List[int], conf: np.ndarray, alpha: float) -> Tuple[Li
         if conf[i] > conf[best]:
             best = i
     return [best], True
+
+
+def entropy(z: np.ndarray) -> np.ndarray:
+    """Per row: Shannon entropy (nats) of softmax(z) over the 256 byte logits."""
+    zs = z - z.max(axis=1, keepdims=True)
+    p = np.exp(zs)
+    p /= p.sum(axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.where(p > 0, p * np.log(p), 0.0)
+    return -t.sum(axis=1)
+
+
+def eb_select(masked: List[int], ent: np.ndarray, gamma: float) -> Tuple[List[int], List[int], List[float]]:
+    """Positions committed by one EB step: the masked positions sorted by entropy
+    (position breaks ties), the longest leading run whose running sum of
+    entropies is <= gamma, at least the first.  Also returns the order and the
+    running sums (for near-tie flags)."""
+    order = sorted(masked, key=lambda i: (float(ent[i]), i))
+    cums, c = [], 0.0
+    for i in order:
+        c += float(ent[i])
+        cums.append(c)
+    n = 0
+    while n < len(order) and cums[n] <= gamma:
+        n += 1
+    return order[: max(n, 1)], order, cums
 
 
 def accept_length(draft: List[int], y: List[int]) -> Tuple[int, int]:
@@ -182,8 +220,10 @@ class OracleSequence:
             self.flags.append(Flag(pos, "argmax", float(gap)))
 
     # ----------------------------------------------------------- BLT-D
-    def diffuse(self, B: int, alpha: float, max_steps: Optional[int] = None):
+    def diffuse(self, B: int, alpha: float, max_steps: Optional[int] = None, unmask: str = "confidence", gamma: float = 0.0):
         """Fill one masked block of B bytes; returns (block, steps, y_last).
+        ``unmask`` selects confidence unmasking (threshold ``alpha``) or EB
+        sampling (bound ``gamma``).
 
         ``y_last`` is the greedy prediction of the last pending committed row
         (None when no row was pending), used by BLT-DV verification.
@@ -210,14 +250,25 @@ class OracleSequence:
                     self._flag_argmax(N, float(g_[0]))
             conf, pred, gap = head_stats(z[len(rows) - B :])
             masked = [i for i in range(B) if block[i] is None]
-            chosen, fallback = unmask_select(masked, conf, alpha)
-            for i in masked:
-                if abs(conf[i] - alpha) < NEAR_ALPHA:
-                    self.flags.append(Flag(N + i, "threshold", float(conf[i])))
-            if fallback and len(masked) > 1:
-                c = np.sort(conf[masked])
-                if c[-1] - c[-2] < NEAR_ALPHA:
-                    self.flags.append(Flag(N + chosen[0], "fallback", float(c[-1] - c[-2])))
+            if unmask == "entropy":
+                ent = entropy(z[len(rows) - B :])
+                chosen, order, cums = eb_select(masked, ent, gamma)
+                n = len(chosen)
+                # the cut could move: a running sum near gamma, or entropies near the cut close together
+                for j in (n - 1, n):
+                    if 0 <= j < len(order) and abs(cums[j] - gamma) < NEAR_EB:
+                        self.flags.append(Flag(N + order[j], "eb_bound", float(cums[j] - gamma)))
+                if n < len(order) and abs(float(ent[order[n]]) - float(ent[order[n - 1]])) < NEAR_EB:
+                    self.flags.append(Flag(N + order[n], "eb_order", float(ent[order[n]] - ent[order[n - 1]])))
+            else:
+                chosen, fallback = unmask_select(masked, conf, alpha)
+                for i in masked:
+                    if abs(conf[i] - alpha) < NEAR_ALPHA:
+                        self.flags.append(Flag(N + i, "threshold", float(conf[i])))
+                if fallback and len(masked) > 1:
+                    c = np.sort(conf[masked])
+                    if c[-1] - c[-2] < NEAR_ALPHA:
+                        self.flags.append(Flag(N + chosen[0], "fallback", float(c[-1] - c[-2])))
             for i in chosen:
                 self._flag_argmax(N + i, float(gap[i]))
                 block[i] = int(pred[i])
@@ -285,7 +336,7 @@ class OracleSequence:
         out: List[int] = []
         while len(out) < G:
             if wl.mode == "D":
-                new, steps, _ = self.diffuse(wl.block, wl.alpha)
+                new, steps, _ = self.diffuse(wl.block, wl.alpha, unmask=wl.unmask, gamma=wl.gamma)
                 info = dict(steps=steps)
             elif wl.mode == "AR":
                 new = [self.ar_step()]

@@ -122,3 +122,22 @@ def test_config5_sweep_points(name):
         om = OracleModel(wl.shape, ws)
         want, o = _oracle_run(wl, om, 0, G)
         _check(res.out[0], want, o, wl, name)
+
+
+def test_config2_eb_sampling(dec9):
+    """BLT-D-4 with EB sampling (gamma 4.5), prefix 1024, 64 bytes, persistent kernel."""
+    from block_diffusion_byte_b200 import binding as B
+    from block_diffusion_byte_b200.driver import Engine, generate
+
+    ws, om = dec9
+    wl = CONFIGS["d4eb_b1"]
+    G = 64
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + G + 4 * wl.block + 16, max_block=16, max_rows=1024,
+                 persistent=True)
+    try:
+        res = generate(eng, wl, [_prefix(wl, 0)], G, seq_ids=[0])
+        assert B.blt_dec_stats(eng.h)["persistent_calls"] > 0
+    finally:
+        eng.close()
+    want, o = _oracle_run(wl, om, 0, G)
+    _check(res.out[0], want, o, wl, "config 2, EB")

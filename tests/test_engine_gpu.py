@@ -173,7 +173,7 @@ def test_d4_b1_first_block_logits_and_bytes(d4_setup):
     assert [int(r["steps"][0]) for r in res.rounds] == [r["steps"] for r in rec][: len(res.rounds)] or res.out[0] != want
 
 
-def _call_logits(wl, ws, persistent, mode, k, alpha, G=24, batch=2):
+def _call_logits(wl, ws, persistent, mode, k, alpha, G=24, batch=2, **wkw):
     """Logits of every engine call of a short generation (diffuse / draft / verify), via out_logits."""
     import ctypes
 
@@ -182,7 +182,7 @@ def _call_logits(wl, ws, persistent, mode, k, alpha, G=24, batch=2):
 
     eng = Engine(wl.shape, ws, max_batch=batch, max_ctx=wl.prefix_len + G + 64, max_block=16, max_rows=256, persistent=persistent)
     try:
-        w = replace(wl, mode=mode, block=k, alpha=alpha)
+        w = replace(wl, mode=mode, block=k, alpha=alpha, **wkw)
         res = generate(eng, w, [_prefix(wl, s) for s in range(batch)], G, record=True)
         st = B.blt_dec_stats(eng.h)
     finally:
@@ -235,3 +235,55 @@ def test_persistent_block_logits_bitwise(tiny_setup, d4_setup, which):
     assert sa == sb
     n = int(sa)
     assert np.array_equal(a[:n], b[:n])
+
+
+# ------------------------------------------------------------------ entropy-bounded (EB) sampling
+@pytest.mark.parametrize("k,gamma", [(4, 4.0), (8, 6.0), (6, 0.0)])
+def test_tiny_eb_generation_matches_oracle(tiny_setup, k, gamma):
+    """BLT-D with EB sampling (blt_dec_diffuse_block_eb) against the oracle's EB rule."""
+    from block_diffusion_byte_b200.driver import generate
+
+    wl, ws, om = tiny_setup
+    w = replace(wl, mode="D", block=k, alpha=0.0, unmask="entropy", gamma=gamma)
+    G = 32
+    pre = _prefix(wl, 0)
+    eng = _engine(w, ws)
+    try:
+        res = generate(eng, w, [pre], G)
+    finally:
+        eng.close()
+    o = OracleSequence(om, w, 0, pre)
+    o.prefill()
+    want = o.generate(G)
+    _compare_bytes(res.out[0], o, want, wl.prefix_len, f"EB-{k}-{gamma}")
+    if not o.flags:
+        assert res.stats["passes"] == o.c.passes
+
+
+@pytest.mark.parametrize("k,gamma,batch", [(4, 4.0, 2), (8, 6.0, 1)])
+def test_persistent_eb_matches_per_phase_bitwise(tiny_setup, k, gamma, batch):
+    """EB sampling runs in the persistent kernel's bookkeeping and in the per-phase
+    unmask kernel with the same arithmetic: bytes, pass counts and logits agree bitwise."""
+    wl, ws, om = tiny_setup
+    a, sa = _call_logits(wl, ws, True, "D", k, 0.0, batch=batch, unmask="entropy", gamma=gamma)
+    b, sb = _call_logits(wl, ws, False, "D", k, 0.0, batch=batch, unmask="entropy", gamma=gamma)
+    assert a.out == b.out
+    assert sa["passes"] == sb["passes"]
+    assert sa["persistent_calls"] > 0 and sb["persistent_calls"] == 0
+    for ra, rb in zip(a.rounds, b.rounds):
+        for key in ra:
+            assert np.array_equal(ra[key], rb[key]), key
+
+
+def test_eb_rejects_bad_gamma(tiny_setup):
+    from block_diffusion_byte_b200 import binding as B
+
+    wl, ws, om = tiny_setup
+    eng = _engine(wl, ws)
+    try:
+        r, keep = eng.rows([[1, 2, 3]], [[0, 0, 0]], [[]])
+        for bad in (float("nan"), -1.0, float("inf")):
+            with pytest.raises(B.BltError):
+                B.blt_dec_diffuse_block_eb(eng.h, 1, r, 4, bad, 0, eng.d_out)
+    finally:
+        eng.close()

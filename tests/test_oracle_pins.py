@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from oracle.model import BLOCK, CAUSAL, OracleModel, Row, SeqState, decoder_pass, dense_reference_pass, may_attend, rmsnorm, rope, silu
-from oracle.policies import OracleSequence, accept_length, head_stats, proxy_gb, unmask_select
+from oracle.policies import OracleSequence, accept_length, eb_select, entropy, head_stats, proxy_gb, unmask_select
 from workload import CONFIGS, WeightSet, prefix_bytes
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
@@ -328,3 +328,73 @@ def test_proxy_bandwidth_from_counted_passes():
     assert proxy_gb(8, 1.0, 2, 1.0, 1.0) == pytest.approx(2 * proxy_gb(4, 1.0, 1, 1.0, 1.0))
     # the 1B model's global term is smaller
     assert proxy_gb(0, 0, 1, g["p_enc_1b"], g["p_global_1b"]) < proxy_gb(0, 0, 1, g["p_enc_3b"], g["p_global_3b"])
+
+
+def test_entropy_closed_forms_and_library():
+    """Entropy (nats) of softmax(z): uniform -> ln 256, two equal maxima far above the
+    rest -> ln 2, a single dominant logit -> 0; random logits agree with SciPy."""
+    from scipy.stats import entropy as sp_entropy
+
+    z = np.zeros((3, 256))
+    z[1, :] = -1e4
+    z[1, [7, 200]] = 0.0
+    z[2, 5] = 1e4
+    e = entropy(z)
+    assert abs(e[0] - np.log(256)) < 1e-12
+    assert abs(e[1] - np.log(2)) < 1e-12
+    assert abs(e[2]) < 1e-12
+    r = np.random.default_rng(3).normal(0, 3, (20, 256))
+    p = np.exp(r - r.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    assert np.allclose(entropy(r), sp_entropy(p, axis=1), rtol=1e-12, atol=1e-12)
+
+
+def test_eb_select_worked_cases():
+    """EB sampling: sort by entropy, commit the leading run within gamma, at least one."""
+    ent = np.array([2.0, 0.5, 1.0, 3.0])
+    assert eb_select([0, 1, 2, 3], ent, 1.6)[0] == [1, 2]          # running sums 0.5, 1.5, 3.5, 6.5
+    assert eb_select([0, 1, 2, 3], ent, 1.5)[0] == [1, 2]          # the bound is inclusive
+    assert eb_select([0, 1, 2, 3], ent, 0.1)[0] == [1]             # nothing within gamma: the lowest one
+    assert eb_select([0, 1, 2, 3], ent, 100.0)[0] == [1, 2, 0, 3]  # everything
+    assert eb_select([0, 3], ent, 2.5)[0] == [0]                   # only masked positions count
+    assert eb_select([2, 0, 1], np.array([1.0, 1.0, 1.0]), 2.0)[0] == [0, 1]  # ties: lower position first
+
+
+def test_eb_select_is_the_largest_feasible_set():
+    """The committed set has the largest size over all subsets of the masked positions
+    whose summed entropy is <= gamma (brute force), and when several subsets share
+    that size it is the one with the lowest entropies."""
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        k = int(rng.integers(1, 8))
+        ent = rng.uniform(0.0, 3.0, k)
+        masked = sorted(rng.choice(k, int(rng.integers(1, k + 1)), replace=False).tolist())
+        gamma = float(rng.uniform(0.0, 6.0))
+        chosen = eb_select(masked, ent, gamma)[0]
+        best = 0
+        for n in range(len(masked) + 1):
+            for sub in itertools.combinations(masked, n):
+                if sum(ent[list(sub)]) <= gamma:
+                    best = max(best, n)
+        assert len(chosen) == max(best, 1)
+        if best >= 1:
+            assert sum(ent[chosen]) <= gamma + 1e-12
+            rest = [i for i in masked if i not in chosen]
+            assert all(ent[i] >= max(ent[chosen]) for i in rest)
+
+
+def test_eb_extremes(tiny):
+    """EB with an unbounded gamma fills the block in one pass, the same block as the
+    confidence rule with alpha 0; with gamma 0 (every entropy is > 0) it commits one
+    position per pass, so a block of B takes B passes."""
+    a = _seq(tiny, alpha=0.0)
+    a.prefill()
+    blk_c, steps_c, _ = a.diffuse(6, 0.0)
+    b = _seq(tiny, alpha=0.0)
+    b.prefill()
+    blk_e, steps_e, _ = b.diffuse(6, 0.0, unmask="entropy", gamma=1e9)
+    assert steps_c == steps_e == 1 and blk_c == blk_e
+    c = _seq(tiny, alpha=0.0)
+    c.prefill()
+    _, steps0, _ = c.diffuse(6, 0.0, unmask="entropy", gamma=0.0)
+    assert steps0 == 6

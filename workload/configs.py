@@ -52,6 +52,8 @@ class Workload:
     patch_kind: str  # "uniform8" or "entropy12"
     seed: int = 0
     cfg_index: int = 0
+    unmask: str = "confidence"  # BLT-D block unmasking: "confidence" (threshold alpha) or "entropy" (EB, bound gamma)
+    gamma: float = 0.0  # EB sampling: bound on the cumulative entropy (nats) of the positions committed per pass
 
 
 TINY = ModelShape(n_layers=2, d_model=128, n_heads=4, d_ffn=512, d_global=256, weight_dtype="f32")
@@ -68,6 +70,9 @@ CONFIGS = {
     # BLT-S k=8 greedy self-speculation; prefix 4096; batch 1 and 16; 512 bytes.
     "s8_b1": Workload("s8_b1", DEC9, "S", 8, 0.0, 512, 1, 4096, "entropy12", 0, 3),
     "s8_b16": Workload("s8_b16", DEC9, "S", 8, 0.0, 512, 16, 4096, "entropy12", 0, 3),
+    # BLT-D-4 with entropy-bounded sampling (gamma 4.5 nats: about two positions per pass on
+    # this model, whose block rows carry about 2 nats each); otherwise config 2.
+    "d4eb_b1": Workload("d4eb_b1", DEC9, "D", 4, 0.0, 512, 1, 1024, "entropy12", 0, 1, unmask="entropy", gamma=4.5),
 }
 
 # Decoder-step throughput sweep: batch x block x prefix, d_global 4096.
