@@ -215,6 +215,7 @@ def main():
     ap.add_argument("--workload", default="d4_b1", choices=sorted(CONFIGS))
     ap.add_argument("--ref-seconds", type=float, default=25.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ar-baseline", action="store_true", help="skip the greedy AR decoding of the same job")
     ap.add_argument("--path", default="persistent", choices=["persistent", "phased"],
                     help="decoder passes in the persistent kernel (one launch per call) or as per-phase kernels")
     args = ap.parse_args()
@@ -346,6 +347,39 @@ def main():
         },
         "clocks": clocks,
     }
+    if world == 1 and not args.no_ar_baseline and wl.mode != "AR":
+        # the same job decoded one byte per pass (plain greedy AR BLT) on the same
+        # engine: wall-clock speedup beside the decoder-NFE ratio (the pages' proxy)
+        from dataclasses import replace
+
+        wl_ar = replace(wl, mode="AR", block=1, alpha=0.0)
+
+        def ar_step():
+            B.blt_dec_rewind(eng.h, nb, [0] * nb, [0] * nb)
+            return generate(eng, wl_ar, prefixes, seq_ids=seq_ids)
+
+        ar_step()
+        sa0 = B.blt_dec_stats(eng.h)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(eng.stream)
+        ar_step()
+        e1.record(eng.stream)
+        barrier()
+        ar_ms = e0.elapsed_time(e1)
+        sa1 = B.blt_dec_stats(eng.h)
+        ar_passes = sa1["passes"] - sa0["passes"]
+        ar_value = wl.gen_bytes * nb / (ar_ms / 1000.0)
+        line["ar_baseline"] = {
+            "value": ar_value,
+            "unit": "bytes/s",
+            "ms_per_step": ar_ms,
+            "passes_per_step": ar_passes,
+            "speedup_wallclock": value / ar_value,
+            "decoder_nfe_ratio": ar_passes / (passes / args.steps),
+            "note": "same engine, prefix and length; greedy AR decoding (one byte per decoder pass); "
+            "decoder_nfe_ratio = AR passes / this mode's passes, the decoder term of the pages' proxy",
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(wl, seconds_cap=args.ref_seconds)
     eng.close()
