@@ -86,17 +86,30 @@ class Engine:
         self.d_next = torch.zeros(max_batch, dtype=torch.uint8, device=dev)
         self.d_vslots = torch.zeros((max_batch, max_block), dtype=torch.int32, device=dev)
         self.h2d_bytes = 0
+        self._staging = {}  # destination data_ptr -> (pinned staging buffer, event of its last copy)
         self.d2h_bytes = 0
 
     # -- staging
     def _put(self, dst: torch.Tensor, arr: np.ndarray) -> torch.Tensor:
+        """Copy ``arr`` into the first rows of ``dst`` through a reusable pinned staging
+        buffer (one per destination; it is rewritten only after its last copy ran)."""
         n = arr.shape[0]
         if n == 0:
             return dst[:0]
-        src = torch.from_numpy(np.ascontiguousarray(arr)).pin_memory()
+        arr = np.ascontiguousarray(arr)
+        key = dst.data_ptr()
+        st = self._staging.get(key)
+        if st is None or st[0].numel() < arr.size or st[0].dtype != dst.dtype:
+            st = (torch.empty(max(arr.size, 1 << 12), dtype=dst.dtype).pin_memory(), torch.cuda.Event())
+            self._staging[key] = st
+        buf, done = st
+        done.synchronize()
+        src = buf[: arr.size]
+        src.numpy()[:] = arr.reshape(-1)
         with torch.cuda.stream(self.stream):
-            dst[:n].copy_(src, non_blocking=True)
-        self.h2d_bytes += src.numel() * src.element_size()
+            dst[:n].view(-1)[: arr.size].copy_(src, non_blocking=True)
+            done.record(self.stream)
+        self.h2d_bytes += arr.nbytes
         return dst[:n]
 
     def _get(self, t: torch.Tensor) -> np.ndarray:

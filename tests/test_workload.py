@@ -105,6 +105,7 @@ def test_scalar_and_batched_generators_agree():
             for x in w:
                 h = mix64((h ^ np.uint64(x & 0xFFFFFFFFFFFFFFFF)) + GAMMA)
         assert int(h[0]) == int(kb)
-    a = latent_vectors(0, 1, 3, list(range(12)), [int(k) for k in keys[:12]], 256)
-    b = np.stack([latent_vector(0, 1, 3, i, int(k), 256) for i, k in enumerate(keys[:12])])
+    # 48 x 2048 values: large enough for the transform to run on several host threads
+    a = latent_vectors(0, 1, 3, list(range(48)), [int(k) for k in keys[:48]], 2048)
+    b = np.stack([latent_vector(0, 1, 3, i, int(k), 2048) for i, k in enumerate(keys[:48])])
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))

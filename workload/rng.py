@@ -92,20 +92,24 @@ def normals(key: int, count: int) -> np.ndarray:
 
 
 def normals_many(keys: np.ndarray, count: int) -> np.ndarray:
-    """``normals`` of every key in ``keys`` at once: float64 [len(keys), count]."""
+    """``normals`` of every key in ``keys`` at once: float64 [len(keys), count].
+
+    The float64 transform runs in torch on the host cores (multi-threaded);
+    every element is computed by the same routine whatever the batch size or
+    thread count, so a value never depends on how it was requested."""
+    import torch
+
     keys = np.asarray(keys, dtype=np.uint64).reshape(-1, 1)
     npair = (count + 1) // 2
     i = np.arange(1, 2 * npair + 1, dtype=np.uint64).reshape(1, -1)
     with np.errstate(over="ignore"):
         raw = mix64(keys + i * GAMMA).reshape(keys.shape[0], npair, 2)
-    u1 = 1.0 - uniform53(raw[:, :, 0])  # (0, 1]
-    u2 = uniform53(raw[:, :, 1])
-    r = np.sqrt(-2.0 * np.log(u1))
+    u1 = torch.from_numpy(1.0 - uniform53(raw[:, :, 0]))  # (0, 1]
+    u2 = torch.from_numpy(uniform53(raw[:, :, 1]))
+    r = torch.sqrt(-2.0 * torch.log(u1))
     t = (2.0 * np.pi) * u2
-    out = np.empty((keys.shape[0], npair, 2), dtype=np.float64)
-    out[:, :, 0] = r * np.cos(t)
-    out[:, :, 1] = r * np.sin(t)
-    return out.reshape(keys.shape[0], -1)[:, :count]
+    out = torch.stack([r * torch.cos(t), r * torch.sin(t)], dim=2)
+    return out.reshape(keys.shape[0], -1)[:, :count].numpy()
 
 
 def round_bf16(x: np.ndarray) -> np.ndarray:
