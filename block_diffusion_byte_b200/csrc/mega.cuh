@@ -29,7 +29,8 @@ namespace bltdec {
 
 constexpr int kMegaConsumers = 8;
 constexpr int kMegaThreads = (kMegaConsumers + 1) * 32;
-constexpr int kStageTiles = 32;                 // k16 tiles of one unit per ring slot
+constexpr int kStageTiles = 64;                 // k16 tiles of one unit per ring slot
+constexpr int kTPW = kStageTiles / 8;           // tiles of a stage per consumer warp
 constexpr int kRingBytes = 128 * 1024;          // weight ring
 constexpr int kMegaMaxNG = 2;                   // <= 16 rows per pass
 constexpr unsigned kSpinLimit = 1u << 26;       // polls before a wait gives up
@@ -482,7 +483,7 @@ __device__ __forceinline__ void build_frags(const MegaArgs& m, const MegaSmem& s
   }
 }
 
-// Phase with K <= 1024 (at most two ring stages per unit).  All eight warps
+// Phase with K <= 1024 (a unit is at most 8 / kTPW ring stages).  All eight warps
 // work on every unit: warp w owns the k-steps s = w (mod 8) -- lane group w
 // of the canonical order -- so it waits only for the inputs of its own
 // k-steps and keeps their fragments in registers.  The CTA's units (up to
@@ -501,7 +502,7 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
   const int u0 = first_unit(p, cta, G);
   if (u0 >= p.units) return true;
   const int nunits = (p.units - u0 + G - 1) / G;
-  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // 1 or 2
+  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // <= 8 / kTPW
   const unsigned it0 = it;
   it += (unsigned)(nunits * nst);
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -536,7 +537,7 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
 #pragma unroll
       for (int n = 0; n < NG; ++n) acc[jv][n][0] = acc[jv][n][1] = acc[jv][n][2] = acc[jv][n][3] = 0.f;
 #pragma unroll
-    for (int st = 0; st < 2; ++st) {
+    for (int st = 0; st < 8 / kTPW; ++st) {
       if (st < nst) {
         const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
 #pragma unroll
@@ -546,18 +547,18 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
             const int slot = itu % sm.S;
             if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
             const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-            uint4 w[4][PL];
+            uint4 w[kTPW][PL];
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kTPW; ++q)
 #pragma unroll
               for (int pl = 0; pl < PL; ++pl)
                 w[q][pl] = *reinterpret_cast<const uint4*>(stage + (size_t)min(8 * q + warp, ntiles - 1) * tile_bytes + pl * 512 + lane * 16);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kTPW; ++q)
               if (8 * q + warp < ntiles)
 #pragma unroll
                 for (int n = 0; n < NG; ++n)
-                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[st * 4 + q][n].x, xf[st * 4 + q][n].y, xf[st * 4 + q][n].z, xf[st * 4 + q][n].w});
+                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[st * kTPW + q][n].x, xf[st * kTPW + q][n].y, xf[st * kTPW + q][n].z, xf[st * kTPW + q][n].w});
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.empty + slot);
           }
@@ -629,9 +630,9 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
   for (int n = 0; n < NG; ++n) src[n] = x_src(m, sm, p, n * 8 + g < nr ? n * 8 + g : 0);
   // unconditional loads (dead rows read row 0, k-steps past the end re-read
   // the last one; neither reaches an output) so all of a stage's are in flight together
-  auto load = [&](int st, float2 (&xa)[4][NG], float2 (&xb)[4][NG]) {
+  auto load = [&](int st, float2 (&xa)[kTPW][NG], float2 (&xb)[kTPW][NG]) {
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < kTPW; ++jj) {
       const int ks = min(st * kStageTiles + 8 * jj + warp, p.ksteps - 1);
 #pragma unroll
       for (int n = 0; n < NG; ++n) {
@@ -644,12 +645,12 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
   // inputs prefetched D stages ahead in registers (an L2 round trip is much
   // longer than one stage's MMAs); stages run in groups of D so the register
   // ring is indexed at compile time
-  constexpr int D = 2 / NG;
+  constexpr int D = (kTPW == 4) ? 2 / NG : 1;
   for (int u = u0; u < p.units; u += G) {
     float acc[NG][4], ss[NG];
 #pragma unroll
     for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
-    float2 xa[D][4][NG], xb[D][4][NG];
+    float2 xa[D][kTPW][NG], xb[D][kTPW][NG];
 #pragma unroll
     for (int d = 0; d < D; ++d)
       if (d < nst) ok = load(d, xa[d], xb[d]) && ok;
@@ -662,22 +663,22 @@ __device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const 
         const int slot = it % sm.S;
         if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
         const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-        float2 (&ca)[4][NG] = xa[d];
-        float2 (&cb)[4][NG] = xb[d];
+        float2 (&ca)[kTPW][NG] = xa[d];
+        float2 (&cb)[kTPW][NG] = xb[d];
         if ((st + 1) * kStageTiles <= p.ksteps) {  // full stage: weight loads first, then the chain
-          uint4 w[4][PL];
+          uint4 w[kTPW][PL];
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
+          for (int jj = 0; jj < kTPW; ++jj)
 #pragma unroll
             for (int q = 0; q < PL; ++q)
               w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)(8 * jj + warp) * tile_bytes + q * 512 + lane * 16);
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
+          for (int jj = 0; jj < kTPW; ++jj)
 #pragma unroll
             for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w[jj], make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
         } else {
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
+          for (int jj = 0; jj < kTPW; ++jj) {
             const int tile = 8 * jj + warp;
             if (st * kStageTiles + tile < p.ksteps) {
               uint4 w[PL];
