@@ -109,3 +109,33 @@ def test_scalar_and_batched_generators_agree():
     a = latent_vectors(0, 1, 3, list(range(48)), [int(k) for k in keys[:48]], 2048)
     b = np.stack([latent_vector(0, 1, 3, i, int(k), 2048) for i, k in enumerate(keys[:48])])
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_driver_latent_slots_and_latents_match_oracle():
+    """The host harness (driver.SeqHost) derives latent slots and the latents to send with
+    its own code; on random commit sequences it agrees with the oracle's rule."""
+    from dataclasses import replace
+
+    from block_diffusion_byte_b200.driver import SeqHost
+    from oracle.model import OracleModel
+    from oracle.policies import OracleSequence
+    from workload import CONFIGS, Patcher, WeightSet
+
+    for kind in ("uniform8", "entropy12"):
+        wl = replace(CONFIGS["tiny_d4"], patch_kind=kind)
+        om = OracleModel(wl.shape, WeightSet(wl.shape).materialize())
+        rng = np.random.default_rng(7)
+        pre = [int(b) for b in rng.integers(0, 256, 40)]
+        o = OracleSequence(om, wl, 0, pre)
+        h = SeqHost(Patcher(kind, wl.seed, wl.cfg_index, 0), wl.seed, wl.cfg_index, 0, wl.shape.d_global)
+        h.commit(pre)
+        for _ in range(30):  # commits of 1..6 bytes, as blocks and accepted drafts arrive
+            new = [int(b) for b in rng.integers(0, 256, int(rng.integers(1, 7)))]
+            o.commit(new)
+            h.commit(new)
+        # nothing was taken, so the host holds every byte's slot and every latent
+        slots, lats = list(h.pend_slots), list(h.lat_ready)
+        assert slots == o.lat
+        assert len(lats) == len(o.st.latents) == o.n_closed
+        for a, b in zip(lats, o.st.latents):
+            assert np.array_equal(np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64))
