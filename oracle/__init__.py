@@ -19,10 +19,13 @@ What it computes, and where it is read from (page titles and sections):
   memory-bandwidth formula (restated on the wangzhan123.com page, section
   "六、测量效能之方式").
 
-Readings where the pages are silent (SwiGLU FFN, pre-norm RMSNorm with eps
-1e-5, rotate-half RoPE with theta 1e4, ``conf >= alpha``, tie-breaks, latent
-slot of open patches ...) are listed in the design doc.  The decoder-layer
+Readings where the pages are silent: a SwiGLU FFN, pre-norm RMSNorm with eps
+1e-5, rotate-half RoPE with theta 1e4, ``conf >= alpha``, argmax ties to the
+lowest byte and fallback ties to the lowest position, and open patches seeing
+the newest closed latent.  The decoder-layer
 internals (RMSNorm, SwiGLU, RoPE) follow those readings: the pages fix none of
 them, so their parity against the pages is unpinned; the tests pin the oracle's
-implementation of each against library routines and closed-form invariants.
+implementation of each against library routines and closed-form invariants,
+and the whole pass against a second statement in torch fp64
+(``tests/test_oracle_restatement.py``).
 """
