@@ -8,11 +8,16 @@ Between blocks the host re-patches the committed bytes and supplies the
 latents of newly closed patches (the synthetic stand-in for the entropy
 patcher + encoder + global model), as in BLT-D inference.
 
-value  decoded bytes/s over all ranks, prefix inputs already on the device
-e2e    the same job through the public API from pinned host buffers
-       (prefix H2D and result D2H inside the timed region)
+value     decoded bytes/s over all ranks, prefix inputs already on the device
+e2e       the same job through the public API from pinned host buffers
+          (prefix H2D and result D2H inside the timed region)
 roofline  the decoder pass (all kernels of one pass) against measured HBM
-       bandwidth: algorithmic bytes per pass / mean pass time (CUDA events)
+          bandwidth: algorithmic bytes per pass / mean pass time (CUDA events)
+batch16   the BLT-S k=8 job at batch 16 (prefix 4096, 512 bytes per sequence),
+          timed the same way
+modes     BLT-S k=8, BLT-DV-16 (one step) and greedy AR on the default job's
+          prefix and length, with the decoder-NFE ratio and the pages' proxy
+          memory bandwidth recomputed from counted passes
 
 Multi-GPU: replicas only (sequences are independent; no collective on the
 data path).  Each rank decodes its own batch; value = all ranks' bytes / the
@@ -115,54 +120,79 @@ class Clocks:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def oracle_rate(wl, seconds_cap: float = 25.0):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload.
+class OracleTimer:
+    """The fp64 oracle, as it stands, timed on a bounded sample of the workload.
 
-    Sample: the full prefill of sequence 0's prefix plus the first blocks
-    (rounds) of decoding until ``seconds_cap`` is reached; the rate is
-    extrapolated to the whole job: gen_bytes / (t_prefill + t_per_byte * gen_bytes).
+    The prefill of sequence 0's prefix runs once (timed); every ``step()`` then
+    decodes a few rounds from a copy of the prefilled state (timed), and the
+    rate is extrapolated to the whole job:
+    gen_bytes / (t_prefill + t_per_byte * gen_bytes), per sequence.
     """
-    from oracle.model import OracleModel
-    from oracle.policies import OracleSequence
 
-    try:
-        from threadpoolctl import threadpool_info
+    def __init__(self, wl, min_bytes: int = 8):
+        import copy
 
-        blas_threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:
-        blas_threads = os.cpu_count() or 1
-    ws = WeightSet(wl.shape, seed=wl.seed).materialize()
-    m = OracleModel(wl.shape, ws)
-    pre = [int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, 0, wl.prefix_len)]
-    o = OracleSequence(m, wl, 0, pre)
-    t0 = time.perf_counter()
-    o.prefill()
-    t_pre = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    made = 0
-    while made < wl.gen_bytes and (time.perf_counter() - t0) < seconds_cap:
-        made += len(o.generate(min(wl.block if wl.mode != "AR" else 1, wl.gen_bytes - made)))
-    t_dec = time.perf_counter() - t1
-    per_byte = t_dec / max(made, 1)
-    rate = wl.gen_bytes * wl.batch / (wl.batch * (t_pre + per_byte * wl.gen_bytes))
-    return {
-        "value": rate,
-        "unit": "bytes/s",
-        "cores": int(blas_threads),
-        "host_cpus": os.cpu_count(),
-        "kind": "oracle",
-        "sample": f"seq 0: full prefill of {wl.prefix_len} bytes ({t_pre:.1f} s) + {made} decoded bytes ({t_dec:.1f} s), "
-        f"extrapolated to {wl.gen_bytes} bytes x batch {wl.batch}",
-    }
+        from oracle.model import OracleModel
+        from oracle.policies import OracleSequence
+
+        self.copy = copy
+        self.wl = wl
+        try:
+            from threadpoolctl import threadpool_info
+
+            self.cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        except Exception:
+            self.cores = os.cpu_count() or 1
+        ws = WeightSet(wl.shape, seed=wl.seed).materialize()
+        pre = [int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, 0, wl.prefix_len)]
+        t0 = time.perf_counter()
+        self.o = OracleSequence(OracleModel(wl.shape, ws), wl, 0, pre)
+        self.o.prefill()
+        self.t_pre = time.perf_counter() - t0
+        self.min_bytes = min_bytes
+
+    def step(self):
+        o = self.copy.deepcopy(self.o)
+        t0 = time.perf_counter()
+        made = 0
+        unit = self.wl.block if self.wl.mode != "AR" else 1
+        while made < self.min_bytes:
+            made += len(o.generate(unit))
+        dt = time.perf_counter() - t0
+        self.last_dt = dt
+        per_byte = dt / made
+        wl = self.wl
+        rate = wl.gen_bytes / (self.t_pre + per_byte * wl.gen_bytes)
+        return {
+            "value": rate,
+            "unit": "bytes/s",
+            "cores": int(self.cores),
+            "host_cpus": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"seq 0: prefill of {wl.prefix_len} bytes once ({self.t_pre:.1f} s), then {made} decoded bytes "
+            f"({dt:.2f} s) from a copy of the prefilled state, extrapolated to {wl.gen_bytes} bytes per sequence",
+        }
+
+
+def oracle_rate(wl, seconds_cap: float = 20.0):
+    """cpu_baseline of the engine arm: the prefill once, then decoded rounds doubling
+    until the sample would pass about seconds_cap of CPU time."""
+    t = OracleTimer(wl, min_bytes=max(8, int(wl.block)))
+    r = t.step()
+    while t.t_pre + 3 * t.last_dt < seconds_cap and t.min_bytes < wl.gen_bytes:
+        t.min_bytes *= 2
+        r = t.step()
+    return r
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    timer = OracleTimer(wl)
     steps = []
     for i in range(args.warmup + args.steps):
-        r = oracle_rate(wl, seconds_cap=args.ref_seconds)
+        r = timer.step()
         if i >= args.warmup:
             steps.append(r)
     v = statistics.mean(s["value"] for s in steps)
@@ -206,6 +236,142 @@ def workload_config(wl):
     }
 
 
+def proxy_gb_counted(passes: int, latents: int, p_dec: float) -> float:
+    """The pages' proxy memory bandwidth, GB = 2 [N_dec P_dec + N_enc (P_enc + P_global)] / 1e9,
+    from counted decoder passes and global-model calls (one per latent consumed), with the
+    1B model's encoder and global sizes (19M, 1.28B) and this decoder's streamed parameters."""
+    return 2.0 * (passes * p_dec + latents * (19e6 + 1.28e9)) / 1e9
+
+
+def time_job(eng, wl, prefixes, seq_ids, steps, warmup, barrier, generate, B):
+    """Warm-up, then `steps` whole jobs bracketed by CUDA events on the engine's stream."""
+    import torch
+
+    nb = len(prefixes)
+
+    def one():
+        B.blt_dec_rewind(eng.h, nb, [0] * nb, [0] * nb)
+        return generate(eng, wl, prefixes, seq_ids=seq_ids)
+
+    for _ in range(warmup):
+        one()
+    st0 = B.blt_dec_stats(eng.h)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = d2h = 0
+    ev0.record(eng.stream)
+    for _ in range(steps):
+        r = one()
+        h2d += r.h2d_bytes
+        d2h += r.d2h_bytes
+    ev1.record(eng.stream)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    st1 = B.blt_dec_stats(eng.h)
+    d = {k: st1[k] - st0[k] for k in st1}
+    return ms, d, h2d, d2h, one
+
+
+def pass_figures(d, steps, ms, peak, pk_kind):
+    """Per-pass figures of the decoder passes in d (prefill excluded)."""
+    passes = d["passes"]
+    tp = max(d["timed_passes"], 1)
+    pass_ms = d["pass_ns"] / 1e6 / tp
+    weight_b = d["weight_bytes"] / max(passes, 1)
+    kv_b = d["kv_read_bytes"] / tp
+    alg_bytes = weight_b + kv_b
+    achieved = alg_bytes / (pass_ms / 1000.0) / 1e9 if pass_ms > 0 else 0.0
+    roof = {
+        "bound": "hbm",
+        "achieved": achieved,
+        "peak": peak,
+        "peak_kind": pk_kind,
+        "unit": "GB/s",
+        "frac": achieved / peak,
+        "frac_of_8tbs": achieved / 8000.0,
+        "alg_bytes_per_pass": alg_bytes,
+        "pass_ms": pass_ms,
+    }
+    dec = {
+        "passes_per_step": passes / steps,
+        "passes_per_s": passes / (ms / 1000.0),
+        "rows_per_pass": (d["rows"] - d["prefill_rows"]) / tp,
+        "weight_bytes_per_pass": weight_b,
+        "kv_bytes_per_pass": kv_b,
+        "launches_per_step": d["kernel_launches"] / steps,
+        "persistent_calls_per_step": d["persistent_calls"] / steps,
+    }
+    return roof, dec
+
+
+class _TimingWeights:
+    """Weights of a given shape for timing only: one random set of layer tensors, shared by
+    every layer (the engine copies each layer separately), so a 1.2B-parameter model costs
+    one layer's worth of host memory and generation time.  Values do not change the time."""
+
+    def __init__(self, shape, seed=0):
+        from workload.gen import GLOBAL_TENSORS, LAYER_TENSORS, tensor_shape
+
+        rng = np.random.default_rng(seed)
+        self.shape = shape
+        self._layer = {}
+        for n in LAYER_TENSORS:
+            dims = tensor_shape(shape, n)
+            if n.endswith("norm") or n == "norm_c":
+                self._layer[n] = np.ones(dims, np.float32)
+            else:
+                self._layer[n] = (rng.standard_normal(dims, dtype=np.float32) / np.sqrt(shape.d_model)).astype(np.float32)
+        self._glob = {n: (rng.standard_normal(tensor_shape(shape, n), dtype=np.float32) / np.sqrt(shape.d_model)).astype(np.float32)
+                      for n in GLOBAL_TENSORS}
+        self._glob["final_norm"] = np.ones(shape.d_model, np.float32)
+
+    def get(self, name, layer=-1):
+        return self._glob[name] if layer < 0 else self._layer[name]
+
+    def layer(self, l):
+        return dict(self._layer)
+
+
+def global_step_timing(barrier, generate, B, Engine, peak, tokens: int = 256, steps: int = 48):
+    """One step of a global transformer at the pages' 1B size on the device, so the
+    N_enc (P_enc + P_global) term of the proxy can be timed: 24 layers, d 2048, 16 heads,
+    FFN 5632 (1.23B parameters per step, bf16), one new token per step after `tokens`
+    cached ones (the global model sees one latent per patch), run through this engine's
+    own per-phase kernels (greedy AR steps of one row)."""
+    import torch
+    from dataclasses import replace
+
+    from workload import ModelShape, Workload
+
+    shape = ModelShape(n_layers=24, d_model=2048, n_heads=16, d_ffn=5632, d_global=128, weight_dtype="bf16")
+    wl = Workload("global_1b_step", shape, "AR", 1, 0.0, steps, 1, tokens, "uniform8", 0, 9)
+    ws = _TimingWeights(shape)
+    eng = Engine(shape, ws, max_batch=1, max_ctx=tokens + steps + 32, max_block=16, max_rows=1024, time_passes=True,
+                 persistent=False)
+    try:
+        pre = [[int(b) for b in prefix_bytes(0, 9, 0, tokens)]]
+        generate(eng, wl, pre, 4)  # warm-up
+        B.blt_dec_rewind(eng.h, 1, [0], [0])
+        st0 = B.blt_dec_stats(eng.h)
+        generate(eng, wl, pre, steps)
+        st1 = B.blt_dec_stats(eng.h)
+    finally:
+        eng.close()
+    d = {k: st1[k] - st0[k] for k in st1}
+    step_ms = d["pass_ns"] / 1e6 / max(d["timed_passes"], 1)
+    params = shape.pass_weight_params() + 256 * shape.d_model
+    return {
+        "shape": {"layers": 24, "d_model": 2048, "heads": 16, "d_ffn": 5632, "params": params},
+        "step_ms": step_ms,
+        "weight_gb_per_step": 2.0 * params / 1e9,
+        "achieved_gbs": 2.0 * params / (step_ms / 1000.0) / 1e9,
+        "frac_of_peak": 2.0 * params / (step_ms / 1000.0) / 1e9 / peak,
+        "path": "per-phase kernels (d 2048 exceeds the persistent kernel's d <= 1024)",
+        "note": "synthetic stand-in for the pages' 1B global model (1.28B); random weights shared across layers "
+        "(timing only); one token per step over a cache of %d tokens" % tokens,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -213,9 +379,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
     ap.add_argument("--workload", default="d4_b1", choices=sorted(CONFIGS))
-    ap.add_argument("--ref-seconds", type=float, default=25.0)
+    ap.add_argument("--ref-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-ar-baseline", action="store_true", help="skip the greedy AR decoding of the same job")
+    ap.add_argument("--no-extras", action="store_true", help="skip the batch-16 job and the BLT-S / BLT-DV / AR comparison")
+    ap.add_argument("--no-ar-baseline", action="store_true", help="same as --no-extras (kept for old command lines)")
     ap.add_argument("--path", default="persistent", choices=["persistent", "phased"],
                     help="decoder passes in the persistent kernel (one launch per call) or as per-phase kernels")
     args = ap.parse_args()
@@ -246,41 +413,27 @@ def main():
         build()
     if dist:
         dist.barrier()
-    ws = WeightSet(wl.shape, seed=wl.seed).materialize()
-    nb = wl.batch
-    max_ctx = wl.prefix_len + wl.gen_bytes + 4 * wl.block + 16
-    eng = Engine(wl.shape, ws, max_batch=nb, max_ctx=max_ctx, max_block=max(wl.block, 16), max_rows=1024, time_passes=True,
-                 persistent=args.path == "persistent")
-    seq_ids = shard_ids(rank, world, nb)
-    prefixes = [[int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, s, wl.prefix_len)] for s in seq_ids]
-
-    def one_step():
-        B.blt_dec_rewind(eng.h, nb, [0] * nb, [0] * nb)
-        return generate(eng, wl, prefixes, seq_ids=seq_ids)
+    persistent = args.path == "persistent"
 
     def barrier():
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        one_step()
-    st0 = B.blt_dec_stats(eng.h)
-    barrier()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h2d = d2h = 0
+    def engine_for(w, ws_):
+        max_ctx = w.prefix_len + w.gen_bytes + 4 * max(w.block, 16) + 16
+        return Engine(w.shape, ws_, max_batch=w.batch, max_ctx=max_ctx, max_block=max(w.block, 16), max_rows=1024,
+                      time_passes=True, persistent=persistent)
+
+    ws = WeightSet(wl.shape, seed=wl.seed).materialize()
+    nb = wl.batch
+    eng = engine_for(wl, ws)
+    seq_ids = shard_ids(rank, world, nb)
+    prefixes = [[int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, s, wl.prefix_len)] for s in seq_ids]
+
     with Clocks(local) as clk:
-        ev0.record(eng.stream)
-        for _ in range(args.steps):
-            r = one_step()
-            h2d += r.h2d_bytes
-            d2h += r.d2h_bytes
-        ev1.record(eng.stream)
-        barrier()
-    ms = ev0.elapsed_time(ev1)
-    st1 = B.blt_dec_stats(eng.h)
+        ms, d, h2d, d2h, one_step = time_job(eng, wl, prefixes, seq_ids, args.steps, args.warmup, barrier, generate, B)
     clocks = clk.summary()
-    d = {k: st1[k] - st0[k] for k in st1}
     ms = max_over_ranks(ms, "cuda")
     total_bytes = wl.gen_bytes * nb * world * args.steps
     value = total_bytes / (ms / 1000.0)
@@ -291,20 +444,18 @@ def main():
     t0 = time.perf_counter()
     e2e_steps = max(1, min(args.steps, 3))
     for _ in range(e2e_steps):
-        r = one_step()
+        one_step()
     barrier()
     e2e_s = max_over_ranks((time.perf_counter() - t0) / e2e_steps, "cuda")
     e2e_value = wl.gen_bytes * nb * world / e2e_s
 
     pk, pk_kind = peaks()
-    passes = d["passes"]
-    pass_ms = d["pass_ns"] / 1e6 / max(d["timed_passes"], 1)
-    weight_b = d["weight_bytes"] / max(passes, 1)
-    kv_b = d["kv_read_bytes"] / max(d["timed_passes"], 1)
-    rows_per_pass = d["rows"] / max(d["timed_passes"], 1)
-    alg_bytes = weight_b + kv_b
-    achieved = alg_bytes / (pass_ms / 1000.0) / 1e9 if pass_ms > 0 else 0.0
     peak = float(pk["hbm_gbs"])
+    roof, dec = pass_figures(d, args.steps, ms, peak, pk_kind)
+    roof["traffic"] = measured_traffic(wl.name, bool(d["persistent_calls"]))
+    roof["traffic_unit"] = "bytes per pass (dram__bytes_read.sum + dram__bytes_write.sum)"
+    roof["kernel"] = "k_mega (persistent decoder pass)" if d["persistent_calls"] else "decoder pass (all kernels of one pass)"
+    dec["path"] = args.path
     line = {
         "metric": "decoded bytes/s",
         "value": value,
@@ -321,65 +472,81 @@ def main():
         "config": workload_config(wl),
         "e2e": {"value": e2e_value, "unit": "bytes/s", "h2d_bytes_per_step": h2d // args.steps, "d2h_bytes_per_step": d2h // args.steps},
         "gpu_launches": d["kernel_launches"],
-        "roofline": {
-            "bound": "hbm",
-            "achieved": achieved,
-            "peak": peak,
-            "peak_kind": pk_kind,
-            "unit": "GB/s",
-            "frac": achieved / peak,
-            "frac_of_8tbs": achieved / 8000.0,
-            "traffic": measured_traffic(wl.name, bool(d["persistent_calls"])),
-            "traffic_unit": "bytes per pass (dram__bytes_read.sum + dram__bytes_write.sum)",
-            "kernel": "k_mega (persistent decoder pass)" if d["persistent_calls"] else "decoder pass (all kernels of one pass)",
-            "alg_bytes_per_pass": alg_bytes,
-            "pass_ms": pass_ms,
-        },
-        "decoder": {
-            "passes_per_step": passes / args.steps,
-            "passes_per_s": passes / (ms / 1000.0),
-            "rows_per_pass": rows_per_pass,
-            "weight_bytes_per_pass": weight_b,
-            "kv_bytes_per_pass": kv_b,
-            "launches_per_step": d["kernel_launches"] / args.steps,
-            "path": args.path,
-            "persistent_calls_per_step": d["persistent_calls"] / args.steps,
-        },
+        "roofline": roof,
+        "decoder": dec,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_ar_baseline and wl.mode != "AR":
-        # the same job decoded one byte per pass (plain greedy AR BLT) on the same
-        # engine: wall-clock speedup beside the decoder-NFE ratio (the pages' proxy)
+    p_dec = float(wl.shape.pass_weight_params() + 256 * wl.shape.d_model)
+    if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
         from dataclasses import replace
 
-        wl_ar = replace(wl, mode="AR", block=1, alpha=0.0)
-
-        def ar_step():
-            B.blt_dec_rewind(eng.h, nb, [0] * nb, [0] * nb)
-            return generate(eng, wl_ar, prefixes, seq_ids=seq_ids)
-
-        ar_step()
-        sa0 = B.blt_dec_stats(eng.h)
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(eng.stream)
-        ar_step()
-        e1.record(eng.stream)
-        barrier()
-        ar_ms = e0.elapsed_time(e1)
-        sa1 = B.blt_dec_stats(eng.h)
-        ar_passes = sa1["passes"] - sa0["passes"]
-        ar_value = wl.gen_bytes * nb / (ar_ms / 1000.0)
-        line["ar_baseline"] = {
-            "value": ar_value,
-            "unit": "bytes/s",
-            "ms_per_step": ar_ms,
-            "passes_per_step": ar_passes,
-            "speedup_wallclock": value / ar_value,
-            "decoder_nfe_ratio": ar_passes / (passes / args.steps),
-            "note": "same engine, prefix and length; greedy AR decoding (one byte per decoder pass); "
-            "decoder_nfe_ratio = AR passes / this mode's passes, the decoder term of the pages' proxy",
+        # BLT-S k=8, BLT-DV-16 (one step) and greedy AR on the same engine, prefix and length:
+        # wall clock beside the decoder-NFE ratio and the pages' proxy bandwidth from counted passes
+        modes = {}
+        for name, w in (("AR", replace(wl, name="ar_b1", mode="AR", block=1, alpha=0.0)),
+                        ("BLT-D-4", wl),
+                        ("BLT-S-8", replace(wl, name="s8_p1024", mode="S", block=8, alpha=0.0)),
+                        ("BLT-DV-16", replace(wl, name="dv16_p1024", mode="DV", block=16, alpha=0.0))):
+            e2 = engine_for(w, ws)
+            try:
+                msm, dm, _, _, _ = time_job(e2, w, prefixes, seq_ids, 1, 1, barrier, generate, B)
+            finally:
+                e2.close()
+            modes[name] = {
+                "value": w.gen_bytes * nb / (msm / 1000.0),
+                "unit": "bytes/s",
+                "ms_per_step": msm,
+                "decoder_passes": dm["passes"],
+                "global_calls": dm["latents"],
+                "proxy_gb": proxy_gb_counted(dm["passes"], dm["latents"], p_dec),
+            }
+        ar = modes["AR"]
+        for name, mrec in modes.items():
+            mrec["speedup_wallclock_vs_ar"] = mrec["value"] / ar["value"]
+            mrec["decoder_nfe_ratio_vs_ar"] = ar["decoder_passes"] / max(mrec["decoder_passes"], 1)
+            mrec["proxy_reduction_vs_ar"] = 1.0 - mrec["proxy_gb"] / ar["proxy_gb"]
+        line["modes"] = {
+            "note": "same engine, weights, prefix 1024 and 512 bytes; proxy_gb = 2 [decoder passes x decoder params + "
+            "global calls x (19M + 1.28B)] / 1e9 (the pages' formula, 1B encoder/global sizes, calls counted as latents consumed)",
+            **modes,
         }
+    if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
+        # decoded bytes/s at batch 16: BLT-S k=8, prefix 4096, 512 bytes per sequence
+        w16 = CONFIGS["s8_b16"]
+        e16 = engine_for(w16, ws)
+        try:
+            ids16 = list(range(w16.batch))
+            pre16 = [[int(b) for b in prefix_bytes(w16.seed, w16.cfg_index, s, w16.prefix_len)] for s in ids16]
+            ms16, d16, h16, o16, _ = time_job(e16, w16, pre16, ids16, 2, 1, barrier, generate, B)
+        finally:
+            e16.close()
+        roof16, dec16 = pass_figures(d16, 2, ms16, peak, pk_kind)
+        dec16["path"] = args.path
+        line["batch16"] = {
+            "config": workload_config(w16),
+            "value": w16.gen_bytes * w16.batch * 2 / (ms16 / 1000.0),
+            "unit": "bytes/s",
+            "steps": 2,
+            "warmup": 1,
+            "ms_per_step": ms16 / 2,
+            "roofline": roof16,
+            "decoder": dec16,
+            "note": "drafting passes (16 rows) run in the persistent kernel, verification passes (128 rows) in the per-phase "
+            "kernels; roofline over all decoder passes of the job",
+        }
+    if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
+        # the N_enc term of the pages' proxy, timed: one global-model step at the 1B size
+        gs = global_step_timing(barrier, generate, B, Engine, peak)
+        line["global_step"] = gs
+        if "modes" in line:
+            for name, mrec in line["modes"].items():
+                if isinstance(mrec, dict) and "decoder_passes" in mrec:
+                    # wall clock of the whole BLT step: the decoder job as measured plus one global step per latent
+                    mrec["with_global_ms"] = mrec["ms_per_step"] + mrec["global_calls"] * gs["step_ms"]
+            ar_tot = line["modes"]["AR"]["with_global_ms"]
+            for name, mrec in line["modes"].items():
+                if isinstance(mrec, dict) and "with_global_ms" in mrec:
+                    mrec["speedup_with_global_vs_ar"] = ar_tot / mrec["with_global_ms"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(wl, seconds_cap=args.ref_seconds)
     eng.close()

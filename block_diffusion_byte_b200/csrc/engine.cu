@@ -11,6 +11,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "bltdec.h"
 #include "kernels.cuh"
 #include "mega.cuh"
@@ -18,6 +20,15 @@
 using namespace bltdec;
 
 namespace {
+
+// NVTX range for the lifetime of a scope (per C-ABI call, per decoder pass);
+// free unless a profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 struct Mat {
   uint4* w = nullptr;
@@ -88,12 +99,15 @@ struct blt_dec {
   bool mega_ok = false;
   int nsm = 0;
   LayerW* d_layers = nullptr;
-  unsigned* flags = nullptr;
-  unsigned* attn_cnt = nullptr;
+  unsigned* flags = nullptr;  // [0] decision epoch, [1] pass-end arrivals
   unsigned* dec_val = nullptr;
   int* abort_flag = nullptr;
   unsigned epoch = 0;
-  int f_qkv = 0, f_o = 0, f_w13 = 0, f_w2 = 0, f_head = 0, f_att = 0, f_dec = 0, mega_groups = 0;
+  unsigned long long* xbuf = nullptr;  // exchange words of the persistent kernel (one allocation)
+  size_t xbuf_words = 0;
+  unsigned long long *x_h = nullptr, *x_q = nullptr, *x_k = nullptr, *x_v = nullptr, *x_att = nullptr, *x_act = nullptr,
+                     *x_w2p = nullptr, *x_logit = nullptr, *x_part = nullptr;
+  int x_cmax = 0;
   // debug: BLTDEC_TRACE=<file> appends device timestamps of each persistent launch's first pass
   unsigned long long* trace = nullptr;
   std::string trace_path;
@@ -216,7 +230,8 @@ constexpr int gemm_stages() {
 template <int NG, int PL, int EPI>
 size_t gemm_smem() {
   constexpr int RB = 8 * NG;
-  return (size_t)gemm_stages<NG, PL, EPI>() * RB * kXStride * 4 + 8 * RB * 4;
+  // activation stages, the RMS partials [8][RB], and the K-segment fold buffer [8][16][RB]
+  return (size_t)gemm_stages<NG, PL, EPI>() * RB * kXStride * 4 + 8 * RB * 4 + 8 * 16 * RB * 4;
 }
 
 template <int NG, int PL, int EPI>
@@ -349,6 +364,7 @@ int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head
   return run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head);
 }
 int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
+  NvtxRange nvtx_("decoder pass (per-phase kernels)");
   const int d = h->d;
   // embed + per layer (cross add, attention partial + combine) + head statistics; GEMMs count themselves
   h->launches += 1 + 3 * (unsigned long long)h->L + (want_head ? 1 : 0);
@@ -631,9 +647,10 @@ __global__ void k_copy_logits(const float* src, float* dst, int n) {
 // ---------------------------------------------------------------------------- persistent pass kernel
 template <int NG, int PL, int DH, typename KVT>
 size_t mega_smem(const blt_dec* h) {
-  const size_t attn = (size_t)(kAttnRows * DH + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * kv_stride<DH, KVT>() * sizeof(KVT);
-  const size_t xin = (size_t)kMegaUnits * 8 * 16 * 8 * NG * 4;  // multi-unit reduction buffer
-  return (size_t)kRingBytes + 8 * 16 * 8 * kMegaMaxNG * 4 + 8 * 8 * kMegaMaxNG * 4 + 16 * 4 + std::max(attn, xin);
+  (void)h;
+  const size_t red = (size_t)kMaxPieces * 8 * 16 * 8 * NG * 4;
+  const size_t att = (size_t)(kMegaRows * DH + kMegaRows * 128) * 4;
+  return (size_t)kRingSlots * kSlotBytes + std::max(red, att) + 8 * 8 * kMegaMaxNG * 4 + 2 * (size_t)kMaxPieces * kMegaRows * 16 * 4;
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -654,16 +671,18 @@ int mega_prepare_pd(blt_dec* h) {
 
 // Decide whether the persistent kernel applies to this model and set it up.
 int mega_setup(blt_dec* h) {
+  const int es = h->kv_f32 ? 4 : 2;
+  const int nseg = h->F > kSegCols ? h->F / kSegCols : 1;
   if (!(h->cfg.flags & BLT_FLAG_PERSISTENT) || h->d > 1024 || h->d % 128 != 0 || h->F % 128 != 0 || h->F > 4096 ||
-      (h->dh != 32 && h->dh != 64) ||
-      h->CH > 128)
+      (h->F > kSegCols && h->F % kSegCols != 0) || (h->dh != 32 && h->dh != 64) || h->CH != 128 || 128 % h->PT != 0 ||
+      2 * h->CH * h->dh * es > kSlotBytes)
     return BLT_OK;
   int dev = 0;
   CK(cudaGetDevice(&dev));
   int coop = 0;
   CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev));
   CK(cudaDeviceGetAttribute(&h->nsm, cudaDevAttrMultiProcessorCount, dev));
-  if (!coop) return BLT_OK;
+  if (!coop || h->nsm < nseg) return BLT_OK;
   int rc;
   if (h->planes == 1) {
     rc = h->kv_f32 ? (h->dh == 64 ? mega_prepare_pd<1, 64, float>(h) : mega_prepare_pd<1, 32, float>(h))
@@ -682,20 +701,26 @@ int mega_setup(blt_dec* h) {
     lw[l] = LayerW{h->qkv[l].w, h->o[l].w, h->w13[l].w, h->w2[l].w, h->attn_norm[l], h->ffn_norm[l]};
   TRY(dalloc(h, &h->d_layers, h->L));
   CK(cudaMemcpy(h->d_layers, lw.data(), sizeof(LayerW) * h->L, cudaMemcpyHostToDevice));
-  const int d = h->d, F = h->F;
-  h->mega_groups = kMegaMaxNG * 8 + 1;  // <= 16 rows: at most 16 sequences, one group each
-  h->f_qkv = 0;
-  h->f_o = h->f_qkv + 3 * d / 16;
-  h->f_w13 = h->f_o + d / 16;
-  h->f_w2 = h->f_w13 + 2 * F / 16;
-  h->f_head = h->f_w2 + d / 16;
-  h->f_att = h->f_head + 16;
-  h->f_dec = h->f_att + h->mega_groups * h->H;
-  const int nflags = h->f_dec + 1;
-  TRY(dalloc(h, &h->flags, nflags));
-  CK(cudaMemset(h->flags, 0, nflags * 4));
-  TRY(dalloc(h, &h->attn_cnt, h->mega_groups * h->H));
-  CK(cudaMemset(h->attn_cnt, 0, h->mega_groups * h->H * 4));
+  // exchange words: [rows][d] x5 (stream, q, k, v, attention), [rows][F], [nseg-1][rows][d], [rows][256],
+  // and the chunk partials [rows][H][CMAX][2 + dh]
+  const size_t R = kMegaRows, d = h->d;
+  h->x_cmax = (h->cfg.max_ctx + h->CH - 1) / h->CH;
+  const size_t n_part = R * h->H * (size_t)h->x_cmax * (2 + h->dh);
+  h->xbuf_words = 5 * R * d + R * h->F + (size_t)std::max(nseg - 1, 1) * R * d + R * 256 + n_part;
+  TRY(dalloc(h, &h->xbuf, h->xbuf_words));
+  CK(cudaMemset(h->xbuf, 0, h->xbuf_words * 8));
+  unsigned long long* p = h->xbuf;
+  h->x_h = p, p += R * d;
+  h->x_q = p, p += R * d;
+  h->x_k = p, p += R * d;
+  h->x_v = p, p += R * d;
+  h->x_att = p, p += R * d;
+  h->x_act = p, p += R * h->F;
+  h->x_w2p = p, p += (size_t)std::max(nseg - 1, 1) * R * d;
+  h->x_logit = p, p += R * 256;
+  h->x_part = p;
+  TRY(dalloc(h, &h->flags, 2));
+  CK(cudaMemset(h->flags, 0, 8));
   TRY(dalloc(h, &h->dec_val, 1));
   TRY(dalloc(h, &h->abort_flag, 1));
   CK(cudaMemset(h->abort_flag, 0, 4));
@@ -710,7 +735,7 @@ int mega_setup(blt_dec* h) {
 }
 
 bool use_mega(const blt_dec* h, int rows_ub, int batch) {
-  return h->mega_ok && rows_ub <= 8 * kMegaMaxNG && batch <= 8 * kMegaMaxNG;
+  return h->mega_ok && rows_ub <= kMegaRows && batch <= kMegaRows;
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -726,6 +751,7 @@ int mega_launch_t(blt_dec* h, MegaArgs& m) {
 // All passes of one call in one launch (rows of pass 1 already planned).
 int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes, int rows_ub, const int* vlat, float* out_logits,
              int* out_acc, unsigned char* out_next) {
+  NvtxRange nvtx_("decoder passes (persistent kernel, one launch)");
   MegaArgs m{};
   m.layers = h->d_layers;
   m.whead = h->head.w;
@@ -738,14 +764,19 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.planes = h->planes;
   m.eps = h->cfg.norm_eps;
   m.ga = base_args(h);
-  m.ga.q = h->q;
   m.aa = attn_args(h);
   m.rows = h->rows;
   m.sd = h->sd;
-  m.h = h->h;
-  m.q = h->q;
-  m.att = h->att;
-  m.act = h->act;
+  m.x_h = h->x_h;
+  m.x_q = h->x_q;
+  m.x_k = h->x_k;
+  m.x_v = h->x_v;
+  m.x_part = h->x_part;
+  m.x_att = h->x_att;
+  m.x_act = h->x_act;
+  m.x_w2p = h->x_w2p;
+  m.x_logit = h->x_logit;
+  m.CMAX = h->x_cmax;
   m.logits = h->logits;
   m.conf = h->conf;
   m.ent = h->ent;
@@ -753,18 +784,22 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.pred = h->pred;
   m.gap = h->gap;
   m.flags = h->flags;
-  m.f_qkv = h->f_qkv;
-  m.f_o = h->f_o;
-  m.f_w13 = h->f_w13;
-  m.f_w2 = h->f_w2;
-  m.f_head = h->f_head;
-  m.f_att = h->f_att;
-  m.f_dec = h->f_dec;
-  m.attn_cnt = h->attn_cnt;
   m.dec_val = h->dec_val;
+  // epochs: unique per (call, pass, layer, stage); restart from zeroed words long before they wrap
+  const unsigned span = (unsigned)(max_passes + 1) * (unsigned)(h->L + 1) * 8u + 16u;
+  if (h->epoch > 0xF0000000u - span) {
+    CK(cudaMemsetAsync(h->xbuf, 0, h->xbuf_words * 8, h->stream));
+    CK(cudaMemsetAsync(h->flags, 0, 8, h->stream));
+    h->epoch = 1;
+  }
   m.epoch0 = h->epoch;
-  h->epoch += (unsigned)(max_passes + 1) * (h->L + 1) + 1;
+  h->epoch += span;
+  CK(cudaMemsetAsync(h->flags + 1, 0, 4, h->stream));  // pass-end arrivals of this launch
+  CK(cudaMemsetAsync(h->abort_flag, 0, 4, h->stream));
   m.abort = h->abort_flag;
+  const bool stall = (h->cfg.flags & BLT_FLAG_TEST_STALL) != 0;
+  m.wait_ns = stall ? 2000000ull : 500000000ull;  // 2 ms under the test-only stall, else 0.5 s
+  m.stall_test = stall ? 1 : 0;
   m.trace = h->trace;
   if (h->trace) {
     h->trace_pending = 1;
@@ -928,7 +963,7 @@ struct NaSwap {
     h->n_lat_rows = c.take<int>(1);
     h->CMAX = kNaCMax;
     h->cfg.max_rows = kNaRows;
-    h->proj_rows = std::max(1, (int)((size_t)kNaRows * kNaMaxD / ((size_t)h->L * h->d)));  // tmp holds rows x L*d
+    h->proj_rows = (int)((size_t)kNaRows * kNaMaxD / ((size_t)h->L * h->d));  // tmp holds rows x L*d; >= 1 (L*d checked)
     used = c.off;
   }
   size_t used = 0;
@@ -945,6 +980,7 @@ struct NaSwap {
 extern "C" {
 
 int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda_stream, blt_dec_t** out) {
+  NvtxRange nvtx_("blt_dec_init");
   if (!cfg || !w || !out) return BLT_ERR_INVALID_ARG;
   *out = nullptr;
   blt_dec* h = new blt_dec();
@@ -1146,6 +1182,7 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
 }
 
 int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_prefill");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   if (h->state != 0) return fail(h, BLT_ERR_STATE, "a draft is waiting for verification");
@@ -1159,12 +1196,14 @@ int blt_dec_prefill(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out
 }
 
 int blt_dec_prefill_noalloc(blt_dec_t* h, int batch, const blt_rows_in* rows, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_prefill_noalloc");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   if (h->state != 0) return fail(h, BLT_ERR_STATE, "a draft is waiting for verification");
-  if (h->d > kNaMaxD || h->F > kNaMaxF || h->H > kNaMaxH || h->dh > kNaMaxDh || h->CH != kNaChunk)
+  if (h->d > kNaMaxD || h->F > kNaMaxF || h->H > kNaMaxH || h->dh > kNaMaxDh || h->CH != kNaChunk ||
+      (size_t)h->L * h->d > (size_t)kNaRows * kNaMaxD)
     return fail(h, BLT_ERR_INVALID_ARG, "model exceeds the static prefill arena (d <= %d, d_ffn <= %d, heads <= %d, head dim <= %d, "
-                "attn_chunk %d)", kNaMaxD, kNaMaxF, kNaMaxH, kNaMaxDh, kNaChunk);
+                "attn_chunk %d, n_layers * d <= %d)", kNaMaxD, kNaMaxF, kNaMaxH, kNaMaxDh, kNaChunk, kNaRows * kNaMaxD);
   TRY(check_pending(h, rows, true));
   CallDesc cd;
   TRY(make_desc(h, batch, rows->row_offsets, rows->latent_offsets, cd));
@@ -1184,6 +1223,7 @@ int blt_dec_prefill_noalloc(blt_dec_t* h, int batch, const blt_rows_in* rows, fl
 
 int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float alpha, int max_steps,
                           uint8_t* out_block, int32_t* out_steps, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_diffuse_block");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   h->state = 0;  // a waiting draft is discarded
@@ -1214,6 +1254,7 @@ int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, i
 
 int blt_dec_diffuse_block_eb(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float gamma, int max_steps,
                              uint8_t* out_block, int32_t* out_steps, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_diffuse_block_eb");
   if (!h) return BLT_ERR_INVALID_ARG;
   if (!(gamma >= 0.f) || gamma == INFINITY) {
     h->err.clear();
@@ -1227,6 +1268,7 @@ int blt_dec_diffuse_block_eb(blt_dec_t* h, int batch, const blt_rows_in* pending
 
 int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode, int k, float alpha, int max_steps,
                   uint8_t* out_draft, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_draft");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   h->state = 0;  // a waiting draft is discarded
@@ -1292,6 +1334,7 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
 
 int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const float* new_latents,
                           const int32_t* latent_offsets, int32_t* out_accepted, uint8_t* out_next, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_verify_accept");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   if (h->state != 1) return fail(h, BLT_ERR_STATE, "no draft is waiting for verification");
@@ -1327,6 +1370,7 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
 }
 
 int blt_dec_rewind(blt_dec_t* h, int batch, const int32_t* kv_len, const int32_t* n_latents) {
+  NvtxRange nvtx_("blt_dec_rewind");
   if (!h) return BLT_ERR_INVALID_ARG;
   h->err.clear();
   if (batch < 1 || batch > h->cfg.max_batch) return fail(h, BLT_ERR_INVALID_ARG, "batch %d", batch);
@@ -1368,10 +1412,12 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->timed_passes = (h->cfg.flags & BLT_FLAG_TIME_PASSES) ? c[0] : 0;
   out->pass_ns = h->pass_ns;
   out->persistent_calls = h->persistent_calls;
+  out->prefill_kv_read_bytes = c[7];
   return BLT_OK;
 }
 
 int blt_dec_sync(blt_dec_t* h) {
+  NvtxRange nvtx_("blt_dec_sync");
   if (!h) return BLT_ERR_INVALID_ARG;
   CK(cudaStreamSynchronize(h->stream));
   if (h->trace && h->trace_pending) {

@@ -17,9 +17,12 @@
 //   is rs * (((a_0 + a_1) + ...) + a_7).  The RMS scale rs = 1/sqrt(ss/K + eps)
 //   takes ss from the same fragments: every lane adds x^2 of its four values in
 //   k order, the four lanes of a row are summed by xor-shuffles (1 then 2) and
-//   the eight groups in order.  Nothing depends on which other rows share the
-//   pass, or on which kernel (per-phase or persistent) runs it, so a row's
-//   results are bit-identical in every pass shape.
+//   the eight groups in order.  K beyond 1024 is cut into segments of 1024
+//   columns (64 k-steps): each segment is reduced as above, and the segment
+//   sums are added in order, ((S_0 + S_1) + S_2) + ..., before the scale.
+//   Nothing depends on which other rows share the pass, or on which kernel
+//   (per-phase or persistent) runs it, so a row's results are bit-identical
+//   in every pass shape.
 #pragma once
 
 #include "common.cuh"
@@ -43,6 +46,7 @@ struct RowsDev {  // per-pass row metadata (arrays of max_rows; counts are devic
 };
 
 constexpr int kMaxCallBatch = 256;
+constexpr int kSegCols = 1024;  // canonical K segment (columns)
 
 struct CallDesc {  // by value as a kernel parameter
   int batch;
@@ -62,7 +66,7 @@ struct SeqDev {
   unsigned char* blk;     // [batch][kMaxBlock] block / draft bytes
   unsigned char* masked;  // [batch][kMaxBlock]
   int* status;
-  unsigned long long* counters;  // passes, rows, prefill_rows, latents, calls, weight_bytes, kv_bytes
+  unsigned long long* counters;  // passes, rows, prefill_rows, latents, calls, weight_bytes, kv_bytes (decoder passes), kv_bytes (prefill)
 };
 
 enum PlanMode : int { PL_PREFILL = 0, PL_FIRST = 1, PL_BLOCK = 2, PL_ARDRAFT = 3, PL_VERIFY = 4 };
@@ -139,8 +143,9 @@ __device__ __forceinline__ void mma_step(float (&c)[4], const uint4 (&w)[PL], co
   if constexpr (PL == 2) mma16816(c, w[1], x.b0h, x.b1h);
 }
 
-__device__ __forceinline__ size_t kv_offset(const GemmArgs& a, int page, int kvsel, int h, int off, int dim) {
-  return ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * a.dh + (size_t)off * a.dh + dim;
+// Element offset of (page, layer, K|V, head, position in page, dim) in the KV pool.
+__device__ __forceinline__ size_t kv_offset(const GemmArgs& a, int page, int layer, int kvsel, int h, int off, int dim) {
+  return ((((size_t)page * a.L + layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * a.dh + (size_t)off * a.dh + dim;
 }
 
 __device__ __forceinline__ const float* c_row(const float* c_lat, int max_lat, int L, int layer, int d, int seq, int lat) {
@@ -208,7 +213,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         set_status(a.status, kErrDevice);
         return;
       }
-      const size_t off = kv_offset(a, page, 0, h, pos % a.PT, 0);
+      const size_t off = kv_offset(a, page, a.layer, 0, h, pos % a.PT, 0);
       kv_store(a, off + j, o0);
       kv_store(a, off + j + half, o1);
     } else {
@@ -218,8 +223,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         return;
       }
       const int n0 = lt * 16 + r16, n1 = n0 + 8;
-      kv_store(a, kv_offset(a, page, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
-      kv_store(a, kv_offset(a, page, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
+      kv_store(a, kv_offset(a, page, a.layer, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
+      kv_store(a, kv_offset(a, page, a.layer, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
     }
   }
 }
@@ -267,6 +272,79 @@ __device__ __forceinline__ void tile_reduce(const float (&acc)[NG][4], const flo
     }
     epi(r16, col, v0 * rs, v1 * rs);
   }
+}
+
+// K segments (K > 1024): fold a finished segment into the running totals.
+// Every warp's accumulators go to red [8][16][RB]; each thread sums its output
+// pairs (p = tid, tid + 256) over the warps in order -- the segment sum S_j --
+// and adds it to its totals (the first segment is taken as is); accumulators
+// restart at zero.  red must not alias the activation staging.
+template <int NG>
+__device__ __forceinline__ void seg_fold(float (&acc)[NG][4], float* red, float (&tot)[2][2], int& nsegs_done, int tid) {
+  constexpr int RB = 8 * NG;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    const int c = n * 8 + 2 * t;
+    red[(warp * 16 + g) * RB + c] = acc[n][0];
+    red[(warp * 16 + g) * RB + c + 1] = acc[n][1];
+    red[(warp * 16 + g + 8) * RB + c] = acc[n][2];
+    red[(warp * 16 + g + 8) * RB + c + 1] = acc[n][3];
+    acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int p = tid + i * kThreads;
+    if (p < 8 * RB) {
+      const int r16 = p & 7, col = p >> 3;
+      float v0 = red[r16 * RB + col], v1 = red[(r16 + 8) * RB + col];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) {
+        v0 += red[(w * 16 + r16) * RB + col];
+        v1 += red[(w * 16 + r16 + 8) * RB + col];
+      }
+      tot[i][0] = nsegs_done ? tot[i][0] + v0 : v0;
+      tot[i][1] = nsegs_done ? tot[i][1] + v1 : v1;
+    }
+  }
+  ++nsegs_done;
+  __syncthreads();
+}
+
+// After the last seg_fold: the RMS scale (if any) and the epilogue of every pair.
+template <int NG, class Fn>
+__device__ __forceinline__ void tile_reduce_totals(const float (&tot)[2][2], const float (&ss)[NG], bool want_ss, float* red, float* ssr,
+                                                   int nr, int K, float eps, int tid, Fn epi) {
+  constexpr int RB = 8 * NG;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  if (want_ss) {
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      float s = ss[n];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (t == 0) ssr[warp * RB + n * 8 + g] = s;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int p = tid + i * kThreads;
+    if (p < 8 * RB) {
+      const int r16 = p & 7, col = p >> 3;
+      if (col >= nr) continue;
+      float rs = 1.0f;
+      if (want_ss) {
+        float s = ssr[col];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) s += ssr[w * RB + col];
+        rs = 1.0f / sqrtf(s / (float)K + eps);
+      }
+      epi(r16, col, tot[i][0] * rs, tot[i][1] * rs);
+    }
+  }
+  (void)red;
 }
 
 // Per-phase GEMM kernel (passes with many rows, latent projection, prefill).
@@ -317,8 +395,14 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   float acc[NG][4], ss[NG];
 #pragma unroll
   for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
+  float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // K > 1024: this thread's output pairs, segments summed in order
+  int nsegs_done = 0;
+  constexpr int kSegWin = kSegCols / kKWin;     // windows per segment (a multiple of DEPTH)
 
   for (int wi0 = 0; wi0 < nwin; wi0 += DEPTH) {
+    if (wi0 > 0 && wi0 % kSegWin == 0) {  // segment boundary: fold the finished segment
+      seg_fold<NG>(acc, xs + (size_t)STAGES * RB * kXStride + 8 * RB, tot, nsegs_done, tid);
+    }
 #pragma unroll
     for (int dd = 0; dd < DEPTH; ++dd) {
       const int wi = wi0 + dd;
@@ -356,8 +440,15 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   }
   cp_async_wait<0>();
   __syncthreads();
-  tile_reduce<NG>(acc, ss, norm, xs, ssr, nr, a.K, a.eps, tid, kThreads, [] { __syncthreads(); },
-                  [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
+  if (a.K <= kSegCols) {
+    tile_reduce<NG>(acc, ss, norm, xs, ssr, nr, a.K, a.eps, tid, kThreads, [] { __syncthreads(); },
+                    [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
+    return;
+  }
+  // last segment, then the ordered segment sum and the scale
+  seg_fold<NG>(acc, xs, tot, nsegs_done, tid);
+  tile_reduce_totals<NG>(tot, ss, norm, xs, ssr, nr, a.K, a.eps, tid,
+                         [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
 }
 
 // ------------------------------------------------------------------------ row-wise kernels
@@ -451,15 +542,14 @@ __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, 
 // fmaf chain in c order.  `per` threads share a key (thread `part` takes rows
 // part, part + per, ...).  The key is widened 32 columns at a time and the
 // running sums live in ps between column blocks (an exact round trip), which
-// keeps the loop small for the instruction cache.
-template <int DH, typename KVT>
-__device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, const KVT* ks, float* ps, const int* lim, int nr,
-                                            int nk, int tid, int nthr) {
-  constexpr int ST = kv_stride<DH, KVT>();
+// keeps the loop small for the instruction cache.  ST: row stride of ks.
+template <int DH, typename KVT, int ST = kv_stride<DH, KVT>()>
+__device__ __forceinline__ void attn_scores(int CH, const float* qs, const KVT* ks, float* ps, const int* lim, int nr, int nk, int tid,
+                                            int nthr) {
   constexpr int CB = DH < 32 ? DH : 32;  // columns per block
-  const int per = max(1, nthr / a.CH);
-  for (int idx = tid; idx < a.CH * per; idx += nthr) {
-    const int key = idx % a.CH, part = idx / a.CH;
+  const int per = max(1, nthr / CH);
+  for (int idx = tid; idx < CH * per; idx += nthr) {
+    const int key = idx % CH, part = idx / CH;
     if (key < nk) {
       for (int c0 = 0; c0 < DH; c0 += CB) {
         float kf[CB];
@@ -468,7 +558,7 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
 #pragma unroll 1
         for (int r = part; r < nr; r += per) {
           const float* q = qs + r * DH + c0;
-          float sr = (c0 == 0) ? 0.f : ps[r * a.CH + key];
+          float sr = (c0 == 0) ? 0.f : ps[r * CH + key];
 #pragma unroll
           for (int c4 = 0; c4 < CB / 4; ++c4) {
             const float4 qv = *reinterpret_cast<const float4*>(q + c4 * 4);
@@ -477,12 +567,12 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
             sr = fmaf(qv.z, kf[c4 * 4 + 2], sr);
             sr = fmaf(qv.w, kf[c4 * 4 + 3], sr);
           }
-          ps[r * a.CH + key] = sr;
+          ps[r * CH + key] = sr;
         }
       }
     }
     for (int r = part; r < nr; r += per)
-      if (!(key < nk && key < lim[r])) ps[r * a.CH + key] = -INFINITY;
+      if (!(key < nk && key < lim[r])) ps[r * CH + key] = -INFINITY;
   }
 }
 
@@ -491,12 +581,11 @@ __device__ __forceinline__ void attn_scores(const AttnArgs& a, const float* qs, 
 // lo B operands), hi then lo per 16-dim step, steps in dim order; one warp
 // per (key tile, row group).  Keys past nk or past a row's limit get -inf.
 // K rows past nk are never loaded: their scores are discarded.
-template <int DH>
-__device__ __forceinline__ void attn_scores_mma(const AttnArgs& a, const float* qs, const __nv_bfloat16* ks, float* ps, const int* lim,
-                                                int nr, int nk, int tid, int nthr) {
-  constexpr int ST = kv_stride<DH, __nv_bfloat16>();
+template <int DH, int ST = kv_stride<DH, __nv_bfloat16>()>
+__device__ __forceinline__ void attn_scores_mma(int CH, const float* qs, const __nv_bfloat16* ks, float* ps, const int* lim, int nr,
+                                                int nk, int tid, int nthr) {
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3, nw = nthr >> 5;
-  const int nkt = a.CH / 16, nrg = (nr + 7) / 8;
+  const int nkt = CH / 16, nrg = (nr + 7) / 8;
 #pragma unroll 1
   for (int item = warp; item < nkt * nrg; item += nw) {
     const int key0 = (item % nkt) * 16, rg = item / nkt;
@@ -519,7 +608,7 @@ __device__ __forceinline__ void attn_scores_mma(const AttnArgs& a, const float* 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int key = key0 + g + (e >= 2 ? 8 : 0), r = rg * 8 + 2 * t + (e & 1);
-      if (r < nr) ps[r * a.CH + key] = (key < nk && key < lim[r]) ? acc[e] : -INFINITY;
+      if (r < nr) ps[r * CH + key] = (key < nk && key < lim[r]) ? acc[e] : -INFINITY;
     }
   }
 }
@@ -527,11 +616,11 @@ __device__ __forceinline__ void attn_scores_mma(const AttnArgs& a, const float* 
 // o^T (16 columns x 8 rows) = V^T (16 columns x 16 keys, bf16 A operand
 // gathered from smem) . p^T (keys x rows, split into bf16 hi and lo), key
 // tiles in order; one warp per (column tile, row group).  V rows from nk up
-// to the next multiple of 16 are zero (their p is 0 as well).
-template <int DH>
-__device__ __forceinline__ void attn_pv_mma(const AttnArgs& a, const float* ps, const __nv_bfloat16* vs, int nr, int nk, int row0,
-                                            int h, int chunk, const float* mrow, const float* lrow, int tid, int nthr) {
-  constexpr int ST = kv_stride<DH, __nv_bfloat16>();
+// to the next multiple of 16 are zero (their p is 0 as well).  Outputs go to
+// emit_o(row, column, value); emit_ml(row, m, l) once per row.
+template <int DH, int ST, class EmitO, class EmitML>
+__device__ __forceinline__ void attn_pv_mma(int CH, const float* ps, const __nv_bfloat16* vs, int nr, int nk, const float* mrow,
+                                            const float* lrow, int tid, int nthr, EmitO emit_o, EmitML emit_ml) {
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3, nw = nthr >> 5;
   const int nkt = (nk + 15) / 16, nrg = (nr + 7) / 8;
   const unsigned short* v16 = reinterpret_cast<const unsigned short*>(vs);
@@ -539,7 +628,7 @@ __device__ __forceinline__ void attn_pv_mma(const AttnArgs& a, const float* ps, 
 #pragma unroll 1
   for (int item = warp; item < (DH / 16) * nrg; item += nw) {
     const int c0 = (item % (DH / 16)) * 16, rg = item / (DH / 16);
-    const float* p = ps + min(rg * 8 + g, nr - 1) * a.CH;
+    const float* p = ps + min(rg * 8 + g, nr - 1) * CH;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 2
     for (int kt = 0; kt < nkt; ++kt) {
@@ -555,44 +644,30 @@ __device__ __forceinline__ void attn_pv_mma(const AttnArgs& a, const float* ps, 
     for (int e = 0; e < 4; ++e) {
       const int c = c0 + g + (e >= 2 ? 8 : 0), r = rg * 8 + 2 * t + (e & 1);
       if (r < nr) {
-        const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
-        a.part_o[base * DH + c] = acc[e];
-        if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+        emit_o(r, c, acc[e]);
+        if (c == 0) emit_ml(r, mrow[r], lrow[r]);
       }
     }
   }
 }
 
-// Softmax partial of one (group, head, chunk): scores of every row against
-// keys [t0, t0+nk) (masked per row by nkeys), m = max, l = sum exp(s - m),
-// o = sum exp(s - m) v.  q pre-scaled by 1/sqrt(dh).  smem: qs [32][DH] f32,
-// ps [32][CH] f32, ks/vs [CH][kv_stride] KVT already loaded.
+// Softmax partial of one chunk of keys for rows 0..nr-1 (per row limit lim):
+// m = max score, l = sum exp(s - m), o = sum exp(s - m) v.  On entry qs
+// [rows][DH] holds q pre-scaled by 1/sqrt(dh), lim the rows' key limits
+// (relative to the chunk), ks/vs the chunk's nk keys (row stride ST; for bf16,
+// V rows nk .. next multiple of 16 zeroed), and every thread has passed
+// `sync` since they were written.  Outputs through emit_o / emit_ml.
 struct NoMark {
   __device__ void operator()(int) const {}
 };
 
-template <int DH, typename KVT, class Sync, class Mark = NoMark>
-__device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
-                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync,
-                                     Mark mark = Mark()) {
-  constexpr int ST = kv_stride<DH, KVT>();
-  const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
-  const int t0 = chunk * a.CH;
-  const int nk = min(a.CH, kmax - t0);
-  for (int i = tid; i < nr * DH; i += nthr) {
-    const int r = i / DH, c = i % DH;
-    qs[r * DH + c] = __ldcg(a.q + (size_t)(row0 + r) * a.d + h * DH + c) * a.scale;
-  }
-  if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
-  if constexpr (sizeof(KVT) == 2) {  // zero V rows nk .. next multiple of 16 (read by the last key tile)
-    const int pad = ((nk + 15) & ~15) - nk;
-    for (int i = tid; i < pad * (DH / 8); i += nthr)
-      *reinterpret_cast<uint4*>(const_cast<KVT*>(vs) + (nk + i / (DH / 8)) * ST + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
-  }
-  sync();
+template <int DH, typename KVT, int ST, class Sync, class EmitO, class EmitML, class Mark = NoMark>
+__device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* ks, const KVT* vs, float* mrow, float* lrow,
+                                const int* lim, int nr, int nk, int tid, int nthr, Sync sync, EmitO emit_o, EmitML emit_ml,
+                                Mark mark = Mark()) {
   mark(1);
-  if constexpr (sizeof(KVT) == 2) attn_scores_mma<DH>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
-  else attn_scores<DH, KVT>(a, qs, ks, ps, lim, nr, nk, tid, nthr);
+  if constexpr (sizeof(KVT) == 2) attn_scores_mma<DH, ST>(CH, qs, ks, ps, lim, nr, nk, tid, nthr);
+  else attn_scores<DH, KVT, ST>(CH, qs, ks, ps, lim, nr, nk, tid, nthr);
   sync();
   mark(2);
   const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
@@ -600,14 +675,14 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   for (int r = warp; r < nr; r += nw) {
     float m = -INFINITY;
 #pragma unroll 1
-    for (int k = lane; k < a.CH; k += 32) m = fmaxf(m, ps[r * a.CH + k]);
+    for (int k = lane; k < CH; k += 32) m = fmaxf(m, ps[r * CH + k]);
     m = warp_max(m);
     float l = 0.f;
 #pragma unroll 1
-    for (int k = lane; k < a.CH; k += 32) {
-      const float s = ps[r * a.CH + k];
+    for (int k = lane; k < CH; k += 32) {
+      const float s = ps[r * CH + k];
       const float p = (s == -INFINITY) ? 0.f : expf(s - m);
-      ps[r * a.CH + k] = p;
+      ps[r * CH + k] = p;
       l += p;
     }
     l = warp_sum(l);
@@ -619,7 +694,7 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
   sync();
   mark(3);
   if constexpr (sizeof(KVT) == 2) {
-    attn_pv_mma<DH>(a, ps, vs, nr, nk, row0, h, chunk, mrow, lrow, tid, nthr);
+    attn_pv_mma<DH, ST>(CH, ps, vs, nr, nk, mrow, lrow, tid, nthr, emit_o, emit_ml);
     return;
   }
   // o[r][c] = sum_k p[r][k] v[k][c], one fmaf chain in k order per output.
@@ -638,35 +713,60 @@ __device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk
       if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * ST + c]);
       else v = vs[k * ST + c];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) o[j] = fmaf(ps[rr[j] * a.CH + k], v, o[j]);
+      for (int j = 0; j < 4; ++j) o[j] = fmaf(ps[rr[j] * CH + k], v, o[j]);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int r = r0 + j * rs;
       if (r < nr) {
-        const size_t base = ((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk;
-        a.part_o[base * DH + c] = o[j];
-        if (c == 0) a.part_ml[base] = make_float2(mrow[r], lrow[r]);
+        emit_o(r, c, o[j]);
+        if (c == 0) emit_ml(r, mrow[r], lrow[r]);
       }
     }
   }
 }
 
-// att[row][h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m}
-// for one (row, head), by one warp.  m = largest chunk maximum (chunks with
-// l > 0); lane j holds the weight of chunk j of each 32-chunk block; l is the
-// warp sum of the lanes' l_c w_c sums; o accumulates the chunks in order with
-// the weight broadcast from its lane.  Lane c (and c + 32, ...) owns column c.
-template <int DH>
-__device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int h, int lane) {
+// Softmax partial of one (group, head, chunk) of the per-phase path: q and the
+// row limits from global memory, K/V already in smem (padded rows), partials
+// to a.part_o / a.part_ml.
+template <int DH, typename KVT, class Sync>
+__device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
+                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync) {
+  constexpr int ST = kv_stride<DH, KVT>();
+  const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
+  const int t0 = chunk * a.CH;
+  const int nk = min(a.CH, kmax - t0);
+  for (int i = tid; i < nr * DH; i += nthr) {
+    const int r = i / DH, c = i % DH;
+    qs[r * DH + c] = __ldcg(a.q + (size_t)(row0 + r) * a.d + h * DH + c) * a.scale;
+  }
+  if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
+  if constexpr (sizeof(KVT) == 2) {  // zero V rows nk .. next multiple of 16 (read by the last key tile)
+    const int pad = ((nk + 15) & ~15) - nk;
+    for (int i = tid; i < pad * (DH / 8); i += nthr)
+      *reinterpret_cast<uint4*>(const_cast<KVT*>(vs) + (nk + i / (DH / 8)) * ST + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
+  }
+  sync();
+  attn_chunk_core<DH, KVT, ST>(
+      a.CH, qs, ps, ks, vs, mrow, lrow, lim, nr, nk, tid, nthr, sync,
+      [&](int r, int c, float v) { a.part_o[(((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk) * DH + c] = v; },
+      [&](int r, float m, float l) { a.part_ml[((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk] = make_float2(m, l); });
+}
+
+// att[h*dh + c] = sum_chunks o_c e^{m_c - m} / sum_chunks l_c e^{m_c - m} for
+// one (row, head) by one warp, over nch chunks.  m = largest chunk maximum
+// (chunks with l > 0); lane j holds the weight of chunk j of each 32-chunk
+// block; l is the warp sum of the lanes' l_c w_c sums; o accumulates the
+// chunks in order with the weight broadcast from its lane.  Lane c (and
+// c + 32, ...) owns column c.  ml(ch) -> float2 (m, l); ov(ch, col) -> o;
+// out(col, value).
+template <int DH, class ML, class OV, class Out>
+__device__ __forceinline__ void attn_combine(int nch, int lane, ML ml_at, OV o_at, Out out) {
   constexpr int DPL = DH >= 32 ? DH / 32 : 1;  // columns per lane
-  const int nk = __ldcg(a.rows.nkeys + row);
-  const int nch = (nk + a.CH - 1) / a.CH;
-  const size_t base = ((size_t)row * a.H + h) * a.CMAX;
   float m = -INFINITY;
 #pragma unroll 1
   for (int ch = lane; ch < nch; ch += 32) {
-    const float2 ml = __ldcg(a.part_ml + base + ch);
+    const float2 ml = ml_at(ch);
     if (ml.y > 0.f) m = fmaxf(m, ml.x);
   }
   m = warp_max(m);
@@ -678,7 +778,7 @@ __device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int
   for (int cb = 0; cb < nch; cb += 32) {
     float w = 0.f;
     if (cb + lane < nch) {
-      const float2 ml = __ldcg(a.part_ml + base + cb + lane);
+      const float2 ml = ml_at(cb + lane);
       if (ml.y > 0.f) {
         w = expf(ml.x - m);
         l = fmaf(ml.y, w, l);
@@ -693,7 +793,7 @@ __device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int
         wj[j] = __shfl_sync(0xffffffffu, w, (j0 + j) & 31);
         const int ch = cb + min(j0 + j, nb - 1);
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) ov[j][i] = col_ok ? __ldcg(a.part_o + (base + ch) * DH + lane + 32 * i) : 0.f;
+        for (int i = 0; i < DPL; ++i) ov[j][i] = col_ok ? o_at(ch, lane + 32 * i) : 0.f;
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -705,7 +805,18 @@ __device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int
   l = warp_sum(l);
   if (col_ok)
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) a.att[(size_t)row * a.d + h * DH + lane + 32 * i] = o[i] / l;
+    for (int i = 0; i < DPL; ++i) out(lane + 32 * i, o[i] / l);
+}
+
+template <int DH>
+__device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int h, int lane) {
+  const int nk = __ldcg(a.rows.nkeys + row);
+  const int nch = (nk + a.CH - 1) / a.CH;
+  const size_t base = ((size_t)row * a.H + h) * a.CMAX;
+  attn_combine<DH>(
+      nch, lane, [&](int ch) { return __ldcg(a.part_ml + base + ch); },
+      [&](int ch, int col) { return __ldcg(a.part_o + (base + ch) * DH + col); },
+      [&](int col, float v) { a.att[(size_t)row * a.d + h * DH + col] = v; });
 }
 
 // grid (H, chunks, groups); 128 threads.
@@ -958,12 +1069,13 @@ __device__ void plan_rows(const PlanArgs& p, int B, const int* row_off, const in
       }
       if (p.mode == PL_PREFILL) {
         sd.counters[2] += n_rows;
+        sd.counters[7] += kvk * p.kv_bytes_per_key;
       } else {
         sd.counters[0] += 1;
         sd.counters[5] += p.weight_bytes_per_pass;
+        sd.counters[6] += kvk * p.kv_bytes_per_key;
       }
       sd.counters[1] += n_rows;
-      sd.counters[6] += kvk * p.kv_bytes_per_key;
     }
   }
   sync();

@@ -3,39 +3,56 @@
 // loop, or the verification pass) in one cooperative launch, one CTA per SM.
 //
 // Warp roles: warps 0..7 consume (tensor-core GEMV, attention, bookkeeping),
-// warp 8 produces: it streams this CTA's weight tiles for the whole pass
-// through a shared-memory ring with 1-D bulk TMA copies, so HBM keeps
-// streaming while consumers wait on data dependencies.
+// warp 8 produces: it streams this CTA's weight pieces and the cached K/V
+// pages of its attention items, in the order the consumers use them, through
+// a ring of 32 KB shared-memory slots with 1-D bulk copies (L2 evict-first for
+// weights).  The producer runs ahead of the consumers across phase boundaries
+// (weights do not depend on activations), so HBM keeps streaming while the
+// consumers wait for their inputs.
 //
-// Work: each projection is cut into units of 16 output rows (a tile row of
-// the fragment-ordered weights).  The units of all phases of a pass
-// (QKV, O, W13, W2 per layer, then the byte head) are dealt round-robin to
-// the CTAs, continuing across phases, so every CTA streams about the same
-// number of bytes at every point of the pass.
+// Hand-offs between CTAs use self-validating words: every activation value
+// is written as one 64-bit word (epoch << 32 | fp32 bits) with a relaxed
+// store, and a consumer polls the words it needs until each carries the
+// expected epoch.  A hand-off costs one L2 round trip after the data lands:
+// no fence, no flag, no second load.  Epochs are unique per (call, pass,
+// layer, stage), so a stale word is never mistaken for a fresh one; a buffer
+// is rewritten only after every reader of its previous contents has finished
+// (each rewrite depends, through the pass's all-to-all data flow, on outputs
+// those readers produced after reading).
 //
-// Dependencies are per-unit epoch flags in global memory (release store by
-// the producing CTA, acquire poll by the consumer), not grid barriers: a
-// QKV k-step waits only for the W2 unit that wrote its 16 input columns,
-// an O-projection k-step for the attention head it reads, and so on.  Every
-// wait is bounded; a wait that runs out sets the abort word and the status,
-// and all CTAs leave.  The arithmetic of every unit, attention chunk,
-// combine and bookkeeping step is the device code the per-phase kernels use,
-// so both paths give bit-identical results.
+// Work per layer (G CTAs):
+//   QKV   3d/16 units of 16 output rows, unit u on CTA u mod G
+//   ATT   items (sequence group, head, 128-key chunk), item i on CTA i mod G;
+//         the CTA of chunk 0 combines the head's chunks
+//   O     d/16 units, W13 2F/16 units (continuing the round robin)
+//   W2    K cut into segments of 1024 columns; segment q has its own G/nseg
+//         CTAs; the CTA of the last segment of a unit sums the segments in
+//         order and applies the residual.
+// The arithmetic of every unit, chunk, combine and bookkeeping step is the
+// canonical order of kernels.cuh, so this path and the per-phase kernels give
+// bit-identical results.  Every wait is bounded: a wait that runs out sets
+// the abort word and the device status (BLT_ERR_DEVICE), and all CTAs leave.
 #pragma once
 
 #include "kernels.cuh"
 
 namespace bltdec {
 
+typedef unsigned long long u64;
+
 constexpr int kMegaConsumers = 8;
 constexpr int kMegaThreads = (kMegaConsumers + 1) * 32;
-constexpr int kStageTiles = 64;                 // k16 tiles of one unit per ring slot
-constexpr int kTPW = kStageTiles / 8;           // tiles of a stage per consumer warp
-constexpr int kRingBytes = 128 * 1024;          // weight ring
-constexpr int kMegaMaxNG = 2;                   // <= 16 rows per pass
-constexpr unsigned kSpinLimit = 1u << 26;       // polls before a wait gives up
+constexpr int kSlotBytes = 32 * 1024;
+constexpr int kRingSlots = 5;
+constexpr int kMegaMaxNG = 2;                  // <= 16 rows per pass
+constexpr int kMegaRows = 8 * kMegaMaxNG;
+constexpr int kMaxPieces = 4;                  // GEMV pieces of one phase reduced together
+constexpr int kSegSteps = kSegCols / 16;       // k-steps per canonical K segment
 
 enum MegaMode : int { MM_DIFFUSE = 0, MM_DRAFT_AR = 1, MM_VERIFY = 2 };
+// Stage of an exchange word (part of its epoch).
+enum Stage : int { ST_QKV = 0, ST_PART = 1, ST_ATT = 2, ST_HO = 3, ST_ACT = 4, ST_W2P = 5, ST_HW = 6, ST_LOGIT = 7 };
+enum PhaseKind : int { PH_QKV = 0, PH_O = 1, PH_W13 = 2, PH_W2 = 3, PH_HEAD = 4 };
 
 struct LayerW {
   const uint4* qkv;
@@ -52,27 +69,34 @@ struct MegaArgs {
   const float* final_norm;
   int L, d, H, dh, F, planes;
   float eps;
-  GemmArgs ga;  // epilogue context: pointers shared by all phases
-  AttnArgs aa;
+  GemmArgs ga;  // embedding, latent cache, KV pool, page table, rotary tables, shapes
+  AttnArgs aa;  // chunk size, scale
   RowsDev rows;
   SeqDev sd;
-  float* h;
-  float* q;
-  float* att;
-  float* act;
-  float* logits;
+  // exchange buffers (64-bit words: epoch << 32 | fp32 bits)
+  u64* x_h;      // [rows][d] residual stream
+  u64* x_q;      // [rows][d] queries (RoPE applied)
+  u64* x_k;      // [rows][d] keys of this pass's rows (RoPE applied, rounded like the cache)
+  u64* x_v;      // [rows][d] values of this pass's rows (rounded like the cache)
+  u64* x_part;   // [rows][H][CMAX][2 + dh] chunk partials (m, l, o)
+  u64* x_att;    // [rows][d] attention output
+  u64* x_act;    // [rows][F] SwiGLU activations
+  u64* x_w2p;    // [nseg - 1][rows][d] W2 segment sums
+  u64* x_logit;  // [rows][256]
+  int CMAX;
+  float* logits;  // [rows][256] plain copy for the bookkeeping
   float* conf;
-  float* ent;  // per-row entropy of the byte head (EB sampling)
-  int eb;      // block unmasking by EB sampling (bound alpha) instead of confidence
-  int* pred;
+  float* ent;
   float* gap;
-  unsigned* flags;  // epoch flags, see flag offsets below
-  int f_qkv, f_o, f_w13, f_w2, f_head, f_att, f_dec;
-  unsigned* attn_cnt;  // [max_groups][H] arrival counters
-  unsigned* dec_val;   // continue word written with the decision flag
+  int* pred;
+  int eb;               // block unmasking by EB sampling (bound alpha) instead of confidence
+  unsigned* flags;      // [0] decision epoch, [1] pass-end arrivals (zeroed before the launch)
+  unsigned* dec_val;    // continue word written with the decision
   unsigned epoch0;
   int* abort;
-  unsigned long long* trace;  // debug timestamps [cta][kTraceEvents] of pass 0 (NULL: off)
+  unsigned long long wait_ns;  // wall time after which a wait gives up
+  int stall_test;       // test only: unit 0 of the first O phase never publishes (a wait must run out)
+  unsigned long long* trace;
   int mode, batch, k, max_passes;
   float alpha;
   const int* vlat;
@@ -82,7 +106,7 @@ struct MegaArgs {
   PlanArgs plan;  // template for the device-side plans of passes >= 2
 };
 
-// ---------------------------------------------------------------------------- sync primitives
+// ---------------------------------------------------------------------------- primitives
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 __device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count));
@@ -92,9 +116,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, unsigned bytes) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_n(uint64_t* b, unsigned n) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(b)), "r"(n) : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint64_t* b, unsigned parity) {
   unsigned ok;
@@ -111,6 +132,11 @@ __device__ __forceinline__ void tma_1d(void* dst, const void* src, unsigned byte
                "l"(src), "r"(bytes), "r"(smem_u32(b)), "l"(pol)
                : "memory");
 }
+__device__ __forceinline__ void tma_1d_plain(void* dst, const void* src, unsigned bytes, uint64_t* b) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(b))
+               : "memory");
+}
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
@@ -119,15 +145,61 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// Barrier of the 256 consumer threads that also ANDs a flag across them: every
+// control decision after a wait is taken the same way by all consumers.
+__device__ __forceinline__ bool consumer_and(bool v) {
+  unsigned r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((unsigned)v)
+      : "memory");
+  return r != 0;
+}
+// generic-proxy writes of this CTA's shared memory become visible to later bulk copies into it
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+// global data written through the generic proxy, read next by bulk copies
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
 
-// Bounded waits.  Return false when the wait gave up (abort raised).
-__device__ __forceinline__ bool wait_flag(const MegaArgs& m, const unsigned* f, unsigned target) {
+// exchange words
+__device__ __forceinline__ u64 xw_pack(float v, unsigned e) { return ((u64)e << 32) | (u64)__float_as_uint(v); }
+__device__ __forceinline__ bool xw_ok(u64 w, unsigned e) { return (unsigned)(w >> 32) == e; }
+__device__ __forceinline__ float xw_val(u64 w) { return __uint_as_float((unsigned)(w & 0xFFFFFFFFull)); }
+__device__ __forceinline__ void xw_st(u64* p, float v, unsigned e) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;\n" ::"l"(p), "l"(xw_pack(v, e)) : "memory");
+}
+__device__ __forceinline__ u64 xw_ld(const u64* p) {
+  u64 w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];\n" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+__device__ __forceinline__ void xw_ld2(const u64* p, u64& a, u64& b) {  // p 16-byte aligned; each word read atomically
+  asm volatile("ld.relaxed.gpu.global.v2.b64 {%0, %1}, [%2];\n" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// State of one bounded wait: polls so far and when the first one failed.
+struct Spin {
   unsigned n = 0;
-  while ((int)(ld_acquire(f) - target) < 0) {
-    if (++n > 64) __nanosleep(64);
-    if ((n & 1023) == 0 && *(volatile int*)m.abort) return false;
-    if (n > kSpinLimit) {
+  unsigned long long t0 = 0;
+};
+// One step of a bounded wait: back off, count, watch the abort word and the
+// clock.  A wait gives up (abort word + BLT_ERR_DEVICE) after m.wait_ns of
+// wall time.  False: give up.
+__device__ __forceinline__ bool spin_step(const MegaArgs& m, Spin& sp) {
+  __nanosleep(sp.n < 32 ? 32 : 128);
+  if (sp.n++ == 0) sp.t0 = gtimer();
+  if ((sp.n & 31) == 0) {
+    if (*(volatile int*)m.abort) return false;
+    if (gtimer() - sp.t0 > m.wait_ns) {
       atomicExch(m.abort, 1);
       set_status(m.sd.status, kErrDevice);
       return false;
@@ -135,63 +207,83 @@ __device__ __forceinline__ bool wait_flag(const MegaArgs& m, const unsigned* f, 
   }
   return true;
 }
+
+// Poll one word until it carries epoch e.
+__device__ __forceinline__ bool xw_wait(const MegaArgs& m, const u64* p, unsigned e, float& v) {
+  Spin spins;
+  while (true) {
+    const u64 w = xw_ld(p);
+    if (xw_ok(w, e)) {
+      v = xw_val(w);
+      return true;
+    }
+    if (!spin_step(m, spins)) return false;
+  }
+}
+// Poll the words idx = tid + 256 i (i < N, idx < n) until each carries epoch
+// e; at(idx) is a word's address, put(idx, value) takes its value.  Every load
+// of a round is in flight at once; a round re-reads only the words not ready.
+template <int N, class At, class Put>
+__device__ __forceinline__ bool poll_words(const MegaArgs& m, int n, unsigned e, int tid, At at, Put put) {
+  unsigned pending = 0;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (tid + 256 * i < n) pending |= 1u << i;
+  Spin spins;
+  if (pending) {  // wait on one word first: a waiting thread issues one load per round, not N
+    const int i0 = __ffs(pending) - 1;
+    const u64* p0 = at(tid + 256 * i0);
+    while (!xw_ok(xw_ld(p0), e))
+      if (!spin_step(m, spins)) return false;
+  }
+  while (pending) {
+    u64 w[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u) w[i] = xw_ld(at(tid + 256 * i));
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (((pending >> i) & 1u) && xw_ok(w[i], e)) {
+        put(tid + 256 * i, xw_val(w[i]));
+        pending &= ~(1u << i);
+      }
+    if (pending && !spin_step(m, spins)) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ bool wait_mbar(const MegaArgs& m, uint64_t* b, unsigned parity) {
   unsigned n = 0;
+  unsigned long long t0 = 0;
   while (!mbar_try(b, parity)) {
-    if ((++n & 1023) == 0 && *(volatile int*)m.abort) return false;
-    if (n > kSpinLimit) {
-      atomicExch(m.abort, 1);
-      set_status(m.sd.status, kErrDevice);
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void fence_acquire() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_acq_rel() { asm volatile("fence.acq_rel.gpu;\n" ::: "memory"); }
-__device__ __forceinline__ void st_relaxed(unsigned* p, unsigned v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
-}
-
-// Warp-wide wait until flag(i) >= target for every i < n: each lane polls
-// its share with relaxed loads (all in flight at once), then one acquire
-// fence orders the data reads that follow.  Bounded like wait_flag.
-template <class FlagFn>
-__device__ __forceinline__ bool warp_wait(const MegaArgs& m, int n, FlagFn flag, unsigned target) {
-  const int lane = threadIdx.x & 31;
-  unsigned spins = 0;
-  while (true) {
-    bool mine = true;
-#pragma unroll 1
-    for (int i = lane; i < n; i += 32) mine &= (int)(ld_relaxed(flag(i)) - target) >= 0;
-    if (__all_sync(0xffffffffu, mine)) break;
-    ++spins;
-    if (spins > 8) __nanosleep(128);
-    if ((spins & 255) == 0 && *(volatile int*)m.abort) return false;
-    if (spins > (kSpinLimit >> 6)) {
-      if (lane == 0) {
+    if (n++ == 0) t0 = gtimer();
+    if ((n & 255) == 0) {
+      if (*(volatile int*)m.abort) return false;
+      if (gtimer() - t0 > m.wait_ns) {
         atomicExch(m.abort, 1);
         set_status(m.sd.status, kErrDevice);
+        return false;
       }
-      return false;
     }
   }
-  fence_acquire();
-  __syncwarp();
   return true;
 }
+__device__ __forceinline__ bool wait_flag(const MegaArgs& m, const unsigned* f, unsigned target, bool eq) {
+  Spin spins;
+  while (true) {
+    const unsigned v = ld_acquire(f);
+    if (eq ? v == target : (int)(v - target) >= 0) return true;
+    if (!spin_step(m, spins)) return false;
+  }
+}
 
-// Device-side timestamps (debug): trace[cta][event] = %globaltimer.
+__device__ __forceinline__ unsigned epoch(const MegaArgs& m, int pass, int layer, int stage) {
+  return m.epoch0 + 1u + (((unsigned)pass * (unsigned)(m.L + 1) + (unsigned)layer) << 3) + (unsigned)stage;
+}
+
+// Device-side timestamps (debug): compiled in only with -DBLTDEC_MEGA_TRACE.
 constexpr int kTraceEvents = 1024;
-__shared__ int s_trace_n;  // this CTA's event count of the traced pass (debug only)
-// Event word: code << 48 | low 48 bits of %globaltimer.  Recorded by thread 0 in pass 0.
-// Compiled in only with -DBLTDEC_MEGA_TRACE (the marks cost instruction-cache space).
+__shared__ int s_trace_n;
 __device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code) {
 #ifdef BLTDEC_MEGA_TRACE
   if (m.trace && pass == 0 && threadIdx.x == 0) {
@@ -200,322 +292,538 @@ __device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code
     const int i = s_trace_n++;
     if (i < kTraceEvents) m.trace[(size_t)blockIdx.x * kTraceEvents + i] = ((unsigned long long)code << 48) | (t & 0xFFFFFFFFFFFFull);
   }
+#else
+  (void)m;
+  (void)pass;
+  (void)code;
 #endif
 }
 enum TraceCode : int {
-  TR_PASS = 1, TR_PHASE_BEGIN = 2, TR_INPUTS = 3, TR_XBUILT = 4, TR_KLOOP = 5, TR_REDUCED = 6, TR_UNIT_DONE = 7,
-  TR_ATT_BEGIN = 8, TR_ATT_QKV = 9, TR_ATT_LOADED = 10, TR_ATT_COMPUTED = 11, TR_ATT_DONE = 12, TR_HEAD = 13, TR_BOOK = 14,
-  TR_XLOADED = 15, TR_ATT_STEP = 16
+  TR_PASS = 1, TR_PH = 2, TR_IN = 3, TR_MMA = 4, TR_DONE = 5, TR_ATT = 6, TR_ATT_DONE = 7, TR_COMB = 8, TR_BOOK = 9,
+  TR_SENT = 10, TR_GATH = 11, TR_PRE = 12, TR_ISLOT = 13, TR_IPOLL = 14, TR_ICORE = 15
 };
 
 // ---------------------------------------------------------------------------- schedule
-enum PhaseKind : int { PH_QKV = 0, PH_O = 1, PH_W13 = 2, PH_W2 = 3, PH_HEAD = 4 };
-
-struct Phase {
-  int kind, layer, units, ksteps, base;
-  const uint4* w;
+// Which units (pieces) of a phase a CTA owns: first, first + step, ... (count).
+struct Assign {
+  int first, step, count;
 };
+__device__ __forceinline__ Assign rr_assign(int units, int off, int cta, int G) {
+  Assign a;
+  a.first = ((cta - off) % G + G) % G;
+  a.step = G;
+  a.count = a.first < units ? (units - a.first + G - 1) / G : 0;
+  return a;
+}
+struct Phase {
+  int kind, layer;
+  const uint4* w;
+  int units;      // output units of 16 rows
+  int ksteps;     // K / 16 of the whole matrix
+  int seg;        // K segment of this CTA's pieces
+  int seg_steps;  // k-steps per piece
+  Assign a;
+};
+__device__ __forceinline__ int n_w2_segments(const MegaArgs& m) { return m.F > kSegCols ? m.F / kSegCols : 1; }
 
-// Phase ph of a pass: ph = 4*l + {0: QKV, 1: O, 2: W13, 3: W2}; ph = 4L: head.
-__device__ __forceinline__ Phase phase_of(const MegaArgs& m, int ph) {
+// Phase `kind` of layer `layer` for this CTA (kind PH_HEAD: layer ignored).
+__device__ __forceinline__ Phase phase_of(const MegaArgs& m, int kind, int layer, int cta, int G) {
   Phase p;
-  const int L = m.L, d = m.d, F = m.F;
-  const int per_layer = 3 * d / 16 + d / 16 + 2 * F / 16 + d / 16;
-  p.layer = ph / 4;
-  p.base = p.layer * per_layer;
-  if (ph >= 4 * L) {
-    p.kind = PH_HEAD;
-    p.layer = L;
-    p.units = 256 / 16;
-    p.ksteps = d / 16;
-    p.base = L * per_layer;
-    p.w = m.whead;
-    return p;
+  p.kind = kind;
+  p.layer = layer;
+  p.seg = 0;
+  const int d = m.d, F = m.F;
+  if (kind == PH_HEAD) {
+    p.w = m.whead, p.units = 256 / 16, p.ksteps = d / 16;
+    p.a = rr_assign(p.units, (4 * d / 16 + 2 * F / 16) % G, cta, G);
+  } else {
+    const LayerW& lw = m.layers[layer];
+    if (kind == PH_QKV) {
+      p.w = lw.qkv, p.units = 3 * d / 16, p.ksteps = d / 16;
+      p.a = rr_assign(p.units, 0, cta, G);
+    } else if (kind == PH_O) {
+      p.w = lw.o, p.units = d / 16, p.ksteps = d / 16;
+      p.a = rr_assign(p.units, (3 * d / 16) % G, cta, G);
+    } else if (kind == PH_W13) {
+      p.w = lw.w13, p.units = 2 * F / 16, p.ksteps = d / 16;
+      p.a = rr_assign(p.units, (4 * d / 16) % G, cta, G);
+    } else {
+      p.w = lw.w2, p.units = d / 16, p.ksteps = F / 16;
+      const int nseg = n_w2_segments(m), cps = G / nseg;
+      const int q = cta / cps;
+      p.seg = q;
+      if (q < nseg) {
+        p.a.first = cta % cps;
+        p.a.step = cps;
+        p.a.count = p.a.first < p.units ? (p.units - p.a.first + cps - 1) / cps : 0;
+      } else {
+        p.a.first = 0, p.a.step = 1, p.a.count = 0;
+      }
+    }
   }
-  const LayerW lw = m.layers[p.layer];
-  p.kind = ph % 4;
-  switch (p.kind) {
-    case PH_QKV:
-      p.units = 3 * d / 16, p.ksteps = d / 16, p.w = lw.qkv;
-      break;
-    case PH_O:
-      p.base += 3 * d / 16, p.units = d / 16, p.ksteps = d / 16, p.w = lw.o;
-      break;
-    case PH_W13:
-      p.base += 4 * d / 16, p.units = 2 * F / 16, p.ksteps = d / 16, p.w = lw.w13;
-      break;
-    default:
-      p.base += 4 * d / 16 + 2 * F / 16, p.units = d / 16, p.ksteps = F / 16, p.w = lw.w2;
-      break;
-  }
+  p.seg_steps = min(p.ksteps, kSegSteps);
   return p;
 }
-
-__device__ __forceinline__ int first_unit(const Phase& p, int cta, int G) {
-  return ((cta - p.base) % G + G) % G;
+template <int PL>
+__device__ __forceinline__ int tiles_per_slot() {
+  return kSlotBytes / (512 * PL);
+}
+template <int PL>
+__device__ __forceinline__ int piece_slots(int tiles) {
+  return (tiles + tiles_per_slot<PL>() - 1) / tiles_per_slot<PL>();
 }
 
-__device__ __forceinline__ unsigned epoch(const MegaArgs& m, int pass, int layer) {
-  return m.epoch0 + (unsigned)(pass * (m.L + 1) + layer + 1);
+// Attention items of a pass: (group, head, chunk), groups in order, then heads, then chunks.
+__device__ __forceinline__ int att_total(const MegaArgs& m, const int* g_kmax, int n_groups) {
+  int total = 0;
+  for (int g = 0; g < n_groups; ++g) total += m.H * ((g_kmax[g] + m.aa.CH - 1) / m.aa.CH);
+  return total;
 }
-
-// ---------------------------------------------------------------------------- producer
-__device__ void mega_producer(const MegaArgs& m, unsigned char* ring, uint64_t* full, uint64_t* empty, int S, int lane) {
-  const int G = gridDim.x, cta = blockIdx.x;
-  const unsigned tile_bytes = 512u * m.planes;
-  const uint64_t pol = l2_evict_first();
-  unsigned it = 0;
-  bool ok = true;
-  for (int pass = 0; pass < m.max_passes && ok; ++pass) {
-    if (pass > 0) {
-      unsigned go = 0;
-      if (lane == 0) {
-        ok = wait_flag(m, m.flags + m.f_dec, epoch(m, pass - 1, m.L));
-        go = ok ? __ldcg(m.dec_val) : 0u;
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      go = __shfl_sync(0xffffffffu, go, 0);
-      if (!ok || go == 0u) break;
+__device__ __forceinline__ void att_decode(const MegaArgs& m, const int* g_kmax, int n_groups, int item, int& g, int& h, int& c) {
+  int rem = item;
+  for (g = 0; g < n_groups; ++g) {
+    const int nch = (g_kmax[g] + m.aa.CH - 1) / m.aa.CH;
+    if (rem < m.H * nch) {
+      h = rem / nch;
+      c = rem % nch;
+      return;
     }
-#pragma unroll 1
-    for (int ph = 0; ph <= 4 * m.L && ok; ++ph) {
-      const Phase p = phase_of(m, ph);
-      const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
-#pragma unroll 1
-      for (int u = first_unit(p, cta, G); u < p.units && ok; u += G) {
-        const unsigned char* src = reinterpret_cast<const unsigned char*>(p.w) + (size_t)u * p.ksteps * tile_bytes;
-#pragma unroll 1
-        for (int st = 0; st < nst; ++st, ++it) {
-          const int slot = it % S;
-          const unsigned tiles = min(kStageTiles, p.ksteps - st * kStageTiles);
-          if (lane == 0) {
-            ok = wait_mbar(m, empty + slot, ((it / S) & 1) ^ 1);
-            if (ok) {
-              mbar_expect_tx(full + slot, tiles * tile_bytes);
-              tma_1d(ring + (size_t)slot * kStageTiles * tile_bytes, src + (size_t)st * kStageTiles * tile_bytes, tiles * tile_bytes,
-                     full + slot, pol);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-        }
-      }
-    }
+    rem -= m.H * nch;
   }
-  // leave no copy in flight: every issued stage must have landed
-  if (lane == 0) {
-    const unsigned issued = it;
-    const unsigned from = issued > (unsigned)S ? issued - S : 0;
-#pragma unroll 1
-    for (unsigned j = from; j < issued; ++j) {
-      unsigned n = 0;
-      while (!mbar_try(full + j % S, (j / S) & 1) && ++n < kSpinLimit) {
-      }
-    }
-  }
+  g = 0, h = 0, c = 0;
+}
+// Item index of (g, h, 0): its CTA combines the head's chunks.
+__device__ __forceinline__ int att_item0(const MegaArgs& m, const int* g_kmax, int g, int h) {
+  int base = 0;
+  for (int j = 0; j < g; ++j) base += m.H * ((g_kmax[j] + m.aa.CH - 1) / m.aa.CH);
+  return base + h * ((g_kmax[g] + m.aa.CH - 1) / m.aa.CH);
 }
 
-// ---------------------------------------------------------------------------- consumer helpers
+// ---------------------------------------------------------------------------- shared memory
 struct MegaSmem {
   unsigned char* ring;
   uint64_t* full;
   uint64_t* empty;
-  int S;
-  float* red;  // [8][16][16]
-  float* ssr;  // [8][16]
-  uint4* xs;   // phase input fragments [k-steps][NG][32 lanes] (shares space with the attention buffers)
-  float* rsv;  // [16] RMS scale per row
-  float* qs;
-  float* ps;
-  void* ks;
-  void* vs;
+  float* red;    // [kMaxPieces][8][16][RB]; the attention scratch aliases it
+  float* ssr;    // [8][RB]
+  float* hpre;   // [kMaxPieces][rows][16] epilogue residual inputs
+  float* cpre;   // [kMaxPieces][rows][16] cross terms of the next layer (W2)
+  float* qs;     // [rows][DH]
+  float* ps;     // [rows][CH]
   float* mrow;
   float* lrow;
   int* lim;
   int* plan_sh;
-  int* misc;  // [0]: last-arrival flag, [1]: any-active
-  int* rseq;  // this pass's row metadata, copied once per pass
+  int* misc;
+  int* rseq;  // this pass's row metadata
   int* rpos;
   int* rlat;
   int* rbyte;
+  int* rnkeys;
+  int* gmeta;  // [5][kMegaRows + 1]: g_seq, g_row0, g_nrows, g_kmax, g_fresh
+  int n_rows, n_groups;
 };
 
-// Source rows of a phase input: value = a[k] (+ c[k] for the cross term).
-struct XSrc {
-  const float* a;
-  const float* c;
-};
-
-// Input row of a phase (before the gain): QKV reads B_l = D_{l-1} + c_l (D_0 =
-// embedding), O reads the attention output, W13 and the head read the
-// residual stream, W2 reads the SwiGLU activations.
-__device__ __forceinline__ XSrc x_src(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int row) {
-  XSrc x{nullptr, nullptr};
-  const int d = m.d;
-  if (p.kind == PH_QKV) {
-    x.a = (p.layer == 0) ? m.ga.embed + (size_t)sm.rbyte[row] * d : m.h + (size_t)row * d;
-    x.c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, p.layer, d, sm.rseq[row], sm.rlat[row]);
-  } else if (p.kind == PH_O) {
-    x.a = m.att + (size_t)row * d;
-  } else if (p.kind == PH_W2) {
-    x.a = m.act + (size_t)row * m.F;
-  } else {
-    x.a = m.h + (size_t)row * d;
-  }
-  return x;
-}
-__device__ __forceinline__ float2 ld2(const float* p) { return __ldcg(reinterpret_cast<const float2*>(p)); }
-
-// Flag of the i-th input that k-steps s0, s0 + 8, ... of phase p depend on:
-// QKV and the head read the residual stream (W2 units), O reads attention
-// heads (one per group), W13 the O units, W2 the W13 unit pairs.
-__device__ __forceinline__ const unsigned* input_flag(const MegaArgs& m, const Phase& p, int s0, int n_groups, int i) {
-  const unsigned* f = m.flags;
-  switch (p.kind) {
-    case PH_O: {
-      const int spk = m.dh / 16;  // k-steps per head
-      return f + m.f_att + (i % n_groups) * m.H + (s0 + 8 * (i / n_groups)) / spk;
+// ---------------------------------------------------------------------------- producer
+template <int PL, int DH, typename KVT>
+__device__ void mega_producer(const MegaArgs& m, MegaSmem& sm, int lane) {
+  const int G = gridDim.x, cta = blockIdx.x;
+  const uint64_t pol = l2_evict_first();
+  unsigned it = 0;
+  bool ok = true;
+  int gk[kMegaRows + 1], gs[kMegaRows + 1], gf[kMegaRows + 1];  // group kmax, sequence, fresh (lane 0)
+  int ng = 0;
+  auto load_groups = [&]() {
+    ng = min(__ldcg(m.rows.n_groups), kMegaRows);
+    for (int g = 0; g < ng; ++g) {
+      gk[g] = __ldcg(m.rows.g_kmax + g);
+      gs[g] = __ldcg(m.rows.g_seq + g);
+      gf[g] = __ldcg(m.rows.g_fresh + g);
     }
-    case PH_W13:
-      return f + m.f_o + s0 + 8 * i;
-    case PH_W2:
-      return f + m.f_w13 + 2 * (s0 + 8 * (i >> 1)) + (i & 1);
-    default:  // QKV (layer > 0), head
-      return f + m.f_w2 + s0 + 8 * i;
+  };
+  auto next_slot = [&](unsigned bytes) -> unsigned char* {  // lane 0: a free slot armed for `bytes`
+    const int slot = it % kRingSlots;
+    if (!wait_mbar(m, sm.empty + slot, ((it / kRingSlots) & 1) ^ 1)) {
+      ok = false;
+      return nullptr;
+    }
+    mbar_expect_tx(sm.full + slot, bytes);
+    ++it;
+    return sm.ring + (size_t)slot * kSlotBytes;
+  };
+  auto issue_phase = [&](const Phase& p) {
+    const unsigned tile_bytes = 512u * PL;
+    for (int i = 0; i < p.a.count && ok; ++i) {
+      const int u = p.a.first + i * p.a.step;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(p.w) +
+                                 ((size_t)u * p.ksteps + (size_t)p.seg * p.seg_steps) * tile_bytes;
+      const int tps = tiles_per_slot<PL>();
+      for (int t0 = 0; t0 < p.seg_steps && ok; t0 += tps) {
+        const unsigned bytes = (unsigned)min(tps, p.seg_steps - t0) * tile_bytes;
+        unsigned char* dst = next_slot(bytes);
+        if (dst) tma_1d(dst, src + (size_t)t0 * tile_bytes, bytes, sm.full + ((it - 1) % kRingSlots), pol);
+      }
+    }
+  };
+  auto issue_attention = [&](int layer) {
+    const int total = att_total(m, gk, ng);
+    const int CH = m.aa.CH, PT = m.ga.PT;
+    const unsigned page_bytes = (unsigned)(PT * DH * sizeof(KVT));
+    for (int item = cta; item < total && ok; item += G) {
+      int g, h, c;
+      att_decode(m, gk, ng, item, g, h, c);
+      const int t0 = c * CH;
+      const int tc = min(min(t0 + CH, gk[g]), gf[g]);  // cached keys of this chunk: [t0, tc)
+      const int np = tc > t0 ? (tc - t0 + PT - 1) / PT : 0;
+      int pages[8];
+      int nvalid = 0;
+      for (int j = 0; j < np; ++j) {
+        const int pi = t0 / PT + j;
+        pages[j] = (pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + gs[g] * m.ga.max_pages + pi) : -1;
+        nvalid += pages[j] >= 0;
+      }
+      unsigned char* dst = next_slot(2u * nvalid * page_bytes);
+      if (!dst) break;
+      uint64_t* bar = sm.full + ((it - 1) % kRingSlots);
+      for (int j = 0; j < np; ++j) {
+        if (pages[j] < 0) continue;
+        const size_t hoff = (((size_t)pages[j] * m.L + layer) * 2) * m.H;
+        const KVT* kv = static_cast<const KVT*>(m.ga.kv);
+        const KVT* ksrc = kv + ((hoff + 0 * m.H + h) * PT) * DH;
+        const KVT* vsrc = kv + ((hoff + 1 * m.H + h) * PT) * DH;
+        tma_1d_plain(dst + (size_t)j * page_bytes, ksrc, page_bytes, bar);
+        tma_1d_plain(dst + (size_t)CH * DH * sizeof(KVT) + (size_t)j * page_bytes, vsrc, page_bytes, bar);
+      }
+    }
+  };
+  if (lane == 0) {
+    load_groups();
+    for (int pass = 0; pass < m.max_passes && ok; ++pass) {
+      for (int l = 0; l < m.L && ok; ++l) {
+        issue_phase(phase_of(m, PH_QKV, l, cta, G));
+        if (pass > 0 && l == 0) {
+          // weights of the next pass went out already; the items need its plan
+          if (!wait_flag(m, m.flags + 0, epoch(m, pass - 1, m.L, ST_LOGIT), true)) {
+            ok = false;
+            break;
+          }
+          if (__ldcg(m.dec_val) == 0u) break;
+          fence_proxy_async_global();
+          load_groups();
+        }
+        issue_attention(l);
+        issue_phase(phase_of(m, PH_O, l, cta, G));
+        issue_phase(phase_of(m, PH_W13, l, cta, G));
+        issue_phase(phase_of(m, PH_W2, l, cta, G));
+      }
+      if (!ok) break;
+      if (pass > 0 && __ldcg(m.dec_val) == 0u) break;
+      issue_phase(phase_of(m, PH_HEAD, 0, cta, G));
+    }
+    // leave no copy in flight: every issued slot must have landed
+    const unsigned from = it > (unsigned)kRingSlots ? it - kRingSlots : 0;
+    const unsigned long long t0 = gtimer();
+    for (unsigned j = from; j < it; ++j)
+      while (!mbar_try(sm.full + j % kRingSlots, (j / kRingSlots) & 1) && gtimer() - t0 < 2ull * m.wait_ns + 1000000ull) {
+      }
   }
+  __syncwarp();
 }
 
-// Wait (whole warp) until the inputs of k-steps s0, s0 + 8, ... (n of them)
-// of phase p in this pass are written.  One polling loop for every phase
-// kind keeps the kernel's code small.
-__device__ __forceinline__ bool wait_inputs(const MegaArgs& m, const Phase& p, int pass, int s0, int n, int n_groups) {
-  if (p.kind == PH_QKV && p.layer == 0) return true;
-  int count = n;
-  unsigned target = epoch(m, pass, p.layer);
-  if (p.kind == PH_O) count = n * n_groups;
-  else if (p.kind == PH_W2) count = 2 * n;
-  else if (p.kind == PH_QKV) target = epoch(m, pass, p.layer - 1);
-  else if (p.kind == PH_HEAD) target = epoch(m, pass, m.L - 1);
-  return warp_wait(m, count, [&](int i) { return input_flag(m, p, s0, n_groups, i); }, target);
-}
+// ---------------------------------------------------------------------------- consumer: GEMV phases
+// Input row of a phase before the gain, read as exchange words: x[row][col0 + k].
+struct XSrc {
+  const u64* x;  // NULL: layer-0 input embed[byte] + c_0
+  int ld, col0;
+  unsigned e;
+};
 
-__device__ __forceinline__ const float* phase_gain(const MegaArgs& m, const Phase& p) {
-  if (p.kind == PH_QKV) return m.layers[p.layer].attn_norm;
-  if (p.kind == PH_W13) return m.layers[p.layer].ffn_norm;
-  if (p.kind == PH_HEAD) return m.final_norm;
-  return nullptr;
-}
-
-// Epilogue of one output pair, dispatched at run time so that one copy of the
-// phase loop serves every projection (the kernel's code must stay small
-// enough for the SM's instruction caches).
-__device__ __forceinline__ void mega_epilogue(const GemmArgs& ga, int epi, int u, int r16, int row, float v0, float v1) {
-  switch (epi) {
-    case EPI_QKV:
-      gemm_epilogue<EPI_QKV>(ga, u, r16, row, v0, v1);
-      break;
-    case EPI_XRESID:
-      gemm_epilogue<EPI_XRESID>(ga, u, r16, row, v0, v1);
-      break;
-    case EPI_SWIGLU:
-      gemm_epilogue<EPI_SWIGLU>(ga, u, r16, row, v0, v1);
-      break;
-    case EPI_RESID:
-      gemm_epilogue<EPI_RESID>(ga, u, r16, row, v0, v1);
-      break;
-    default:
-      gemm_epilogue<EPI_STORE>(ga, u, r16, row, v0, v1);
-      break;
-  }
-}
-
-// Phase input of this warp's k-steps warp, warp + 8, ... (nkw <= 8 of them) as
-// split-bf16 B fragments in registers, and its lanes' sums of squares (the
-// canonical order: per lane, k-steps in increasing order).  Every load is
-// issued unconditionally (a dead row reads row 0, a k-step past the warp's
-// share re-reads its last one; neither reaches an output) so all are in
-// flight at once.  HASC: QKV input, which adds the cross term c_l.
-template <int NG, bool HASC>
-__device__ __forceinline__ void build_frags(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int nr, int nkw,
-                                            const float* gain, uint4 (&xf)[8][NG], float (&ss)[NG], int warp, int lane) {
+// Wait for and load this warp's k-steps (warp, warp + 8, ...; nkw of them) of
+// every live row as B fragments, plus the lanes' sums of squares (canonical
+// order).  Rows >= nr get zeros.
+template <int NG>
+__device__ __forceinline__ bool gather_frags(const MegaArgs& m, const MegaSmem& sm, const XSrc& xs, int nr, int nkw, const float* gain,
+                                             uint4 (&xf)[8][NG], float (&ss)[NG], int warp, int lane, int pass) {
   const int g = lane >> 2, t = lane & 3;
-  const bool norm = gain != nullptr;
-  XSrc src[NG];
+  float2 xa[8][NG], xb[8][NG];
+  unsigned pending = 0;
 #pragma unroll
-  for (int n = 0; n < NG; ++n) {
-    ss[n] = 0.f;
-    const int row = n * 8 + g;
-    src[n] = x_src(m, sm, p, row < nr ? row : 0);
+  for (int j = 0; j < 8; ++j)
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      xa[j][n] = xb[j][n] = make_float2(0.f, 0.f);
+      if (j < nkw && n * 8 + g < nr) pending |= 3u << ((j * NG + n) * 2);
+    }
+  if (!xs.x) {  // layer 0: embedding + cross term, finished data
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int n = 0; n < NG; ++n)
+        if ((pending >> ((j * NG + n) * 2)) & 1u) {
+          const int row = n * 8 + g, k0 = (warp + 8 * j) * 16 + 2 * t;
+          const float* e = m.ga.embed + (size_t)sm.rbyte[row] * m.d;
+          const float* c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, 0, m.d, sm.rseq[row], sm.rlat[row]);
+          xa[j][n] = make_float2(__ldg(e + k0) + __ldcg(c + k0), __ldg(e + k0 + 1) + __ldcg(c + k0 + 1));
+          xb[j][n] = make_float2(__ldg(e + k0 + 8) + __ldcg(c + k0 + 8), __ldg(e + k0 + 9) + __ldcg(c + k0 + 9));
+        }
+    pending = 0;
   }
+  Spin spins;
+  bool ok = true;
+  if (__any_sync(0xffffffffu, pending != 0u)) {  // warp-uniform: the loop below has a full-mask vote
+    // Sentinels: lane j < nkw polls one word of k-step warp + 8 j (row 0, its last column) until
+    // every k-step of the warp has data; only then do all lanes load everything.  While waiting,
+    // a warp issues at most 8 loads per round.
+    const u64* sp = xs.x + xs.col0 + (warp + 8 * lane) * 16 + 15;
+    bool ready = lane >= nkw;
+    while (true) {
+      if (!ready) ready = xw_ok(xw_ld(sp), xs.e);
+      if (__all_sync(0xffffffffu, ready)) break;
+      if (!spin_step(m, spins)) {
+        ok = false;
+        break;
+      }
+    }
+  }
+  trace_mark(m, pass, TR_SENT << 8);
+  while (pending && ok) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    if (half * 4 < nkw) {
-      float2 ra[4][NG], rb[4][NG];
-      float4 gv[4];
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = min(half * 4 + jj, nkw - 1);
-        const int k0 = (warp + 8 * j) * 16 + 2 * t;
+      for (int n = 0; n < NG; ++n)
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          ra[jj][n] = ld2(src[n].a + k0);
-          rb[jj][n] = ld2(src[n].a + k0 + 8);
-          if constexpr (HASC) {
-            const float2 c0 = ld2(src[n].c + k0), c8 = ld2(src[n].c + k0 + 8);
-            ra[jj][n] = make_float2(ra[jj][n].x + c0.x, ra[jj][n].y + c0.y);
-            rb[jj][n] = make_float2(rb[jj][n].x + c8.x, rb[jj][n].y + c8.y);
+        for (int hf = 0; hf < 2; ++hf) {
+          const unsigned bit = 1u << ((j * NG + n) * 2 + hf);
+          if (pending & bit) {
+            const int row = n * 8 + g, k0 = (warp + 8 * j) * 16 + 2 * t + 8 * hf;
+            u64 a, b;
+            xw_ld2(xs.x + (size_t)row * xs.ld + xs.col0 + k0, a, b);
+            if (xw_ok(a, xs.e) && xw_ok(b, xs.e)) {
+              const float2 v = make_float2(xw_val(a), xw_val(b));
+              if (hf == 0) xa[j][n] = v;
+              else xb[j][n] = v;
+              pending &= ~bit;
+            }
           }
         }
-        gv[jj] = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (norm) gv[jj] = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
-      }
+    if (pending && !spin_step(m, spins)) {
+      ok = false;
+      break;
+    }
+  }
+  trace_mark(m, pass, TR_GATH << 8);
+  const bool norm = gain != nullptr;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = half * 4 + jj;
+  for (int n = 0; n < NG; ++n) ss[n] = 0.f;
 #pragma unroll
-        for (int n = 0; n < NG; ++n) {
-          const float2 a = ra[jj][n], b = rb[jj][n];
-          if (norm && j < nkw) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
-          const XFrag f = make_xfrag(a.x * gv[jj].x, a.y * gv[jj].y, b.x * gv[jj].z, b.y * gv[jj].w);
-          xf[j][n] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
+  for (int j = 0; j < 8; ++j) {
+    float4 gv = make_float4(1.f, 1.f, 1.f, 1.f);
+    const int k0 = (warp + 8 * j) * 16 + 2 * t;
+    if (norm && j < nkw) gv = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      const float2 a = xa[j][n], b = xb[j][n];
+      if (norm && j < nkw) ss[n] = ss_add(ss[n], a.x, a.y, b.x, b.y);
+      const XFrag f = make_xfrag(a.x * gv.x, a.y * gv.y, b.x * gv.z, b.y * gv.w);
+      xf[j][n] = make_uint4(f.b0h, f.b1h, f.b0l, f.b1l);
+    }
+  }
+  return ok;
+}
+
+// Epilogue side inputs, into smem before the MMAs: the residual the output is
+// added to (O: the stream after the previous layer; W2 finisher: after O) and
+// the next layer's cross term (W2 finisher).
+template <int NG>
+__device__ __forceinline__ bool prefetch_side(const MegaArgs& m, MegaSmem& sm, const Phase& p, int jv0, int nu, int pass, int nr, int tid) {
+  const int l = p.layer, d = m.d;
+  const bool is_o = p.kind == PH_O;
+  const bool fin = p.kind == PH_W2 && p.seg == n_w2_segments(m) - 1;
+  if (!is_o && !fin) return true;
+  const int n = nu * kMegaRows * 16;
+  auto col_of = [&](int i) { return (p.a.first + (jv0 + i / (kMegaRows * 16)) * p.a.step) * 16 + i % 16; };
+  auto row_of = [&](int i) { return (i / 16) % kMegaRows; };
+  if (fin)
+    for (int i = tid; i < n; i += 256) {
+      const int row = row_of(i);
+      sm.cpre[i] = (l + 1 < m.L && row < nr)
+                       ? __ldcg(c_row(m.ga.c_lat, m.ga.max_lat, m.L, l + 1, d, sm.rseq[row], sm.rlat[row]) + col_of(i))
+                       : 0.f;
+    }
+  if (is_o && l == 0) {  // the stream before layer 0 is embed + c_0
+    for (int i = tid; i < n; i += 256) {
+      const int row = row_of(i);
+      sm.hpre[i] = row < nr ? __ldg(m.ga.embed + (size_t)sm.rbyte[row] * d + col_of(i)) +
+                                  __ldcg(c_row(m.ga.c_lat, m.ga.max_lat, m.L, 0, d, sm.rseq[row], sm.rlat[row]) + col_of(i))
+                            : 0.f;
+    }
+    return true;
+  }
+  const unsigned e = is_o ? epoch(m, pass, l - 1, ST_HW) : epoch(m, pass, l, ST_HO);
+  // dead rows read row 0's word (always written) and are never used
+  return poll_words<kMaxPieces * kMegaRows * 16 / 256>(
+      m, n, e, tid, [&](int i) { return m.x_h + (size_t)(row_of(i) < nr ? row_of(i) : 0) * d + col_of(i); },
+      [&](int i, float v) { sm.hpre[i] = v; });
+}
+
+// Output pair (tile rows r16, r16 + 8) of unit u for row `row`.
+template <int NG>
+__device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int jv, int u, int r16, int row,
+                                              float v0, float v1, int pass) {
+  const int d = m.d, l = p.layer;
+  switch (p.kind) {
+    case PH_QKV: {
+      const unsigned e = epoch(m, pass, l, ST_QKV);
+      const GemmArgs& a = m.ga;
+      const int tiles_sec = d / 16;
+      const int sec = u / tiles_sec, lt = u % tiles_sec;
+      const int pos = sm.rpos[row], seq = sm.rseq[row];
+      if (sec < 2) {  // q and k tiles hold rotary pairs (j, j + dh/2) in rows (r16, r16 + 8)
+        const int tph = m.dh / 16;
+        const int h = lt / tph, j = (lt % tph) * 8 + r16;
+        const int half = m.dh / 2;
+        const size_t ri = (size_t)pos * half + j;
+        const float c = __ldg(a.rope_cos + ri), s = __ldg(a.rope_sin + ri);
+        const float o0 = v0 * c - v1 * s, o1 = v1 * c + v0 * s;
+        const size_t xo = (size_t)row * d + h * m.dh + j;
+        if (sec == 0) {
+          xw_st(m.x_q + xo, o0, e);
+          xw_st(m.x_q + xo + half, o1, e);
+          return true;
         }
+        const int pi = pos / a.PT;
+        const int page = (pi < a.max_pages) ? __ldcg(a.page_table + seq * a.max_pages + pi) : -1;
+        float r0 = o0, r1 = o1;
+        if (page < 0) {
+          set_status(a.status, kErrDevice);
+        } else {
+          const size_t off = kv_offset(a, page, l, 0, h, pos % a.PT, 0);
+          kv_store(a, off + j, o0);
+          kv_store(a, off + j + half, o1);
+        }
+        if (!a.kv_f32) {
+          r0 = __bfloat162float(__float2bfloat16_rn(o0));
+          r1 = __bfloat162float(__float2bfloat16_rn(o1));
+        }
+        xw_st(m.x_k + xo, r0, e);
+        xw_st(m.x_k + xo + half, r1, e);
+      } else {
+        const int n0 = lt * 16 + r16, n1 = n0 + 8;
+        const int pi = pos / a.PT;
+        const int page = (pi < a.max_pages) ? __ldcg(a.page_table + seq * a.max_pages + pi) : -1;
+        if (page < 0) {
+          set_status(a.status, kErrDevice);
+        } else {
+          kv_store(a, kv_offset(a, page, l, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
+          kv_store(a, kv_offset(a, page, l, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
+        }
+        float r0 = v0, r1 = v1;
+        if (!a.kv_f32) {
+          r0 = __bfloat162float(__float2bfloat16_rn(v0));
+          r1 = __bfloat162float(__float2bfloat16_rn(v1));
+        }
+        xw_st(m.x_v + (size_t)row * d + n0, r0, e);
+        xw_st(m.x_v + (size_t)row * d + n1, r1, e);
       }
+      return true;
+    }
+    case PH_O: {
+      if (m.stall_test && pass == 0 && l == 0 && u == 0) return true;  // test only: never publish
+      const unsigned e = epoch(m, pass, l, ST_HO);
+      const float* hp = sm.hpre + (jv * kMegaRows + row) * 16;
+      xw_st(m.x_h + (size_t)row * d + u * 16 + r16, hp[r16] + v0, e);
+      xw_st(m.x_h + (size_t)row * d + u * 16 + r16 + 8, hp[r16 + 8] + v1, e);
+      return true;
+    }
+    case PH_W13: {
+      xw_st(m.x_act + (size_t)row * m.F + u * 8 + r16, silu(v0) * v1, epoch(m, pass, l, ST_ACT));
+      return true;
+    }
+    case PH_W2: {
+      const int nseg = n_w2_segments(m);
+      if (p.seg < nseg - 1) {
+        const unsigned e = epoch(m, pass, l, ST_W2P);
+        u64* dst = m.x_w2p + ((size_t)p.seg * kMegaRows + row) * d + u * 16 + r16;
+        xw_st(dst, v0, e);
+        xw_st(dst + 8, v1, e);
+        return true;
+      }
+      // finisher: the segment sums in order, then the residual and the next layer's cross term
+      float t0 = v0, t1 = v1;
+      bool ok = true;
+      if (nseg > 1) {
+        constexpr int kMaxSeg = 4;  // d_ffn <= 4096
+        const unsigned e = epoch(m, pass, l, ST_W2P);
+        float sv[2 * (kMaxSeg - 1)];
+        unsigned pending = (1u << (2 * (nseg - 1))) - 1u;
+        Spin spins;
+        while (pending) {
+          u64 w[2 * (kMaxSeg - 1)];
+#pragma unroll
+          for (int i = 0; i < 2 * (kMaxSeg - 1); ++i)
+            if ((pending >> i) & 1u) w[i] = xw_ld(m.x_w2p + ((size_t)(i >> 1) * kMegaRows + row) * d + u * 16 + r16 + 8 * (i & 1));
+#pragma unroll
+          for (int i = 0; i < 2 * (kMaxSeg - 1); ++i)
+            if (((pending >> i) & 1u) && xw_ok(w[i], e)) {
+              sv[i] = xw_val(w[i]);
+              pending &= ~(1u << i);
+            }
+          if (pending && !spin_step(m, spins)) {
+            ok = false;
+            break;
+          }
+        }
+        float a0 = sv[0], a1 = sv[1];
+#pragma unroll
+        for (int q = 1; q < kMaxSeg - 1; ++q)
+          if (q < nseg - 1) {
+            a0 = a0 + sv[2 * q];
+            a1 = a1 + sv[2 * q + 1];
+          }
+        t0 = a0 + v0;
+        t1 = a1 + v1;
+      }
+      const float* hp = sm.hpre + (jv * kMegaRows + row) * 16;
+      const float* cp = sm.cpre + (jv * kMegaRows + row) * 16;
+      float h0 = hp[r16] + t0, h1 = hp[r16 + 8] + t1;
+      if (l + 1 < m.L) {
+        h0 = h0 + cp[r16];
+        h1 = h1 + cp[r16 + 8];
+      }
+      const unsigned e = epoch(m, pass, l, ST_HW);
+      xw_st(m.x_h + (size_t)row * d + u * 16 + r16, h0, e);
+      xw_st(m.x_h + (size_t)row * d + u * 16 + r16 + 8, h1, e);
+      return ok;
+    }
+    default: {
+      const unsigned e = epoch(m, pass, m.L, ST_LOGIT);
+      xw_st(m.x_logit + (size_t)row * 256 + u * 16 + r16, v0, e);
+      xw_st(m.x_logit + (size_t)row * 256 + u * 16 + r16 + 8, v1, e);
+      return true;
     }
   }
 }
 
-// Phase with K <= 1024 (a unit is at most 8 / kTPW ring stages).  All eight warps
-// work on every unit: warp w owns the k-steps s = w (mod 8) -- lane group w
-// of the canonical order -- so it waits only for the inputs of its own
-// k-steps and keeps their fragments in registers.  The CTA's units (up to
-// kMegaUnits at a time) run together: one accumulator per unit per warp, so
-// the units' MMA chains interleave; then one cross-warp reduction (the
-// operation order of tile_reduce: warps in order, the RMS scale from the
-// warps' sums of squares in order), one epilogue pass, one fence and the
-// units' flags.
-constexpr int kMegaUnits = 4;
-
+// One GEMV phase of this CTA: gather the input once, run its pieces from the
+// ring (all eight warps on every piece, warp w on the k-steps = w mod 8 --
+// lane group w of the canonical order), reduce across warps in order, apply
+// the epilogue.  `it`: ring slots consumed so far.
 template <int NG, int PL>
-__device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int epi, int pass, unsigned& it, int nr,
-                                int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
+__device__ bool run_gemv(const MegaArgs& m, MegaSmem& sm, const Phase& p, const XSrc& xs, const float* gain, int pass, unsigned& it,
+                         int tid) {
   constexpr int RB = 8 * NG;
-  const int G = gridDim.x, cta = blockIdx.x;
-  const int u0 = first_unit(p, cta, G);
-  if (u0 >= p.units) return true;
-  const int nunits = (p.units - u0 + G - 1) / G;
-  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;  // <= 8 / kTPW
-  const unsigned it0 = it;
-  it += (unsigned)(nunits * nst);
+  if (p.a.count == 0) return true;
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const float* gain = phase_gain(m, p);
-  const bool norm = gain != nullptr;
-  const int nkw = (p.ksteps - warp + 7) / 8;  // k-steps of this warp (<= 8)
-  trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
-  bool ok = wait_inputs(m, p, pass, warp, nkw, n_groups);
-  trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
+  const int nr = sm.n_rows;
+  const int nkw = (p.seg_steps - warp + 7) / 8;
+  trace_mark(m, pass, TR_PH << 8 | p.kind);
+  // the epilogue's side inputs are older data: fetch them while the phase input is still on its way
+  bool ok = prefetch_side<NG>(m, sm, p, 0, min(kMaxPieces, p.a.count), pass, nr, tid);
+  trace_mark(m, pass, TR_PRE << 8 | p.kind);
   uint4 xf[8][NG];
   float ss[NG];
-  if (p.kind == PH_QKV) build_frags<NG, true>(m, sm, p, nr, nkw, gain, xf, ss, warp, lane);
-  else build_frags<NG, false>(m, sm, p, nr, nkw, gain, xf, ss, warp, lane);
+  ok = gather_frags<NG>(m, sm, xs, nr, nkw, gain, xf, ss, warp, lane, pass) && ok;
+  const bool norm = gain != nullptr;
   if (norm) {
 #pragma unroll
     for (int n = 0; n < NG; ++n) {
@@ -525,50 +833,56 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
       if (t == 0) sm.ssr[warp * RB + n * 8 + g] = v;
     }
   }
-  trace_mark(m, pass, TR_XLOADED << 8 | p.kind);
+  trace_mark(m, pass, TR_IN << 8 | p.kind);
+  const int nsl = piece_slots<PL>(p.seg_steps);
   const unsigned tile_bytes = 512u * PL;
-  float* red = reinterpret_cast<float*>(sm.xs);  // [unit][warp][16][RB]
-#pragma unroll 1
-  for (int ug = 0; ug < nunits; ug += kMegaUnits) {
-    const int nu = min(kMegaUnits, nunits - ug);
-    float acc[kMegaUnits][NG][4];
+  for (int jv0 = 0; jv0 < p.a.count; jv0 += kMaxPieces) {
+    const int nu = min(kMaxPieces, p.a.count - jv0);
+    if (jv0 > 0) ok = prefetch_side<NG>(m, sm, p, jv0, nu, pass, nr, tid) && ok;
+    float acc[kMaxPieces][NG][4];
 #pragma unroll
-    for (int jv = 0; jv < kMegaUnits; ++jv)
+    for (int jv = 0; jv < kMaxPieces; ++jv)
 #pragma unroll
       for (int n = 0; n < NG; ++n) acc[jv][n][0] = acc[jv][n][1] = acc[jv][n][2] = acc[jv][n][3] = 0.f;
 #pragma unroll
-    for (int st = 0; st < 8 / kTPW; ++st) {
-      if (st < nst) {
-        const int ntiles = min(kStageTiles, p.ksteps - st * kStageTiles);
+    for (int jv = 0; jv < kMaxPieces; ++jv) {
+      if (jv < nu) {
+        constexpr int TPS = kSlotBytes / (512 * PL);           // tiles per slot
+        constexpr int TPW = TPS / 8;                           // tiles of a slot per warp
+        constexpr int MAXSL = (kSegSteps + TPS - 1) / TPS;     // slots per piece at most
 #pragma unroll
-        for (int jv = 0; jv < kMegaUnits; ++jv) {
-          if (jv < nu) {
-            const unsigned itu = it0 + (unsigned)((ug + jv) * nst + st);
-            const int slot = itu % sm.S;
-            if (!wait_mbar(m, sm.full + slot, (itu / sm.S) & 1)) ok = false;
-            const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-            uint4 w[kTPW][PL];
+        for (int sl = 0; sl < MAXSL; ++sl) {
+          if (sl < nsl) {
+            const unsigned itu = it++;
+            const int slot = itu % kRingSlots;
+            if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
+            const unsigned char* stage = sm.ring + (size_t)slot * kSlotBytes;
+            const int ntiles = min(TPS, p.seg_steps - sl * TPS);
+            uint4 w[TPW][PL];
 #pragma unroll
-            for (int q = 0; q < kTPW; ++q)
+            for (int q = 0; q < TPW; ++q)
 #pragma unroll
               for (int pl = 0; pl < PL; ++pl)
                 w[q][pl] = *reinterpret_cast<const uint4*>(stage + (size_t)min(8 * q + warp, ntiles - 1) * tile_bytes + pl * 512 + lane * 16);
 #pragma unroll
-            for (int q = 0; q < kTPW; ++q)
+            for (int q = 0; q < TPW; ++q) {
+              const int j = sl * TPW + q;  // this warp's j-th k-step of the piece: k-step 8 j + warp
               if (8 * q + warp < ntiles)
 #pragma unroll
                 for (int n = 0; n < NG; ++n)
-                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[st * kTPW + q][n].x, xf[st * kTPW + q][n].y, xf[st * kTPW + q][n].z, xf[st * kTPW + q][n].w});
+                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[j][n].x, xf[j][n].y, xf[j][n].z, xf[j][n].w});
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.empty + slot);
           }
         }
       }
     }
+    trace_mark(m, pass, TR_MMA << 8 | p.kind);
 #pragma unroll
-    for (int jv = 0; jv < kMegaUnits; ++jv) {
+    for (int jv = 0; jv < kMaxPieces; ++jv) {
       if (jv < nu) {
-        float* rw = red + (size_t)(jv * 8 + warp) * 16 * RB;
+        float* rw = sm.red + (size_t)(jv * 8 + warp) * 16 * RB;
 #pragma unroll
         for (int n = 0; n < NG; ++n) {
           const int c = n * 8 + 2 * t;
@@ -584,7 +898,7 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
       const int jv = pi / (8 * RB), q = pi % (8 * RB);
       const int r16 = q & 7, col = q >> 3;
       if (col >= nr) continue;
-      const float* ru = red + (size_t)jv * 8 * 16 * RB;
+      const float* ru = sm.red + (size_t)jv * 8 * 16 * RB;
       float v0 = ru[r16 * RB + col], v1 = ru[(r16 + 8) * RB + col];
 #pragma unroll
       for (int w = 1; w < kWarps; ++w) {
@@ -598,196 +912,229 @@ __device__ bool run_phase_units(const MegaArgs& m, const MegaSmem& sm, const Pha
         for (int w = 1; w < kWarps; ++w) sv += sm.ssr[w * RB + col];
         rs = 1.0f / sqrtf(sv / (float)(p.ksteps * 16) + m.eps);
       }
-      mega_epilogue(ga, epi, u0 + (ug + jv) * G, r16, col, v0 * rs, v1 * rs);
+      const int u = p.a.first + (jv0 + jv) * p.a.step;
+      ok = mega_epilogue<NG>(m, sm, p, jv, u, r16, col, v0 * rs, v1 * rs, pass) && ok;
     }
-    consumer_sync();  // epilogue stores done, red free again
-    if (tid == 0) {
-      fence_acq_rel();
-      for (int jv = 0; jv < nu; ++jv) st_relaxed(flag_base + u0 + (ug + jv) * G, epoch(m, pass, p.layer));
-    }
-    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
+    consumer_sync();  // red, hpre, cpre free again
   }
+  trace_mark(m, pass, TR_DONE << 8 | p.kind);
   return ok;
 }
 
-// Streamed-input phase (W2, K = F > 1024): inputs loaded stage by stage, one
-// stage ahead.
-template <int NG, int PL>
-__device__ bool run_phase_streamed(const MegaArgs& m, const MegaSmem& sm, const Phase& p, int pass, unsigned& it, int nr,
-                                   int n_groups, const GemmArgs& ga, unsigned* flag_base, int tid) {
-  const int G = gridDim.x, cta = blockIdx.x;
-  const int u0 = first_unit(p, cta, G);
-  if (u0 >= p.units) return true;
-  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const unsigned tile_bytes = 512u * PL;
-  const int nst = (p.ksteps + kStageTiles - 1) / kStageTiles;
+// ---------------------------------------------------------------------------- consumer: attention
+// attn_combine for one (row, head) by one warp, with the chunk partials read as
+// exchange words: for each block of 32 chunks every lane polls its chunk's
+// (m, l) and its columns of every chunk's o in one round of loads, then the
+// arithmetic of attn_combine runs in the same order on the registers.
+template <int DH>
+__device__ __forceinline__ bool combine_row_xw(const MegaArgs& m, const u64* base, int nch, int lane, unsigned e, u64* out, unsigned e_out) {
+  constexpr int DPL = DH >= 32 ? DH / 32 : 1;  // columns per lane
+  constexpr int REC = 2 + DH;
+  const bool col_ok = lane < DH;
   bool ok = true;
-  trace_mark(m, pass, TR_PHASE_BEGIN << 8 | p.kind);
-  ok = wait_inputs(m, p, pass, warp, (p.ksteps - warp + 7) / 8, n_groups);  // all of this warp's k-steps
-  trace_mark(m, pass, TR_INPUTS << 8 | p.kind);
-  XSrc src[NG];
-#pragma unroll
-  for (int n = 0; n < NG; ++n) src[n] = x_src(m, sm, p, n * 8 + g < nr ? n * 8 + g : 0);
-  // unconditional loads (dead rows read row 0, k-steps past the end re-read
-  // the last one; neither reaches an output) so all of a stage's are in flight together
-  auto load = [&](int st, float2 (&xa)[kTPW][NG], float2 (&xb)[kTPW][NG]) {
-#pragma unroll
-    for (int jj = 0; jj < kTPW; ++jj) {
-      const int ks = min(st * kStageTiles + 8 * jj + warp, p.ksteps - 1);
-#pragma unroll
-      for (int n = 0; n < NG; ++n) {
-        xa[jj][n] = ld2(src[n].a + ks * 16 + 2 * t);
-        xb[jj][n] = ld2(src[n].a + ks * 16 + 2 * t + 8);
+  auto poll_ml = [&](int ch, float& mm, float& ll) {
+    Spin spins;
+    while (true) {
+      u64 a, b;
+      a = xw_ld(base + (size_t)ch * REC);
+      b = xw_ld(base + (size_t)ch * REC + 1);
+      if (xw_ok(a, e) && xw_ok(b, e)) {
+        mm = xw_val(a), ll = xw_val(b);
+        return true;
       }
+      if (!spin_step(m, spins)) return false;
     }
-    return ok;
   };
-  // inputs prefetched D stages ahead in registers (an L2 round trip is much
-  // longer than one stage's MMAs); stages run in groups of D so the register
-  // ring is indexed at compile time
-  constexpr int D = (kTPW == 4) ? 2 / NG : 1;
-  for (int u = u0; u < p.units; u += G) {
-    float acc[NG][4], ss[NG];
-#pragma unroll
-    for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
-    float2 xa[D][kTPW][NG], xb[D][kTPW][NG];
-#pragma unroll
-    for (int d = 0; d < D; ++d)
-      if (d < nst) ok = load(d, xa[d], xb[d]) && ok;
+  float mmax = -INFINITY;
+  float m0 = 0.f, l0 = 0.f;  // the lane's chunk of the first block, kept for the second pass
 #pragma unroll 1
-    for (int s0 = 0; s0 < nst; s0 += D) {
+  for (int ch = lane; ch < nch; ch += 32) {
+    float mm, ll;
+    ok = poll_ml(ch, mm, ll) && ok;
+    if (ch < 32) m0 = mm, l0 = ll;
+    if (ll > 0.f) mmax = fmaxf(mmax, mm);
+  }
+  mmax = warp_max(mmax);
+  float l = 0.f, o[DPL];
 #pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int st = s0 + d;
-      if (st < nst) {
-        const int slot = it % sm.S;
-        if (!wait_mbar(m, sm.full + slot, (it / sm.S) & 1)) ok = false;
-        const unsigned char* stage = sm.ring + (size_t)slot * kStageTiles * tile_bytes;
-        float2 (&ca)[kTPW][NG] = xa[d];
-        float2 (&cb)[kTPW][NG] = xb[d];
-        if ((st + 1) * kStageTiles <= p.ksteps) {  // full stage: weight loads first, then the chain
-          uint4 w[kTPW][PL];
+  for (int i = 0; i < DPL; ++i) o[i] = 0.f;
+#pragma unroll 1
+  for (int cb = 0; cb < nch; cb += 32) {
+    const int nb = min(32, nch - cb);
+    float w = 0.f;
+    if (cb + lane < nch) {
+      float mm = m0, ll = l0;
+      if (cb > 0) ok = poll_ml(cb + lane, mm, ll) && ok;
+      if (ll > 0.f) {
+        w = expf(mm - mmax);
+        l = fmaf(ll, w, l);
+      }
+    }
+    // this lane's columns of the block's o, 16 chunks per round of loads (re-read only what is not ready)
+    constexpr int SUB = 16;
+#pragma unroll 1
+    for (int sb = 0; sb < nb; sb += SUB) {
+      float ov[SUB][DPL];
+      unsigned pending = 0;
 #pragma unroll
-          for (int jj = 0; jj < kTPW; ++jj)
+      for (int j = 0; j < SUB; ++j)
 #pragma unroll
-            for (int q = 0; q < PL; ++q)
-              w[jj][q] = *reinterpret_cast<const uint4*>(stage + (size_t)(8 * jj + warp) * tile_bytes + q * 512 + lane * 16);
-#pragma unroll
-          for (int jj = 0; jj < kTPW; ++jj)
-#pragma unroll
-            for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w[jj], make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
-        } else {
-#pragma unroll
-          for (int jj = 0; jj < kTPW; ++jj) {
-            const int tile = 8 * jj + warp;
-            if (st * kStageTiles + tile < p.ksteps) {
-              uint4 w[PL];
-#pragma unroll
-              for (int q = 0; q < PL; ++q) w[q] = *reinterpret_cast<const uint4*>(stage + (size_t)tile * tile_bytes + q * 512 + lane * 16);
-#pragma unroll
-              for (int n = 0; n < NG; ++n) mma_step<PL>(acc[n], w, make_xfrag(ca[jj][n].x, ca[jj][n].y, cb[jj][n].x, cb[jj][n].y));
-            }
-          }
+        for (int i = 0; i < DPL; ++i) {
+          ov[j][i] = 0.f;
+          if (sb + j < nb && col_ok) pending |= 1u << (j * DPL + i);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sm.empty + slot);
-        ++it;
-        if (st + D < nst) ok = load(st + D, xa[d], xb[d]) && ok;
+      Spin spins;
+      while (pending) {
+        u64 wv[SUB][DPL];
+#pragma unroll
+        for (int j = 0; j < SUB; ++j)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i)
+            if ((pending >> (j * DPL + i)) & 1u) wv[j][i] = xw_ld(base + (size_t)(cb + sb + j) * REC + 2 + lane + 32 * i);
+#pragma unroll
+        for (int j = 0; j < SUB; ++j)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i)
+            if (((pending >> (j * DPL + i)) & 1u) && xw_ok(wv[j][i], e)) {
+              ov[j][i] = xw_val(wv[j][i]);
+              pending &= ~(1u << (j * DPL + i));
+            }
+        if (pending && !spin_step(m, spins)) {
+          ok = false;
+          break;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < SUB; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, (sb + j) & 31);
+        if (sb + j < nb)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) o[i] = fmaf(ov[j][i], wj, o[i]);
       }
     }
-    }
-    trace_mark(m, pass, TR_KLOOP << 8 | p.kind);
-    tile_reduce<NG>(acc, ss, false, sm.red, sm.ssr, nr, p.ksteps * 16, m.eps, tid, 256, consumer_sync,
-                    [&](int r16, int col, float v0, float v1) { mega_epilogue(ga, EPI_RESID, u, r16, col, v0, v1); });
-    trace_mark(m, pass, TR_REDUCED << 8 | p.kind);
-    consumer_sync();
-    if (tid == 0) st_release(flag_base + u, epoch(m, pass, p.layer));
-    trace_mark(m, pass, TR_UNIT_DONE << 8 | p.kind);
   }
+  l = warp_sum(l);
+  if (col_ok)
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) xw_st(out + lane + 32 * i, o[i] / l, e_out);
   return ok;
 }
 
-// Attention of layer l: items (group, head, chunk) dealt round-robin; the
-// last CTA to finish a (group, head) combines its chunks and raises the flag.
+
+// This CTA's attention items of layer l, then the combines it owns.
 template <int DH, typename KVT>
-__device__ bool run_attention(const MegaArgs& m, const MegaSmem& sm, int layer, int pass, int n_groups, int tid) {
+__device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, unsigned& it, int tid) {
   const int G = gridDim.x, cta = blockIdx.x;
-  AttnArgs a = m.aa;
-  a.layer = layer;
-  const int tph = DH / 16;
-  const int tiles_sec = m.d / 16;
-  int total = 0;
-  for (int g = 0; g < n_groups; ++g) total += m.H * ((__ldcg(m.rows.g_kmax + g) + a.CH - 1) / a.CH);
+  const int CH = m.aa.CH, H = m.H, d = m.d;
+  const int* gk = sm.gmeta + 3 * (kMegaRows + 1);
+  const int ng = sm.n_groups;
+  const int total = att_total(m, gk, ng);
+  const int warp = tid >> 5, lane = tid & 31;
   bool ok = true;
-  KVT* ks = static_cast<KVT*>(sm.ks);
-  KVT* vs = static_cast<KVT*>(sm.vs);
+  const unsigned e_qkv = epoch(m, pass, l, ST_QKV), e_part = epoch(m, pass, l, ST_PART);
+  trace_mark(m, pass, TR_ATT << 8);
   for (int item = cta; item < total; item += G) {
-    int g = 0, rem = item, nch = 0;
-    for (; g < n_groups; ++g) {
-      nch = (__ldcg(m.rows.g_kmax + g) + a.CH - 1) / a.CH;
-      if (rem < m.H * nch) break;
-      rem -= m.H * nch;
+    int g, h, c;
+    att_decode(m, gk, ng, item, g, h, c);
+    const int row0 = sm.gmeta[1 * (kMegaRows + 1) + g], nr = sm.gmeta[2 * (kMegaRows + 1) + g];
+    const int kmax = gk[g], fresh = sm.gmeta[4 * (kMegaRows + 1) + g];
+    const int t0 = c * CH, nk = min(CH, kmax - t0);
+    const unsigned itu = it++;
+    const int slot = itu % kRingSlots;
+    KVT* ks = reinterpret_cast<KVT*>(sm.ring + (size_t)slot * kSlotBytes);
+    KVT* vs = ks + CH * DH;
+    // this pass's keys and values, and q, as exchange words; the cached pages are in the slot
+    if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
+    trace_mark(m, pass, TR_ISLOT << 8);
+    const int f0 = max(t0, fresh), f1 = t0 + nk;
+    const int nf = f1 > f0 ? (f1 - f0) * DH : 0;  // this pass's keys in the chunk, times DH
+    // one poll for this pass's keys and values in the chunk and the rows' queries
+    ok = poll_words<(2 * kMegaRows * 64 + kMegaRows * 64) / 256>(
+             m, 2 * nf + nr * DH, e_qkv, tid,
+             [&](int i) {
+               if (i < 2 * nf) {
+                 const int sel = i >= nf, rem = i - sel * nf;
+                 return (sel ? m.x_v : m.x_k) + (size_t)(row0 + (f0 + rem / DH - fresh)) * d + h * DH + rem % DH;
+               }
+               const int q = i - 2 * nf;
+               return m.x_q + (size_t)(row0 + q / DH) * d + h * DH + q % DH;
+             },
+             [&](int i, float v) {
+               if (i < 2 * nf) {
+                 const int sel = i >= nf, rem = i - sel * nf;
+                 KVT* dst = (sel ? vs : ks) + (size_t)(f0 + rem / DH - t0) * DH + rem % DH;
+                 if constexpr (sizeof(KVT) == 2) *dst = __float2bfloat16_rn(v);
+                 else *dst = v;
+               } else {
+                 sm.qs[i - 2 * nf] = v * m.aa.scale;
+               }
+             }) &&
+         ok;
+    trace_mark(m, pass, TR_IPOLL << 8);
+    if (tid < kMegaRows) sm.lim[tid] = (tid < nr) ? sm.rnkeys[row0 + tid] - t0 : 0;
+    if constexpr (sizeof(KVT) == 2) {  // zero V rows nk .. next multiple of 16 (read by the last key tile)
+      const int pad = ((nk + 15) & ~15) - nk;
+      for (int i = tid; i < pad * (DH / 8); i += 256)
+        *reinterpret_cast<uint4*>(vs + (size_t)(nk + i / (DH / 8)) * DH + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
     }
-    const int h = rem / nch, c = rem % nch;
-    const int seq = __ldcg(m.rows.g_seq + g), kmax = __ldcg(m.rows.g_kmax + g), fresh = __ldcg(m.rows.g_fresh + g);
-    const int t0 = c * a.CH, t1 = min(t0 + a.CH, kmax);
-    trace_mark(m, pass, TR_ATT_BEGIN << 8);
-    // keys cached before this pass can be fetched before q/k/v of this pass exist
-    attn_load_kv<DH, KVT>(a, seq, h, t0, t0, min(t1, fresh), ks, vs, tid, 256);
-    cp_async_commit();
-    if (tid < 32)
-      ok = warp_wait(m, 3 * tph, [&](int i) { return m.flags + m.f_qkv + (i / tph) * tiles_sec + h * tph + i % tph; },
-                     epoch(m, pass, layer)) && ok;
     consumer_sync();
-    trace_mark(m, pass, TR_ATT_QKV << 8);
-    attn_load_kv<DH, KVT>(a, seq, h, t0, max(t0, fresh), t1, ks, vs, tid, 256);
-    cp_async_commit();
-    cp_async_wait<0>();
+    u64* part = m.x_part + (((size_t)row0 * H + h) * m.CMAX + c) * (2 + DH);
+    const size_t rstride = (size_t)H * m.CMAX * (2 + DH);
+    attn_chunk_core<DH, KVT, DH>(
+        CH, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, nr, nk, tid, 256, consumer_sync,
+        [&](int r, int col, float v) { xw_st(part + r * rstride + 2 + col, v, e_part); },
+        [&](int r, float mm, float ll) {
+          xw_st(part + r * rstride, mm, e_part);
+          xw_st(part + r * rstride + 1, ll, e_part);
+        });
+    trace_mark(m, pass, TR_ICORE << 8);
+    fence_proxy_async_smem();  // the slot was written by these threads; the producer refills it by bulk copy
     consumer_sync();
-    trace_mark(m, pass, TR_ATT_LOADED << 8);
-    attn_partial_compute<DH, KVT, decltype(&consumer_sync)>(
-        a, g, h, c, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, tid, 256, consumer_sync,
-        [&](int step) { trace_mark(m, pass, TR_ATT_STEP << 8 | step); });
-    consumer_sync();
-    trace_mark(m, pass, TR_ATT_COMPUTED << 8);
-    if (tid == 0) {
-      __threadfence();
-      const unsigned old = atomicAdd(m.attn_cnt + g * m.H + h, 1u);
-      sm.misc[0] = (old == (unsigned)(nch - 1));
-      __threadfence();
-    }
-    consumer_sync();
-    if (sm.misc[0]) {
-      const int row0 = __ldcg(m.rows.g_row0 + g), nr = __ldcg(m.rows.g_nrows + g);
-      for (int r = tid >> 5; r < nr; r += 8) attn_combine_row<DH>(a, row0 + r, h, tid & 31);
-      consumer_sync();
-      if (tid == 0) {
-        m.attn_cnt[g * m.H + h] = 0u;
-        st_release(m.flags + m.f_att + g * m.H + h, epoch(m, pass, layer));
-      }
-    }
-    consumer_sync();
-    trace_mark(m, pass, TR_ATT_DONE << 8 | sm.misc[0]);
+    if (lane == 0) mbar_arrive(sm.empty + slot);
   }
+  trace_mark(m, pass, TR_ATT_DONE << 8);
+  // combines: (g, h) whose chunk 0 this CTA ran; one warp per row
+  const unsigned e_att = epoch(m, pass, l, ST_ATT);
+  for (int g = 0; g < ng; ++g) {
+    const int nch = (gk[g] + CH - 1) / CH;
+    const int row0 = sm.gmeta[1 * (kMegaRows + 1) + g], nr = sm.gmeta[2 * (kMegaRows + 1) + g];
+    for (int h = 0; h < H; ++h) {
+      if (att_item0(m, gk, g, h) % G != cta) continue;
+      for (int r = warp; r < nr; r += kMegaConsumers) {
+        const int row = row0 + r;
+        const int rnch = (sm.rnkeys[row] + CH - 1) / CH;
+        const u64* base = m.x_part + (((size_t)row * H + h) * m.CMAX) * (2 + DH);
+        ok = combine_row_xw<DH>(m, base, rnch, lane, e_part, m.x_att + (size_t)row * d + h * DH, e_att) && ok;
+      }
+      (void)nch;
+    }
+  }
+  trace_mark(m, pass, TR_COMB << 8);
   return ok;
 }
 
+// ---------------------------------------------------------------------------- bookkeeping (CTA 0)
 // After the head of pass `pass`: statistics, the mode's bookkeeping, the
-// decision to go on, the plan of the next pass (CTA 0 only).
-__device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass, int nr, int tid) {
+// decision to go on, the plan of the next pass.
+__device__ bool mega_bookkeeping(const MegaArgs& m, MegaSmem& sm, int pass, int nr, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
-  if (tid < 32) warp_wait(m, 16, [&](int u) { return m.flags + m.f_head + u; }, epoch(m, pass, m.L));
+  bool ok = true;
+  // every CTA's stores of this pass (the KV cache included) happen before the decision
+  if (tid == 0) ok = wait_flag(m, m.flags + 1, (unsigned)(gridDim.x * (pass + 1)), false);
+  const unsigned e = epoch(m, pass, m.L, ST_LOGIT);
+  ok = poll_words<kMegaRows>(m, nr * 256, e, tid, [&](int i) { return m.x_logit + i; }, [&](int i, float v) { m.logits[i] = v; }) && ok;
   if (tid == 0) sm.misc[1] = 0;
-  consumer_sync();
+  __threadfence_block();
+  ok = consumer_and(ok);
   for (int r = warp; r < nr; r += 8) {
-    float c, g, e;
+    float c, g, en;
     int p;
-    head_stats_row(m.logits + (size_t)r * 256, lane, c, p, g, e);
+    head_stats_row(m.logits + (size_t)r * 256, lane, c, p, g, en);
     if (lane == 0) {
       m.conf[r] = c;
       m.pred[r] = p;
       m.gap[r] = g;
-      m.ent[r] = e;
+      m.ent[r] = en;
     }
   }
   __threadfence_block();
@@ -812,7 +1159,7 @@ __device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass
   }
   __threadfence_block();
   consumer_sync();
-  if (cont) {
+  if (cont && ok) {
     PlanArgs p = m.plan;
     if (m.mode == MM_DIFFUSE) {
       p.mode = PL_BLOCK;
@@ -824,46 +1171,41 @@ __device__ void mega_bookkeeping(const MegaArgs& m, const MegaSmem& sm, int pass
   }
   consumer_sync();
   if (tid == 0) {
-    *(volatile unsigned*)m.dec_val = cont ? 1u : 0u;
+    *(volatile unsigned*)m.dec_val = (cont && ok) ? 1u : 0u;
     __threadfence();
-    st_release(m.flags + m.f_dec, epoch(m, pass, m.L));
+    st_release(m.flags + 0, e);
   }
+  return ok;
 }
 
+// ---------------------------------------------------------------------------- the kernel
 template <int NG, int PL, int DH, typename KVT>
 __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   extern __shared__ __align__(1024) unsigned char mega_smem[];
-  __shared__ uint64_t bars[2 * 16];
+  __shared__ uint64_t bars[2 * kRingSlots];
   __shared__ int plan_sh[3 * (kMaxCallBatch + 1)];
   __shared__ int misc[4];
-  __shared__ float mrow[kAttnRows], lrow[kAttnRows];
-  __shared__ int lim[kAttnRows];
-  __shared__ int rmeta[4][8 * kMegaMaxNG];
-  __shared__ int rpage[8 * kMegaMaxNG];                       // KV page of each row's position
-  __shared__ float rope_c[8 * kMegaMaxNG * 32], rope_s[8 * kMegaMaxNG * 32];  // [row][dh/2], dh <= 64
+  __shared__ float mrow[kMegaRows], lrow[kMegaRows];
+  __shared__ int lim[kMegaRows];
+  __shared__ int rmeta[5][kMegaRows];
+  __shared__ int gmeta[5 * (kMegaRows + 1)];
 
-  const unsigned tile_bytes = 512u * PL;
-  const unsigned slot_bytes = kStageTiles * tile_bytes;
   MegaSmem sm;
-  sm.S = min(16, (int)(kRingBytes / slot_bytes));
   sm.ring = mega_smem;
-  unsigned char* p = mega_smem + kRingBytes;
+  unsigned char* p = mega_smem + (size_t)kRingSlots * kSlotBytes;
   sm.red = reinterpret_cast<float*>(p);
-  p += 8 * 16 * 8 * kMegaMaxNG * 4;
+  sm.qs = sm.red;  // attention scratch aliases the reduction buffer
+  sm.ps = sm.qs + kMegaRows * DH;
+  p += (size_t)kMaxPieces * 8 * 16 * 8 * NG * 4 > (size_t)(kMegaRows * DH + kMegaRows * 128) * 4
+           ? (size_t)kMaxPieces * 8 * 16 * 8 * NG * 4
+           : (size_t)(kMegaRows * DH + kMegaRows * 128) * 4;
   sm.ssr = reinterpret_cast<float*>(p);
   p += 8 * 8 * kMegaMaxNG * 4;
-  sm.rsv = reinterpret_cast<float*>(p);
-  p += 16 * 4;
-  sm.xs = reinterpret_cast<uint4*>(p);  // the phases' reduction buffer shares space with the attention buffers
-  sm.qs = reinterpret_cast<float*>(p);
-  p += kAttnRows * DH * 4;
-  sm.ps = reinterpret_cast<float*>(p);
-  p += kAttnRows * m.aa.CH * 4;
-  sm.ks = p;
-  p += m.aa.CH * kv_stride<DH, KVT>() * sizeof(KVT);
-  sm.vs = p;
+  sm.hpre = reinterpret_cast<float*>(p);
+  p += kMaxPieces * kMegaRows * 16 * 4;
+  sm.cpre = reinterpret_cast<float*>(p);
   sm.full = bars;
-  sm.empty = bars + 16;
+  sm.empty = bars + kRingSlots;
   sm.mrow = mrow;
   sm.lrow = lrow;
   sm.lim = lim;
@@ -873,11 +1215,13 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.rpos = rmeta[1];
   sm.rlat = rmeta[2];
   sm.rbyte = rmeta[3];
+  sm.rnkeys = rmeta[4];
+  sm.gmeta = gmeta;
 
   const int tid = threadIdx.x;
   if (tid == 0) {
     s_trace_n = 0;
-    for (int i = 0; i < sm.S; ++i) {
+    for (int i = 0; i < kRingSlots; ++i) {
       mbar_init(sm.full + i, 1);
       mbar_init(sm.empty + i, kMegaConsumers);
     }
@@ -886,14 +1230,15 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   __syncthreads();
 
   if (tid >= 256) {  // producer warp
-    mega_producer(m, sm.ring, sm.full, sm.empty, sm.S, tid & 31);
+    mega_producer<PL, DH, KVT>(m, sm, tid & 31);
     return;
   }
+  const int G = gridDim.x;
   unsigned it = 0;
   bool ok = true;
   for (int pass = 0; pass < m.max_passes && ok; ++pass) {
     if (pass > 0) {
-      if (tid == 0) misc[2] = wait_flag(m, m.flags + m.f_dec, epoch(m, pass - 1, m.L)) ? (int)__ldcg(m.dec_val) : -1;
+      if (tid == 0) misc[2] = wait_flag(m, m.flags + 0, epoch(m, pass - 1, m.L, ST_LOGIT), true) ? (int)__ldcg(m.dec_val) : -1;
       consumer_sync();
       const int go = misc[2];
       consumer_sync();
@@ -902,70 +1247,52 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
         break;
       }
     }
-    const int nr = __ldcg(m.rows.n_rows);
-    const int n_groups = __ldcg(m.rows.n_groups);
-    if (tid < 8 * kMegaMaxNG) {  // rows past nr get harmless in-range values (inputs are loaded unconditionally)
-      const bool live = tid < nr;
+    // this pass's rows (live rows only; the rest never reach an output)
+    sm.n_rows = min(__ldcg(m.rows.n_rows), kMegaRows);
+    sm.n_groups = min(__ldcg(m.rows.n_groups), kMegaRows);
+    if (tid < kMegaRows) {
+      const bool live = tid < sm.n_rows;
       sm.rseq[tid] = live ? __ldcg(m.rows.seq + tid) : 0;
       sm.rpos[tid] = live ? __ldcg(m.rows.pos + tid) : 0;
       sm.rlat[tid] = live ? __ldcg(m.rows.lat + tid) : 0;
       sm.rbyte[tid] = live ? __ldcg(m.rows.byte + tid) : 0;
+      sm.rnkeys[tid] = live ? __ldcg(m.rows.nkeys + tid) : 0;
     }
-    consumer_sync();
-    {  // this pass's rotary factors and KV pages per row (dead rows: position 0)
-      const int half = m.dh / 2;
-      for (int i = tid; i < 8 * kMegaMaxNG * half; i += 256) {
-        const size_t src = (size_t)sm.rpos[i / half] * half + i % half;
-        rope_c[i] = __ldg(m.ga.rope_cos + src);
-        rope_s[i] = __ldg(m.ga.rope_sin + src);
-      }
-      if (tid < 8 * kMegaMaxNG) {
-        const int pi = sm.rpos[tid] / m.ga.PT;
-        rpage[tid] = (pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + sm.rseq[tid] * m.ga.max_pages + pi) : -1;
-      }
+    if (tid < sm.n_groups) {
+      gmeta[0 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_seq + tid);
+      gmeta[1 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_row0 + tid);
+      gmeta[2 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_nrows + tid);
+      gmeta[3 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_kmax + tid);
+      gmeta[4 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_fresh + tid);
     }
     consumer_sync();
     trace_mark(m, pass, TR_PASS << 8);
-    // Steps of a pass: per layer QKV, attention, O, W13, W2; then the byte
-    // head.  One call site per routine keeps a single copy of each in the
-    // kernel, small enough for the SM's instruction caches.
-    GemmArgs ga = m.ga;
-    ga.row_seq = sm.rseq;
-    ga.row_pos = sm.rpos;
-    ga.row_lat = sm.rlat;
-    ga.row_byte = sm.rbyte;
-    ga.rope_cos = rope_c;
-    ga.rope_sin = rope_s;
-    ga.rope_by_row = 1;
-    ga.row_page = rpage;
-    for (int step = 0; step <= 5 * m.L && ok; ++step) {
-      const int l = step / 5, k = step - 5 * l;
-      if (k == 1) {
-        ok = run_attention<DH, KVT>(m, sm, l, pass, n_groups, tid) && ok;
-        continue;
-      }
-      const bool head = l == m.L;
-      const Phase p = phase_of(m, head ? 4 * m.L : 4 * l + (k == 0 ? 0 : k - 1));
-      ga.layer = head ? 0 : l;
-      int epi = EPI_STORE;
-      unsigned* fb = m.flags + m.f_head;
-      if (head) {
-        ga.out = m.logits, ga.ldo = 256;
-      } else if (k == 0) {
-        epi = EPI_QKV, fb = m.flags + m.f_qkv;
-      } else if (k == 2) {
-        epi = EPI_XRESID, fb = m.flags + m.f_o, ga.out = m.h, ga.ldo = m.d;
-      } else if (k == 3) {
-        epi = EPI_SWIGLU, fb = m.flags + m.f_w13, ga.out = m.act, ga.ldo = m.F;
-      } else {
-        epi = EPI_RESID, fb = m.flags + m.f_w2, ga.out = m.h, ga.ldo = m.d;
-      }
-      if (k == 4 && !head && p.ksteps > 64) ok = run_phase_streamed<NG, PL>(m, sm, p, pass, it, nr, n_groups, ga, fb, tid) && ok;
-      else ok = run_phase_units<NG, PL>(m, sm, p, epi, pass, it, nr, n_groups, ga, fb, tid) && ok;
+    const int nr = sm.n_rows;
+    for (int l = 0; l < m.L && ok; ++l) {
+      XSrc xs;
+      xs.x = (l == 0) ? nullptr : m.x_h;
+      xs.ld = m.d, xs.col0 = 0, xs.e = (l == 0) ? 0u : epoch(m, pass, l - 1, ST_HW);
+      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_QKV, l, blockIdx.x, G), xs, m.layers[l].attn_norm, pass, it, tid) && ok);
+      ok = consumer_and(run_attention<DH, KVT>(m, sm, l, pass, it, tid) && ok);
+      xs.x = m.x_att, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, l, ST_ATT);
+      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_O, l, blockIdx.x, G), xs, nullptr, pass, it, tid) && ok);
+      xs.x = m.x_h, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, l, ST_HO);
+      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_W13, l, blockIdx.x, G), xs, m.layers[l].ffn_norm, pass, it, tid) && ok);
+      const Phase pw2 = phase_of(m, PH_W2, l, blockIdx.x, G);
+      xs.x = m.x_act, xs.ld = m.F, xs.col0 = pw2.seg * kSegCols, xs.e = epoch(m, pass, l, ST_ACT);
+      ok = consumer_and(run_gemv<NG, PL>(m, sm, pw2, xs, nullptr, pass, it, tid) && ok);
     }
     if (!ok) break;
-    trace_mark(m, pass, TR_HEAD << 8);
-    if (blockIdx.x == 0 && ok) mega_bookkeeping(m, sm, pass, nr, tid);
+    XSrc xs;
+    xs.x = m.x_h, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, m.L - 1, ST_HW);
+    ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_HEAD, 0, blockIdx.x, G), xs, m.final_norm, pass, it, tid) && ok);
+    // this CTA's stores of the pass (KV cache included) are done: arrive
+    if (tid == 0) {
+      __threadfence();
+      red_release_add(m.flags + 1, 1u);
+    }
+    if (!ok) break;
+    if (blockIdx.x == 0) ok = consumer_and(mega_bookkeeping(m, sm, pass, nr, tid) && ok);
     trace_mark(m, pass, TR_BOOK << 8);
   }
 }

@@ -61,13 +61,13 @@ class Engine:
 
     def __init__(self, shape: ModelShape, weights: WeightSet, max_batch: int, max_ctx: int, max_block: int,
                  max_rows: int = 1024, max_latents: Optional[int] = None, page_tokens: int = 64, attn_chunk: int = 0,
-                 device: str = "cuda", time_passes: bool = False, persistent: bool = False):
+                 device: str = "cuda", time_passes: bool = False, persistent: bool = False, extra_flags: int = 0):
         self.shape = shape
         self.max_batch, self.max_ctx, self.max_block, self.max_rows = max_batch, max_ctx, max_block, max_rows
         self.max_latents = max_latents or (max_ctx // 2 + 64)
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
-        flags = (B.BLT_FLAG_TIME_PASSES if time_passes else 0) | (B.BLT_FLAG_PERSISTENT if persistent else 0)
+        flags = (B.BLT_FLAG_TIME_PASSES if time_passes else 0) | (B.BLT_FLAG_PERSISTENT if persistent else 0) | extra_flags
         cfg = engine_config(shape, max_batch, max_ctx, self.max_latents, max_rows, max_block, page_tokens, 0, attn_chunk, flags)
         layers = []
         for l in range(shape.n_layers):
@@ -254,6 +254,8 @@ def generate(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: Op
             for i, s in enumerate(seqs):
                 s.commit([int(d[i, 0])])
                 s.out.append(int(d[i, 0]))
+            if record:
+                rounds.append(dict(next=d[:, 0].copy()))
         elif wl.mode in ("S", "DV"):
             mode = B.BLT_DRAFT_AR if wl.mode == "S" else B.BLT_DRAFT_DIFFUSION
             B.blt_dec_draft(h, nb, r, mode, k, wl.alpha, 0, eng.d_out)

@@ -98,6 +98,10 @@ typedef struct {
 
 #define BLT_FLAG_TIME_PASSES 1 /* bracket the decoder passes of every call with CUDA events (counters.pass_ns) */
 #define BLT_FLAG_PERSISTENT 2  /* run small passes (<= 16 rows) in the persistent pass kernel (one launch per call) */
+#define BLT_FLAG_TEST_STALL 4  /* test only: in the persistent kernel, one output of the first pass's first O
+                                  projection is never published and the waits give up after about a
+                                  millisecond: the call's passes stop and blt_dec_sync reports
+                                  BLT_ERR_DEVICE (exercises the bounded waits; never set in production) */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */
@@ -126,11 +130,12 @@ typedef struct {
   uint64_t latents;        /* latents projected (global-model outputs consumed) */
   uint64_t calls;          /* C-ABI calls that ran decoder work */
   uint64_t weight_bytes;   /* weight bytes streamed by decoder passes (algorithmic) */
-  uint64_t kv_read_bytes;  /* K/V bytes read by self-attention (algorithmic) */
+  uint64_t kv_read_bytes;  /* K/V bytes read by the self-attention of decoder passes (algorithmic; prefill excluded) */
   uint64_t kernel_launches; /* engine kernels launched (host count) */
   uint64_t timed_passes;   /* decoder passes inside timed calls (BLT_FLAG_TIME_PASSES) */
   uint64_t pass_ns;        /* summed device time of those calls' passes, ns (latent projection excluded) */
   uint64_t persistent_calls; /* calls whose decoder passes ran in the persistent kernel (BLT_FLAG_PERSISTENT) */
+  uint64_t prefill_kv_read_bytes; /* K/V bytes read by the self-attention of prefill chunks (algorithmic) */
 } blt_dec_counters;
 
 /* Create an engine.  Copies and re-lays out the weights on the device
@@ -163,8 +168,11 @@ int blt_dec_prefill(blt_dec_t *h, int batch, const blt_rows_in *rows, float *out
  * 32-row chunks.
  *
  * Limits (else INVALID_ARG): d_model <= 1024, d_ffn <= 4096, n_heads <= 16,
- * head dim <= 64, attn_chunk 128 (the default), and each sequence's cached
- * length plus its rows <= 4096 positions.  The arena is about 5.2 MB and every
+ * head dim <= 64, n_layers * d_model <= 32768 (the latent-projection
+ * temporary), attn_chunk 128 (the default), and each sequence's cached
+ * length plus its rows <= 4096 positions.  The logits and the KV cache it
+ * writes are bit-identical to blt_dec_prefill's (a row's arithmetic does not
+ * depend on which rows share its pass).  The arena is about 5.2 MB and every
  * GPU that loads the library holds it until the process exits.
  * The first call on a device resolves the arena's device address
  * (cudaGetSymbolAddress) with that device current; make that first call

@@ -21,3 +21,15 @@ def tiny():
     wl = CONFIGS["tiny_d4"]
     ws = WeightSet(wl.shape, seed=0, gain_std=0.1).materialize()
     return wl, ws, OracleModel(wl.shape, ws)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """List every parity comparison with its flagged positions and divergences."""
+    try:
+        from _parity import REPORT
+    except ImportError:
+        return
+    if REPORT:
+        terminalreporter.section("engine vs oracle parity (flagged near-tie positions listed)")
+        for line in REPORT:
+            terminalreporter.write_line(line)

@@ -45,13 +45,31 @@ def test_binding_covers_every_export(lib):
     binding.load_library()
 
 
-def test_struct_layouts_match_header():
+def test_struct_layouts_match_header(tmp_path):
+    """The binding's ctypes structs have the sizes and field offsets a C compiler gives the
+    header's structs (checked by compiling the header with gcc)."""
+    import subprocess
+
     from block_diffusion_byte_b200 import binding as B
 
-    assert ctypes.sizeof(B.blt_dec_config) == 18 * 4
-    assert ctypes.sizeof(B.blt_dec_weights) == 4 * 8
-    assert ctypes.sizeof(B.blt_rows_in) == 5 * 8
-    assert ctypes.sizeof(B.blt_dec_counters) == 11 * 8
+    structs = {"blt_dec_config": B.blt_dec_config, "blt_dec_weights": B.blt_dec_weights, "blt_rows_in": B.blt_rows_in,
+               "blt_dec_counters": B.blt_dec_counters}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "bltdec.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} %zu\\n", sizeof({name}));')
+        for f, _ in cls._fields_:
+            lines.append(f'  printf("{name}.{f} %zu\\n", offsetof({name}, {f}));')
+    lines.append("  return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-I", inc, "-o", str(exe), str(src)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines())
+    for name, cls in structs.items():
+        assert int(got[name]) == ctypes.sizeof(cls), name
+        for f, _ in cls._fields_:
+            assert int(got[f"{name}.{f}"]) == getattr(cls, f).offset, (name, f)
 
 
 def test_init_rejects_bad_config_without_touching_the_gpu(lib):

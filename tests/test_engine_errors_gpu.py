@@ -99,3 +99,34 @@ def test_context_capacity_is_no_space(eng):
     with pytest.raises(B.BltError) as ei:
         B.blt_dec_diffuse_block(e.h, 1, r, 4, 0.7, 0, e.d_out)
     assert ei.value.code == B.BLT_ERR_NO_SPACE
+
+
+def test_persistent_kernel_wait_runs_out():
+    """A bounded wait of the persistent pass kernel that runs out ends the call with
+    BLT_ERR_DEVICE instead of hanging: under the test-only flag one output of the first
+    O projection is never published, so every consumer of it waits about a millisecond and
+    gives up, and all CTAs leave.  A fresh handle then decodes normally."""
+    import time
+
+    from block_diffusion_byte_b200 import binding as B
+    from block_diffusion_byte_b200.driver import Engine, generate
+
+    wl = CONFIGS["tiny_d4"]
+    ws = WeightSet(wl.shape).materialize()
+    prefix = [int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, 0, wl.prefix_len)]
+    e = Engine(wl.shape, ws, max_batch=1, max_ctx=160, max_block=8, max_rows=64, persistent=True, extra_flags=B.BLT_FLAG_TEST_STALL)
+    try:
+        t0 = time.perf_counter()
+        with pytest.raises(B.BltError) as ei:
+            generate(e, wl, [prefix], 4)
+        assert ei.value.code == B.BLT_ERR_DEVICE
+        assert time.perf_counter() - t0 < 30.0
+        assert B.blt_dec_stats(e.h)["persistent_calls"] >= 1
+    finally:
+        e.close()
+    f = Engine(wl.shape, ws, max_batch=1, max_ctx=160, max_block=8, max_rows=64, persistent=True)
+    try:
+        res = generate(f, wl, [prefix], 8)
+        assert B.blt_dec_sync(f.h) == 0 and len(res.out[0]) == 8
+    finally:
+        f.close()
