@@ -41,7 +41,14 @@ namespace bltdec {
 typedef unsigned long long u64;
 
 constexpr int kMegaConsumers = 8;
-constexpr int kMegaThreads = (kMegaConsumers + 1) * 32;
+// Three warpgroups: two of consumers, and one holding the producer warp (its three other
+// warps leave at once).  Launched at 168 registers a thread (65536 / 384), the producer's
+// warpgroup gives registers back and the consumers take them (setmaxnreg):
+// 128 * 56 + 256 * 224 = 384 * 168.
+constexpr int kMegaThreads = 12 * 32;
+constexpr int kProducerRegs = 56;
+constexpr int kConsumerRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kMegaThreads * 168, "register split exceeds the launch's registers");
 constexpr int kSlotBytes = 32 * 1024;
 constexpr int kRingSlots = 5;
 constexpr int kMegaMaxNG = 2;                  // <= 16 rows per pass
@@ -420,6 +427,9 @@ struct MegaSmem {
   int* rlat;
   int* rbyte;
   int* rnkeys;
+  int* rpage;    // KV page of each row's position (-1: none)
+  float* rope_c; // [rows][dh/2] rotary factors of each row's position
+  float* rope_s;
   int* gmeta;  // [5][kMegaRows + 1]: g_seq, g_row0, g_nrows, g_kmax, g_fresh
   int n_rows, n_groups;
 };
@@ -540,75 +550,82 @@ struct XSrc {
 
 // Wait for and load this warp's k-steps (warp, warp + 8, ...; nkw of them) of
 // every live row as B fragments, plus the lanes' sums of squares (canonical
-// order).  Rows >= nr get zeros.
+// order).  Rows >= nr get zeros.  A lane loads all its words in one round
+// (a dead row reads row 0 and a k-step past nkw re-reads the last one: both
+// are always written, never used) and reloads the round only if a word is not
+// ready yet -- rare once the sentinels have passed.
 template <int NG>
 __device__ __forceinline__ bool gather_frags(const MegaArgs& m, const MegaSmem& sm, const XSrc& xs, int nr, int nkw, const float* gain,
                                              uint4 (&xf)[8][NG], float (&ss)[NG], int warp, int lane, int pass) {
   const int g = lane >> 2, t = lane & 3;
   float2 xa[8][NG], xb[8][NG];
-  unsigned pending = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int n = 0; n < NG; ++n) {
-      xa[j][n] = xb[j][n] = make_float2(0.f, 0.f);
-      if (j < nkw && n * 8 + g < nr) pending |= 3u << ((j * NG + n) * 2);
-    }
+  bool ok = true;
   if (!xs.x) {  // layer 0: embedding + cross term, finished data
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int n = 0; n < NG; ++n) {
+      const int row = n * 8 + g;
+      const bool live = row < nr;
+      const int rr = live ? row : 0;
+      const float* e = m.ga.embed + (size_t)sm.rbyte[rr] * m.d;
+      const float* c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, 0, m.d, sm.rseq[rr], sm.rlat[rr]);
 #pragma unroll
-      for (int n = 0; n < NG; ++n)
-        if ((pending >> ((j * NG + n) * 2)) & 1u) {
-          const int row = n * 8 + g, k0 = (warp + 8 * j) * 16 + 2 * t;
-          const float* e = m.ga.embed + (size_t)sm.rbyte[row] * m.d;
-          const float* c = c_row(m.ga.c_lat, m.ga.max_lat, m.L, 0, m.d, sm.rseq[row], sm.rlat[row]);
-          xa[j][n] = make_float2(__ldg(e + k0) + __ldcg(c + k0), __ldg(e + k0 + 1) + __ldcg(c + k0 + 1));
-          xb[j][n] = make_float2(__ldg(e + k0 + 8) + __ldcg(c + k0 + 8), __ldg(e + k0 + 9) + __ldcg(c + k0 + 9));
-        }
-    pending = 0;
-  }
-  Spin spins;
-  bool ok = true;
-  if (__any_sync(0xffffffffu, pending != 0u)) {  // warp-uniform: the loop below has a full-mask vote
-    // Sentinels: lane j < nkw polls one word of k-step warp + 8 j (row 0, its last column) until
-    // every k-step of the warp has data; only then do all lanes load everything.  While waiting,
-    // a warp issues at most 8 loads per round.
-    const u64* sp = xs.x + xs.col0 + (warp + 8 * lane) * 16 + 15;
-    bool ready = lane >= nkw;
-    while (true) {
-      if (!ready) ready = xw_ok(xw_ld(sp), xs.e);
-      if (__all_sync(0xffffffffu, ready)) break;
-      if (!spin_step(m, spins)) {
-        ok = false;
-        break;
+      for (int j = 0; j < 8; ++j) {
+        const int k0 = (warp + 8 * min(j, nkw - 1)) * 16 + 2 * t;
+        const float2 a = make_float2(__ldg(e + k0) + __ldcg(c + k0), __ldg(e + k0 + 1) + __ldcg(c + k0 + 1));
+        const float2 b = make_float2(__ldg(e + k0 + 8) + __ldcg(c + k0 + 8), __ldg(e + k0 + 9) + __ldcg(c + k0 + 9));
+        xa[j][n] = (live && j < nkw) ? a : make_float2(0.f, 0.f);
+        xb[j][n] = (live && j < nkw) ? b : make_float2(0.f, 0.f);
       }
     }
-  }
-  trace_mark(m, pass, TR_SENT << 8);
-  while (pending && ok) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int n = 0; n < NG; ++n)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const unsigned bit = 1u << ((j * NG + n) * 2 + hf);
-          if (pending & bit) {
-            const int row = n * 8 + g, k0 = (warp + 8 * j) * 16 + 2 * t + 8 * hf;
-            u64 a, b;
-            xw_ld2(xs.x + (size_t)row * xs.ld + xs.col0 + k0, a, b);
-            if (xw_ok(a, xs.e) && xw_ok(b, xs.e)) {
-              const float2 v = make_float2(xw_val(a), xw_val(b));
-              if (hf == 0) xa[j][n] = v;
-              else xb[j][n] = v;
-              pending &= ~bit;
-            }
-          }
+  } else {
+    Spin spins;
+    {
+      // Sentinels: lane j < nkw polls one word of k-step warp + 8 j (row 0, its last column) until
+      // every k-step of the warp has data; only then do all lanes load everything.  While waiting,
+      // a warp issues at most 8 loads per round.
+      const u64* sp = xs.x + xs.col0 + (warp + 8 * min(lane, 7)) * 16 + 15;
+      bool ready = lane >= nkw;
+      while (true) {
+        if (!ready) ready = xw_ok(xw_ld(sp), xs.e);
+        if (__all_sync(0xffffffffu, ready)) break;
+        if (!spin_step(m, spins)) {
+          ok = false;
+          break;
         }
-    if (pending && !spin_step(m, spins)) {
-      ok = false;
-      break;
+      }
+    }
+    trace_mark(m, pass, TR_SENT << 8);
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      const int row = n * 8 + g;
+      const bool live = row < nr;
+      const u64* base = xs.x + (size_t)(live ? row : 0) * xs.ld + xs.col0 + 2 * t;
+      while (ok) {
+        u64 wa[8][2], wb[8][2];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) xw_ld2(base + (warp + 8 * min(j, nkw - 1)) * 16 + 8 * hf, wa[j][hf], wb[j][hf]);
+        bool all = true;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) all = all && xw_ok(wa[j][hf], xs.e) && xw_ok(wb[j][hf], xs.e);
+        if (all) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const bool use = live && j < nkw;
+            xa[j][n] = use ? make_float2(xw_val(wa[j][0]), xw_val(wb[j][0])) : make_float2(0.f, 0.f);
+            xb[j][n] = use ? make_float2(xw_val(wa[j][1]), xw_val(wb[j][1])) : make_float2(0.f, 0.f);
+          }
+          break;
+        }
+        if (!spin_step(m, spins)) ok = false;
+      }
+      if (!ok) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xa[j][n] = xb[j][n] = make_float2(0.f, 0.f);
+      }
     }
   }
   trace_mark(m, pass, TR_GATH << 8);
@@ -677,13 +694,12 @@ __device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem&
       const GemmArgs& a = m.ga;
       const int tiles_sec = d / 16;
       const int sec = u / tiles_sec, lt = u % tiles_sec;
-      const int pos = sm.rpos[row], seq = sm.rseq[row];
+      const int pos = sm.rpos[row];
       if (sec < 2) {  // q and k tiles hold rotary pairs (j, j + dh/2) in rows (r16, r16 + 8)
         const int tph = m.dh / 16;
         const int h = lt / tph, j = (lt % tph) * 8 + r16;
         const int half = m.dh / 2;
-        const size_t ri = (size_t)pos * half + j;
-        const float c = __ldg(a.rope_cos + ri), s = __ldg(a.rope_sin + ri);
+        const float c = sm.rope_c[row * 32 + j], s = sm.rope_s[row * 32 + j];
         const float o0 = v0 * c - v1 * s, o1 = v1 * c + v0 * s;
         const size_t xo = (size_t)row * d + h * m.dh + j;
         if (sec == 0) {
@@ -691,8 +707,7 @@ __device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem&
           xw_st(m.x_q + xo + half, o1, e);
           return true;
         }
-        const int pi = pos / a.PT;
-        const int page = (pi < a.max_pages) ? __ldcg(a.page_table + seq * a.max_pages + pi) : -1;
+        const int page = sm.rpage[row];
         float r0 = o0, r1 = o1;
         if (page < 0) {
           set_status(a.status, kErrDevice);
@@ -709,8 +724,7 @@ __device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem&
         xw_st(m.x_k + xo + half, r1, e);
       } else {
         const int n0 = lt * 16 + r16, n1 = n0 + 8;
-        const int pi = pos / a.PT;
-        const int page = (pi < a.max_pages) ? __ldcg(a.page_table + seq * a.max_pages + pi) : -1;
+        const int page = sm.rpage[row];
         if (page < 0) {
           set_status(a.status, kErrDevice);
         } else {
@@ -1187,8 +1201,9 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   __shared__ int misc[4];
   __shared__ float mrow[kMegaRows], lrow[kMegaRows];
   __shared__ int lim[kMegaRows];
-  __shared__ int rmeta[5][kMegaRows];
+  __shared__ int rmeta[6][kMegaRows];
   __shared__ int gmeta[5 * (kMegaRows + 1)];
+  __shared__ float rope_tab[2][kMegaRows * 32];  // dh <= 64
 
   MegaSmem sm;
   sm.ring = mega_smem;
@@ -1216,6 +1231,9 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.rlat = rmeta[2];
   sm.rbyte = rmeta[3];
   sm.rnkeys = rmeta[4];
+  sm.rpage = rmeta[5];
+  sm.rope_c = rope_tab[0];
+  sm.rope_s = rope_tab[1];
   sm.gmeta = gmeta;
 
   const int tid = threadIdx.x;
@@ -1229,10 +1247,12 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   }
   __syncthreads();
 
-  if (tid >= 256) {  // producer warp
-    mega_producer<PL, DH, KVT>(m, sm, tid & 31);
+  if (tid >= 256) {  // the producer's warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kProducerRegs));
+    if (tid < 288) mega_producer<PL, DH, KVT>(m, sm, tid & 31);
     return;
   }
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kConsumerRegs));
   const int G = gridDim.x;
   unsigned it = 0;
   bool ok = true;
@@ -1257,6 +1277,17 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
       sm.rlat[tid] = live ? __ldcg(m.rows.lat + tid) : 0;
       sm.rbyte[tid] = live ? __ldcg(m.rows.byte + tid) : 0;
       sm.rnkeys[tid] = live ? __ldcg(m.rows.nkeys + tid) : 0;
+    }
+    consumer_sync();
+    if (tid < kMegaRows) {  // the KV page of each row's position (dead rows: position 0)
+      const int pi = sm.rpos[tid] / m.ga.PT;
+      sm.rpage[tid] = (pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + sm.rseq[tid] * m.ga.max_pages + pi) : -1;
+    }
+    for (int i = tid; i < kMegaRows * (m.dh / 2); i += 256) {  // rotary factors of each row's position
+      const int r = i / (m.dh / 2), j = i % (m.dh / 2);
+      const size_t src = (size_t)sm.rpos[r] * (m.dh / 2) + j;
+      sm.rope_c[r * 32 + j] = __ldg(m.ga.rope_cos + src);
+      sm.rope_s[r * 32 + j] = __ldg(m.ga.rope_sin + src);
     }
     if (tid < sm.n_groups) {
       gmeta[0 * (kMegaRows + 1) + tid] = __ldcg(m.rows.g_seq + tid);
