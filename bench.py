@@ -420,10 +420,11 @@ def main():
         if dist:
             dist.barrier()
 
-    def engine_for(w, ws_):
-        max_ctx = w.prefix_len + w.gen_bytes + 4 * max(w.block, 16) + 16
+    def engine_for(w, ws_, tensor_cores=True):
+        # a batch decodes until its slowest sequence has gen_bytes: room for the faster sequences' extra rounds
+        max_ctx = w.prefix_len + (2 * w.gen_bytes if w.batch > 1 else w.gen_bytes) + 4 * max(w.block, 16) + 16
         return Engine(w.shape, ws_, max_batch=w.batch, max_ctx=max_ctx, max_block=max(w.block, 16), max_rows=1024,
-                      time_passes=True, persistent=persistent)
+                      time_passes=True, persistent=persistent, tensor_cores=tensor_cores)
 
     ws = WeightSet(wl.shape, seed=wl.seed).materialize()
     nb = wl.batch
@@ -513,15 +514,20 @@ def main():
     if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
         # decoded bytes/s at batch 16: BLT-S k=8, prefix 4096, 512 bytes per sequence
         w16 = CONFIGS["s8_b16"]
-        e16 = engine_for(w16, ws)
-        try:
-            ids16 = list(range(w16.batch))
-            pre16 = [[int(b) for b in prefix_bytes(w16.seed, w16.cfg_index, s, w16.prefix_len)] for s in ids16]
-            ms16, d16, h16, o16, _ = time_job(e16, w16, pre16, ids16, 2, 1, barrier, generate, B)
-        finally:
-            e16.close()
+        ids16 = list(range(w16.batch))
+        pre16 = [[int(b) for b in prefix_bytes(w16.seed, w16.cfg_index, s, w16.prefix_len)] for s in ids16]
+        runs16 = {}
+        for tc in (True, False):  # verification passes (128 rows) on the tcgen05 GEMM, then on the GEMV kernels
+            e16 = engine_for(w16, ws, tensor_cores=tc)
+            try:
+                runs16[tc] = time_job(e16, w16, pre16, ids16, 2, 1, barrier, generate, B)
+            finally:
+                e16.close()
+        ms16, d16, h16, o16, _ = runs16[True]
         roof16, dec16 = pass_figures(d16, 2, ms16, peak, pk_kind)
         dec16["path"] = args.path
+        dec16["tc_gemms_per_step"] = d16["tc_gemms"] / 2
+        ms16g = runs16[False][0]
         line["batch16"] = {
             "config": workload_config(w16),
             "value": w16.gen_bytes * w16.batch * 2 / (ms16 / 1000.0),
@@ -531,8 +537,11 @@ def main():
             "ms_per_step": ms16 / 2,
             "roofline": roof16,
             "decoder": dec16,
-            "note": "drafting passes (16 rows) run in the persistent kernel, verification passes (128 rows) in the per-phase "
-            "kernels; roofline over all decoder passes of the job",
+            "gemv_value": w16.gen_bytes * w16.batch * 2 / (ms16g / 1000.0),
+            "gemv_ms_per_step": ms16g / 2,
+            "tcgen05_speedup": ms16g / ms16,
+            "note": "drafting passes (16 rows) run in the persistent kernel; verification passes (128 rows) project on the "
+            "tcgen05 GEMM (value) or on the mma.sync GEMV kernels (gemv_value); roofline over all decoder passes of the job",
         }
     if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
         # the N_enc term of the pages' proxy, timed: one global-model step at the 1B size

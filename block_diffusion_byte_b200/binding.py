@@ -29,6 +29,7 @@ BLT_DRAFT_DIFFUSION = 1
 BLT_FLAG_TIME_PASSES = 1
 BLT_FLAG_PERSISTENT = 2
 BLT_FLAG_TEST_STALL = 4  # test only: the persistent kernel's bounded waits must run out
+BLT_FLAG_TENSOR_CORES = 8  # decode passes of >= 128 rows: projections on the tcgen05 GEMM
 BLT_LAYER_NT = 12
 LAYER_ORDER = ("wq_c", "wk_c", "wv_c", "wo_c", "norm_c", "attn_norm", "wqkv", "wo", "ffn_norm", "w1", "w3", "w2")
 
@@ -104,6 +105,7 @@ class blt_dec_counters(C.Structure):
         ("pass_ns", C.c_uint64),
         ("persistent_calls", C.c_uint64),
         ("prefill_kv_read_bytes", C.c_uint64),
+        ("tc_gemms", C.c_uint64),
     ]
 
     def as_dict(self):

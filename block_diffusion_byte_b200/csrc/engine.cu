@@ -16,6 +16,7 @@
 #include "bltdec.h"
 #include "kernels.cuh"
 #include "mega.cuh"
+#include "tc_gemm.cuh"
 
 using namespace bltdec;
 
@@ -33,6 +34,10 @@ struct NvtxRange {
 struct Mat {
   uint4* w = nullptr;
   int N = 0, K = 0, planes = 1;
+  // BLT_FLAG_TENSOR_CORES: the same rows (same order), row-major bf16, and its TMA map (box 64 x tc_bn)
+  __nv_bfloat16* wr = nullptr;
+  int tc_bn = 0;
+  CUtensorMap tmap{};
   size_t bytes() const { return (size_t)N * K * 2 * planes; }
 };
 
@@ -108,6 +113,16 @@ struct blt_dec {
   unsigned long long *x_h = nullptr, *x_q = nullptr, *x_k = nullptr, *x_v = nullptr, *x_att = nullptr, *x_act = nullptr,
                      *x_w2p = nullptr, *x_logit = nullptr, *x_part = nullptr;
   int x_cmax = 0;
+  // tcgen05 GEMM (BLT_FLAG_TENSOR_CORES): prepared activation planes [RL][max(d, F)] and row scales
+  bool tc = false;
+  bool in_prefill = false;
+  __nv_bfloat16 *tc_hi = nullptr, *tc_lo = nullptr;
+  float* tc_rs = nullptr;
+  CUtensorMap tc_hi_d{}, tc_lo_d{}, tc_hi_f{}, tc_lo_f{};  // views with row stride d and F
+  unsigned long long tc_gemms = 0;
+  // persistent kernel: sleep between polls of a wait (ns; first 32 polls, then the rest).
+  // Tuning knob: BLTDEC_SPIN_NS="<first>,<rest>".
+  unsigned spin_ns[2] = {32, 128};
   // debug: BLTDEC_TRACE=<file> appends device timestamps of each persistent launch's first pass
   unsigned long long* trace = nullptr;
   std::string trace_path;
@@ -154,8 +169,33 @@ int dalloc(blt_dec* h, T** p, size_t count) {
 // Pack W (rows given by src_row(tile_row) of a [*, K] fp32 matrix) into
 // m16k16 tensor-core A-fragment order: tile (mt, ks), plane p, lane l holds
 // rows g, g+8 and columns 2t, 2t+1, 2t+8, 2t+9 (g = l/4, t = l%4).
+// TMA map of a row-major bf16 matrix [outer][inner]: boxes of 64 inner elements
+// (one 128-byte swizzle atom) x box_outer rows, zero fill outside.
+typedef CUresult (*TensorMapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                         const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                         CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+int tc_map(blt_dec* h, CUtensorMap* map, const void* base, int inner, int outer, int box_outer) {
+  static TensorMapEncodeTiled encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    CK(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (!fn || q != cudaDriverEntryPointSuccess) return fail(h, BLT_ERR_CUDA, "cuTensorMapEncodeTiled not available");
+    encode = reinterpret_cast<TensorMapEncodeTiled>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)inner * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, BLT_ERR_CUDA, "cuTensorMapEncodeTiled: error %d", (int)r);
+  return BLT_OK;
+}
+
 template <class RowFn>
-int pack_matrix(blt_dec* h, Mat& m, int N, int K, int planes, RowFn src_row) {
+int pack_matrix(blt_dec* h, Mat& m, int N, int K, int planes, RowFn src_row, bool tc_copy = false) {
   m.N = N;
   m.K = K;
   m.planes = planes;
@@ -183,6 +223,18 @@ int pack_matrix(blt_dec* h, Mat& m, int N, int K, int planes, RowFn src_row) {
   }
   TRY(dalloc(h, &m.w, buf.size() * 2 / 16));
   CK(cudaMemcpy(m.w, buf.data(), buf.size() * 2, cudaMemcpyHostToDevice));
+  if (tc_copy && h->tc && planes == 1 && K % kTcBK == 0) {
+    std::vector<uint16_t> rm((size_t)N * K);
+    for (int r = 0; r < N; ++r) {
+      const float* src = src_row(r);
+      for (int k = 0; k < K; ++k) rm[(size_t)r * K + k] = bf16_rne(src[k]);
+    }
+    m.tc_bn = N >= 2048 ? 128 : N >= 512 ? 64 : 32;
+    if (N % m.tc_bn) return BLT_OK;  // stays on the GEMV path
+    TRY(dalloc(h, &m.wr, rm.size()));
+    CK(cudaMemcpy(m.wr, rm.data(), rm.size() * 2, cudaMemcpyHostToDevice));
+    TRY(tc_map(h, &m.tmap, m.wr, K, N, m.tc_bn));
+  }
   return BLT_OK;
 }
 
@@ -242,6 +294,14 @@ int set_gemm_attr(blt_dec* h) {
 }
 
 template <int EPI>
+int set_tc_attrs(blt_dec* h) {
+  CK(cudaFuncSetAttribute(k_tc_gemm<32, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(32)));
+  CK(cudaFuncSetAttribute(k_tc_gemm<64, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(64)));
+  CK(cudaFuncSetAttribute(k_tc_gemm<128, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(128)));
+  return BLT_OK;
+}
+
+template <int EPI>
 int set_attrs_epi(blt_dec* h) {
   TRY((set_gemm_attr<1, 1, EPI>(h)));
   TRY((set_gemm_attr<2, 1, EPI>(h)));
@@ -261,9 +321,37 @@ void launch_ng(blt_dec* h, const GemmArgs& a, int rows_ub) {
   k_gemm<NG, PL, EPI, gemm_stages<NG, PL, EPI>()><<<grid, kThreads, gemm_smem<NG, PL, EPI>(), h->stream>>>(a);
 }
 
+template <int BN, int EPI>
+void launch_tc(blt_dec* h, const Mat& m, const GemmArgs& a, int rows_ub) {
+  const bool kd = m.K == h->d;
+  dim3 grid(m.N / BN, (rows_ub + kTcBM - 1) / kTcBM);
+  k_tc_gemm<BN, EPI><<<grid, 128, tc_smem_bytes(BN), h->stream>>>(kd ? h->tc_hi_d : h->tc_hi_f, kd ? h->tc_lo_d : h->tc_lo_f,
+                                                                  m.tmap, a, h->tc_rs, 500000000ull);
+}
+
+// The projection on the tcgen05 GEMM: activation prep, then the tiles.
+template <int EPI>
+int tc_gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
+  a.w = nullptr;
+  a.N = m.N;
+  a.K = m.K;
+  a.status = h->sd.status;
+  k_tc_prep<<<rows_ub, 256, 0, h->stream>>>(a.X, a.ldx, m.K, a.gain, a.eps, a.n_rows, rows_ub, h->tc_hi, h->tc_lo, h->tc_rs);
+  if (m.tc_bn == 128) launch_tc<128, EPI>(h, m, a, rows_ub);
+  else if (m.tc_bn == 64) launch_tc<64, EPI>(h, m, a, rows_ub);
+  else launch_tc<32, EPI>(h, m, a, rows_ub);
+  h->launches += 2;
+  h->tc_gemms += 1;
+  CK(cudaGetLastError());
+  return BLT_OK;
+}
+
 template <int EPI>
 int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
   if (rows_ub <= 0) return BLT_OK;
+  if constexpr (EPI == EPI_STORE || EPI == EPI_RESID || EPI == EPI_SWIGLU || EPI == EPI_QKV) {
+    if (h->tc && !h->in_prefill && rows_ub >= kTcMinRows && m.wr) return tc_gemm<EPI>(h, m, a, rows_ub);
+  }
   a.w = m.w;
   a.N = m.N;
   a.K = m.K;
@@ -650,7 +738,8 @@ size_t mega_smem(const blt_dec* h) {
   (void)h;
   const size_t red = (size_t)kMaxPieces * 8 * 16 * 8 * NG * 4;
   const size_t att = (size_t)(kMegaRows * DH + kMegaRows * 128) * 4;
-  return (size_t)kRingSlots * kSlotBytes + std::max(red, att) + 8 * 8 * kMegaMaxNG * 4 + 2 * (size_t)kMaxPieces * kMegaRows * 16 * 4;
+  return (size_t)kRingSlots * kSlotBytes + std::max(red, att) + 8 * 8 * kMegaMaxNG * 4 + 2 * (size_t)kMaxPieces * kMegaRows * 16 * 4 +
+         1024 * 4;  // ring, reduction / attention scratch, ssr, hpre, cpre, gain (d <= 1024)
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -726,6 +815,10 @@ int mega_setup(blt_dec* h) {
   CK(cudaMemset(h->abort_flag, 0, 4));
   h->epoch = 1;
   h->mega_ok = true;
+  if (const char* sp = getenv("BLTDEC_SPIN_NS")) {
+    unsigned a = 0, b = 0;
+    if (sscanf(sp, "%u,%u", &a, &b) == 2 && a <= 100000 && b <= 100000) h->spin_ns[0] = a, h->spin_ns[1] = b;
+  }
   if (const char* tp = getenv("BLTDEC_TRACE")) {
     h->trace_path = tp;
     TRY(dalloc(h, &h->trace, (size_t)h->nsm * kTraceEvents));
@@ -799,6 +892,8 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   m.abort = h->abort_flag;
   const bool stall = (h->cfg.flags & BLT_FLAG_TEST_STALL) != 0;
   m.wait_ns = stall ? 2000000ull : 500000000ull;  // 2 ms under the test-only stall, else 0.5 s
+  m.spin_ns0 = h->spin_ns[0];
+  m.spin_ns1 = h->spin_ns[1];
   m.stall_test = stall ? 1 : 0;
   m.trace = h->trace;
   if (h->trace) {
@@ -843,6 +938,11 @@ int prefill_impl(blt_dec* h, int batch, const blt_rows_in* rows, float* out_logi
   int kmax = 0;
   for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
   const int chunk = h->cfg.max_rows;
+  struct PrefillScope {  // prefill stays on the GEMV path (any chunking gives the same bits)
+    blt_dec* h;
+    explicit PrefillScope(blt_dec* hh) : h(hh) { h->in_prefill = true; }
+    ~PrefillScope() { h->in_prefill = false; }
+  } scope(h);
   for (int r0 = 0; r0 < total; r0 += chunk) {
     const int r1 = std::min(total, r0 + chunk);
     PlanArgs p = plan_args(h, PL_PREFILL, 0);
@@ -1023,6 +1123,7 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
       h->own_stream = true;
     }
     const int d = h->d, dg = h->dg, F = h->F, L = h->L, dh = h->dh, pl = h->planes;
+    h->tc = (c.flags & BLT_FLAG_TENSOR_CORES) && pl == 1 && c.max_rows >= kTcMinRows && d % kTcBK == 0 && F % kTcBK == 0;
     h->qkv.resize(L);
     h->o.resize(L);
     h->w13.resize(L);
@@ -1044,15 +1145,15 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
         const int head = tile / tph, tt = tile % tph;
         const int j = tt * 8 + (r16 & 7) + (r16 >= 8 ? dh / 2 : 0);
         return wqkv + ((size_t)sec * d + head * dh + j) * d;
-      }));
-      TRY(pack_matrix(h, h->o[l], d, d, pl, [&](int r) { return lw[BLT_LAYER_WO] + (size_t)r * d; }));
+      }, true));
+      TRY(pack_matrix(h, h->o[l], d, d, pl, [&](int r) { return lw[BLT_LAYER_WO] + (size_t)r * d; }, true));
       // SwiGLU: tile rows 0..7 = W1 rows j..j+7, rows 8..15 = the same rows of W3
       TRY(pack_matrix(h, h->w13[l], 2 * F, d, pl, [&](int r) -> const float* {
         const int tile = r / 16, r16 = r % 16;
         const int j = tile * 8 + (r16 & 7);
         return (r16 < 8 ? lw[BLT_LAYER_W1] : lw[BLT_LAYER_W3]) + (size_t)j * d;
-      }));
-      TRY(pack_matrix(h, h->w2[l], d, F, pl, [&](int r) { return lw[BLT_LAYER_W2] + (size_t)r * F; }));
+      }, true));
+      TRY(pack_matrix(h, h->w2[l], d, F, pl, [&](int r) { return lw[BLT_LAYER_W2] + (size_t)r * F; }, true));
       TRY(upload(h, &h->attn_norm[l], lw[BLT_LAYER_ATTN_NORM], d));
       TRY(upload(h, &h->ffn_norm[l], lw[BLT_LAYER_FFN_NORM], d));
     }
@@ -1061,7 +1162,7 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
                     [&](int r) { return w->layer[(size_t)(r / d) * BLT_LAYER_NT + BLT_LAYER_WV_C] + (size_t)(r % d) * dg; }));
     TRY(pack_matrix(h, h->oc_all, L * d, d, pl,
                     [&](int r) { return w->layer[(size_t)(r / d) * BLT_LAYER_NT + BLT_LAYER_WO_C] + (size_t)(r % d) * d; }));
-    TRY(pack_matrix(h, h->head, 256, d, pl, [&](int r) { return w->head + (size_t)r * d; }));
+    TRY(pack_matrix(h, h->head, 256, d, pl, [&](int r) { return w->head + (size_t)r * d; }, true));
     {
       // the embedding is read once per row: keep it fp32, values rounded like the weights
       std::vector<float> e((size_t)h->V * d);
@@ -1165,6 +1266,22 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(set_attrs_epi<EPI_SWIGLU>(h));
     TRY(set_attrs_epi<EPI_QKV>(h));
     TRY(set_attrs_epi<EPI_LATC>(h));
+    if (h->tc) {
+      const int KM = std::max(d, F);
+      TRY(dalloc(h, &h->tc_hi, (size_t)RL * KM));
+      TRY(dalloc(h, &h->tc_lo, (size_t)RL * KM));
+      TRY(dalloc(h, &h->tc_rs, RL));
+      CK(cudaMemset(h->tc_hi, 0, (size_t)RL * KM * 2));
+      CK(cudaMemset(h->tc_lo, 0, (size_t)RL * KM * 2));
+      TRY(tc_map(h, &h->tc_hi_d, h->tc_hi, d, RL, kTcBM));
+      TRY(tc_map(h, &h->tc_lo_d, h->tc_lo, d, RL, kTcBM));
+      TRY(tc_map(h, &h->tc_hi_f, h->tc_hi, F, RL, kTcBM));
+      TRY(tc_map(h, &h->tc_lo_f, h->tc_lo, F, RL, kTcBM));
+      TRY(set_tc_attrs<EPI_STORE>(h));
+      TRY(set_tc_attrs<EPI_RESID>(h));
+      TRY(set_tc_attrs<EPI_SWIGLU>(h));
+      TRY(set_tc_attrs<EPI_QKV>(h));
+    }
     TRY(set_attn_attrs<float>(h, attn_smem_bytes(h)));
     TRY(set_attn_attrs<__nv_bfloat16>(h, attn_smem_bytes(h)));
     TRY(mega_setup(h));
@@ -1413,6 +1530,7 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->pass_ns = h->pass_ns;
   out->persistent_calls = h->persistent_calls;
   out->prefill_kv_read_bytes = c[7];
+  out->tc_gemms = h->tc_gemms;
   return BLT_OK;
 }
 

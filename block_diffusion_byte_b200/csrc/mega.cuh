@@ -34,6 +34,8 @@
 // the abort word and the device status (BLT_ERR_DEVICE), and all CTAs leave.
 #pragma once
 
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace bltdec {
@@ -102,6 +104,7 @@ struct MegaArgs {
   unsigned epoch0;
   int* abort;
   unsigned long long wait_ns;  // wall time after which a wait gives up
+  unsigned spin_ns0, spin_ns1;  // sleep between polls: the first 32 polls of a wait, then the rest
   int stall_test;       // test only: unit 0 of the first O phase never publishes (a wait must run out)
   unsigned long long* trace;
   int mode, batch, k, max_passes;
@@ -115,6 +118,11 @@ struct MegaArgs {
 
 // ---------------------------------------------------------------------------- primitives
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
 __device__ __forceinline__ void mbar_init(uint64_t* b, unsigned count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(b)), "r"(count));
 }
@@ -202,7 +210,7 @@ struct Spin {
 // clock.  A wait gives up (abort word + BLT_ERR_DEVICE) after m.wait_ns of
 // wall time.  False: give up.
 __device__ __forceinline__ bool spin_step(const MegaArgs& m, Spin& sp) {
-  __nanosleep(sp.n < 32 ? 32 : 128);
+  __nanosleep(sp.n < 32 ? m.spin_ns0 : m.spin_ns1);
   if (sp.n++ == 0) sp.t0 = gtimer();
   if ((sp.n & 31) == 0) {
     if (*(volatile int*)m.abort) return false;
@@ -259,6 +267,41 @@ __device__ __forceinline__ bool poll_words(const MegaArgs& m, int n, unsigned e,
   return true;
 }
 
+// poll_words for pairs of adjacent words (at(i) 16-byte aligned): one 16-byte
+// load per pair; put(i, v0, v1) once both words carry epoch e.
+template <int N, class At, class Put>
+__device__ __forceinline__ bool poll_pairs(const MegaArgs& m, int n, unsigned e, int tid, At at, Put put) {
+  unsigned pending = 0;
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (tid + 256 * i < n) pending |= 1u << i;
+  Spin spins;
+  if (pending) {  // wait on one pair first
+    const int i0 = __ffs(pending) - 1;
+    const u64* p0 = at(tid + 256 * i0);
+    while (true) {
+      u64 a, b;
+      xw_ld2(p0, a, b);
+      if (xw_ok(a, e) && xw_ok(b, e)) break;
+      if (!spin_step(m, spins)) return false;
+    }
+  }
+  while (pending) {
+    u64 w0[N], w1[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if ((pending >> i) & 1u) xw_ld2(at(tid + 256 * i), w0[i], w1[i]);
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (((pending >> i) & 1u) && xw_ok(w0[i], e) && xw_ok(w1[i], e)) {
+        put(tid + 256 * i, xw_val(w0[i]), xw_val(w1[i]));
+        pending &= ~(1u << i);
+      }
+    if (pending && !spin_step(m, spins)) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ bool wait_mbar(const MegaArgs& m, uint64_t* b, unsigned parity) {
   unsigned n = 0;
   unsigned long long t0 = 0;
@@ -307,7 +350,8 @@ __device__ __forceinline__ void trace_mark(const MegaArgs& m, int pass, int code
 }
 enum TraceCode : int {
   TR_PASS = 1, TR_PH = 2, TR_IN = 3, TR_MMA = 4, TR_DONE = 5, TR_ATT = 6, TR_ATT_DONE = 7, TR_COMB = 8, TR_BOOK = 9,
-  TR_SENT = 10, TR_GATH = 11, TR_PRE = 12, TR_ISLOT = 13, TR_IPOLL = 14, TR_ICORE = 15
+  TR_SENT = 10, TR_GATH = 11, TR_PRE = 12, TR_ISLOT = 13, TR_IPOLL = 14, TR_ICORE = 15, TR_CBEG = 16,
+  TR_CROW = 17, TR_CML = 18, TR_CSUB = 19, TR_ISTAGE = 20, TR_MW = 21
 };
 
 // ---------------------------------------------------------------------------- schedule
@@ -399,13 +443,6 @@ __device__ __forceinline__ void att_decode(const MegaArgs& m, const int* g_kmax,
   }
   g = 0, h = 0, c = 0;
 }
-// Item index of (g, h, 0): its CTA combines the head's chunks.
-__device__ __forceinline__ int att_item0(const MegaArgs& m, const int* g_kmax, int g, int h) {
-  int base = 0;
-  for (int j = 0; j < g; ++j) base += m.H * ((g_kmax[j] + m.aa.CH - 1) / m.aa.CH);
-  return base + h * ((g_kmax[g] + m.aa.CH - 1) / m.aa.CH);
-}
-
 // ---------------------------------------------------------------------------- shared memory
 struct MegaSmem {
   unsigned char* ring;
@@ -415,6 +452,7 @@ struct MegaSmem {
   float* ssr;    // [8][RB]
   float* hpre;   // [kMaxPieces][rows][16] epilogue residual inputs
   float* cpre;   // [kMaxPieces][rows][16] cross terms of the next layer (W2)
+  float* gain;   // [d] the phase's norm gain; warp w's k-steps written and read by warp w only
   float* qs;     // [rows][DH]
   float* ps;     // [rows][CH]
   float* mrow;
@@ -580,10 +618,11 @@ __device__ __forceinline__ bool gather_frags(const MegaArgs& m, const MegaSmem& 
   } else {
     Spin spins;
     {
-      // Sentinels: lane j < nkw polls one word of k-step warp + 8 j (row 0, its last column) until
+      // Sentinels: lane j < nkw polls one word of k-step warp + 8 j (its last column) until
       // every k-step of the warp has data; only then do all lanes load everything.  While waiting,
       // a warp issues at most 8 loads per round.
-      const u64* sp = xs.x + xs.col0 + (warp + 8 * min(lane, 7)) * 16 + 15;
+      // (row blockIdx mod nr: the CTAs' polls spread over the rows instead of meeting on row 0's words)
+      const u64* sp = xs.x + (size_t)(blockIdx.x % nr) * xs.ld + xs.col0 + (warp + 8 * min(lane, 7)) * 16 + 15;
       bool ready = lane >= nkw;
       while (true) {
         if (!ready) ready = xw_ok(xw_ld(sp), xs.e);
@@ -630,13 +669,17 @@ __device__ __forceinline__ bool gather_frags(const MegaArgs& m, const MegaSmem& 
   }
   trace_mark(m, pass, TR_GATH << 8);
   const bool norm = gain != nullptr;
+  if (norm) {  // the warp's gain values, copied in before the wait (stage_gain)
+    cp_async_wait<0>();
+    __syncwarp();
+  }
 #pragma unroll
   for (int n = 0; n < NG; ++n) ss[n] = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     float4 gv = make_float4(1.f, 1.f, 1.f, 1.f);
     const int k0 = (warp + 8 * j) * 16 + 2 * t;
-    if (norm && j < nkw) gv = make_float4(__ldg(gain + k0), __ldg(gain + k0 + 1), __ldg(gain + k0 + 8), __ldg(gain + k0 + 9));
+    if (norm && j < nkw) gv = make_float4(sm.gain[k0], sm.gain[k0 + 1], sm.gain[k0 + 8], sm.gain[k0 + 9]);
 #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const float2 a = xa[j][n], b = xb[j][n];
@@ -646,6 +689,15 @@ __device__ __forceinline__ bool gather_frags(const MegaArgs& m, const MegaSmem& 
     }
   }
   return ok;
+}
+
+// The norm gain of this warp's k-steps (warp + 8 j, j < nkw) into shared memory
+// by asynchronous copies, one 16-byte piece per lane, issued before the phase's
+// input wait so that their latency hides behind it.
+__device__ __forceinline__ void stage_gain(const MegaSmem& sm, const float* gain, int nkw, int warp, int lane) {
+  const int j = lane >> 2, o = (warp + 8 * j) * 16 + 4 * (lane & 3);
+  if (j < nkw) cp_async16(sm.gain + o, gain + o, 16);
+  cp_async_commit();
 }
 
 // Epilogue side inputs, into smem before the MMAs: the residual the output is
@@ -831,6 +883,7 @@ __device__ bool run_gemv(const MegaArgs& m, MegaSmem& sm, const Phase& p, const 
   const int nr = sm.n_rows;
   const int nkw = (p.seg_steps - warp + 7) / 8;
   trace_mark(m, pass, TR_PH << 8 | p.kind);
+  if (gain) stage_gain(sm, gain, nkw, warp, lane);
   // the epilogue's side inputs are older data: fetch them while the phase input is still on its way
   bool ok = prefetch_side<NG>(m, sm, p, 0, min(kMaxPieces, p.a.count), pass, nr, tid);
   trace_mark(m, pass, TR_PRE << 8 | p.kind);
@@ -858,36 +911,83 @@ __device__ bool run_gemv(const MegaArgs& m, MegaSmem& sm, const Phase& p, const 
     for (int jv = 0; jv < kMaxPieces; ++jv)
 #pragma unroll
       for (int n = 0; n < NG; ++n) acc[jv][n][0] = acc[jv][n][1] = acc[jv][n][2] = acc[jv][n][3] = 0.f;
+    if constexpr (PL == 1) {
+      // one slot per piece: wait for the group's slots, then walk the k-steps with the pieces
+      // interleaved, so that their MMA chains overlap (each chain is the same as run alone)
+      constexpr int TPW = kSlotBytes / 512 / 8;  // tiles of a slot per warp
+      uint32_t stage[kMaxPieces];  // this lane's address in each piece's slot (shared memory)
 #pragma unroll
-    for (int jv = 0; jv < kMaxPieces; ++jv) {
-      if (jv < nu) {
-        constexpr int TPS = kSlotBytes / (512 * PL);           // tiles per slot
-        constexpr int TPW = TPS / 8;                           // tiles of a slot per warp
-        constexpr int MAXSL = (kSegSteps + TPS - 1) / TPS;     // slots per piece at most
+      for (int jv = 0; jv < kMaxPieces; ++jv) {
+        stage[jv] = smem_u32(sm.ring) + lane * 16 + warp * 512;
+        if (jv < nu) {
+          const unsigned itu = it + jv;
+          const int slot = itu % kRingSlots;
+          if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
+          stage[jv] += slot * kSlotBytes;
+        }
+      }
+      trace_mark(m, pass, TR_MW << 8);
+      const int ntiles = p.seg_steps;  // <= 64: one slot
+      auto chains = [&](auto nu_c) {
+        constexpr int NU = decltype(nu_c)::value;
 #pragma unroll
-        for (int sl = 0; sl < MAXSL; ++sl) {
-          if (sl < nsl) {
-            const unsigned itu = it++;
-            const int slot = itu % kRingSlots;
-            if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
-            const unsigned char* stage = sm.ring + (size_t)slot * kSlotBytes;
-            const int ntiles = min(TPS, p.seg_steps - sl * TPS);
-            uint4 w[TPW][PL];
+        for (int q = 0; q < TPW; ++q) {
+          if (8 * q + warp < ntiles) {  // k-step 8 q + warp of every piece
+            uint4 w[NU][1];
 #pragma unroll
-            for (int q = 0; q < TPW; ++q)
+            for (int jv = 0; jv < NU; ++jv) w[jv][0] = lds128(stage[jv] + q * 4096);
 #pragma unroll
-              for (int pl = 0; pl < PL; ++pl)
-                w[q][pl] = *reinterpret_cast<const uint4*>(stage + (size_t)min(8 * q + warp, ntiles - 1) * tile_bytes + pl * 512 + lane * 16);
+            for (int n = 0; n < NG; ++n) {
+              const XFrag xq{xf[q][n].x, xf[q][n].y, xf[q][n].z, xf[q][n].w};
 #pragma unroll
-            for (int q = 0; q < TPW; ++q) {
-              const int j = sl * TPW + q;  // this warp's j-th k-step of the piece: k-step 8 j + warp
-              if (8 * q + warp < ntiles)
-#pragma unroll
-                for (int n = 0; n < NG; ++n)
-                  mma_step<PL>(acc[jv][n], w[q], XFrag{xf[j][n].x, xf[j][n].y, xf[j][n].z, xf[j][n].w});
+              for (int jv = 0; jv < NU; ++jv) mma_step<1>(acc[jv][n], w[jv], xq);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sm.empty + slot);
+          }
+        }
+      };
+      if (nu == 1) chains(std::integral_constant<int, 1>{});
+      else if (nu == 2) chains(std::integral_constant<int, 2>{});
+      else if (nu == 3) chains(std::integral_constant<int, 3>{});
+      else chains(std::integral_constant<int, 4>{});
+      __syncwarp();
+      if (lane == 0)
+#pragma unroll
+        for (int jv = 0; jv < kMaxPieces; ++jv)
+          if (jv < nu) mbar_arrive(sm.empty + (it + jv) % kRingSlots);
+      it += nu;
+    } else {
+#pragma unroll
+      for (int jv = 0; jv < kMaxPieces; ++jv) {
+        if (jv < nu) {
+          constexpr int TPS = kSlotBytes / (512 * PL);           // tiles per slot
+          constexpr int TPW = TPS / 8;                           // tiles of a slot per warp
+          constexpr int MAXSL = (kSegSteps + TPS - 1) / TPS;     // slots per piece at most
+#pragma unroll
+          for (int sl = 0; sl < MAXSL; ++sl) {
+            if (sl < nsl) {
+              const unsigned itu = it++;
+              const int slot = itu % kRingSlots;
+              if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
+              trace_mark(m, pass, TR_MW << 8 | (jv * MAXSL + sl));
+              const unsigned char* stage = sm.ring + (size_t)slot * kSlotBytes;
+              const int ntiles = min(TPS, p.seg_steps - sl * TPS);
+              uint4 w[TPW][PL];
+#pragma unroll
+              for (int q = 0; q < TPW; ++q)
+#pragma unroll
+                for (int pl = 0; pl < PL; ++pl)
+                  w[q][pl] = *reinterpret_cast<const uint4*>(stage + (size_t)min(8 * q + warp, ntiles - 1) * tile_bytes + pl * 512 + lane * 16);
+#pragma unroll
+              for (int q = 0; q < TPW; ++q) {
+                const int j = sl * TPW + q;  // this warp's j-th k-step of the piece: k-step 8 j + warp
+                if (8 * q + warp < ntiles)
+#pragma unroll
+                  for (int n = 0; n < NG; ++n)
+                    mma_step<PL>(acc[jv][n], w[q], XFrag{xf[j][n].x, xf[j][n].y, xf[j][n].z, xf[j][n].w});
+              }
+              __syncwarp();
+              if (lane == 0) mbar_arrive(sm.empty + slot);
+            }
           }
         }
       }
@@ -937,21 +1037,25 @@ __device__ bool run_gemv(const MegaArgs& m, MegaSmem& sm, const Phase& p, const 
 
 // ---------------------------------------------------------------------------- consumer: attention
 // attn_combine for one (row, head) by one warp, with the chunk partials read as
-// exchange words: for each block of 32 chunks every lane polls its chunk's
-// (m, l) and its columns of every chunk's o in one round of loads, then the
-// arithmetic of attn_combine runs in the same order on the registers.
+// exchange words.  Each chunk's (m, l) pair and each pair of o columns is one
+// 16-byte load (a record is 2 + DH words, so both start on 16 bytes).  Lane j
+// holds chunk j of each 32-chunk block for the weights; lane c owns columns
+// 2c and 2c + 1 and reads eight chunks per round of loads.  The arithmetic is
+// attn_combine's, in the same order: the maximum over chunks with l > 0, the
+// lanes' l sums then a warp sum, and per column one fmaf chain in chunk order.
 template <int DH>
-__device__ __forceinline__ bool combine_row_xw(const MegaArgs& m, const u64* base, int nch, int lane, unsigned e, u64* out, unsigned e_out) {
-  constexpr int DPL = DH >= 32 ? DH / 32 : 1;  // columns per lane
+__device__ __forceinline__ bool combine_row_xw(const MegaArgs& m, const u64* base, int nch, int lane, unsigned e, u64* out, unsigned e_out,
+                                               int pass) {
+  static_assert(DH == 32 || DH == 64, "column pairs per lane");
   constexpr int REC = 2 + DH;
-  const bool col_ok = lane < DH;
+  constexpr int RND = 5;  // chunks per round of loads (more spills registers)
+  const bool col_ok = 2 * lane < DH;
   bool ok = true;
   auto poll_ml = [&](int ch, float& mm, float& ll) {
     Spin spins;
     while (true) {
       u64 a, b;
-      a = xw_ld(base + (size_t)ch * REC);
-      b = xw_ld(base + (size_t)ch * REC + 1);
+      xw_ld2(base + (size_t)ch * REC, a, b);
       if (xw_ok(a, e) && xw_ok(b, e)) {
         mm = xw_val(a), ll = xw_val(b);
         return true;
@@ -963,15 +1067,14 @@ __device__ __forceinline__ bool combine_row_xw(const MegaArgs& m, const u64* bas
   float m0 = 0.f, l0 = 0.f;  // the lane's chunk of the first block, kept for the second pass
 #pragma unroll 1
   for (int ch = lane; ch < nch; ch += 32) {
-    float mm, ll;
+    float mm = 0.f, ll = 0.f;
     ok = poll_ml(ch, mm, ll) && ok;
     if (ch < 32) m0 = mm, l0 = ll;
     if (ll > 0.f) mmax = fmaxf(mmax, mm);
   }
   mmax = warp_max(mmax);
-  float l = 0.f, o[DPL];
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) o[i] = 0.f;
+  trace_mark(m, pass, TR_CML << 8);
+  float l = 0.f, o0 = 0.f, o1 = 0.f;
 #pragma unroll 1
   for (int cb = 0; cb < nch; cb += 32) {
     const int nb = min(32, nch - cb);
@@ -984,56 +1087,48 @@ __device__ __forceinline__ bool combine_row_xw(const MegaArgs& m, const u64* bas
         l = fmaf(ll, w, l);
       }
     }
-    // this lane's columns of the block's o, 16 chunks per round of loads (re-read only what is not ready)
-    constexpr int SUB = 16;
 #pragma unroll 1
-    for (int sb = 0; sb < nb; sb += SUB) {
-      float ov[SUB][DPL];
+    for (int sb = 0; sb < nb; sb += RND) {
+      const u64* p = base + (size_t)(cb + sb) * REC + 2 + 2 * lane;
       unsigned pending = 0;
 #pragma unroll
-      for (int j = 0; j < SUB; ++j)
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) {
-          ov[j][i] = 0.f;
-          if (sb + j < nb && col_ok) pending |= 1u << (j * DPL + i);
-        }
+      for (int j = 0; j < RND; ++j)
+        if (sb + j < nb && col_ok) pending |= 1u << j;
+      u64 va[RND], vb[RND];
       Spin spins;
-      while (pending) {
-        u64 wv[SUB][DPL];
+      while (true) {
 #pragma unroll
-        for (int j = 0; j < SUB; ++j)
+        for (int j = 0; j < RND; ++j)  // every load of the round first, then the checks
+          if ((pending >> j) & 1u) xw_ld2(p + (size_t)j * REC, va[j], vb[j]);
+        unsigned bad = 0;
 #pragma unroll
-          for (int i = 0; i < DPL; ++i)
-            if ((pending >> (j * DPL + i)) & 1u) wv[j][i] = xw_ld(base + (size_t)(cb + sb + j) * REC + 2 + lane + 32 * i);
-#pragma unroll
-        for (int j = 0; j < SUB; ++j)
-#pragma unroll
-          for (int i = 0; i < DPL; ++i)
-            if (((pending >> (j * DPL + i)) & 1u) && xw_ok(wv[j][i], e)) {
-              ov[j][i] = xw_val(wv[j][i]);
-              pending &= ~(1u << (j * DPL + i));
-            }
-        if (pending && !spin_step(m, spins)) {
+        for (int j = 0; j < RND; ++j)
+          if (((pending >> j) & 1u) && (!xw_ok(va[j], e) || !xw_ok(vb[j], e))) bad |= 1u << j;
+        pending = bad;
+        if (!pending) break;
+        if (!spin_step(m, spins)) {
           ok = false;
           break;
         }
       }
+      trace_mark(m, pass, TR_CSUB << 8);
 #pragma unroll
-      for (int j = 0; j < SUB; ++j) {
+      for (int j = 0; j < RND; ++j) {
         const float wj = __shfl_sync(0xffffffffu, w, (sb + j) & 31);
-        if (sb + j < nb)
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) o[i] = fmaf(ov[j][i], wj, o[i]);
+        if (sb + j < nb) {
+          o0 = fmaf(xw_val(va[j]), wj, o0);
+          o1 = fmaf(xw_val(vb[j]), wj, o1);
+        }
       }
     }
   }
   l = warp_sum(l);
-  if (col_ok)
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) xw_st(out + lane + 32 * i, o[i] / l, e_out);
+  if (col_ok) {
+    xw_st(out + 2 * lane, o0 / l, e_out);
+    xw_st(out + 2 * lane + 1, o1 / l, e_out);
+  }
   return ok;
 }
-
 
 // This CTA's attention items of layer l, then the combines it owns.
 template <int DH, typename KVT>
@@ -1061,26 +1156,37 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
     if (!wait_mbar(m, sm.full + slot, (itu / kRingSlots) & 1)) ok = false;
     trace_mark(m, pass, TR_ISLOT << 8);
     const int f0 = max(t0, fresh), f1 = t0 + nk;
-    const int nf = f1 > f0 ? (f1 - f0) * DH : 0;  // this pass's keys in the chunk, times DH
-    // one poll for this pass's keys and values in the chunk and the rows' queries
-    ok = poll_words<(2 * kMegaRows * 64 + kMegaRows * 64) / 256>(
-             m, 2 * nf + nr * DH, e_qkv, tid,
+    constexpr int HP = DH / 2;  // column pairs of a head
+    const int nfp = f1 > f0 ? (f1 - f0) * HP : 0;  // this pass's keys in the chunk, times HP
+    // one poll for this pass's keys and values in the chunk and the rows' queries, by column pairs
+    ok = poll_pairs<(3 * kMegaRows * HP + 255) / 256>(
+             m, 2 * nfp + nr * HP, e_qkv, tid,
              [&](int i) {
-               if (i < 2 * nf) {
-                 const int sel = i >= nf, rem = i - sel * nf;
-                 return (sel ? m.x_v : m.x_k) + (size_t)(row0 + (f0 + rem / DH - fresh)) * d + h * DH + rem % DH;
-               }
-               const int q = i - 2 * nf;
-               return m.x_q + (size_t)(row0 + q / DH) * d + h * DH + q % DH;
-             },
-             [&](int i, float v) {
-               if (i < 2 * nf) {
-                 const int sel = i >= nf, rem = i - sel * nf;
-                 KVT* dst = (sel ? vs : ks) + (size_t)(f0 + rem / DH - t0) * DH + rem % DH;
-                 if constexpr (sizeof(KVT) == 2) *dst = __float2bfloat16_rn(v);
-                 else *dst = v;
+               const u64* src = m.x_q;
+               int r, c;
+               if (i < 2 * nfp) {
+                 const int sel = i >= nfp, rem = i - sel * nfp;
+                 src = sel ? m.x_v : m.x_k;
+                 r = row0 + f0 - fresh + rem / HP, c = rem % HP;
                } else {
-                 sm.qs[i - 2 * nf] = v * m.aa.scale;
+                 const int q = i - 2 * nfp;
+                 r = row0 + q / HP, c = q % HP;
+               }
+               return src + (size_t)r * d + h * DH + 2 * c;
+             },
+             [&](int i, float v0, float v1) {
+               if (i < 2 * nfp) {
+                 const int sel = i >= nfp, rem = i - sel * nfp;
+                 KVT* dst = (sel ? vs : ks) + (size_t)(f0 - t0 + rem / HP) * DH + 2 * (rem % HP);
+                 if constexpr (sizeof(KVT) == 2) {
+                   *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(v0, v1);
+                 } else {
+                   dst[0] = v0;
+                   dst[1] = v1;
+                 }
+               } else {
+                 const int q = i - 2 * nfp;
+                 *reinterpret_cast<float2*>(sm.qs + 2 * q) = make_float2(v0 * m.aa.scale, v1 * m.aa.scale);
                }
              }) &&
          ok;
@@ -1100,27 +1206,26 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
         [&](int r, float mm, float ll) {
           xw_st(part + r * rstride, mm, e_part);
           xw_st(part + r * rstride + 1, ll, e_part);
-        });
+        },
+        [&](int stage) { trace_mark(m, pass, TR_ISTAGE << 8 | stage); });
     trace_mark(m, pass, TR_ICORE << 8);
     fence_proxy_async_smem();  // the slot was written by these threads; the producer refills it by bulk copy
     consumer_sync();
     if (lane == 0) mbar_arrive(sm.empty + slot);
   }
   trace_mark(m, pass, TR_ATT_DONE << 8);
-  // combines: (g, h) whose chunk 0 this CTA ran; one warp per row
+  // combines: pair p = g H + h belongs to CTA p mod G; one warp per row
   const unsigned e_att = epoch(m, pass, l, ST_ATT);
-  for (int g = 0; g < ng; ++g) {
-    const int nch = (gk[g] + CH - 1) / CH;
+  trace_mark(m, pass, TR_CBEG << 8);
+  for (int pr = cta; pr < ng * H; pr += G) {
+    const int g = pr / H, h = pr % H;
     const int row0 = sm.gmeta[1 * (kMegaRows + 1) + g], nr = sm.gmeta[2 * (kMegaRows + 1) + g];
-    for (int h = 0; h < H; ++h) {
-      if (att_item0(m, gk, g, h) % G != cta) continue;
-      for (int r = warp; r < nr; r += kMegaConsumers) {
-        const int row = row0 + r;
-        const int rnch = (sm.rnkeys[row] + CH - 1) / CH;
-        const u64* base = m.x_part + (((size_t)row * H + h) * m.CMAX) * (2 + DH);
-        ok = combine_row_xw<DH>(m, base, rnch, lane, e_part, m.x_att + (size_t)row * d + h * DH, e_att) && ok;
-      }
-      (void)nch;
+    for (int r = warp; r < nr; r += kMegaConsumers) {
+      const int row = row0 + r;
+      const int rnch = (sm.rnkeys[row] + CH - 1) / CH;
+      const u64* base = m.x_part + (((size_t)row * H + h) * m.CMAX) * (2 + DH);
+      trace_mark(m, pass, TR_CROW << 8);
+      ok = combine_row_xw<DH>(m, base, rnch, lane, e_part, m.x_att + (size_t)row * d + h * DH, e_att, pass) && ok;
     }
   }
   trace_mark(m, pass, TR_COMB << 8);
@@ -1136,7 +1241,11 @@ __device__ bool mega_bookkeeping(const MegaArgs& m, MegaSmem& sm, int pass, int 
   // every CTA's stores of this pass (the KV cache included) happen before the decision
   if (tid == 0) ok = wait_flag(m, m.flags + 1, (unsigned)(gridDim.x * (pass + 1)), false);
   const unsigned e = epoch(m, pass, m.L, ST_LOGIT);
-  ok = poll_words<kMegaRows>(m, nr * 256, e, tid, [&](int i) { return m.x_logit + i; }, [&](int i, float v) { m.logits[i] = v; }) && ok;
+  for (int half = 0; half < 2; ++half)  // two rounds of at most eight words per thread
+    ok = poll_words<kMegaRows / 2>(m, max(0, min(nr, (half + 1) * kMegaRows / 2) - half * kMegaRows / 2) * 256, e, tid,
+                                   [&](int i) { return m.x_logit + half * (kMegaRows / 2) * 256 + i; },
+                                   [&](int i, float v) { m.logits[half * (kMegaRows / 2) * 256 + i] = v; }) &&
+         ok;
   if (tid == 0) sm.misc[1] = 0;
   __threadfence_block();
   ok = consumer_and(ok);
@@ -1219,6 +1328,8 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.hpre = reinterpret_cast<float*>(p);
   p += kMaxPieces * kMegaRows * 16 * 4;
   sm.cpre = reinterpret_cast<float*>(p);
+  p += kMaxPieces * kMegaRows * 16 * 4;
+  sm.gain = reinterpret_cast<float*>(p);
   sm.full = bars;
   sm.empty = bars + kRingSlots;
   sm.mrow = mrow;

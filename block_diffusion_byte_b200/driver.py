@@ -61,13 +61,17 @@ class Engine:
 
     def __init__(self, shape: ModelShape, weights: WeightSet, max_batch: int, max_ctx: int, max_block: int,
                  max_rows: int = 1024, max_latents: Optional[int] = None, page_tokens: int = 64, attn_chunk: int = 0,
-                 device: str = "cuda", time_passes: bool = False, persistent: bool = False, extra_flags: int = 0):
+                 device: str = "cuda", time_passes: bool = False, persistent: bool = False, extra_flags: int = 0,
+                 tensor_cores: bool = True):
         self.shape = shape
         self.max_batch, self.max_ctx, self.max_block, self.max_rows = max_batch, max_ctx, max_block, max_rows
         self.max_latents = max_latents or (max_ctx // 2 + 64)
         self.device = torch.device(device)
         self.stream = torch.cuda.Stream(device=self.device)
+        # tensor_cores: decode passes of >= 128 rows project on the tcgen05 GEMM (bf16 weights; ignored otherwise)
         flags = (B.BLT_FLAG_TIME_PASSES if time_passes else 0) | (B.BLT_FLAG_PERSISTENT if persistent else 0) | extra_flags
+        if tensor_cores:
+            flags |= B.BLT_FLAG_TENSOR_CORES
         cfg = engine_config(shape, max_batch, max_ctx, self.max_latents, max_rows, max_block, page_tokens, 0, attn_chunk, flags)
         layers = []
         for l in range(shape.n_layers):

@@ -102,6 +102,10 @@ typedef struct {
                                   projection is never published and the waits give up after about a
                                   millisecond: the call's passes stop and blt_dec_sync reports
                                   BLT_ERR_DEVICE (exercises the bounded waits; never set in production) */
+#define BLT_FLAG_TENSOR_CORES 8 /* decode passes of >= 128 rows run their projections (QKV, O, SwiGLU, W2, head)
+                                   on the tcgen05 GEMM (bf16 weights only; prefill stays on the GEMV path
+                                   so that any chunking of a prefix gives the same bits).  Costs a second,
+                                   row-major bf16 copy of those weights. */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */
@@ -136,6 +140,7 @@ typedef struct {
   uint64_t pass_ns;        /* summed device time of those calls' passes, ns (latent projection excluded) */
   uint64_t persistent_calls; /* calls whose decoder passes ran in the persistent kernel (BLT_FLAG_PERSISTENT) */
   uint64_t prefill_kv_read_bytes; /* K/V bytes read by the self-attention of prefill chunks (algorithmic) */
+  uint64_t tc_gemms;       /* projections run on the tcgen05 GEMM (BLT_FLAG_TENSOR_CORES) */
 } blt_dec_counters;
 
 /* Create an engine.  Copies and re-lays out the weights on the device

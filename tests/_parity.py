@@ -156,7 +156,7 @@ def compare_generation(name: str, wl, model, seq: int, prefix: Sequence[int], G:
 
 
 def engine_gen_factory(shape, ws, wl, seq_ids: Sequence[int], prefixes_other: Optional[dict] = None, s_index: int = 0,
-                       persistent: bool = False, max_rows: int = 1024, extra_ctx: int = 0):
+                       persistent: bool = False, max_rows: int = 1024, extra_ctx: int = 0, tensor_cores: bool = True):
     """An ``engine_gen`` for compare_generation: a fresh engine per call, the sequence under
     test at batch index s_index and the other sequences with their own prefixes."""
     from block_diffusion_byte_b200.driver import Engine, generate
@@ -169,9 +169,10 @@ def engine_gen_factory(shape, ws, wl, seq_ids: Sequence[int], prefixes_other: Op
                 prefs.append(list(prefix))
             else:
                 prefs.append([int(b) for b in prefix_bytes(wl.seed, wl.cfg_index, s, wl.prefix_len)])
-        max_ctx = max(len(p) for p in prefs) + G + 4 * wl.block + 32 + extra_ctx
+        # in a batch every sequence decodes until the slowest has G bytes: room for the faster ones' extra rounds
+        max_ctx = max(len(p) for p in prefs) + (2 * G if len(prefs) > 1 else G) + 4 * wl.block + 32 + extra_ctx
         eng = Engine(shape, ws, max_batch=len(seq_ids), max_ctx=max_ctx, max_block=max(16, wl.block), max_rows=max_rows,
-                     persistent=persistent)
+                     persistent=persistent, tensor_cores=tensor_cores)
         try:
             return generate(eng, wl, prefs, G, record=True, seq_ids=list(seq_ids))
         finally:

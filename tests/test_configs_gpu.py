@@ -90,11 +90,13 @@ def test_config2_eb_full_job(dec9):
     _stored_compare("d4eb_b1_seq0", wl, 0, 0, gen)
 
 
-def test_config3_dv16_batch8_full(dec9):
+@pytest.mark.parametrize("tensor_cores", [False, True], ids=["gemv", "tcgen05"])
+def test_config3_dv16_batch8_full(dec9, tensor_cores):
     """BLT-DV-16 one-step drafts + verification, prefix 2048, batch 8, sequence 0 for all
-    1024 bytes (accept lengths compared round by round)."""
+    1024 bytes (accept lengths compared round by round).  Its passes hold 8 x 16 = 128 rows:
+    the projections run on the GEMV kernels, or with BLT_FLAG_TENSOR_CORES on the tcgen05 GEMM."""
     wl = CONFIGS["dv16_b8"]
-    gen = engine_gen_factory(wl.shape, dec9, wl, list(range(8)), s_index=0, persistent=True)
+    gen = engine_gen_factory(wl.shape, dec9, wl, list(range(8)), s_index=0, persistent=True, tensor_cores=tensor_cores)
     _stored_compare("dv16_b8_seq0", wl, 0, 0, gen)
 
 
@@ -108,7 +110,9 @@ def test_config4_s8_batch1_full(dec9, persistent):
 
 def test_config4_s8_batch16_full(dec9):
     """BLT-S k=8, prefix 4096, batch 16: sequence 3 for all 512 bytes inside the batch, and
-    the whole batch byte-identical to greedy AR decoding on the engine."""
+    the whole batch byte-identical to greedy AR decoding on the engine.  (For the exact
+    identity both jobs run on the GEMV kernels: the verification passes' 128 rows would
+    otherwise take the tcgen05 GEMM, whose fp32 sums differ in order from the AR passes'.)"""
     from block_diffusion_byte_b200.driver import Engine, generate
 
     wl = CONFIGS["s8_b16"]
@@ -119,7 +123,8 @@ def test_config4_s8_batch16_full(dec9):
         outs = {}
         for mode, k in (("S", 8), ("AR", 1)):
             w = replace(wl, mode=mode, block=k)
-            eng = Engine(wl.shape, dec9, max_batch=16, max_ctx=wl.prefix_len + 128 + 64, max_block=16, max_rows=1024, persistent=True)
+            eng = Engine(wl.shape, dec9, max_batch=16, max_ctx=wl.prefix_len + 2 * 128 + 64, max_block=16, max_rows=1024, persistent=True,
+                         tensor_cores=False)
             try:
                 outs[mode] = generate(eng, w, prefs, 128).out
             finally:
