@@ -115,7 +115,6 @@ struct blt_dec {
   int x_cmax = 0;
   // tcgen05 GEMM (BLT_FLAG_TENSOR_CORES): prepared activation planes [RL][max(d, F)] and row scales
   bool tc = false;
-  bool in_prefill = false;
   __nv_bfloat16 *tc_hi = nullptr, *tc_lo = nullptr;
   float* tc_rs = nullptr;
   CUtensorMap tc_hi_d{}, tc_lo_d{}, tc_hi_f{}, tc_lo_f{};  // views with row stride d and F
@@ -350,7 +349,7 @@ template <int EPI>
 int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
   if (rows_ub <= 0) return BLT_OK;
   if constexpr (EPI == EPI_STORE || EPI == EPI_RESID || EPI == EPI_SWIGLU || EPI == EPI_QKV) {
-    if (h->tc && !h->in_prefill && rows_ub >= kTcMinRows && m.wr) return tc_gemm<EPI>(h, m, a, rows_ub);
+    if (h->tc && rows_ub >= kTcMinRows && m.wr) return tc_gemm<EPI>(h, m, a, rows_ub);
   }
   a.w = m.w;
   a.N = m.N;
@@ -938,11 +937,6 @@ int prefill_impl(blt_dec* h, int batch, const blt_rows_in* rows, float* out_logi
   int kmax = 0;
   for (int s = 0; s < batch; ++s) kmax = std::max(kmax, h->kv_ub[s] + cd.row_off[s + 1] - cd.row_off[s]);
   const int chunk = h->cfg.max_rows;
-  struct PrefillScope {  // prefill stays on the GEMV path (any chunking gives the same bits)
-    blt_dec* h;
-    explicit PrefillScope(blt_dec* hh) : h(hh) { h->in_prefill = true; }
-    ~PrefillScope() { h->in_prefill = false; }
-  } scope(h);
   for (int r0 = 0; r0 < total; r0 += chunk) {
     const int r1 = std::min(total, r0 + chunk);
     PlanArgs p = plan_args(h, PL_PREFILL, 0);

@@ -48,8 +48,8 @@ constexpr int kMegaConsumers = 8;
 // warpgroup gives registers back and the consumers take them (setmaxnreg):
 // 128 * 56 + 256 * 224 = 384 * 168.
 constexpr int kMegaThreads = 12 * 32;
-constexpr int kProducerRegs = 56;
-constexpr int kConsumerRegs = 224;
+constexpr int kProducerRegs = 64;
+constexpr int kConsumerRegs = 216;
 static_assert(128 * kProducerRegs + 256 * kConsumerRegs <= kMegaThreads * 168, "register split exceeds the launch's registers");
 constexpr int kSlotBytes = 32 * 1024;
 constexpr int kRingSlots = 5;
@@ -430,6 +430,12 @@ __device__ __forceinline__ int att_total(const MegaArgs& m, const int* g_kmax, i
   for (int g = 0; g < n_groups; ++g) total += m.H * ((g_kmax[g] + m.aa.CH - 1) / m.aa.CH);
   return total;
 }
+// This CTA's attention items: a contiguous range of the item order (g, h, c), so that a
+// CTA's consecutive items are mostly consecutive chunks of one (group, head).
+__device__ __forceinline__ void att_range(int total, int G, int cta, int& i0, int& i1) {
+  i0 = (int)((long long)cta * total / G);
+  i1 = (int)((long long)(cta + 1) * total / G);
+}
 __device__ __forceinline__ void att_decode(const MegaArgs& m, const int* g_kmax, int n_groups, int item, int& g, int& h, int& c) {
   int rem = item;
   for (g = 0; g < n_groups; ++g) {
@@ -469,6 +475,7 @@ struct MegaSmem {
   float* rope_c; // [rows][dh/2] rotary factors of each row's position
   float* rope_s;
   int* gmeta;  // [5][kMegaRows + 1]: g_seq, g_row0, g_nrows, g_kmax, g_fresh
+  int* ppages;  // [16] the producer's KV-page lookups (next item, current item)
   int n_rows, n_groups;
 };
 
@@ -517,28 +524,43 @@ __device__ void mega_producer(const MegaArgs& m, MegaSmem& sm, int lane) {
     const int total = att_total(m, gk, ng);
     const int CH = m.aa.CH, PT = m.ga.PT;
     const unsigned page_bytes = (unsigned)(PT * DH * sizeof(KVT));
-    for (int item = cta; item < total && ok; item += G) {
-      int g, h, c;
+    int i0, i1;
+    att_range(total, G, cta, i0, i1);
+    // the page-table entries of an item are loaded one item ahead: their latency passes
+    // while the previous item waits for its slot
+    int g = 0, h = 0, c = 0, np = 0;
+    int* pages = sm.ppages;  // [2][8] in shared memory: the next item's, then the current item's
+    auto lookup = [&](int item) {
       att_decode(m, gk, ng, item, g, h, c);
       const int t0 = c * CH;
       const int tc = min(min(t0 + CH, gk[g]), gf[g]);  // cached keys of this chunk: [t0, tc)
-      const int np = tc > t0 ? (tc - t0 + PT - 1) / PT : 0;
-      int pages[8];
-      int nvalid = 0;
-      for (int j = 0; j < np; ++j) {
+      np = tc > t0 ? (tc - t0 + PT - 1) / PT : 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
         const int pi = t0 / PT + j;
-        pages[j] = (pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + gs[g] * m.ga.max_pages + pi) : -1;
-        nvalid += pages[j] >= 0;
+        pages[j] = (j < np && pi < m.ga.max_pages) ? __ldcg(m.ga.page_table + gs[g] * m.ga.max_pages + pi) : -1;
       }
+    };
+    if (i0 < i1) lookup(i0);
+    for (int item = i0; item < i1 && ok; ++item) {
+      const int ih = h, inp = np;
+      int* ipages = pages + 8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ipages[j] = pages[j];
+      if (item + 1 < i1) lookup(item + 1);
+      int nvalid = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) nvalid += (j < inp && ipages[j] >= 0);
       unsigned char* dst = next_slot(2u * nvalid * page_bytes);
       if (!dst) break;
       uint64_t* bar = sm.full + ((it - 1) % kRingSlots);
-      for (int j = 0; j < np; ++j) {
-        if (pages[j] < 0) continue;
-        const size_t hoff = (((size_t)pages[j] * m.L + layer) * 2) * m.H;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= inp || ipages[j] < 0) continue;
+        const size_t hoff = (((size_t)ipages[j] * m.L + layer) * 2) * m.H;
         const KVT* kv = static_cast<const KVT*>(m.ga.kv);
-        const KVT* ksrc = kv + ((hoff + 0 * m.H + h) * PT) * DH;
-        const KVT* vsrc = kv + ((hoff + 1 * m.H + h) * PT) * DH;
+        const KVT* ksrc = kv + ((hoff + 0 * m.H + ih) * PT) * DH;
+        const KVT* vsrc = kv + ((hoff + 1 * m.H + ih) * PT) * DH;
         tma_1d_plain(dst + (size_t)j * page_bytes, ksrc, page_bytes, bar);
         tma_1d_plain(dst + (size_t)CH * DH * sizeof(KVT) + (size_t)j * page_bytes, vsrc, page_bytes, bar);
       }
@@ -1142,9 +1164,14 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
   bool ok = true;
   const unsigned e_qkv = epoch(m, pass, l, ST_QKV), e_part = epoch(m, pass, l, ST_PART);
   trace_mark(m, pass, TR_ATT << 8);
-  for (int item = cta; item < total; item += G) {
+  int i0, i1;
+  att_range(total, G, cta, i0, i1);
+  int qg = -1, qh = -1;  // (group, head) whose queries sm.qs holds
+  for (int item = i0; item < i1; ++item) {
     int g, h, c;
     att_decode(m, gk, ng, item, g, h, c);
+    const bool new_q = g != qg || h != qh;
+    qg = g, qh = h;
     const int row0 = sm.gmeta[1 * (kMegaRows + 1) + g], nr = sm.gmeta[2 * (kMegaRows + 1) + g];
     const int kmax = gk[g], fresh = sm.gmeta[4 * (kMegaRows + 1) + g];
     const int t0 = c * CH, nk = min(CH, kmax - t0);
@@ -1158,9 +1185,10 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
     const int f0 = max(t0, fresh), f1 = t0 + nk;
     constexpr int HP = DH / 2;  // column pairs of a head
     const int nfp = f1 > f0 ? (f1 - f0) * HP : 0;  // this pass's keys in the chunk, times HP
-    // one poll for this pass's keys and values in the chunk and the rows' queries, by column pairs
+    // one poll for this pass's keys and values in the chunk and (for a new (group, head)) the
+    // rows' queries, by column pairs
     ok = poll_pairs<(3 * kMegaRows * HP + 255) / 256>(
-             m, 2 * nfp + nr * HP, e_qkv, tid,
+             m, 2 * nfp + (new_q ? nr * HP : 0), e_qkv, tid,
              [&](int i) {
                const u64* src = m.x_q;
                int r, c;
@@ -1303,7 +1331,7 @@ __device__ bool mega_bookkeeping(const MegaArgs& m, MegaSmem& sm, int pass, int 
 
 // ---------------------------------------------------------------------------- the kernel
 template <int NG, int PL, int DH, typename KVT>
-__global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
+__global__ void __launch_bounds__(kMegaThreads, 1) k_mega(const __grid_constant__ MegaArgs m) {
   extern __shared__ __align__(1024) unsigned char mega_smem[];
   __shared__ uint64_t bars[2 * kRingSlots];
   __shared__ int plan_sh[3 * (kMaxCallBatch + 1)];
@@ -1313,6 +1341,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   __shared__ int rmeta[6][kMegaRows];
   __shared__ int gmeta[5 * (kMegaRows + 1)];
   __shared__ float rope_tab[2][kMegaRows * 32];  // dh <= 64
+  __shared__ int ppages[16];
 
   MegaSmem sm;
   sm.ring = mega_smem;
@@ -1346,6 +1375,7 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
   sm.rope_c = rope_tab[0];
   sm.rope_s = rope_tab[1];
   sm.gmeta = gmeta;
+  sm.ppages = ppages;
 
   const int tid = threadIdx.x;
   if (tid == 0) {
@@ -1410,24 +1440,36 @@ __global__ void __launch_bounds__(kMegaThreads, 1) k_mega(MegaArgs m) {
     consumer_sync();
     trace_mark(m, pass, TR_PASS << 8);
     const int nr = sm.n_rows;
-    for (int l = 0; l < m.L && ok; ++l) {
+    // The pass as one loop of GEMV steps (per layer QKV, O, W13, W2; then the head), so that
+    // run_gemv and run_attention are each inlined once: the kernel's code stays small enough
+    // for the instruction caches to keep a phase's working set.
+    const int nsteps = 4 * m.L + 1;
+    for (int st = 0; st < nsteps && ok; ++st) {
+      const int l = st >> 2, k = st & 3;
       XSrc xs;
-      xs.x = (l == 0) ? nullptr : m.x_h;
-      xs.ld = m.d, xs.col0 = 0, xs.e = (l == 0) ? 0u : epoch(m, pass, l - 1, ST_HW);
-      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_QKV, l, blockIdx.x, G), xs, m.layers[l].attn_norm, pass, it, tid) && ok);
-      ok = consumer_and(run_attention<DH, KVT>(m, sm, l, pass, it, tid) && ok);
-      xs.x = m.x_att, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, l, ST_ATT);
-      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_O, l, blockIdx.x, G), xs, nullptr, pass, it, tid) && ok);
-      xs.x = m.x_h, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, l, ST_HO);
-      ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_W13, l, blockIdx.x, G), xs, m.layers[l].ffn_norm, pass, it, tid) && ok);
-      const Phase pw2 = phase_of(m, PH_W2, l, blockIdx.x, G);
-      xs.x = m.x_act, xs.ld = m.F, xs.col0 = pw2.seg * kSegCols, xs.e = epoch(m, pass, l, ST_ACT);
-      ok = consumer_and(run_gemv<NG, PL>(m, sm, pw2, xs, nullptr, pass, it, tid) && ok);
+      xs.ld = m.d, xs.col0 = 0;
+      const float* gain = nullptr;
+      Phase ph;
+      if (l == m.L) {  // the byte head
+        ph = phase_of(m, PH_HEAD, 0, blockIdx.x, G);
+        xs.x = m.x_h, xs.e = epoch(m, pass, m.L - 1, ST_HW), gain = m.final_norm;
+      } else if (k == 0) {
+        ph = phase_of(m, PH_QKV, l, blockIdx.x, G);
+        xs.x = (l == 0) ? nullptr : m.x_h, xs.e = (l == 0) ? 0u : epoch(m, pass, l - 1, ST_HW), gain = m.layers[l].attn_norm;
+      } else if (k == 1) {
+        ph = phase_of(m, PH_O, l, blockIdx.x, G);
+        xs.x = m.x_att, xs.e = epoch(m, pass, l, ST_ATT);
+      } else if (k == 2) {
+        ph = phase_of(m, PH_W13, l, blockIdx.x, G);
+        xs.x = m.x_h, xs.e = epoch(m, pass, l, ST_HO), gain = m.layers[l].ffn_norm;
+      } else {
+        ph = phase_of(m, PH_W2, l, blockIdx.x, G);
+        xs.x = m.x_act, xs.ld = m.F, xs.col0 = ph.seg * kSegCols, xs.e = epoch(m, pass, l, ST_ACT);
+      }
+      ok = consumer_and(run_gemv<NG, PL>(m, sm, ph, xs, gain, pass, it, tid) && ok);
+      if (k == 0 && l < m.L) ok = consumer_and(run_attention<DH, KVT>(m, sm, l, pass, it, tid) && ok);
     }
     if (!ok) break;
-    XSrc xs;
-    xs.x = m.x_h, xs.ld = m.d, xs.col0 = 0, xs.e = epoch(m, pass, m.L - 1, ST_HW);
-    ok = consumer_and(run_gemv<NG, PL>(m, sm, phase_of(m, PH_HEAD, 0, blockIdx.x, G), xs, m.final_norm, pass, it, tid) && ok);
     // this CTA's stores of the pass (KV cache included) are done: arrive
     if (tid == 0) {
       __threadfence();

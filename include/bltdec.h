@@ -102,10 +102,10 @@ typedef struct {
                                   projection is never published and the waits give up after about a
                                   millisecond: the call's passes stop and blt_dec_sync reports
                                   BLT_ERR_DEVICE (exercises the bounded waits; never set in production) */
-#define BLT_FLAG_TENSOR_CORES 8 /* decode passes of >= 128 rows run their projections (QKV, O, SwiGLU, W2, head)
-                                   on the tcgen05 GEMM (bf16 weights only; prefill stays on the GEMV path
-                                   so that any chunking of a prefix gives the same bits).  Costs a second,
-                                   row-major bf16 copy of those weights. */
+#define BLT_FLAG_TENSOR_CORES 8 /* passes of >= 128 rows (prefill chunks included) run their projections
+                                   (QKV, O, SwiGLU, W2, head) on the tcgen05 GEMM (bf16 weights only).
+                                   Results then agree with the GEMV path to rounding, not bit for bit.
+                                   Costs a second, row-major bf16 copy of those weights. */
 
 typedef struct {
   const float *embed;      /* host [vocab, d] */
@@ -175,9 +175,12 @@ int blt_dec_prefill(blt_dec_t *h, int batch, const blt_rows_in *rows, float *out
  * Limits (else INVALID_ARG): d_model <= 1024, d_ffn <= 4096, n_heads <= 16,
  * head dim <= 64, n_layers * d_model <= 32768 (the latent-projection
  * temporary), attn_chunk 128 (the default), and each sequence's cached
- * length plus its rows <= 4096 positions.  The logits and the KV cache it
- * writes are bit-identical to blt_dec_prefill's (a row's arithmetic does not
- * depend on which rows share its pass).  The arena is about 5.2 MB and every
+ * length plus its rows <= 4096 positions.  Its 32-row chunks always take the
+ * GEMV kernels, so the logits and the KV cache it writes are bit-identical to
+ * blt_dec_prefill's on a handle without BLT_FLAG_TENSOR_CORES (a row's
+ * arithmetic does not depend on which rows share its pass); with that flag,
+ * blt_dec_prefill's chunks of >= 128 rows take the tcgen05 GEMM and agree to
+ * rounding.  The arena is about 5.2 MB and every
  * GPU that loads the library holds it until the process exits.
  * The first call on a device resolves the arena's device address
  * (cudaGetSymbolAddress) with that device current; make that first call

@@ -5,8 +5,10 @@ whose device-memory budget is spent, or that sized the handle's scratch small;
 a host thread that must not allocate after start-up).  For them the per-call
 scratch of this entry point lives in a static device arena of fixed size.
 Through the C ABI it must give the same logits and the same engine state as
-blt_dec_prefill, bit for bit (a row's arithmetic does not depend on which rows
-share its pass, so chunking the rows differently changes no bit), on two calls
+blt_dec_prefill on a handle without BLT_FLAG_TENSOR_CORES, bit for bit (a row's
+arithmetic does not depend on which rows share its pass, so chunking the rows
+differently changes no bit; the flag would send blt_dec_prefill's chunks of 128
+rows and more to the tcgen05 GEMM, which agrees to rounding only), on two calls
 in a row; it must also serve a handle whose own scratch holds a single row, and
 leave the device's free memory unchanged.  This file runs alone in a fresh
 process or after the other tests.
@@ -59,7 +61,7 @@ def test_prefill_noalloc_matches_prefill_twice(name, max_rows):
     ws = WeightSet(wl.shape).materialize()
     n = wl.prefix_len - 1
     # the reference: the regular prefill on a handle with room for 256 rows per pass
-    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 32, max_block=8, max_rows=256)
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 32, max_block=8, max_rows=256, tensor_cores=False)
     try:
         (r, keep), (pb, ps) = _rows(eng, wl, 0)
         ref = torch.zeros((n, 256), dtype=torch.float32, device="cuda")
@@ -71,7 +73,7 @@ def test_prefill_noalloc_matches_prefill_twice(name, max_rows):
     finally:
         eng.close()
     # the entry point under test, on a handle whose own scratch holds max_rows rows
-    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 32, max_block=8, max_rows=max_rows)
+    eng = Engine(wl.shape, ws, max_batch=1, max_ctx=wl.prefix_len + 32, max_block=8, max_rows=max_rows, tensor_cores=False)
     try:
         for call in range(2):
             B.blt_dec_rewind(eng.h, 1, [0], [0])
