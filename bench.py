@@ -540,8 +540,10 @@ def main():
             "gemv_value": w16.gen_bytes * w16.batch * 2 / (ms16g / 1000.0),
             "gemv_ms_per_step": ms16g / 2,
             "tcgen05_speedup": ms16g / ms16,
-            "note": "drafting passes (16 rows) run in the persistent kernel; verification passes (128 rows) project on the "
-            "tcgen05 GEMM (value) or on the mma.sync GEMV kernels (gemv_value); roofline over all decoder passes of the job",
+            "note": "drafting passes (16 rows over 16 x ~4100 cached bytes: ~57 attention items per SM) run in the per-phase "
+            "kernels, whose attention blocks overlap on each SM (the persistent kernel takes small passes with <= 8 items per SM); "
+            "verification passes (128 rows) and prefill chunks project on the tcgen05 GEMM (value) or on the mma.sync GEMV "
+            "kernels (gemv_value); roofline over all decoder passes of the job",
         }
     if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
         # the N_enc term of the pages' proxy, timed: one global-model step at the 1B size

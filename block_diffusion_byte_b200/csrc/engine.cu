@@ -398,9 +398,10 @@ GemmArgs base_args(blt_dec* h) {
   return a;
 }
 
-size_t attn_smem_bytes(const blt_dec* h) {
+// Shared memory of k_attn_partial for groups of at most `rows` rows.
+size_t attn_smem_bytes(const blt_dec* h, int rows = kAttnRows) {
   const int es = h->kv_f32 ? 4 : 2;
-  return (size_t)(kAttnRows * h->dh + kAttnRows * h->CH) * 4 + (size_t)2 * h->CH * (h->dh + 16 / es) * es;
+  return (size_t)(rows * h->dh + rows * h->CH) * 4 + (size_t)2 * h->CH * (h->dh + 16 / es) * es;
 }
 AttnArgs attn_args(blt_dec* h) {
   AttnArgs aa{};
@@ -423,34 +424,53 @@ AttnArgs attn_args(blt_dec* h) {
   aa.status = h->sd.status;
   return aa;
 }
-template <typename KVT>
-void launch_attn_t(blt_dec* h, dim3 ag, size_t smem, const AttnArgs& aa) {
-  if (h->dh == 64) k_attn_partial<64, KVT><<<ag, 128, smem, h->stream>>>(aa);
-  else if (h->dh == 32) k_attn_partial<32, KVT><<<ag, 128, smem, h->stream>>>(aa);
-  else if (h->dh == 128) k_attn_partial<128, KVT><<<ag, 128, smem, h->stream>>>(aa);
-  else k_attn_partial<16, KVT><<<ag, 128, smem, h->stream>>>(aa);
+template <typename KVT, int ROWS>
+void launch_attn_r(blt_dec* h, dim3 ag, const AttnArgs& aa) {
+  const size_t smem = attn_smem_bytes(h, ROWS);
+  if (h->dh == 64) k_attn_partial<64, KVT, ROWS><<<ag, 128, smem, h->stream>>>(aa);
+  else if (h->dh == 32) k_attn_partial<32, KVT, ROWS><<<ag, 128, smem, h->stream>>>(aa);
+  else if (h->dh == 128) k_attn_partial<128, KVT, ROWS><<<ag, 128, smem, h->stream>>>(aa);
+  else k_attn_partial<16, KVT, ROWS><<<ag, 128, smem, h->stream>>>(aa);
 }
-void launch_attn(blt_dec* h, dim3 ag, size_t smem, const AttnArgs& aa) {
-  if (h->kv_f32) launch_attn_t<float>(h, ag, smem, aa);
-  else launch_attn_t<__nv_bfloat16>(h, ag, smem, aa);
+// grp_rows_ub: the most rows any attention group of the pass can hold; a smaller bound
+// selects a variant with less shared memory, so more blocks share an SM.
+template <typename KVT>
+void launch_attn_t(blt_dec* h, dim3 ag, const AttnArgs& aa, int grp_rows_ub) {
+  if (grp_rows_ub <= 8) launch_attn_r<KVT, 8>(h, ag, aa);
+  else if (grp_rows_ub <= 16) launch_attn_r<KVT, 16>(h, ag, aa);
+  else launch_attn_r<KVT, kAttnRows>(h, ag, aa);
+}
+void launch_attn(blt_dec* h, dim3 ag, const AttnArgs& aa, int grp_rows_ub) {
+  if (h->kv_f32) launch_attn_t<float>(h, ag, aa, grp_rows_ub);
+  else launch_attn_t<__nv_bfloat16>(h, ag, aa, grp_rows_ub);
+}
+template <typename KVT, int ROWS>
+int set_attn_attrs_r(blt_dec* h) {
+  const int smem = (int)attn_smem_bytes(h, ROWS);
+  CK(cudaFuncSetAttribute(k_attn_partial<16, KVT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<32, KVT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<64, KVT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  CK(cudaFuncSetAttribute(k_attn_partial<128, KVT, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  return BLT_OK;
 }
 template <typename KVT>
-int set_attn_attrs(blt_dec* h, size_t smem) {
-  CK(cudaFuncSetAttribute(k_attn_partial<16, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  CK(cudaFuncSetAttribute(k_attn_partial<32, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  CK(cudaFuncSetAttribute(k_attn_partial<64, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  CK(cudaFuncSetAttribute(k_attn_partial<128, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+int set_attn_attrs(blt_dec* h) {
+  TRY((set_attn_attrs_r<KVT, 8>(h)));
+  TRY((set_attn_attrs_r<KVT, 16>(h)));
+  TRY((set_attn_attrs_r<KVT, kAttnRows>(h)));
   return BLT_OK;
 }
 
 // ---------------------------------------------------------------------------- one decoder pass
 // Runs every layer over the rows planned on the device (at most rows_ub rows,
 // keys below keys_ub, at most groups_ub attention groups).
-int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head);
-int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
-  return run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head);
+int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head, int grp_rows_ub);
+// grp_rows_ub: rows per attention group at most (a sequence's rows in the pass, capped at
+// the planner's group size).
+int run_pass(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head, int grp_rows_ub = kAttnRows) {
+  return run_pass_body(h, rows_ub, keys_ub, groups_ub, want_head, std::min(grp_rows_ub, kAttnRows));
 }
-int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head) {
+int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want_head, int grp_rows_ub) {
   NvtxRange nvtx_("decoder pass (per-phase kernels)");
   const int d = h->d;
   // embed + per layer (cross add, attention partial + combine) + head statistics; GEMMs count themselves
@@ -470,7 +490,7 @@ int run_pass_body(blt_dec* h, int rows_ub, int keys_ub, int groups_ub, bool want
     a.q = h->q;
     TRY(gemm<EPI_QKV>(h, h->qkv[l], a, rows_ub));
     aa.layer = l;
-    launch_attn(h, dim3(h->H, nchunks, groups_ub), attn_smem_bytes(h), aa);
+    launch_attn(h, dim3(h->H, nchunks, groups_ub), aa, grp_rows_ub);
     const dim3 cg(rows_ub, h->H);
     if (h->dh == 64) k_attn_combine<64><<<cg, 32, 0, h->stream>>>(aa);
     else if (h->dh == 32) k_attn_combine<32><<<cg, 32, 0, h->stream>>>(aa);
@@ -660,13 +680,13 @@ int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, f
   p.pend_bytes = pend->bytes;
   p.pend_lat = pend->row_latent;
   TRY(plan(h, p, cd));
-  TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true));
+  TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true, npmax + k));
   k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits, h->eb ? h->ent : nullptr);
   h->launches += 1;
   for (int st = 1; st < max_steps; ++st) {
     PlanArgs pb = plan_args(h, PL_BLOCK, k);
     TRY(plan(h, pb, cd));
-    TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true));
+    TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true, k));
     k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits,
                                           h->eb ? h->ent : nullptr);
     h->launches += 1;
@@ -826,8 +846,17 @@ int mega_setup(blt_dec* h) {
   return BLT_OK;
 }
 
+// The persistent kernel runs a CTA's attention items one after another, each with a fixed
+// latency of a few microseconds; with many long sequences (batch 16 at 4096 cached bytes:
+// ~57 items per CTA per layer) the per-phase kernels, whose attention blocks overlap on
+// every SM, are faster (measured 18 vs 25 ms per 8-pass draft call there, while at batch 1
+// and 1024 bytes the persistent kernel is 2.5x faster).  Above 8 items per SM: per-phase.
 bool use_mega(const blt_dec* h, int rows_ub, int batch) {
-  return h->mega_ok && rows_ub <= kMegaRows && batch <= kMegaRows;
+  if (!h->mega_ok || rows_ub > kMegaRows || batch > kMegaRows) return false;
+  long long items = 0;
+  const int per_seq = (rows_ub + batch - 1) / batch;
+  for (int s = 0; s < batch; ++s) items += (long long)h->H * ((h->kv_ub[s] + per_seq + h->CH - 1) / h->CH);
+  return items <= 8LL * h->nsm;
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -1276,8 +1305,8 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
       TRY(set_tc_attrs<EPI_SWIGLU>(h));
       TRY(set_tc_attrs<EPI_QKV>(h));
     }
-    TRY(set_attn_attrs<float>(h, attn_smem_bytes(h)));
-    TRY(set_attn_attrs<__nv_bfloat16>(h, attn_smem_bytes(h)));
+    TRY(set_attn_attrs<float>(h));
+    TRY(set_attn_attrs<__nv_bfloat16>(h));
     TRY(mega_setup(h));
     CK(cudaDeviceSynchronize());
     return BLT_OK;
@@ -1416,14 +1445,14 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
     p.pend_bytes = pending->bytes;
     p.pend_lat = pending->row_latent;
     TRY(plan(h, p, cd));
-    TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true));
+    TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true, npmax));
     k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, 0, h->pred, h->logits, out_logits);
     h->launches += 1;
     for (int t = 1; t < k; ++t) {
       PlanArgs pa = plan_args(h, PL_ARDRAFT, 0);
       pa.step = t;
       TRY(plan(h, pa, cd));
-      TRY(run_pass(h, batch, keys_ub, batch, true));
+      TRY(run_pass(h, batch, keys_ub, batch, true, 1));
       k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, t, h->pred, h->logits, out_logits);
       h->launches += 1;
     }
@@ -1466,7 +1495,7 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
   if (use_mega(h, batch * k, batch)) {
     TRY(mega_run(h, MM_VERIFY, batch, k, 0.f, 1, batch * k, draft_row_latent, out_logits, out_accepted, out_next));
   } else {
-    TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true));
+    TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true, k));
     k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
     h->launches += 1;
   }

@@ -520,6 +520,26 @@ __host__ __device__ constexpr int kv_stride() {
 // Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
 // ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).  One
 // K or V row per iteration: a single page-table lookup per row.
+// Keys and values t0 .. t0 + n - 1 of (seq, head h) into smem (row stride
+// kv_stride), with the chunk's page ids already in pg[] (pg[j]: the page of
+// positions (t0 / PT + j) PT ..): every copy is issued at once.
+template <int DH, typename KVT>
+__device__ __forceinline__ void attn_load_kv_paged(const AttnArgs& a, const int* pg, int h, int t0, int n, KVT* ks, KVT* vs, int tid,
+                                                   int nthr) {
+  constexpr int PER = 16 / sizeof(KVT);
+  constexpr int CPR = DH / PER;
+  constexpr int ST = kv_stride<DH, KVT>();
+  const KVT* kv = static_cast<const KVT*>(a.kv);
+#pragma unroll 1
+  for (int i = tid; i < 2 * n * CPR; i += nthr) {
+    const int c = i % CPR, r = i / CPR;
+    const int kvsel = r >= n, key = kvsel ? r - n : r, pos = t0 + key;
+    const int page = max(pg[pos / a.PT - t0 / a.PT], 0);
+    const KVT* src = kv + ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * DH + (size_t)(pos % a.PT) * DH;
+    cp_async16((kvsel ? vs : ks) + key * ST + c * PER, src + c * PER, 16);
+  }
+}
+
 template <int DH, typename KVT>
 __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, int t0, int lo, int hi, KVT* ks, KVT* vs, int tid,
                                              int nthr) {
@@ -726,27 +746,41 @@ __device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* k
   }
 }
 
-// Softmax partial of one (group, head, chunk) of the per-phase path: q and the
-// row limits from global memory, K/V already in smem (padded rows), partials
-// to a.part_o / a.part_ml.
-template <int DH, typename KVT, class Sync>
-__device__ void attn_partial_compute(const AttnArgs& a, int gi, int h, int chunk, float* qs, float* ps, const KVT* ks,
-                                     const KVT* vs, float* mrow, float* lrow, int* lim, int tid, int nthr, Sync sync) {
+// Softmax partial of one (group, head, chunk) of the per-phase path, in two
+// steps: attn_partial_stage loads q and the row limits into smem and zeroes the
+// V padding (it may run while the chunk's K/V copies are in flight); after the
+// caller's wait and `sync`, attn_partial_run runs attn_chunk_core with the
+// partials to a.part_o / a.part_ml.  ROWS: the smem capacity in rows (the
+// group's row count must not exceed it).
+template <int DH, typename KVT, int ROWS>
+__device__ __forceinline__ bool attn_partial_stage(const AttnArgs& a, int gi, int h, int chunk, float* qs, KVT* vs, int* lim,
+                                                   int tid, int nthr) {
   constexpr int ST = kv_stride<DH, KVT>();
   const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
+  if (nr > ROWS) {  // the host's bound on rows per group was wrong: no write past the smem
+    if (tid == 0) set_status(a.status, kErrDevice);
+    return false;
+  }
   const int t0 = chunk * a.CH;
   const int nk = min(a.CH, kmax - t0);
   for (int i = tid; i < nr * DH; i += nthr) {
     const int r = i / DH, c = i % DH;
     qs[r * DH + c] = __ldcg(a.q + (size_t)(row0 + r) * a.d + h * DH + c) * a.scale;
   }
-  if (tid < kAttnRows) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
+  if (tid < ROWS) lim[tid] = (tid < nr) ? __ldcg(a.rows.nkeys + row0 + tid) - t0 : 0;
   if constexpr (sizeof(KVT) == 2) {  // zero V rows nk .. next multiple of 16 (read by the last key tile)
     const int pad = ((nk + 15) & ~15) - nk;
     for (int i = tid; i < pad * (DH / 8); i += nthr)
-      *reinterpret_cast<uint4*>(const_cast<KVT*>(vs) + (nk + i / (DH / 8)) * ST + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(vs + (nk + i / (DH / 8)) * ST + (i % (DH / 8)) * 8) = make_uint4(0, 0, 0, 0);
   }
-  sync();
+  return true;
+}
+template <int DH, typename KVT, int ROWS, class Sync>
+__device__ __forceinline__ void attn_partial_run(const AttnArgs& a, int gi, int h, int chunk, const float* qs, float* ps, const KVT* ks,
+                                                 const KVT* vs, float* mrow, float* lrow, const int* lim, int tid, int nthr, Sync sync) {
+  constexpr int ST = kv_stride<DH, KVT>();
+  const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
+  const int nk = min(a.CH, kmax - chunk * a.CH);
   attn_chunk_core<DH, KVT, ST>(
       a.CH, qs, ps, ks, vs, mrow, lrow, lim, nr, nk, tid, nthr, sync,
       [&](int r, int c, float v) { a.part_o[(((size_t)(row0 + r) * a.H + h) * a.CMAX + chunk) * DH + c] = v; },
@@ -820,7 +854,8 @@ __device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int
 }
 
 // grid (H, chunks, groups); 128 threads.
-template <int DH, typename KVT>
+// grid (H, chunks, groups), 128 threads; ROWS: rows per group at most (smem).
+template <int DH, typename KVT, int ROWS>
 __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   const int gi = blockIdx.z;
   if (gi >= *a.rows.n_groups) return;
@@ -830,16 +865,28 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   const int h = blockIdx.x;
   extern __shared__ float4 smem4[];
   float* qs = reinterpret_cast<float*>(smem4);
-  float* ps = qs + kAttnRows * DH;
-  KVT* ks = reinterpret_cast<KVT*>(ps + kAttnRows * a.CH);
+  float* ps = qs + ROWS * DH;
+  KVT* ks = reinterpret_cast<KVT*>(ps + ROWS * a.CH);
   KVT* vs = ks + a.CH * kv_stride<DH, KVT>();
-  __shared__ float mrow[kAttnRows], lrow[kAttnRows];
-  __shared__ int lim[kAttnRows];
-  attn_load_kv<DH, KVT>(a, a.rows.g_seq[gi], h, t0, t0, min(t0 + a.CH, kmax), ks, vs, threadIdx.x, 128);
+  __shared__ float mrow[ROWS], lrow[ROWS];
+  __shared__ int lim[ROWS];
+  __shared__ int pg[16];  // the chunk's KV pages (at most CH / PT + 1 <= 9)
+  const int n = min(t0 + a.CH, kmax) - t0;
+  if (threadIdx.x < (t0 + n - 1) / a.PT - t0 / a.PT + 1) {
+    const int seq = a.rows.g_seq[gi], pi = t0 / a.PT + threadIdx.x;
+    int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
+    if (page < 0) set_status(a.status, kErrDevice);
+    pg[threadIdx.x] = page;
+  }
+  // q and the row limits load while the page ids do; then every K/V copy goes out at once
+  const bool ok = attn_partial_stage<DH, KVT, ROWS>(a, gi, h, blockIdx.y, qs, vs, lim, threadIdx.x, 128);
+  __syncthreads();
+  attn_load_kv_paged<DH, KVT>(a, pg, h, t0, n, ks, vs, threadIdx.x, 128);
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
-  attn_partial_compute<DH, KVT>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128, [] { __syncthreads(); });
+  if (!ok) return;
+  attn_partial_run<DH, KVT, ROWS>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128, [] { __syncthreads(); });
 }
 
 // grid (rows_max, H), one warp.
