@@ -29,7 +29,9 @@ BLT_DRAFT_DIFFUSION = 1
 BLT_FLAG_TIME_PASSES = 1
 BLT_FLAG_PERSISTENT = 2
 BLT_FLAG_TEST_STALL = 4  # test only: the persistent kernel's bounded waits must run out
-BLT_FLAG_TENSOR_CORES = 8  # decode passes of >= 128 rows: projections on the tcgen05 GEMM
+BLT_FLAG_TENSOR_CORES = 8  # passes of >= 128 rows: projections on the tcgen05 GEMM
+BLT_UNMASK_CONFIDENCE = 0
+BLT_UNMASK_EB = 1
 BLT_LAYER_NT = 12
 LAYER_ORDER = ("wq_c", "wk_c", "wv_c", "wo_c", "norm_c", "attn_norm", "wqkv", "wo", "ffn_norm", "w1", "w3", "w2")
 
@@ -41,6 +43,9 @@ EXPORTS = (
     "blt_dec_diffuse_block_eb",
     "blt_dec_draft",
     "blt_dec_verify_accept",
+    "blt_dec_diffuse_block_sampled",
+    "blt_dec_draft_sampled",
+    "blt_dec_verify_sampled",
     "blt_dec_rewind",
     "blt_dec_stats",
     "blt_dec_sync",
@@ -91,6 +96,10 @@ class blt_rows_in(C.Structure):
     ]
 
 
+class blt_sampling(C.Structure):
+    _fields_ = [("temperature", C.c_float), ("top_p", C.c_float), ("uniforms", C.c_void_p)]
+
+
 class blt_dec_counters(C.Structure):
     _fields_ = [
         ("passes", C.c_uint64),
@@ -131,6 +140,10 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.blt_dec_diffuse_block_eb.argtypes = [P, I, C.POINTER(blt_rows_in), I, F, I, P, P, P]
     lib.blt_dec_draft.argtypes = [P, I, C.POINTER(blt_rows_in), I, I, F, I, P, P]
     lib.blt_dec_verify_accept.argtypes = [P, P, P, C.POINTER(C.c_int32), P, P, P]
+    SP = C.POINTER(blt_sampling)
+    lib.blt_dec_diffuse_block_sampled.argtypes = [P, I, C.POINTER(blt_rows_in), I, F, I, I, SP, P, P, P]
+    lib.blt_dec_draft_sampled.argtypes = [P, I, C.POINTER(blt_rows_in), I, I, F, I, SP, P, P]
+    lib.blt_dec_verify_sampled.argtypes = [P, P, P, C.POINTER(C.c_int32), SP, P, P, P]
     lib.blt_dec_rewind.argtypes = [P, I, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
     lib.blt_dec_stats.argtypes = [P, C.POINTER(blt_dec_counters)]
     lib.blt_dec_sync.argtypes = [P]
@@ -233,6 +246,31 @@ def blt_dec_verify_accept(h, draft_row_latent, new_latents, latent_offsets, out_
         h, _ptr(draft_row_latent), _ptr(new_latents), lo, _ptr(out_accepted), _ptr(out_next), _ptr(out_logits)
     )
     _check(h, rc, "blt_dec_verify_accept")
+
+
+def sampling(temperature: float, top_p: float, uniforms_dev) -> blt_sampling:
+    """Sampling parameters; uniforms_dev: device float32 [batch][2 k + 1] in [0, 1)."""
+    return blt_sampling(float(temperature), float(top_p), _ptr(uniforms_dev))
+
+
+def blt_dec_diffuse_block_sampled(h, batch, pending, k, threshold, unmask, max_steps, samp, out_block, out_steps=None,
+                                  out_logits=None) -> None:
+    rc = load_library().blt_dec_diffuse_block_sampled(h, batch, C.byref(pending), k, float(threshold), unmask, max_steps,
+                                                      C.byref(samp), _ptr(out_block), _ptr(out_steps), _ptr(out_logits))
+    _check(h, rc, "blt_dec_diffuse_block_sampled")
+
+
+def blt_dec_draft_sampled(h, batch, pending, mode, k, alpha, max_steps, samp, out_draft, out_logits=None) -> None:
+    rc = load_library().blt_dec_draft_sampled(h, batch, C.byref(pending), mode, k, float(alpha), max_steps, C.byref(samp),
+                                              _ptr(out_draft), _ptr(out_logits))
+    _check(h, rc, "blt_dec_draft_sampled")
+
+
+def blt_dec_verify_sampled(h, draft_row_latent, new_latents, latent_offsets, samp, out_accepted, out_next, out_logits=None) -> None:
+    lo = _i32(latent_offsets)
+    rc = load_library().blt_dec_verify_sampled(h, _ptr(draft_row_latent), _ptr(new_latents), lo, C.byref(samp),
+                                               _ptr(out_accepted), _ptr(out_next), _ptr(out_logits))
+    _check(h, rc, "blt_dec_verify_sampled")
 
 
 def blt_dec_rewind(h, batch, kv_len=None, n_latents=None) -> None:

@@ -17,6 +17,7 @@
 #include "kernels.cuh"
 #include "mega.cuh"
 #include "tc_gemm.cuh"
+#include "sampling.cuh"
 
 using namespace bltdec;
 
@@ -86,6 +87,7 @@ struct blt_dec {
   std::vector<void*> allocs;
   int state = 0;  // 0 ready, 1 draft waiting
   int draft_k = 0, draft_batch = 0;
+  bool draft_sampled = false;  // the waiting draft was drawn (its distributions are in sa.qdist)
   std::vector<int> kv_ub, nlat_ub;
   int* mirror = nullptr;  // pinned [2*max_batch]: kv_len, n_lat
   cudaEvent_t mirror_ev = nullptr;
@@ -119,9 +121,15 @@ struct blt_dec {
   float* tc_rs = nullptr;
   CUtensorMap tc_hi_d{}, tc_lo_d{}, tc_hi_f{}, tc_lo_f{};  // views with row stride d and F
   unsigned long long tc_gemms = 0;
+  // stochastic decoding (the *_sampled entry points): on for the duration of such a call
+  bool samp_on = false;
+  SampleArgs sa{};
   // persistent kernel: sleep between polls of a wait (ns; first 32 polls, then the rest).
   // Tuning knob: BLTDEC_SPIN_NS="<first>,<rest>".
   unsigned spin_ns[2] = {32, 128};
+  // attention items per SM up to which a small pass runs in the persistent kernel.
+  // Tuning knob: BLTDEC_MEGA_ITEMS_PER_SM=<n>.
+  int mega_items_per_sm = 8;
   // debug: BLTDEC_TRACE=<file> appends device timestamps of each persistent launch's first pass
   unsigned long long* trace = nullptr;
   std::string trace_path;
@@ -668,6 +676,22 @@ int max_kv_ub(blt_dec* h, int batch) {
   return m;
 }
 
+// Bookkeeping kernels, greedy or (during a *_sampled call) drawing the committed bytes.
+void launch_unmask(blt_dec* h, int batch, int k, float alpha, int step, float* out_logits) {
+  if (h->samp_on)
+    k_unmask_sampled<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, step, h->sa, h->conf, h->pred, h->logits, out_logits,
+                                                   h->eb ? h->ent : nullptr);
+  else
+    k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, step, h->conf, h->pred, h->logits, out_logits,
+                                          h->eb ? h->ent : nullptr);
+}
+void launch_draft_ar(blt_dec* h, int batch, int step, float* out_logits) {
+  if (h->samp_on)
+    k_draft_ar_sampled<<<batch, 32, 0, h->stream>>>(h->sd, batch, step, h->sa, h->pred, h->logits, out_logits);
+  else
+    k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, step, h->pred, h->logits, out_logits);
+}
+
 // Fill k-byte blocks (BLT-D / BLT-DV draft) with the pending rows in pass 1.
 int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, float alpha, int max_steps, float* out_logits) {
   const int batch = cd.batch;
@@ -681,14 +705,13 @@ int block_loop(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, f
   p.pend_lat = pend->row_latent;
   TRY(plan(h, p, cd));
   TRY(run_pass(h, rows1, keys_ub, groups_bound(cd, k), true, npmax + k));
-  k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, 0, h->conf, h->pred, h->logits, out_logits, h->eb ? h->ent : nullptr);
+  launch_unmask(h, batch, k, alpha, 0, out_logits);
   h->launches += 1;
   for (int st = 1; st < max_steps; ++st) {
     PlanArgs pb = plan_args(h, PL_BLOCK, k);
     TRY(plan(h, pb, cd));
     TRY(run_pass(h, batch * k, keys_ub, batch * ((k + 31) / 32), true, k));
-    k_unmask<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, alpha, st, h->conf, h->pred, h->logits, out_logits,
-                                          h->eb ? h->ent : nullptr);
+    launch_unmask(h, batch, k, alpha, st, out_logits);
     h->launches += 1;
   }
   CK(cudaGetLastError());
@@ -834,6 +857,7 @@ int mega_setup(blt_dec* h) {
   CK(cudaMemset(h->abort_flag, 0, 4));
   h->epoch = 1;
   h->mega_ok = true;
+  if (const char* ip = getenv("BLTDEC_MEGA_ITEMS_PER_SM")) h->mega_items_per_sm = std::max(0, atoi(ip));
   if (const char* sp = getenv("BLTDEC_SPIN_NS")) {
     unsigned a = 0, b = 0;
     if (sscanf(sp, "%u,%u", &a, &b) == 2 && a <= 100000 && b <= 100000) h->spin_ns[0] = a, h->spin_ns[1] = b;
@@ -850,13 +874,14 @@ int mega_setup(blt_dec* h) {
 // latency of a few microseconds; with many long sequences (batch 16 at 4096 cached bytes:
 // ~57 items per CTA per layer) the per-phase kernels, whose attention blocks overlap on
 // every SM, are faster (measured 18 vs 25 ms per 8-pass draft call there, while at batch 1
-// and 1024 bytes the persistent kernel is 2.5x faster).  Above 8 items per SM: per-phase.
+// and 1024 bytes the persistent kernel is 2.5x faster).  Above 8 items per SM (the knob
+// below): per-phase.
 bool use_mega(const blt_dec* h, int rows_ub, int batch) {
-  if (!h->mega_ok || rows_ub > kMegaRows || batch > kMegaRows) return false;
+  if (!h->mega_ok || h->samp_on || rows_ub > kMegaRows || batch > kMegaRows) return false;
   long long items = 0;
   const int per_seq = (rows_ub + batch - 1) / batch;
   for (int s = 0; s < batch; ++s) items += (long long)h->H * ((h->kv_ub[s] + per_seq + h->CH - 1) / h->CH);
-  return items <= 8LL * h->nsm;
+  return items <= (long long)h->mega_items_per_sm * h->nsm;
 }
 
 template <int NG, int PL, int DH, typename KVT>
@@ -1272,6 +1297,9 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(dalloc(h, &sd.masked, (size_t)B * kMaxBlock));
     TRY(dalloc(h, &sd.status, 1));
     TRY(dalloc(h, &sd.counters, 8));
+    TRY(dalloc(h, &h->sa.qdist, (size_t)B * kMaxBlock * 256));
+    TRY(dalloc(h, &h->sa.p0dist, (size_t)B * 256));
+    TRY(dalloc(h, &h->sa.pdist, (size_t)B * 256));
     CK(cudaMemset(sd.kv_len, 0, B * 4));
     CK(cudaMemset(sd.n_lat, 0, B * 4));
     CK(cudaMemset(sd.active, 0, B * 4));
@@ -1410,8 +1438,9 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
                   uint8_t* out_draft, float* out_logits) {
   NvtxRange nvtx_("blt_dec_draft");
   if (!h) return BLT_ERR_INVALID_ARG;
-  h->err.clear();
+  if (!h->samp_on) h->err.clear();
   h->state = 0;  // a waiting draft is discarded
+  h->draft_sampled = false;
   TRY(check_pending(h, pending, true));
   if (mode != BLT_DRAFT_AR && mode != BLT_DRAFT_DIFFUSION) return fail(h, BLT_ERR_INVALID_ARG, "mode %d", mode);
   if (k < 1 || k > h->cfg.max_block) return fail(h, BLT_ERR_INVALID_ARG, "k %d outside 1..%d", k, h->cfg.max_block);
@@ -1446,14 +1475,14 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
     p.pend_lat = pending->row_latent;
     TRY(plan(h, p, cd));
     TRY(run_pass(h, cd.row_off[batch], keys_ub, groups_bound(cd, 0), true, npmax));
-    k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, 0, h->pred, h->logits, out_logits);
+    launch_draft_ar(h, batch, 0, out_logits);
     h->launches += 1;
     for (int t = 1; t < k; ++t) {
       PlanArgs pa = plan_args(h, PL_ARDRAFT, 0);
       pa.step = t;
       TRY(plan(h, pa, cd));
       TRY(run_pass(h, batch, keys_ub, batch, true, 1));
-      k_draft_ar<<<batch, 32, 0, h->stream>>>(h->sd, batch, t, h->pred, h->logits, out_logits);
+      launch_draft_ar(h, batch, t, out_logits);
       h->launches += 1;
     }
   } else {
@@ -1496,7 +1525,11 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
     TRY(mega_run(h, MM_VERIFY, batch, k, 0.f, 1, batch * k, draft_row_latent, out_logits, out_accepted, out_next));
   } else {
     TRY(run_pass(h, batch * k, max_kv_ub(h, batch) + k, batch * ((k + 31) / 32), true, k));
-    k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
+    if (h->samp_on)
+      k_accept_sampled<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->sa, draft_row_latent, h->logits, out_accepted, out_next,
+                                                      out_logits);
+    else
+      k_accept<<<batch, 32, 0, h->stream>>>(h->sd, batch, k, h->pred, draft_row_latent, h->logits, out_accepted, out_next, out_logits);
     h->launches += 1;
   }
   TRY(pass_end(h));
@@ -1555,6 +1588,61 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->prefill_kv_read_bytes = c[7];
   out->tc_gemms = h->tc_gemms;
   return BLT_OK;
+}
+
+// ---------------------------------------------------------------------------- stochastic decoding
+namespace {
+int sampling_on(blt_dec* h, const blt_sampling* s, int k) {
+  if (!s || !s->uniforms) return fail(h, BLT_ERR_INVALID_ARG, "sampling parameters or uniforms are NULL");
+  if (!(s->temperature > 0.f) || s->temperature == INFINITY) return fail(h, BLT_ERR_INVALID_ARG, "temperature must be > 0 and finite");
+  if (!(s->top_p > 0.f && s->top_p <= 1.f)) return fail(h, BLT_ERR_INVALID_ARG, "top_p must be in (0, 1]");
+  h->sa.temperature = s->temperature;
+  h->sa.top_p = s->top_p;
+  h->sa.u = s->uniforms;
+  h->sa.ustride = 2 * k + 1;
+  h->samp_on = true;
+  return BLT_OK;
+}
+struct SamplingScope {  // sampling stays on for exactly one call
+  blt_dec* h;
+  ~SamplingScope() { h->samp_on = false; }
+};
+}  // namespace
+
+int blt_dec_diffuse_block_sampled(blt_dec_t* h, int batch, const blt_rows_in* pending, int k, float threshold, int unmask,
+                                  int max_steps, const blt_sampling* sampling, uint8_t* out_block, int32_t* out_steps,
+                                  float* out_logits) {
+  NvtxRange nvtx_("blt_dec_diffuse_block_sampled");
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (unmask != BLT_UNMASK_CONFIDENCE && unmask != BLT_UNMASK_EB) return fail(h, BLT_ERR_INVALID_ARG, "unmask %d", unmask);
+  TRY(sampling_on(h, sampling, k));
+  SamplingScope scope{h};
+  if (unmask == BLT_UNMASK_EB) return blt_dec_diffuse_block_eb(h, batch, pending, k, threshold, max_steps, out_block, out_steps, out_logits);
+  return blt_dec_diffuse_block(h, batch, pending, k, threshold, max_steps, out_block, out_steps, out_logits);
+}
+
+int blt_dec_draft_sampled(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode, int k, float alpha, int max_steps,
+                          const blt_sampling* sampling, uint8_t* out_draft, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_draft_sampled");
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  TRY(sampling_on(h, sampling, k));
+  SamplingScope scope{h};
+  const int rc = blt_dec_draft(h, batch, pending, mode, k, alpha, max_steps, out_draft, out_logits);
+  h->draft_sampled = rc == BLT_OK;
+  return rc;
+}
+
+int blt_dec_verify_sampled(blt_dec_t* h, const int32_t* draft_row_latent, const float* new_latents, const int32_t* latent_offsets,
+                           const blt_sampling* sampling, int32_t* out_accepted, uint8_t* out_next, float* out_logits) {
+  NvtxRange nvtx_("blt_dec_verify_sampled");
+  if (!h) return BLT_ERR_INVALID_ARG;
+  h->err.clear();
+  if (h->state != 1 || !h->draft_sampled) return fail(h, BLT_ERR_STATE, "no drawn draft is waiting for verification");
+  TRY(sampling_on(h, sampling, h->draft_k));
+  SamplingScope scope{h};
+  return blt_dec_verify_accept(h, draft_row_latent, new_latents, latent_offsets, out_accepted, out_next, out_logits);
 }
 
 int blt_dec_sync(blt_dec_t* h) {

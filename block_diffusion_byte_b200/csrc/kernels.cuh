@@ -681,11 +681,118 @@ struct NoMark {
   __device__ void operator()(int) const {}
 };
 
+// Chunk partial for one or two rows (bf16 K/V), on the CUDA cores: threads 0..127
+// take part whatever nthr is (the arithmetic does not depend on the block size).
+//   scores: thread t = key t, s_r = fmaf chain over the columns in order (q in
+//     fp32, pre-scaled; K widened from bf16).
+//   softmax: m_r = max over keys (warp maxima, then the 4 warps in order);
+//     p = exp(s - m) (0 for masked keys); l_r = warp sums (butterfly), then the 4
+//     warps' sums added in order.
+//   PV: thread t = column pair (t mod 32 [+ 32 j]) x key quarter t / 32 (32
+//     keys, one fmaf chain in key order); the 4 quarters are added in order.
+// Scratch: ps [2][CH] then 16 floats; the K tile, once the scores are taken,
+// holds the PV partials [4][2][DH] (CH >= 16 rows of >= DH bf16 hold them).
+template <int DH, int ST, class Sync, class EmitO, class EmitML>
+__device__ void attn_chunk_small(int CH, const float* qs, float* ps, const __nv_bfloat16* ks, const __nv_bfloat16* vs, float* mrow,
+                                 float* lrow, const int* lim, int nr, int nk, int tid, Sync sync, EmitO emit_o, EmitML emit_ml) {
+  constexpr int NC = DH / 8;   // 16-byte pieces of a key row
+  constexpr int NP = DH / 2;   // column pairs
+  constexpr int PPT = (NP + 31) / 32;
+  const int warp = tid >> 5, lane = tid & 31;
+  float* red = ps + 2 * CH;    // [2 rows][4 warps] maxima, then sums
+  const bool act = tid < 128;
+  float s0 = -INFINITY, s1 = -INFINITY;
+  if (act && tid < nk) {
+    const uint4* kr = reinterpret_cast<const uint4*>(ks + (size_t)tid * ST);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const uint4 w = kr[j];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        const int c = j * 8 + 2 * e;
+        a0 = fmaf(qs[c], f.x, a0);
+        a0 = fmaf(qs[c + 1], f.y, a0);
+        if (nr > 1) {
+          a1 = fmaf(qs[DH + c], f.x, a1);
+          a1 = fmaf(qs[DH + c + 1], f.y, a1);
+        }
+      }
+    }
+    if (tid < lim[0]) s0 = a0;
+    if (nr > 1 && tid < lim[1]) s1 = a1;
+  }
+  // softmax statistics
+  float m0 = warp_max(s0), m1 = warp_max(s1);
+  if (act && lane == 0) red[warp] = m0, red[4 + warp] = m1;
+  sync();
+  m0 = fmaxf(fmaxf(fmaxf(red[0], red[1]), red[2]), red[3]);
+  m1 = fmaxf(fmaxf(fmaxf(red[4], red[5]), red[6]), red[7]);
+  const float p0 = (s0 == -INFINITY) ? 0.f : expf(s0 - m0);
+  const float p1 = (s1 == -INFINITY) ? 0.f : expf(s1 - m1);
+  if (act && tid < CH) {
+    ps[tid] = p0;
+    ps[CH + tid] = p1;
+  }
+  const float l0 = warp_sum(p0), l1 = warp_sum(p1);
+  if (act && lane == 0) red[8 + warp] = l0, red[12 + warp] = l1;
+  sync();
+  if (tid == 0) {
+    mrow[0] = m0, lrow[0] = ((red[8] + red[9]) + red[10]) + red[11];
+    if (nr > 1) mrow[1] = m1, lrow[1] = ((red[12] + red[13]) + red[14]) + red[15];
+  }
+  // PV partials of key quarter `warp`, into the K tile (no thread reads K any more)
+  float* part = reinterpret_cast<float*>(const_cast<__nv_bfloat16*>(ks));
+  const int kq = warp;
+  if (act) {
+#pragma unroll
+    for (int j = 0; j < PPT; ++j) {
+      const int cp = lane + 32 * j;
+      if (cp < NP) {
+        float o00 = 0.f, o01 = 0.f, o10 = 0.f, o11 = 0.f;
+        const int k1 = min(kq * 32 + 32, nk);
+#pragma unroll 4
+        for (int k = kq * 32; k < k1; ++k) {
+          const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vs + (size_t)k * ST + 2 * cp));
+          const float q0 = ps[k], q1 = ps[CH + k];
+          o00 = fmaf(q0, v.x, o00);
+          o01 = fmaf(q0, v.y, o01);
+          if (nr > 1) {
+            o10 = fmaf(q1, v.x, o10);
+            o11 = fmaf(q1, v.y, o11);
+          }
+        }
+        float* pr = part + (size_t)kq * 2 * DH;  // [quarter][row][DH]
+        pr[2 * cp] = o00, pr[2 * cp + 1] = o01;
+        pr[DH + 2 * cp] = o10, pr[DH + 2 * cp + 1] = o11;
+      }
+    }
+  }
+  sync();
+  for (int i = tid; i < nr * DH; i += 128) {
+    if (!act) break;
+    const int r = i / DH, c = i % DH;
+    const float o = ((part[r * DH + c] + part[2 * DH + r * DH + c]) + part[4 * DH + r * DH + c]) + part[6 * DH + r * DH + c];
+    emit_o(r, c, o);
+  }
+  if (tid < nr) emit_ml(tid, mrow[tid], lrow[tid]);
+}
+
+
 template <int DH, typename KVT, int ST, class Sync, class EmitO, class EmitML, class Mark = NoMark>
 __device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* ks, const KVT* vs, float* mrow, float* lrow,
                                 const int* lim, int nr, int nk, int tid, int nthr, Sync sync, EmitO emit_o, EmitML emit_ml,
                                 Mark mark = Mark()) {
   mark(1);
+  if constexpr (sizeof(KVT) == 2) {
+    if (nr <= 2 && CH <= 128) {  // one or two rows: the CUDA-core path (any block size, the same bits)
+      attn_chunk_small<DH, ST>(CH, qs, ps, ks, vs, mrow, lrow, lim, nr, nk, tid, sync, emit_o, emit_ml);
+      mark(3);
+      return;
+    }
+  }
   if constexpr (sizeof(KVT) == 2) attn_scores_mma<DH, ST>(CH, qs, ks, ps, lim, nr, nk, tid, nthr);
   else attn_scores<DH, KVT, ST>(CH, qs, ks, ps, lim, nr, nk, tid, nthr);
   sync();
@@ -1165,9 +1272,11 @@ __global__ void k_lat_plan(CallDesc cd, SeqDev sd, int* lat_seq, int* lat_slot, 
 // ranked by entropy (position breaks ties), running sums of entropy taken in
 // rank order in fp32, every position whose running sum is <= gamma is
 // committed, and at least the first.  Returns whether masked positions remain.
+// newly (optional): the lanes committed by this pass; with greedy_bytes false the
+// caller writes their bytes (sampling).
 __device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, float alpha, int step, const float* conf,
                                            const int* pred, const float* logits, float* out_logits, int lane,
-                                           const float* ent = nullptr) {
+                                           const float* ent = nullptr, unsigned* newly = nullptr, bool greedy_bytes = true) {
   if (step == 0 && lane == 0) {
     const int lr = sd.last_row[s];
     if (lr >= 0) sd.y_last[s] = __ldcg(pred + lr);
@@ -1210,9 +1319,10 @@ __device__ __forceinline__ bool unmask_seq(SeqDev sd, int s, int batch, int k, f
     commit = m && lane == bi;
   }
   if (commit) {
-    sd.blk[s * kMaxBlock + lane] = (unsigned char)__ldcg(pred + row);
+    if (greedy_bytes) sd.blk[s * kMaxBlock + lane] = (unsigned char)__ldcg(pred + row);
     sd.masked[s * kMaxBlock + lane] = 0;
   }
+  if (newly) *newly = __ballot_sync(0xffffffffu, commit);
   const unsigned left = __ballot_sync(0xffffffffu, m && !commit);
   if (out_logits && in) {
     float* dst = out_logits + (((size_t)step * batch + s) * k + lane) * 256;

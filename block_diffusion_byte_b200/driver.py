@@ -27,7 +27,7 @@ from typing import List, Optional, Sequence
 import numpy as np
 import torch
 
-from workload import ModelShape, Patcher, PatchState, WeightSet, Workload, latent_vectors
+from workload import sampling_uniforms, ModelShape, Patcher, PatchState, WeightSet, Workload, latent_vectors
 
 from . import binding as B
 
@@ -302,3 +302,95 @@ def generate(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: Op
     st1 = B.blt_dec_stats(h)
     stats = {k_: st1[k_] - st0[k_] for k_ in st1}
     return GenResult([s.out[:G] for s in seqs], rounds, stats, dt, eng.h2d_bytes - h2d0, eng.d2h_bytes - d2h0)
+
+
+def generate_sampled(eng: Engine, wl: Workload, prefixes: Sequence[Sequence[int]], G: int, temperature: float, top_p: float,
+                     seq_ids: Optional[Sequence[int]] = None, record: bool = False) -> GenResult:
+    """Prefill, then decode G bytes per sequence with drawn bytes: BLT-D (confidence
+    or EB selection), BLT-S / BLT-DV (rejection-sampling verification).  Round r of
+    sequence s uses the workload's uniforms for calls 2 r (block / draft) and
+    2 r + 1 (verification), 2 k + 1 each."""
+    nb = len(prefixes)
+    ids = list(seq_ids) if seq_ids is not None else list(range(nb))
+    sh = wl.shape
+    seqs = [SeqHost(Patcher(wl.patch_kind, wl.seed, wl.cfg_index, i), wl.seed, wl.cfg_index, i, sh.d_global) for i in ids]
+    h = eng.h
+    st0 = B.blt_dec_stats(h)
+    t0 = time.perf_counter()
+    for s, pre in zip(seqs, prefixes):
+        s.commit(list(pre))
+    bl, sl, ll = [], [], []
+    for s in seqs:
+        b, sl_, l = s.take_pending()
+        bl.append(b[:-1])
+        sl.append(sl_[:-1])
+        ll.append(l)
+        s.pend_bytes, s.pend_slots = b[-1:], sl_[-1:]
+    r, keep = eng.rows(bl, sl, ll)
+    B.blt_dec_prefill(h, nb, r)
+    rounds: List[dict] = []
+    k = wl.block
+    rnd = 0
+
+    def uniforms(call: int):
+        # the engine reads them on its own stream: the copy completes first; callers keep the
+        # tensor alive until the call's outputs have been read
+        u = torch.from_numpy(np.stack([sampling_uniforms(wl.seed, wl.cfg_index, i, call, 2 * k + 1) for i in ids])).to(eng.device)
+        torch.cuda.synchronize(eng.device)
+        return u
+
+    while any(len(s.out) < G for s in seqs):
+        pend = [s.take_pending() for s in seqs]
+        r, keep = eng.rows([p[0] for p in pend], [p[1] for p in pend], [p[2] for p in pend])
+        u_d = uniforms(2 * rnd)
+        samp = B.sampling(temperature, top_p, u_d)
+        if wl.mode == "D":
+            rule = B.BLT_UNMASK_EB if wl.unmask == "entropy" else B.BLT_UNMASK_CONFIDENCE
+            thr = wl.gamma if wl.unmask == "entropy" else wl.alpha
+            B.blt_dec_diffuse_block_sampled(h, nb, r, k, thr, rule, 0, samp, eng.d_out, eng.d_steps)
+            blk = eng._get(eng.out_view(nb, k))
+            for i, s in enumerate(seqs):
+                new = [int(v) for v in blk[i]]
+                s.commit(new)
+                s.out += new
+            if record:
+                rounds.append(dict(block=blk.copy()))
+        elif wl.mode in ("S", "DV"):
+            mode = B.BLT_DRAFT_AR if wl.mode == "S" else B.BLT_DRAFT_DIFFUSION
+            B.blt_dec_draft_sampled(h, nb, r, mode, k, wl.alpha, 0, samp, eng.d_out)
+            draft = eng._get(eng.out_view(nb, k))
+            vslots = np.zeros((nb, k), dtype=np.int32)
+            prov: List[List[np.ndarray]] = []
+            for i, s in enumerate(seqs):
+                slots, lats, _ = s.patch(s.pstate, [int(v) for v in draft[i]])
+                vslots[i] = slots
+                prov.append(lats)
+            lo = np.cumsum([0] + [len(p) for p in prov]).tolist()
+            allp = [v for p in prov for v in p]
+            dl = eng._put(eng.d_lat, np.stack(allp).astype(np.float32)) if allp else None
+            dvs = eng._put(eng.d_vslots.view(-1), vslots.reshape(-1))
+            u_v = uniforms(2 * rnd + 1)
+            B.blt_dec_verify_sampled(h, dvs, dl, lo, B.sampling(temperature, top_p, u_v), eng.d_acc, eng.d_next)
+            acc = eng._get(eng.d_acc[:nb])
+            nxt = eng._get(eng.d_next[:nb])
+            for i, s in enumerate(seqs):
+                a = int(acc[i])
+                new = [int(v) for v in draft[i, :a]] + [int(nxt[i])]
+                s_slots, s_lats, st = s.patch(s.pstate, new)
+                kept = (vslots[i, a - 1] + 1 - s.pstate.n_closed) if a >= 1 else 0
+                s.pstate = st
+                s.pend_bytes += new[a:]
+                s.pend_slots += s_slots[a:]
+                s.n_sent += kept
+                s.lat_ready += s_lats[kept:]
+                s.out += new
+            if record:
+                rounds.append(dict(draft=draft.copy(), accepted=acc.copy(), next=nxt.copy()))
+        else:
+            raise ValueError(f"sampled decoding has no mode {wl.mode}")
+        rnd += 1
+    st = B.blt_dec_sync(h)
+    if st != 0:
+        raise B.BltError(st, "generate_sampled", B.blt_dec_last_error(h))
+    st1 = B.blt_dec_stats(h)
+    return GenResult([s.out[:G] for s in seqs], rounds, {k_: st1[k_] - st0[k_] for k_ in st1}, time.perf_counter() - t0, 0, 0)

@@ -256,6 +256,61 @@ int blt_dec_draft(blt_dec_t *h, int batch, const blt_rows_in *pending, int mode,
 int blt_dec_verify_accept(blt_dec_t *h, const int32_t *draft_row_latent, const float *new_latents,
                           const int32_t *latent_offsets, int32_t *out_accepted, uint8_t *out_next, float *out_logits);
 
+/* ---- stochastic decoding -------------------------------------------------
+ * Fast-BLT (discuss.pytorch.kr), "블록 언마스킹 전략": the unmasking rules can be
+ * combined with top-p sampling; "BLT-S와 BLT-DV": with a non-zero temperature the
+ * verification extends through rejection sampling (the page evaluates greedy
+ * decoding only).  Definitions used here (the page gives none):
+ *   dist(z) = softmax(z / temperature) over the 256 byte logits, bytes ranked by
+ *     probability (ties: lower byte first), the shortest leading run whose
+ *     cumulative probability reaches top_p kept and renormalised;
+ *   a draw with uniform u = the smallest byte b whose cumulative probability
+ *     (bytes in increasing order) exceeds u.
+ * Random numbers are inputs: `uniforms` is a device array [batch][2 k + 1] of
+ * values in [0, 1) (k: the call's block / draft size; for verification the
+ * waiting draft's), owned by the caller and read during the call's stream work.
+ * These calls run on the per-phase kernels (never the persistent one). */
+typedef struct {
+  float temperature;     /* > 0 */
+  float top_p;           /* in (0, 1] */
+  const float *uniforms; /* device [batch][2 k + 1] */
+} blt_sampling;
+
+#define BLT_UNMASK_CONFIDENCE 0 /* threshold = alpha */
+#define BLT_UNMASK_EB 1         /* threshold = gamma (entropy bound, nats) */
+
+/* blt_dec_diffuse_block (unmask = CONFIDENCE) or blt_dec_diffuse_block_eb
+ * (unmask = EB), with the positions each pass commits chosen by that rule and
+ * their bytes drawn from dist(logits of their rows) with uniforms[s][i] for
+ * block position i.  Errors: those of the greedy call, INVALID_ARG for bad
+ * sampling parameters. */
+int blt_dec_diffuse_block_sampled(blt_dec_t *h, int batch, const blt_rows_in *pending, int k, float threshold, int unmask,
+                                  int max_steps, const blt_sampling *sampling, uint8_t *out_block, int32_t *out_steps,
+                                  float *out_logits);
+
+/* blt_dec_draft with drawn bytes: BLT_DRAFT_AR draws draft byte t from
+ * dist(logits of pass t's row) with uniforms[s][t]; BLT_DRAFT_DIFFUSION draws
+ * the bytes the unmasking commits, as blt_dec_diffuse_block_sampled (confidence
+ * rule).  The distribution each draft byte was drawn from, and the target of
+ * draft slot 0 (dist of the last committed byte's row), are kept for
+ * blt_dec_verify_sampled. */
+int blt_dec_draft_sampled(blt_dec_t *h, int batch, const blt_rows_in *pending, int mode, int k, float alpha, int max_steps,
+                          const blt_sampling *sampling, uint8_t *out_draft, float *out_logits);
+
+/* Verification of a blt_dec_draft_sampled draft by rejection sampling.  The
+ * causal pass is blt_dec_verify_accept's; then per sequence, for slots
+ * t = 0..k-1 with draft byte x_t, draft distribution q_t and target p_t (slot 0:
+ * the kept target; slot t > 0: dist of verification row t - 1): x_t is
+ * accepted while uniforms[s][t] < min(1, p_t(x_t) / q_t(x_t)); at the first
+ * rejection out_next[s] is drawn from max(p_t - q_t, 0) renormalised (p_t if
+ * that is zero) with uniforms[s][k + t]; if all k are accepted, out_next[s] is
+ * drawn from dist(row k - 1) with uniforms[s][2 k].  out_accepted / out_next /
+ * KV commit as in blt_dec_verify_accept.  Errors: as blt_dec_verify_accept;
+ * STATE when the waiting draft was not drawn. */
+int blt_dec_verify_sampled(blt_dec_t *h, const int32_t *draft_row_latent, const float *new_latents,
+                           const int32_t *latent_offsets, const blt_sampling *sampling, int32_t *out_accepted,
+                           uint8_t *out_next, float *out_logits);
+
 /* Set sequences' cached length and committed latent count (host arrays
  * [batch]; -1 keeps a value).  Values may only shrink.  Drops a waiting draft.
  * Synchronous with respect to the handle's stream.  Errors: INVALID_ARG. */

@@ -50,6 +50,7 @@ import numpy as np
 from workload import Patcher, PatchState, Workload, latent_vector
 
 from .model import BLOCK, CAUSAL, OracleModel, Row, SeqState, decoder_pass
+from .sampling import rejection_verify, sample_byte, tempered_top_p
 
 NEAR_TIE_GAP = 0.05  # top-2 logit gap below which an argmax is a near-tie
 NEAR_ALPHA = 0.03  # |conf - alpha| below which a threshold decision is a near-tie
@@ -220,14 +221,24 @@ class OracleSequence:
             self.flags.append(Flag(pos, "argmax", float(gap)))
 
     # ----------------------------------------------------------- BLT-D
-    def diffuse(self, B: int, alpha: float, max_steps: Optional[int] = None, unmask: str = "confidence", gamma: float = 0.0):
+    def diffuse(self, B: int, alpha: float, max_steps: Optional[int] = None, unmask: str = "confidence", gamma: float = 0.0,
+                samp: Optional[Tuple[float, float, List[float]]] = None):
         """Fill one masked block of B bytes; returns (block, steps, y_last).
         ``unmask`` selects confidence unmasking (threshold ``alpha``) or EB
         sampling (bound ``gamma``).
 
         ``y_last`` is the greedy prediction of the last pending committed row
         (None when no row was pending), used by BLT-DV verification.
+
+        ``samp`` = (temperature, top_p, uniforms): the committed positions are
+        chosen as above, their bytes drawn from the tempered top-p distribution
+        of their rows with uniforms[i] for block position i (oracle.sampling);
+        the distributions are kept in ``self.q_dists`` (per position) and the
+        last pending row's in ``self.p0_dist``.
         """
+        if samp is not None:
+            self.q_dists = [None] * B
+            self.p0_dist = None
         N = len(self.bytes)
         m_slot = self.n_closed - 1  # newest closed latent o_M
         mask_id = self.sh.mask_id
@@ -247,7 +258,12 @@ class OracleSequence:
                 if pend:
                     _, p_, g_ = head_stats(z[len(pend) - 1 : len(pend)])
                     y_last = int(p_[0])
-                    self._flag_argmax(N, float(g_[0]))
+                    if samp is None:
+                        self._flag_argmax(N, float(g_[0]))
+                    else:
+                        self.p0_dist, cut = tempered_top_p(z[len(pend) - 1], samp[0], samp[1])
+                        if cut < 2e-3:
+                            self.flags.append(Flag(N, "top_p", cut))
             conf, pred, gap = head_stats(z[len(rows) - B :])
             masked = [i for i in range(B) if block[i] is None]
             if unmask == "entropy":
@@ -270,8 +286,15 @@ class OracleSequence:
                     if c[-1] - c[-2] < NEAR_ALPHA:
                         self.flags.append(Flag(N + chosen[0], "fallback", float(c[-1] - c[-2])))
             for i in chosen:
-                self._flag_argmax(N + i, float(gap[i]))
-                block[i] = int(pred[i])
+                if samp is None:
+                    self._flag_argmax(N + i, float(gap[i]))
+                    block[i] = int(pred[i])
+                else:
+                    b, dist, kind, margin = sample_byte(z[len(rows) - B + i], samp[0], samp[1], samp[2][i])
+                    if kind:
+                        self.flags.append(Flag(N + i, kind, margin))
+                    block[i] = b
+                    self.q_dists[i] = dist
         return [int(b) for b in block], steps, y_last
 
     # ----------------------------------------------------------- AR
@@ -306,6 +329,56 @@ class OracleSequence:
             self._flag_argmax(l + t, float(gap[t - 1]))
         self.cached = l + a  # the verify pass wrote the accepted rows' final K/V
         return a, nxt
+
+    def verify_sampled(self, draft: List[int], q: List[np.ndarray], p0: np.ndarray, samp: Tuple[float, float, List[float]]):
+        """One causal pass over the draft, then rejection sampling (oracle.sampling):
+        targets p_0 = p0 and p_t = dist(verification row t - 1).  Returns (accepted, next byte)."""
+        T, top_p, u = samp
+        l = len(self.bytes)
+        k = len(draft)
+        slots, prov = self.speculative_slots(draft)
+        n_lat = len(self.st.latents)
+        self.st.latents += prov
+        z = self._pass([Row(draft[t], l + t, slots[t], CAUSAL) for t in range(k)])
+        del self.st.latents[n_lat:]
+        ps = [p0]
+        for t in range(k):
+            d, cut = tempered_top_p(z[t], T, top_p)
+            if cut < 2e-3:
+                self.flags.append(Flag(l + t + 1, "top_p", cut))
+            ps.append(d)
+        a, nxt, fl = rejection_verify(draft, q, ps, u[:k], u[k : 2 * k + 1])
+        for slot, kind, margin in fl:
+            self.flags.append(Flag(l + slot, kind, margin))
+        self.cached = l + a
+        return a, nxt
+
+    def blt_s_round_sampled(self, k: int, T: float, top_p: float, u_draft: List[float], u_verify: List[float]):
+        """Self-speculation with drawn draft bytes, verified by rejection sampling."""
+        l = len(self.bytes)
+        m_slot = self.n_closed - 1
+        N = len(self.bytes)
+        z = self._pass(self._pending())
+        self.cached = N
+        draft, q = [], []
+        for t in range(k):
+            if t > 0:
+                z = self._pass([Row(draft[-1], l + t - 1, m_slot, CAUSAL)])
+            b, dist, kind, margin = sample_byte(z[-1], T, top_p, u_draft[t])
+            if kind:
+                self.flags.append(Flag(l + t, kind, margin))
+            draft.append(b)
+            q.append(dist)
+        a, nxt = self.verify_sampled(draft, q, q[0], (T, top_p, u_verify))
+        return draft, a, nxt
+
+    def blt_dv_round_sampled(self, k: int, alpha: float, T: float, top_p: float, u_draft: List[float], u_verify: List[float]):
+        """Diffusion draft with drawn bytes, verified by rejection sampling."""
+        if len(self.bytes) == self.cached:
+            raise ValueError("BLT-DV needs the last committed byte pending")
+        draft, steps, _ = self.diffuse(k, alpha, samp=(T, top_p, u_draft))
+        a, nxt = self.verify_sampled(draft, self.q_dists, self.p0_dist, (T, top_p, u_verify))
+        return draft, a, nxt, steps
 
     def blt_s_round(self, k: int):
         """Self-speculation: k autoregressive draft bytes, then verification."""

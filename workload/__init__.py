@@ -23,6 +23,7 @@ from .gen import (  # noqa: F401
     PatchState,
     Patcher,
     prefix_bytes,
+    sampling_uniforms,
     latent_vector,
     latent_vectors,
 )

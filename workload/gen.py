@@ -33,13 +33,14 @@ from typing import Dict, List, Sequence, Tuple
 import numpy as np
 
 from .configs import ModelShape
-from .rng import FNV_OFFSET, derive_key, derive_keys, fnv1a64, normals, normals_many, round_bf16, stream, stream_int
+from .rng import FNV_OFFSET, derive_key, derive_keys, fnv1a64, normals, normals_many, round_bf16, stream, stream_int, uniform53
 
 STREAM_WEIGHT = 1
 STREAM_PREFIX = 2
 STREAM_PATCH = 3
 STREAM_LATENT = 4
 STREAM_GAIN = 5
+STREAM_SAMPLE = 6
 
 # Per-layer tensors, PyTorch Linear layout [out, in].
 LAYER_TENSORS = (
@@ -133,6 +134,13 @@ class WeightSet:
         if sh.weight_dtype == "bf16":
             w = round_bf16(w)
         return w.reshape(dims)
+
+
+def sampling_uniforms(seed: int, cfg_index: int, seq: int, call: int, n: int) -> np.ndarray:
+    """``n`` uniforms in [0, 1) for stochastic decoding call ``call`` of sequence
+    ``seq``, as float32 (both sides use exactly these values)."""
+    u = uniform53(stream(derive_key(seed, STREAM_SAMPLE, cfg_index, seq, call), 0, n)).astype(np.float32)
+    return np.minimum(u, np.float32(1.0 - 2.0**-24))
 
 
 def prefix_bytes(seed: int, cfg_index: int, seq: int, n: int) -> np.ndarray:
