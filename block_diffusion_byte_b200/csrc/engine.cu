@@ -117,6 +117,9 @@ struct blt_dec {
   int x_cmax = 0;
   // tcgen05 GEMM (BLT_FLAG_TENSOR_CORES): prepared activation planes [RL][max(d, F)] and row scales
   bool tc = false;
+  // split-K of small GEMV grids over K segments (W2 of small passes): workspace [nseg][seg_rows][seg_n]
+  float* seg_ws = nullptr;
+  int seg_rows = 0, seg_n = 0, seg_nmax = 0, sm_count = 0;
   __nv_bfloat16 *tc_hi = nullptr, *tc_lo = nullptr;
   float* tc_rs = nullptr;
   CUtensorMap tc_hi_d{}, tc_lo_d{}, tc_hi_f{}, tc_lo_f{};  // views with row stride d and F
@@ -324,7 +327,7 @@ int set_attrs_epi(blt_dec* h) {
 template <int NG, int PL, int EPI>
 void launch_ng(blt_dec* h, const GemmArgs& a, int rows_ub) {
   constexpr int RB = 8 * NG;
-  dim3 grid(a.N / 16, (rows_ub + RB - 1) / RB);
+  dim3 grid(a.N / 16, (rows_ub + RB - 1) / RB, a.seg_ws ? a.K / kSegCols : 1);
   k_gemm<NG, PL, EPI, gemm_stages<NG, PL, EPI>()><<<grid, kThreads, gemm_smem<NG, PL, EPI>(), h->stream>>>(a);
 }
 
@@ -365,6 +368,17 @@ int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
   a.status = h->sd.status;
   const int ng = rows_ub <= 8 ? 1 : rows_ub <= 16 ? 2 : rows_ub <= 32 ? 4 : 8;
   h->launches += 1;
+  // A grid of fewer CTAs than half the SMs with K in several canonical segments (W2 of a small
+  // pass): one CTA per (tile, segment), then k_seg_finish adds the segment sums in order --
+  // the same additions in the same order as one CTA folding them, so the same bits.
+  const int nseg = m.K / kSegCols;
+  const long long tiles = (long long)(m.N / 16) * ((rows_ub + 8 * ng - 1) / (8 * ng));
+  const bool split = h->seg_ws && a.gain == nullptr && m.K > kSegCols && m.K % kSegCols == 0 && nseg <= h->seg_nmax &&
+                     m.N <= h->seg_n && rows_ub <= h->seg_rows && 2 * tiles <= h->sm_count;
+  if (split) {
+    a.seg_ws = h->seg_ws;
+    a.seg_rows = h->seg_rows;
+  }
   if (m.planes == 1) {
     if (ng == 1) launch_ng<1, 1, EPI>(h, a, rows_ub);
     else if (ng == 2) launch_ng<2, 1, EPI>(h, a, rows_ub);
@@ -375,6 +389,11 @@ int gemm(blt_dec* h, const Mat& m, GemmArgs a, int rows_ub) {
     else if (ng == 2) launch_ng<2, 2, EPI>(h, a, rows_ub);
     else if (ng == 4) launch_ng<4, 2, EPI>(h, a, rows_ub);
     else launch_ng<8, 2, EPI>(h, a, rows_ub);
+  }
+  if (split) {
+    const long long pairs = (long long)rows_ub * (m.N / 2);
+    k_seg_finish<EPI><<<(unsigned)((pairs + 255) / 256), 256, 0, h->stream>>>(a, nseg);
+    h->launches += 1;
   }
   CK(cudaGetLastError());
   return BLT_OK;
@@ -1317,6 +1336,18 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(set_attrs_epi<EPI_SWIGLU>(h));
     TRY(set_attrs_epi<EPI_QKV>(h));
     TRY(set_attrs_epi<EPI_LATC>(h));
+    {
+      int dev = 0;
+      CK(cudaGetDevice(&dev));
+      CK(cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, dev));
+      // split-K of small W2 grids: rows up to 64 (larger passes fill the GPU without it)
+      if (F > kSegCols && F % kSegCols == 0) {
+        h->seg_nmax = F / kSegCols;
+        h->seg_rows = std::min(RL, 64);
+        h->seg_n = d;
+        TRY(dalloc(h, &h->seg_ws, (size_t)h->seg_nmax * h->seg_rows * d));
+      }
+    }
     if (h->tc) {
       const int KM = std::max(d, F);
       TRY(dalloc(h, &h->tc_hi, (size_t)RL * KM));

@@ -118,6 +118,10 @@ struct GemmArgs {
   const int* lat_slot;
   int max_lat;
   int* status;
+  // split over K segments (K > kSegCols, no gain): CTA z computes segment z's sums into
+  // seg_ws [nseg][seg_rows][N]; k_seg_finish adds them in order and runs the epilogue
+  float* seg_ws;
+  int seg_rows;
 };
 
 // Four gained values of one k16 step -> hi/lo B fragments (k = 2t, 2t+1 | 2t+8, 2t+9).
@@ -364,9 +368,13 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int nwin = a.K / kKWin;
   const int ksteps = a.K / 16;
   const bool norm = a.gain != nullptr;
+  constexpr int kSegWin = kSegCols / kKWin;  // windows per segment (a multiple of DEPTH)
+  // windows [w0, nwin): all of K, or (split) segment blockIdx.z only
+  const bool split = a.seg_ws != nullptr;
+  const int w0 = split ? (int)blockIdx.z * kSegWin : 0;
+  const int nwin = split ? w0 + kSegWin : a.K / kKWin;
 
   const float* xg = a.X + (a.group_tiles ? (size_t)(mt / a.group_tiles) * a.group_xoff : 0);
   auto stage = [&](int wi, int buf) {
@@ -386,10 +394,10 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
 #pragma unroll
   for (int dd = 0; dd < DEPTH; ++dd)
 #pragma unroll
-    for (int p = 0; p < PL; ++p) wb[dd][p] = (dd < nwin) ? wtile(dd, p) : make_uint4(0, 0, 0, 0);
+    for (int p = 0; p < PL; ++p) wb[dd][p] = (w0 + dd < nwin) ? wtile(w0 + dd, p) : make_uint4(0, 0, 0, 0);
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < nwin) stage(s, s);
+    if (w0 + s < nwin) stage(w0 + s, (w0 + s) % STAGES);
     cp_async_commit();
   }
   float acc[NG][4], ss[NG];
@@ -397,10 +405,9 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   for (int n = 0; n < NG; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = ss[n] = 0.f;
   float tot[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // K > 1024: this thread's output pairs, segments summed in order
   int nsegs_done = 0;
-  constexpr int kSegWin = kSegCols / kKWin;     // windows per segment (a multiple of DEPTH)
 
-  for (int wi0 = 0; wi0 < nwin; wi0 += DEPTH) {
-    if (wi0 > 0 && wi0 % kSegWin == 0) {  // segment boundary: fold the finished segment
+  for (int wi0 = w0; wi0 < nwin; wi0 += DEPTH) {
+    if (wi0 > w0 && wi0 % kSegWin == 0) {  // segment boundary: fold the finished segment
       seg_fold<NG>(acc, xs + (size_t)STAGES * RB * kXStride + 8 * RB, tot, nsegs_done, tid);
     }
 #pragma unroll
@@ -440,6 +447,22 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   }
   cp_async_wait<0>();
   __syncthreads();
+  if (split) {  // this segment's sums S_z (the warps added in order), for k_seg_finish
+    seg_fold<NG>(acc, xs, tot, nsegs_done, tid);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int p = tid + i * kThreads;
+      if (p < 8 * RB) {
+        const int r16 = p & 7, col = p >> 3;
+        if (col < nr) {
+          float* w = a.seg_ws + ((size_t)blockIdx.z * a.seg_rows + row0 + col) * a.N + mt * 16 + r16;
+          w[0] = tot[i][0];
+          w[8] = tot[i][1];
+        }
+      }
+    }
+    return;
+  }
   if (a.K <= kSegCols) {
     tile_reduce<NG>(acc, ss, norm, xs, ssr, nr, a.K, a.eps, tid, kThreads, [] { __syncthreads(); },
                     [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
@@ -449,6 +472,25 @@ __global__ void __launch_bounds__(kThreads) k_gemm(GemmArgs a) {
   seg_fold<NG>(acc, xs, tot, nsegs_done, tid);
   tile_reduce_totals<NG>(tot, ss, norm, xs, ssr, nr, a.K, a.eps, tid,
                          [&](int r16, int col, float v0, float v1) { gemm_epilogue<EPI>(a, mt, r16, row0 + col, v0, v1); });
+}
+
+// After a split k_gemm: the segment sums added in order, ((S_0 + S_1) + S_2) + ...,
+// exactly as k_gemm folds them, then the epilogue.  One thread per output pair.
+template <int EPI>
+__global__ void k_seg_finish(GemmArgs a, int nseg) {
+  const int nrows = a.n_rows ? *a.n_rows : a.rows_host;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;  // (row, tile, r16)
+  const int pairs = a.N / 2;
+  const int row = i / pairs, q = i % pairs, mt = q / 8, r16 = q % 8;
+  if (row >= nrows) return;
+  const float* w = a.seg_ws + (size_t)row * a.N + mt * 16 + r16;
+  const size_t zs = (size_t)a.seg_rows * a.N;
+  float v0 = w[0], v1 = w[8];
+  for (int z = 1; z < nseg; ++z) {
+    v0 = v0 + w[z * zs];
+    v1 = v1 + w[z * zs + 8];
+  }
+  gemm_epilogue<EPI>(a, mt, r16, row, v0, v1);
 }
 
 // ------------------------------------------------------------------------ row-wise kernels
@@ -520,15 +562,14 @@ __host__ __device__ constexpr int kv_stride() {
 // Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
 // ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).  One
 // K or V row per iteration: a single page-table lookup per row.
-// Keys and values t0 .. t0 + n - 1 of (seq, head h) into smem (row stride
-// kv_stride), with the chunk's page ids already in pg[] (pg[j]: the page of
+// Keys and values t0 .. t0 + n - 1 of (seq, head h) into smem (row stride ST,
+// kv_stride by default), with the chunk's page ids already in pg[] (pg[j]: the page of
 // positions (t0 / PT + j) PT ..): every copy is issued at once.
-template <int DH, typename KVT>
+template <int DH, typename KVT, int ST = kv_stride<DH, KVT>()>
 __device__ __forceinline__ void attn_load_kv_paged(const AttnArgs& a, const int* pg, int h, int t0, int n, KVT* ks, KVT* vs, int tid,
                                                    int nthr) {
   constexpr int PER = 16 / sizeof(KVT);
   constexpr int CPR = DH / PER;
-  constexpr int ST = kv_stride<DH, KVT>();
   const KVT* kv = static_cast<const KVT*>(a.kv);
 #pragma unroll 1
   for (int i = tid; i < 2 * n * CPR; i += nthr) {
@@ -859,10 +900,9 @@ __device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* k
 // caller's wait and `sync`, attn_partial_run runs attn_chunk_core with the
 // partials to a.part_o / a.part_ml.  ROWS: the smem capacity in rows (the
 // group's row count must not exceed it).
-template <int DH, typename KVT, int ROWS>
+template <int DH, typename KVT, int ROWS, int ST>
 __device__ __forceinline__ bool attn_partial_stage(const AttnArgs& a, int gi, int h, int chunk, float* qs, KVT* vs, int* lim,
                                                    int tid, int nthr) {
-  constexpr int ST = kv_stride<DH, KVT>();
   const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
   if (nr > ROWS) {  // the host's bound on rows per group was wrong: no write past the smem
     if (tid == 0) set_status(a.status, kErrDevice);
@@ -882,10 +922,9 @@ __device__ __forceinline__ bool attn_partial_stage(const AttnArgs& a, int gi, in
   }
   return true;
 }
-template <int DH, typename KVT, int ROWS, class Sync>
+template <int DH, typename KVT, int ROWS, int ST, class Sync>
 __device__ __forceinline__ void attn_partial_run(const AttnArgs& a, int gi, int h, int chunk, const float* qs, float* ps, const KVT* ks,
                                                  const KVT* vs, float* mrow, float* lrow, const int* lim, int tid, int nthr, Sync sync) {
-  constexpr int ST = kv_stride<DH, KVT>();
   const int row0 = __ldcg(a.rows.g_row0 + gi), nr = __ldcg(a.rows.g_nrows + gi), kmax = __ldcg(a.rows.g_kmax + gi);
   const int nk = min(a.CH, kmax - chunk * a.CH);
   attn_chunk_core<DH, KVT, ST>(
@@ -964,6 +1003,7 @@ __device__ __forceinline__ void attn_combine_row(const AttnArgs& a, int row, int
 // grid (H, chunks, groups), 128 threads; ROWS: rows per group at most (smem).
 template <int DH, typename KVT, int ROWS>
 __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
+  constexpr int ST = kv_stride<DH, KVT>();
   const int gi = blockIdx.z;
   if (gi >= *a.rows.n_groups) return;
   const int kmax = a.rows.g_kmax[gi];
@@ -974,26 +1014,28 @@ __global__ void __launch_bounds__(128) k_attn_partial(AttnArgs a) {
   float* qs = reinterpret_cast<float*>(smem4);
   float* ps = qs + ROWS * DH;
   KVT* ks = reinterpret_cast<KVT*>(ps + ROWS * a.CH);
-  KVT* vs = ks + a.CH * kv_stride<DH, KVT>();
+  KVT* vs = ks + a.CH * ST;
   __shared__ float mrow[ROWS], lrow[ROWS];
   __shared__ int lim[ROWS];
   __shared__ int pg[16];  // the chunk's KV pages (at most CH / PT + 1 <= 9)
   const int n = min(t0 + a.CH, kmax) - t0;
-  if (threadIdx.x < (t0 + n - 1) / a.PT - t0 / a.PT + 1) {
-    const int seq = a.rows.g_seq[gi], pi = t0 / a.PT + threadIdx.x;
+  const int p0 = t0 / a.PT, np = (t0 + n - 1) / a.PT - p0 + 1;
+  if (threadIdx.x < np) {
+    const int seq = a.rows.g_seq[gi], pi = p0 + threadIdx.x;
     int page = (pi < a.max_pages) ? a.page_table[seq * a.max_pages + pi] : -1;
     if (page < 0) set_status(a.status, kErrDevice);
     pg[threadIdx.x] = page;
   }
   // q and the row limits load while the page ids do; then every K/V copy goes out at once
-  const bool ok = attn_partial_stage<DH, KVT, ROWS>(a, gi, h, blockIdx.y, qs, vs, lim, threadIdx.x, 128);
+  const bool ok = attn_partial_stage<DH, KVT, ROWS, ST>(a, gi, h, blockIdx.y, qs, vs, lim, threadIdx.x, 128);
   __syncthreads();
   attn_load_kv_paged<DH, KVT>(a, pg, h, t0, n, ks, vs, threadIdx.x, 128);
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
   if (!ok) return;
-  attn_partial_run<DH, KVT, ROWS>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128, [] { __syncthreads(); });
+  attn_partial_run<DH, KVT, ROWS, ST>(a, gi, h, blockIdx.y, qs, ps, ks, vs, mrow, lrow, lim, threadIdx.x, 128,
+                                      [] { __syncthreads(); });
 }
 
 // grid (rows_max, H), one warp.
