@@ -48,6 +48,8 @@ EXPORTS = (
     "blt_dec_verify_sampled",
     "blt_dec_rewind",
     "blt_dec_stats",
+    "blt_dec_upload",
+    "blt_dec_download",
     "blt_dec_sync",
     "blt_dec_last_error",
     "blt_dec_free",
@@ -146,6 +148,8 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
     lib.blt_dec_verify_sampled.argtypes = [P, P, P, C.POINTER(C.c_int32), SP, P, P, P]
     lib.blt_dec_rewind.argtypes = [P, I, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
     lib.blt_dec_stats.argtypes = [P, C.POINTER(blt_dec_counters)]
+    lib.blt_dec_upload.argtypes = [P, P, P, C.c_size_t]
+    lib.blt_dec_download.argtypes = [P, P, P, C.c_size_t]
     lib.blt_dec_sync.argtypes = [P]
     lib.blt_dec_last_error.argtypes = [P]
     lib.blt_dec_last_error.restype = C.c_char_p
@@ -281,6 +285,16 @@ def blt_dec_stats(h) -> dict:
     c = blt_dec_counters()
     _check(h, load_library().blt_dec_stats(h, C.byref(c)), "blt_dec_stats")
     return c.as_dict()
+
+
+def blt_dec_upload(h, dst_device, src_host: int, n: int) -> None:
+    """Host -> device copy of n bytes on the handle's stream (src_host: an address; reusable at once)."""
+    _check(h, load_library().blt_dec_upload(h, _ptr(dst_device), src_host, n), "blt_dec_upload")
+
+
+def blt_dec_download(h, dst_host: int, src_device, n: int) -> None:
+    """Device -> host copy of n bytes after the handle's queued work (dst_host: an address)."""
+    _check(h, load_library().blt_dec_download(h, dst_host, _ptr(src_device), n), "blt_dec_download")
 
 
 def blt_dec_sync(h) -> int:

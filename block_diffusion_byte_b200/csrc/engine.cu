@@ -137,6 +137,18 @@ struct blt_dec {
   unsigned long long* trace = nullptr;
   std::string trace_path;
   int trace_pending = 0;
+  // blt_dec_upload: a ring of pinned bounce buffers, each reused once its last copy has run
+  struct Bounce {
+    void* p = nullptr;
+    size_t cap = 0;
+    cudaEvent_t done = nullptr;
+  };
+  static constexpr int kUpSlots = 4;
+  static constexpr size_t kUpSmall = 256 * 1024;  // ring buffers' size; larger copies use up_large
+  Bounce up[kUpSlots];
+  int up_next = 0;
+  Bounce up_large;  // grows to the largest copy seen (prefill rows and latents)
+  Bounce down;      // blt_dec_download
 };
 
 namespace {
@@ -1702,9 +1714,56 @@ int blt_dec_sync(blt_dec_t* h) {
 
 const char* blt_dec_last_error(blt_dec_t* h) { return h ? h->err.c_str() : "NULL handle"; }
 
+int blt_dec_upload(blt_dec_t* h, void* dst, const void* src, size_t n) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  if (n == 0) return BLT_OK;
+  if (!dst || !src) return fail(h, BLT_ERR_INVALID_ARG, "blt_dec_upload: NULL pointer");
+  const bool small = n <= blt_dec::kUpSmall;
+  blt_dec::Bounce& b = small ? h->up[h->up_next] : h->up_large;
+  if (small) h->up_next = (h->up_next + 1) % blt_dec::kUpSlots;
+  if (b.done) CK(cudaEventSynchronize(b.done));  // the buffer's previous copy has run
+  else CK(cudaEventCreateWithFlags(&b.done, cudaEventDisableTiming));
+  if (b.cap < n) {  // small buffers: once; the large one: when a larger copy comes
+    if (b.p) CK(cudaFreeHost(b.p));
+    b.p = nullptr;
+    b.cap = 0;
+    const size_t cap = small ? blt_dec::kUpSmall : n + n / 4;
+    CK(cudaHostAlloc(&b.p, cap, cudaHostAllocDefault));
+    b.cap = cap;
+  }
+  memcpy(b.p, src, n);
+  CK(cudaMemcpyAsync(dst, b.p, n, cudaMemcpyHostToDevice, h->stream));
+  CK(cudaEventRecord(b.done, h->stream));
+  return BLT_OK;
+}
+
+int blt_dec_download(blt_dec_t* h, void* dst, const void* src, size_t n) {
+  if (!h) return BLT_ERR_INVALID_ARG;
+  if (n && (!dst || !src)) return fail(h, BLT_ERR_INVALID_ARG, "blt_dec_download: NULL pointer");
+  blt_dec::Bounce& b = h->down;
+  if (b.cap < n) {
+    if (b.p) CK(cudaFreeHost(b.p));
+    b.p = nullptr;
+    b.cap = 0;
+    const size_t cap = std::max(n + n / 4, (size_t)1 << 16);
+    CK(cudaHostAlloc(&b.p, cap, cudaHostAllocDefault));
+    b.cap = cap;
+  }
+  if (n) CK(cudaMemcpyAsync(b.p, src, n, cudaMemcpyDeviceToHost, h->stream));
+  CK(cudaStreamSynchronize(h->stream));
+  if (n) memcpy(dst, b.p, n);
+  return BLT_OK;
+}
+
 void blt_dec_free(blt_dec_t* h) {
   if (!h) return;
   if (h->stream) cudaStreamSynchronize(h->stream);
+  for (int i = 0; i <= blt_dec::kUpSlots; ++i) {
+    blt_dec::Bounce& b = i < blt_dec::kUpSlots ? h->up[i] : h->up_large;
+    if (b.p) cudaFreeHost(b.p);
+    if (b.done) cudaEventDestroy(b.done);
+  }
+  if (h->down.p) cudaFreeHost(h->down.p);
   for (void* p : h->allocs) cudaFree(p);
   if (h->mirror) cudaFreeHost(h->mirror);
   if (h->mirror_ev) cudaEventDestroy(h->mirror_ev);

@@ -31,6 +31,8 @@ from workload import sampling_uniforms, ModelShape, Patcher, PatchState, WeightS
 
 from . import binding as B
 
+_NP_DTYPE = {torch.uint8: np.uint8, torch.int32: np.int32, torch.float32: np.float32, torch.int64: np.int64}
+
 
 def engine_config(shape: ModelShape, max_batch: int, max_ctx: int, max_latents: int, max_rows: int, max_block: int,
                   page_tokens: int = 64, kv_pages: int = 0, attn_chunk: int = 0, flags: int = 0) -> B.blt_dec_config:
@@ -80,9 +82,6 @@ class Engine:
         g = {n: np.ascontiguousarray(weights.get(n), dtype=np.float32) for n in ("embed", "head", "final_norm")}
         self.h = B.blt_dec_init(cfg, g["embed"], g["head"], g["final_norm"], layers, self.stream.cuda_stream)
         dev = self.device
-        nrow = max(max_rows, max_batch * max_block) + max_batch
-        self.d_bytes = torch.zeros(nrow, dtype=torch.uint8, device=dev)
-        self.d_slots = torch.zeros(nrow, dtype=torch.int32, device=dev)
         self.d_lat = torch.zeros((max(max_rows, 4 * max_batch * max_block), shape.d_global), dtype=torch.float32, device=dev)
         self.d_out = torch.zeros((max_batch, max_block), dtype=torch.uint8, device=dev)
         self.d_steps = torch.zeros(max_batch, dtype=torch.int32, device=dev)
@@ -90,55 +89,61 @@ class Engine:
         self.d_next = torch.zeros(max_batch, dtype=torch.uint8, device=dev)
         self.d_vslots = torch.zeros((max_batch, max_block), dtype=torch.int32, device=dev)
         self.h2d_bytes = 0
-        self._staging = {}  # destination data_ptr -> (pinned staging buffer, event of its last copy)
         self.d2h_bytes = 0
+        self._h_rows = np.empty(1 << 16, dtype=np.uint8)  # a call's rows, packed (host)
+        self._d_rows = torch.empty(1 << 16, dtype=torch.uint8, device=dev)
 
-    # -- staging
+    # -- staging: every host <-> device copy goes through the engine's blt_dec_upload /
+    # blt_dec_download (pinned bounce buffers, the handle's stream)
     def _put(self, dst: torch.Tensor, arr: np.ndarray) -> torch.Tensor:
-        """Copy ``arr`` into the first rows of ``dst`` through a reusable pinned staging
-        buffer (one per destination; it is rewritten only after its last copy ran)."""
+        """Copy ``arr`` into the first rows of ``dst`` (queued on the engine's stream)."""
         n = arr.shape[0]
         if n == 0:
             return dst[:0]
-        arr = np.ascontiguousarray(arr)
-        key = dst.data_ptr()
-        st = self._staging.get(key)
-        if st is None or st[0].numel() < arr.size or st[0].dtype != dst.dtype:
-            st = (torch.empty(max(arr.size, 1 << 12), dtype=dst.dtype).pin_memory(), torch.cuda.Event())
-            self._staging[key] = st
-        buf, done = st
-        done.synchronize()
-        src = buf[: arr.size]
-        src.numpy()[:] = arr.reshape(-1)
-        with torch.cuda.stream(self.stream):
-            dst[:n].view(-1)[: arr.size].copy_(src, non_blocking=True)
-            done.record(self.stream)
+        arr = np.ascontiguousarray(arr, dtype=_NP_DTYPE[dst.dtype])
+        if arr.nbytes > dst.numel() * dst.element_size():
+            raise ValueError(f"staging overflow: {arr.nbytes} bytes into {dst.numel() * dst.element_size()}")
+        B.blt_dec_upload(self.h, dst.data_ptr(), arr.ctypes.data, arr.nbytes)
         self.h2d_bytes += arr.nbytes
         return dst[:n]
 
     def _get(self, t: torch.Tensor) -> np.ndarray:
-        with torch.cuda.stream(self.stream):
-            out = t.to("cpu", non_blocking=False)
-        self.d2h_bytes += out.numel() * out.element_size()
-        return out.numpy()
+        """A device tensor's values on the host, after the engine's queued work."""
+        if not t.is_contiguous():
+            raise ValueError("_get needs a contiguous tensor")
+        out = np.empty(tuple(t.shape), dtype=_NP_DTYPE[t.dtype])
+        B.blt_dec_download(self.h, out.ctypes.data, t.data_ptr(), out.nbytes)
+        self.d2h_bytes += out.nbytes
+        return out
 
     def rows(self, byte_lists: Sequence[Sequence[int]], slot_lists: Sequence[Sequence[int]], lat_lists: Sequence[Sequence[np.ndarray]]):
+        """Stage a call's rows: bytes, latent slots and new latents packed into one upload."""
         ro = np.cumsum([0] + [len(b) for b in byte_lists]).astype(np.int64)
         lo = np.cumsum([0] + [len(v) for v in lat_lists]).astype(np.int64)
-        bts = np.array([b for bl in byte_lists for b in bl], dtype=np.uint8)
-        sls = np.array([s for sl in slot_lists for s in sl], dtype=np.int32)
+        n = int(ro[-1])
         lats = [v for vl in lat_lists for v in vl]
-        if bts.shape[0] > self.d_bytes.shape[0]:
-            self.d_bytes = torch.zeros(bts.shape[0], dtype=torch.uint8, device=self.device)
-            self.d_slots = torch.zeros(bts.shape[0], dtype=torch.int32, device=self.device)
-        db = self._put(self.d_bytes, bts)
-        ds = self._put(self.d_slots, sls)
-        dl = None
+        dg = self.shape.d_global
+        o_s = (n + 15) & ~15
+        o_l = (o_s + 4 * n + 15) & ~15
+        total = o_l + 4 * dg * len(lats)
+        if self._h_rows.nbytes < total:
+            self._h_rows = np.empty(total + total // 4, dtype=np.uint8)
+        if self._d_rows.numel() < total:
+            torch.cuda.synchronize(self.device)  # the old buffer may still be read by queued work
+            self._d_rows = torch.empty(total + total // 4, dtype=torch.uint8, device=self.device)
+        buf = self._h_rows
+        if n:
+            buf[:n] = np.fromiter((b for bl in byte_lists for b in bl), dtype=np.uint8, count=n)
+            buf[o_s:o_s + 4 * n].view(np.int32)[:] = np.fromiter((v for sl in slot_lists for v in sl), dtype=np.int32, count=n)
         if lats:
-            if len(lats) > self.d_lat.shape[0]:
-                self.d_lat = torch.zeros((len(lats), self.shape.d_global), dtype=torch.float32, device=self.device)
-            dl = self._put(self.d_lat, np.stack(lats).astype(np.float32))
-        return B.rows_in(db, ds, ro.tolist(), dl, lo.tolist())
+            lv = buf[o_l:total].view(np.float32).reshape(len(lats), dg)
+            for i, v in enumerate(lats):
+                lv[i] = v
+        base = self._d_rows.data_ptr()
+        if total:
+            B.blt_dec_upload(self.h, base, buf.ctypes.data, total)
+        self.h2d_bytes += n * 5 + 4 * dg * len(lats)
+        return B.rows_in(base, base + o_s, ro.tolist(), base + o_l if lats else None, lo.tolist())
 
     def out_view(self, nb: int, k: int) -> torch.Tensor:
         """The engine writes [batch, k] byte outputs densely."""

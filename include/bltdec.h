@@ -42,6 +42,7 @@
 #ifndef BLTDEC_H
 #define BLTDEC_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -318,6 +319,19 @@ int blt_dec_rewind(blt_dec_t *h, int batch, const int32_t *kv_len, const int32_t
 
 /* Read the counters (waits for the handle's stream). */
 int blt_dec_stats(blt_dec_t *h, blt_dec_counters *out);
+
+/* Host <-> device copies on the handle's stream, for the rows, latents and
+ * outputs of the calls above (plain runtime helpers; no decoder work).
+ * blt_dec_upload: copies n bytes from host memory src (any memory; it is
+ * read before the call returns, so the caller may reuse it at once) to device
+ * memory dst, through one of the handle's pinned bounce buffers; the device
+ * copy is queued on the stream (later calls on the handle see it).
+ * blt_dec_download: copies n bytes from device memory src to host memory dst
+ * after all queued work; returns once dst holds them.  Both: n = 0 does no
+ * copy; the device pointers must be valid for n bytes.  Errors: INVALID_ARG
+ * (NULL pointer with n > 0), CUDA. */
+int blt_dec_upload(blt_dec_t *h, void *dst_device, const void *src_host, size_t n);
+int blt_dec_download(blt_dec_t *h, void *dst_host, const void *src_device, size_t n);
 
 /* Wait for all queued work; returns BLT_OK or the device status word
  * (BLT_ERR_STEP_LIMIT, BLT_ERR_DEVICE) and clears it. */

@@ -241,3 +241,32 @@ def test_eb_rejects_bad_gamma(tiny_setup):
                 B.blt_dec_diffuse_block_eb(eng.h, 1, r, 4, bad, 0, eng.d_out)
     finally:
         eng.close()
+
+
+def test_upload_download_round_trip(tiny_setup):
+    """blt_dec_upload / blt_dec_download: bytes survive a round trip through device
+    memory at small, bounce-ring and large sizes; the source may be reused at once;
+    n = 0 copies nothing; NULL pointers are INVALID_ARG."""
+    from block_diffusion_byte_b200 import binding as B
+
+    wl, ws, _ = tiny_setup
+    eng = _engine(wl, ws)
+    try:
+        dev = torch.empty(3 << 20, dtype=torch.uint8, device="cuda")
+        rng = np.random.default_rng(5)
+        for n in (1, 4096, 300_000, 3 << 20):
+            src = rng.integers(0, 256, n, dtype=np.uint8)
+            want = src.copy()
+            B.blt_dec_upload(eng.h, dev.data_ptr(), src.ctypes.data, n)
+            src[:] = 0  # reused at once: the upload took its bytes before returning
+            got = np.empty(n, dtype=np.uint8)
+            B.blt_dec_download(eng.h, got.ctypes.data, dev.data_ptr(), n)
+            assert np.array_equal(got, want), n
+        B.blt_dec_upload(eng.h, dev.data_ptr(), 0, 0)
+        B.blt_dec_download(eng.h, 0, dev.data_ptr(), 0)
+        with pytest.raises(B.BltError):
+            B.blt_dec_upload(eng.h, None, src.ctypes.data, 16)
+        with pytest.raises(B.BltError):
+            B.blt_dec_download(eng.h, 0, dev.data_ptr(), 16)
+    finally:
+        eng.close()

@@ -61,10 +61,15 @@ def derive_keys(*columns) -> np.ndarray:
     """``derive_key`` over rows of words: column ``j`` holds word ``j`` of every key
     (ints broadcast).  Elementwise the same operations as ``derive_key``."""
     n = max((len(c) for c in columns if not np.isscalar(c)), default=1)
+    if n <= 8:  # a few keys: Python integers are faster than numpy's per-call overhead
+        return np.asarray([derive_key(*[c if np.isscalar(c) else c[i] for c in columns]) for i in range(n)], dtype=np.uint64)
     h = np.zeros(n, dtype=np.uint64)
     with np.errstate(over="ignore"):
         for c in columns:
-            w = np.asarray([int(v) & 0xFFFFFFFFFFFFFFFF for v in (c if not np.isscalar(c) else [c] * n)], dtype=np.uint64)
+            if np.isscalar(c):
+                w = np.uint64(int(c) & 0xFFFFFFFFFFFFFFFF)  # broadcast: the same word for every key
+            else:
+                w = np.asarray([int(v) & 0xFFFFFFFFFFFFFFFF for v in c], dtype=np.uint64)
             h = mix64((h ^ w) + GAMMA)
     return h
 
