@@ -691,7 +691,7 @@ __device__ __forceinline__ void attn_pv_mma(int CH, const float* ps, const __nv_
     const int c0 = (item % (DH / 16)) * 16, rg = item / (DH / 16);
     const float* p = ps + min(rg * 8 + g, nr - 1) * CH;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
+#pragma unroll 4
     for (int kt = 0; kt < nkt; ++kt) {
       const int k0 = kt * 16 + 2 * t;
       const unsigned short* va = v16 + k0 * ST + c0 + g;
@@ -842,16 +842,31 @@ __device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* k
 #pragma unroll 1
   for (int r = warp; r < nr; r += nw) {
     float m = -INFINITY;
-#pragma unroll 1
-    for (int k = lane; k < CH; k += 32) m = fmaxf(m, ps[r * CH + k]);
-    m = warp_max(m);
     float l = 0.f;
+    if (CH == 128) {  // the usual chunk: a lane's four scores loaded at once, the exps in parallel
+      float s[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[j] = ps[r * CH + lane + 32 * j];
+      m = fmaxf(fmaxf(fmaxf(m, s[0]), s[1]), fmaxf(s[2], s[3]));
+      m = warp_max(m);
+      float p[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        p[j] = (s[j] == -INFINITY) ? 0.f : expf(s[j] - m);
+        ps[r * CH + lane + 32 * j] = p[j];
+      }
+      l = ((p[0] + p[1]) + p[2]) + p[3];  // 0 + p0 = p0: the same sums as the loop below
+    } else {
 #pragma unroll 1
-    for (int k = lane; k < CH; k += 32) {
-      const float s = ps[r * CH + k];
-      const float p = (s == -INFINITY) ? 0.f : expf(s - m);
-      ps[r * CH + k] = p;
-      l += p;
+      for (int k = lane; k < CH; k += 32) m = fmaxf(m, ps[r * CH + k]);
+      m = warp_max(m);
+#pragma unroll 1
+      for (int k = lane; k < CH; k += 32) {
+        const float s = ps[r * CH + k];
+        const float p = (s == -INFINITY) ? 0.f : expf(s - m);
+        ps[r * CH + k] = p;
+        l += p;
+      }
     }
     l = warp_sum(l);
     if (lane == 0) {
