@@ -756,6 +756,9 @@ bool use_mega(const blt_dec* h, int rows_ub, int batch);
 // The block loop on the persistent kernel when the pass is small enough.
 int diffuse_passes(blt_dec* h, const CallDesc& cd, const blt_rows_in* pend, int k, float alpha, int max_steps, float* out_logits) {
   const int batch = cd.batch;
+  // a position's confidence (its largest byte probability) is at least 1/V: with alpha <= 1/V
+  // every masked position commits in the first pass, and the later passes would have no rows
+  if (!h->eb && alpha * (float)h->V <= 1.f) max_steps = 1;
   const int rows1 = cd.row_off[batch] + batch * k;
   if (!use_mega(h, rows1, batch)) return block_loop(h, cd, pend, k, alpha, max_steps, out_logits);
   PlanArgs p = plan_args(h, PL_FIRST, k);
