@@ -148,6 +148,14 @@ __device__ __forceinline__ void mma_step(float (&c)[4], const uint4 (&w)[PL], co
 }
 
 // Element offset of (page, layer, K|V, head, position in page, dim) in the KV pool.
+// K/V rows of 64 bf16 (128 bytes) are stored with their 16-byte pieces permuted by
+// position: piece j of position pos sits at piece j ^ (pos mod 8).  A chunk copied as
+// is into shared memory (128-key chunks start at multiples of 8) then has the eight
+// rows of every 8x8 ldmatrix tile in eight different bank groups.  Other K/V formats
+// are stored plainly.
+__device__ __forceinline__ int kv_dim(const GemmArgs& a, int pos, int dim) {
+  return (a.kv_f32 || a.dh != 64) ? dim : ((((dim >> 3) ^ pos) & 7) << 3) | (dim & 7);
+}
 __device__ __forceinline__ size_t kv_offset(const GemmArgs& a, int page, int layer, int kvsel, int h, int off, int dim) {
   return ((((size_t)page * a.L + layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * a.dh + (size_t)off * a.dh + dim;
 }
@@ -217,9 +225,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         set_status(a.status, kErrDevice);
         return;
       }
-      const size_t off = kv_offset(a, page, a.layer, 0, h, pos % a.PT, 0);
-      kv_store(a, off + j, o0);
-      kv_store(a, off + j + half, o1);
+      kv_store(a, kv_offset(a, page, a.layer, 0, h, pos % a.PT, kv_dim(a, pos, j)), o0);
+      kv_store(a, kv_offset(a, page, a.layer, 0, h, pos % a.PT, kv_dim(a, pos, j + half)), o1);
     } else {
       const int page = row_kv_page(a, row, seq, pos);
       if (page < 0) {
@@ -227,8 +234,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& a, int mt, int r16
         return;
       }
       const int n0 = lt * 16 + r16, n1 = n0 + 8;
-      kv_store(a, kv_offset(a, page, a.layer, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
-      kv_store(a, kv_offset(a, page, a.layer, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
+      kv_store(a, kv_offset(a, page, a.layer, 1, n0 / a.dh, pos % a.PT, kv_dim(a, pos, n0 % a.dh)), v0);
+      kv_store(a, kv_offset(a, page, a.layer, 1, n1 / a.dh, pos % a.PT, kv_dim(a, pos, n1 % a.dh)), v1);
     }
   }
 }
@@ -558,6 +565,19 @@ template <int DH, typename KVT>
 __host__ __device__ constexpr int kv_stride() {
   return DH + 16 / (int)sizeof(KVT);
 }
+// Whether K/V rows are stored with permuted 16-byte pieces (see kv_dim).
+template <int DH, typename KVT>
+__host__ __device__ constexpr bool kv_swizzled() {
+  return DH == 64 && sizeof(KVT) == 2;
+}
+// Element (row, col) of a K/V chunk in shared memory.  ST > 0: rows of ST elements,
+// plain.  ST == 0: rows of 64 elements as stored (piece j of row r at j ^ (r mod 8);
+// the chunk starts at a position that is a multiple of 8).
+template <int ST>
+__device__ __forceinline__ int kv_at(int row, int col) {
+  if constexpr (ST == 0) return row * 64 + ((((col >> 3) ^ row) & 7) << 3) + (col & 7);
+  else return row * ST + col;
+}
 
 // Copy positions [lo, hi) of the chunk starting at t0 of (seq, head) into smem
 // ks/vs (raw KVT, [CH][kv_stride]) with 16-byte cp.async (L2 only).  One
@@ -577,7 +597,8 @@ __device__ __forceinline__ void attn_load_kv_paged(const AttnArgs& a, const int*
     const int kvsel = r >= n, key = kvsel ? r - n : r, pos = t0 + key;
     const int page = max(pg[pos / a.PT - t0 / a.PT], 0);
     const KVT* src = kv + ((((size_t)page * a.L + a.layer) * 2 + kvsel) * a.H + h) * (size_t)a.PT * DH + (size_t)(pos % a.PT) * DH;
-    cp_async16((kvsel ? vs : ks) + key * ST + c * PER, src + c * PER, 16);
+    const int cs = kv_swizzled<DH, KVT>() ? (c ^ (pos & 7)) : c;  // the stored piece
+    cp_async16((kvsel ? vs : ks) + key * ST + c * PER, src + cs * PER, 16);
   }
 }
 
@@ -594,8 +615,9 @@ __device__ __forceinline__ void attn_load_kv(const AttnArgs& a, int seq, int h, 
     const int key = lo - t0 + (kvsel ? i - n : i);
     const KVT* src = kv_chunk_src<DH, KVT>(a, seq, h, t0 + key, kvsel);
     KVT* dst = (kvsel ? vs : ks) + key * ST;
+    const int sw = kv_swizzled<DH, KVT>() ? ((t0 + key) & 7) : 0;  // stored pieces are permuted by position
 #pragma unroll
-    for (int c = 0; c < CPR; ++c) cp_async16(dst + c * PER, src + c * PER, 16);
+    for (int c = 0; c < CPR; ++c) cp_async16(dst + c * PER, src + (c ^ sw) * PER, 16);
   }
 }
 
@@ -637,6 +659,26 @@ __device__ __forceinline__ void attn_scores(int CH, const float* qs, const KVT* 
   }
 }
 
+// Four 8x8 b16 matrices from shared memory as one m16n8k16 A fragment (ldmatrix);
+// lane L gives the address of row L & 7 of matrix L >> 3 (16 bytes, 16-byte aligned).
+// _t: each matrix transposed on the way.
+__device__ __forceinline__ uint4 ldsm_x4(const void* p) {
+  uint4 r;
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(smem_u32(p))
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ uint4 ldsm_x4_t(const void* p) {
+  uint4 r;
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(smem_u32(p))
+               : "memory");
+  return r;
+}
+
 // bf16 K/V on the tensor cores.  Scores: S^T (16 keys x 8 rows) = K (16 x 16
 // dims, bf16 A operand from smem) . q^T (dims x rows, split into bf16 hi and
 // lo B operands), hi then lo per 16-dim step, steps in dim order; one warp
@@ -653,13 +695,12 @@ __device__ __forceinline__ void attn_scores_mma(int CH, const float* qs, const _
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (key0 < nk) {
       const float* q = qs + min(rg * 8 + g, nr - 1) * DH;  // rows past nr: a live row's values, never stored
+      // this lane's row address for ldmatrix: keys key0 + (lane & 7) (+ 8 for matrices 1, 3), dims + 8 for matrices 2, 3
+      const int kr = key0 + (lane & 7) + ((lane >> 3) & 1) * 8, kc = (lane >> 4) * 8;
 #pragma unroll
       for (int s = 0; s < DH / 16; ++s) {
         const int c = s * 16 + 2 * t;
-        const __nv_bfloat16* k0 = ks + (key0 + g) * ST + c;
-        const __nv_bfloat16* k8 = ks + (key0 + g + 8) * ST + c;
-        const uint4 A = make_uint4(*reinterpret_cast<const uint32_t*>(k0), *reinterpret_cast<const uint32_t*>(k8),
-                                   *reinterpret_cast<const uint32_t*>(k0 + 8), *reinterpret_cast<const uint32_t*>(k8 + 8));
+        const uint4 A = ldsm_x4(ks + kv_at<ST>(kr, s * 16 + kc));  // K[key0 + g | + 8][c, c + 1 | c + 8, c + 9]
         const float2 qa = *reinterpret_cast<const float2*>(q + c), qb = *reinterpret_cast<const float2*>(q + c + 8);
         const XFrag xf = make_xfrag(qa.x, qa.y, qb.x, qb.y);
         mma16816(acc, A, xf.b0h, xf.b1h);
@@ -684,18 +725,18 @@ __device__ __forceinline__ void attn_pv_mma(int CH, const float* ps, const __nv_
                                             const float* lrow, int tid, int nthr, EmitO emit_o, EmitML emit_ml) {
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3, nw = nthr >> 5;
   const int nkt = (nk + 15) / 16, nrg = (nr + 7) / 8;
-  const unsigned short* v16 = reinterpret_cast<const unsigned short*>(vs);
-  auto pk = [](unsigned short lo, unsigned short hi) { return (uint32_t)lo | ((uint32_t)hi << 16); };
 #pragma unroll 1
   for (int item = warp; item < (DH / 16) * nrg; item += nw) {
     const int c0 = (item % (DH / 16)) * 16, rg = item / (DH / 16);
     const float* p = ps + min(rg * 8 + g, nr - 1) * CH;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // this lane's row address for ldmatrix.trans: keys (lane & 7) (+ 8 for matrices 2, 3), columns c0 (+ 8 for 1, 3)
+    const int vr = (lane & 7) + (lane >> 4) * 8, vc = c0 + ((lane >> 3) & 1) * 8;
 #pragma unroll 4
     for (int kt = 0; kt < nkt; ++kt) {
       const int k0 = kt * 16 + 2 * t;
-      const unsigned short* va = v16 + k0 * ST + c0 + g;
-      const uint4 A = make_uint4(pk(va[0], va[ST]), pk(va[8], va[ST + 8]), pk(va[8 * ST], va[9 * ST]), pk(va[8 * ST + 8], va[9 * ST + 8]));
+      // V^T fragment: V[k0, k0 + 1 | k0 + 8, k0 + 9][c0 + g | c0 + g + 8]
+      const uint4 A = ldsm_x4_t(vs + kv_at<ST>(kt * 16 + vr, vc));
       const float2 pa = *reinterpret_cast<const float2*>(p + k0), pb = *reinterpret_cast<const float2*>(p + k0 + 8);
       const XFrag xf = make_xfrag(pa.x, pa.y, pb.x, pb.y);
       mma16816(acc, A, xf.b0h, xf.b1h);
@@ -744,11 +785,10 @@ __device__ void attn_chunk_small(int CH, const float* qs, float* ps, const __nv_
   const bool act = tid < 128;
   float s0 = -INFINITY, s1 = -INFINITY;
   if (act && tid < nk) {
-    const uint4* kr = reinterpret_cast<const uint4*>(ks + (size_t)tid * ST);
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int j = 0; j < NC; ++j) {
-      const uint4 w = kr[j];
+      const uint4 w = *reinterpret_cast<const uint4*>(ks + kv_at<ST>(tid, j * 8));  // columns 8j .. 8j + 7
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -796,7 +836,7 @@ __device__ void attn_chunk_small(int CH, const float* qs, float* ps, const __nv_
         const int k1 = min(kq * 32 + 32, nk);
 #pragma unroll 4
         for (int k = kq * 32; k < k1; ++k) {
-          const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vs + (size_t)k * ST + 2 * cp));
+          const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vs + kv_at<ST>(k, 2 * cp)));
           const float q0 = ps[k], q1 = ps[CH + k];
           o00 = fmaf(q0, v.x, o00);
           o01 = fmaf(q0, v.y, o01);
@@ -893,8 +933,8 @@ __device__ void attn_chunk_core(int CH, const float* qs, float* ps, const KVT* k
 #pragma unroll 4
     for (int k = 0; k < nk; ++k) {
       float v;
-      if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[k * ST + c]);
-      else v = vs[k * ST + c];
+      if constexpr (sizeof(KVT) == 2) v = __bfloat162float(vs[kv_at<ST>(k, c)]);
+      else v = vs[kv_at<ST>(k, c)];
 #pragma unroll
       for (int j = 0; j < 4; ++j) o[j] = fmaf(ps[rr[j] * CH + k], v, o[j]);
     }

@@ -762,9 +762,8 @@ __device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem&
         if (page < 0) {
           set_status(a.status, kErrDevice);
         } else {
-          const size_t off = kv_offset(a, page, l, 0, h, pos % a.PT, 0);
-          kv_store(a, off + j, o0);
-          kv_store(a, off + j + half, o1);
+          kv_store(a, kv_offset(a, page, l, 0, h, pos % a.PT, kv_dim(a, pos, j)), o0);
+          kv_store(a, kv_offset(a, page, l, 0, h, pos % a.PT, kv_dim(a, pos, j + half)), o1);
         }
         if (!a.kv_f32) {
           r0 = __bfloat162float(__float2bfloat16_rn(o0));
@@ -778,8 +777,8 @@ __device__ __forceinline__ bool mega_epilogue(const MegaArgs& m, const MegaSmem&
         if (page < 0) {
           set_status(a.status, kErrDevice);
         } else {
-          kv_store(a, kv_offset(a, page, l, 1, n0 / a.dh, pos % a.PT, n0 % a.dh), v0);
-          kv_store(a, kv_offset(a, page, l, 1, n1 / a.dh, pos % a.PT, n1 % a.dh), v1);
+          kv_store(a, kv_offset(a, page, l, 1, n0 / a.dh, pos % a.PT, kv_dim(a, pos, n0 % a.dh)), v0);
+          kv_store(a, kv_offset(a, page, l, 1, n1 / a.dh, pos % a.PT, kv_dim(a, pos, n1 % a.dh)), v1);
         }
         float r0 = v0, r1 = v1;
         if (!a.kv_f32) {
@@ -1137,6 +1136,8 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
   const int ng = sm.n_groups;
   const int total = att_total(m, gk, ng);
   const int warp = tid >> 5, lane = tid & 31;
+  // the slot holds whole pages as stored: 64-element bf16 rows keep their permuted pieces
+  constexpr int KST = kv_swizzled<DH, KVT>() ? 0 : DH;
   bool ok = true;
   const unsigned e_qkv = epoch(m, pass, l, ST_QKV), e_part = epoch(m, pass, l, ST_PART);
   trace_mark(m, pass, TR_ATT << 8);
@@ -1181,7 +1182,7 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
              [&](int i, float v0, float v1) {
                if (i < 2 * nfp) {
                  const int sel = i >= nfp, rem = i - sel * nfp;
-                 KVT* dst = (sel ? vs : ks) + (size_t)(f0 - t0 + rem / HP) * DH + 2 * (rem % HP);
+                 KVT* dst = (sel ? vs : ks) + kv_at<KST>(f0 - t0 + rem / HP, 2 * (rem % HP));
                  if constexpr (sizeof(KVT) == 2) {
                    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(v0, v1);
                  } else {
@@ -1204,7 +1205,7 @@ __device__ bool run_attention(const MegaArgs& m, MegaSmem& sm, int l, int pass, 
     consumer_sync();
     u64* part = m.x_part + (((size_t)row0 * H + h) * m.CMAX + c) * (2 + DH);
     const size_t rstride = (size_t)H * m.CMAX * (2 + DH);
-    attn_chunk_core<DH, KVT, DH>(
+    attn_chunk_core<DH, KVT, KST>(
         CH, sm.qs, sm.ps, ks, vs, sm.mrow, sm.lrow, sm.lim, nr, nk, tid, 256, consumer_sync,
         [&](int r, int col, float v) { xw_st(part + r * rstride + 2 + col, v, e_part); },
         [&](int r, float mm, float ll) {
