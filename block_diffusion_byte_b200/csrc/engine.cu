@@ -108,7 +108,8 @@ struct blt_dec {
   LayerW* d_layers = nullptr;
   unsigned* flags = nullptr;  // [0] decision epoch, [1] pass-end arrivals
   unsigned* dec_val = nullptr;
-  int* abort_flag = nullptr;
+  int* abort_flag = nullptr;  // flags + 2: reset with the pass-end arrivals in one memset
+  unsigned long long calls = 0;  // engine calls served (counted on the host)
   unsigned epoch = 0;
   unsigned long long* xbuf = nullptr;  // exchange words of the persistent kernel (one allocation)
   size_t xbuf_words = 0;
@@ -588,8 +589,7 @@ void refresh_bounds(blt_dec* h) {
 
 int post_mirror(blt_dec* h) {
   const int B = h->cfg.max_batch;
-  CK(cudaMemcpyAsync(h->mirror, h->sd.kv_len, B * 4, cudaMemcpyDeviceToHost, h->stream));
-  CK(cudaMemcpyAsync(h->mirror + B, h->sd.n_lat, B * 4, cudaMemcpyDeviceToHost, h->stream));
+  CK(cudaMemcpyAsync(h->mirror, h->sd.kv_len, 2 * B * 4, cudaMemcpyDeviceToHost, h->stream));  // kv_len, n_lat
   CK(cudaEventRecord(h->mirror_ev, h->stream));
   h->mirror_pending = true;
   return BLT_OK;
@@ -795,7 +795,6 @@ void bump_bounds(blt_dec* h, const CallDesc& cd, int extra_kv) {
   }
 }
 
-__global__ void k_count_call(unsigned long long* c) { c[4] += 1; }
 __global__ void k_snapshot_base(SeqDev sd, int batch) {
   const int s = threadIdx.x + blockIdx.x * blockDim.x;
   if (s < batch) sd.kv_base[s] = sd.kv_len[s];
@@ -884,11 +883,10 @@ int mega_setup(blt_dec* h) {
   h->x_w2p = p, p += (size_t)std::max(nseg - 1, 1) * R * d;
   h->x_logit = p, p += R * 256;
   h->x_part = p;
-  TRY(dalloc(h, &h->flags, 2));
-  CK(cudaMemset(h->flags, 0, 8));
+  TRY(dalloc(h, &h->flags, 3));  // [0] pass plan word, [1] pass-end arrivals, [2] abort word
+  CK(cudaMemset(h->flags, 0, 12));
   TRY(dalloc(h, &h->dec_val, 1));
-  TRY(dalloc(h, &h->abort_flag, 1));
-  CK(cudaMemset(h->abort_flag, 0, 4));
+  h->abort_flag = reinterpret_cast<int*>(h->flags + 2);
   h->epoch = 1;
   h->mega_ok = true;
   if (const char* ip = getenv("BLTDEC_MEGA_ITEMS_PER_SM")) h->mega_items_per_sm = std::max(0, atoi(ip));
@@ -974,8 +972,7 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
   }
   m.epoch0 = h->epoch;
   h->epoch += span;
-  CK(cudaMemsetAsync(h->flags + 1, 0, 4, h->stream));  // pass-end arrivals of this launch
-  CK(cudaMemsetAsync(h->abort_flag, 0, 4, h->stream));
+  CK(cudaMemsetAsync(h->flags + 1, 0, 8, h->stream));  // pass-end arrivals and abort word of this launch
   m.abort = h->abort_flag;
   const bool stall = (h->cfg.flags & BLT_FLAG_TEST_STALL) != 0;
   m.wait_ns = stall ? 2000000ull : 500000000ull;  // 2 ms under the test-only stall, else 0.5 s
@@ -1017,8 +1014,7 @@ int mega_run(blt_dec* h, int mode, int batch, int k, float alpha, int max_passes
 int prefill_impl(blt_dec* h, int batch, const blt_rows_in* rows, float* out_logits, const CallDesc& cd) {
   const int total = cd.row_off[batch];
   TRY(reserve(h, cd, 0, true));
-  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
-  h->launches += 1;
+  h->calls += 1;
   TRY(project_latents(h, cd, rows->new_latents, true));
   k_snapshot_base<<<1, 256, 0, h->stream>>>(h->sd, batch);
   h->launches += 1;
@@ -1319,9 +1315,9 @@ int blt_dec_init(const blt_dec_config* cfg, const blt_dec_weights* w, void* cuda
     TRY(dalloc(h, &h->n_lat_rows, 1));
     SeqDev& sd = h->sd;
     const int B = c.max_batch;
-    TRY(dalloc(h, &sd.kv_len, B));
+    TRY(dalloc(h, &sd.kv_len, 2 * B));  // kv_len then n_lat: the host mirror reads both in one copy
+    sd.n_lat = sd.kv_len + B;
     TRY(dalloc(h, &sd.kv_base, B));
-    TRY(dalloc(h, &sd.n_lat, B));
     TRY(dalloc(h, &sd.active, B));
     TRY(dalloc(h, &sd.steps, B));
     TRY(dalloc(h, &sd.y_last, B));
@@ -1453,8 +1449,7 @@ int blt_dec_diffuse_block(blt_dec_t* h, int batch, const blt_rows_in* pending, i
     return fail(h, BLT_ERR_NO_SPACE, "pass rows %d > max_rows %d", cd.row_off[batch] + batch * k, h->cfg.max_rows);
   refresh_bounds(h);
   TRY(reserve(h, cd, k, true));
-  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
-  h->launches += 1;
+  h->calls += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
   TRY(pass_begin(h));
   TRY(diffuse_passes(h, cd, pending, k, alpha, max_steps, out_logits));
@@ -1502,8 +1497,7 @@ int blt_dec_draft(blt_dec_t* h, int batch, const blt_rows_in* pending, int mode,
   if (rows1 > h->cfg.max_rows) return fail(h, BLT_ERR_NO_SPACE, "pass rows %d > max_rows %d", rows1, h->cfg.max_rows);
   refresh_bounds(h);
   TRY(reserve(h, cd, k, true));
-  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
-  h->launches += 1;
+  h->calls += 1;
   TRY(project_latents(h, cd, pending->new_latents, true));
   TRY(pass_begin(h));
   if (mode == BLT_DRAFT_AR && use_mega(h, std::max(cd.row_off[batch], batch), batch)) {
@@ -1560,8 +1554,7 @@ int blt_dec_verify_accept(blt_dec_t* h, const int32_t* draft_row_latent, const f
   TRY(make_desc(h, batch, nullptr, latent_offsets, cd));
   refresh_bounds(h);
   TRY(reserve(h, cd, k, false));
-  k_count_call<<<1, 1, 0, h->stream>>>(h->sd.counters);
-  h->launches += 1;
+  h->calls += 1;
   TRY(project_latents(h, cd, new_latents, false));
   TRY(pass_begin(h));
   PlanArgs p = plan_args(h, PL_VERIFY, k);
@@ -1603,8 +1596,7 @@ int blt_dec_rewind(blt_dec_t* h, int batch, const int32_t* kv_len, const int32_t
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(h->stream));
   const int B = h->cfg.max_batch;
-  CK(cudaMemcpy(h->mirror, h->sd.kv_len, B * 4, cudaMemcpyDeviceToHost));
-  CK(cudaMemcpy(h->mirror + B, h->sd.n_lat, B * 4, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(h->mirror, h->sd.kv_len, 2 * B * 4, cudaMemcpyDeviceToHost));  // kv_len, n_lat
   for (int s = 0; s < B; ++s) {
     h->kv_ub[s] = h->mirror[s];
     h->nlat_ub[s] = h->mirror[B + s];
@@ -1624,7 +1616,7 @@ int blt_dec_stats(blt_dec_t* h, blt_dec_counters* out) {
   out->rows = c[1];
   out->prefill_rows = c[2];
   out->latents = c[3];
-  out->calls = c[4];
+  out->calls = h->calls;
   out->weight_bytes = c[5];
   out->kv_read_bytes = c[6];
   out->kernel_launches = h->launches;
