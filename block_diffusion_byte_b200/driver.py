@@ -125,7 +125,7 @@ class Engine:
         dg = self.shape.d_global
         o_s = (n + 15) & ~15
         o_l = (o_s + 4 * n + 15) & ~15
-        total = o_l + 4 * dg * len(lats)
+        total = o_l + 4 * dg * len(lats) if lats else o_s + 4 * n
         if self._h_rows.nbytes < total:
             self._h_rows = np.empty(total + total // 4, dtype=np.uint8)
         if self._d_rows.numel() < total:
