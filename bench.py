@@ -332,6 +332,49 @@ class _TimingWeights:
         return dict(self._layer)
 
 
+# decoder-step sweep points timed by the bench (batch, block, prefix): the sample rows of the
+# sweep's roofline table, from one row per pass up to 1024 rows per pass
+SWEEP_POINTS = ((1, 4, 512), (1, 4, 2048), (1, 16, 8192), (16, 8, 2048), (16, 16, 8192), (64, 16, 512))
+
+
+def sweep_timing(barrier, generate, B, Engine, persistent, peak, pk_kind, points=SWEEP_POINTS):
+    """Decoder-pass time at points of the decoder-step sweep (d_global 4096, BLT-D with
+    alpha 0.7, two blocks per sequence): per point one warm-up job, then one job whose
+    decoder passes are timed with CUDA events; the same per-pass figures as the main line."""
+    from workload import SWEEP
+
+    by = {(w.batch, w.block, w.prefix_len): w for w in SWEEP}
+    ws_s = WeightSet(SWEEP[0].shape, seed=SWEEP[0].seed).materialize()
+    out = []
+    for b, k, p in points:
+        w = by[(b, k, p)]
+        ids = list(range(b))
+        pres = [[int(x) for x in prefix_bytes(w.seed, w.cfg_index, s, p)] for s in ids]
+        # a call's rows: the previous block (now causal) and the new block of every sequence
+        eng = Engine(w.shape, ws_s, max_batch=b, max_ctx=p + 4 * w.gen_bytes + 4 * max(k, 16) + 16, max_block=max(k, 16),
+                     max_rows=max(1024, 2 * b * (k + 1)), time_passes=True, persistent=persistent)
+        try:
+            ms, d, _, _, _ = time_job(eng, w, pres, ids, 1, 1, barrier, generate, B)
+        finally:
+            eng.close()
+        roof, dec = pass_figures(d, 1, ms, peak, pk_kind)
+        out.append(
+            {
+                "batch": b,
+                "block": k,
+                "prefix": p,
+                "rows_per_pass": dec["rows_per_pass"],
+                "decoder_passes": d["passes"],
+                "pass_ms": roof["pass_ms"],
+                "alg_mb_per_pass": roof["alg_bytes_per_pass"] / 1e6,
+                "achieved_gbs": roof["achieved"],
+                "frac": roof["frac"],
+                "path": "persistent" if d["persistent_calls"] else "per-phase",
+            }
+        )
+    return out
+
+
 def global_step_timing(barrier, generate, B, Engine, peak, tokens: int = 256, steps: int = 48):
     """One step of a global transformer at the pages' 1B size on the device, so the
     N_enc (P_enc + P_global) term of the proxy can be timed: 24 layers, d 2048, 16 heads,
@@ -544,6 +587,13 @@ def main():
             "kernels, whose attention blocks overlap on each SM (the persistent kernel takes small passes with <= 8 items per SM); "
             "verification passes (128 rows) and prefill chunks project on the tcgen05 GEMM (value) or on the mma.sync GEMV "
             "kernels (gemv_value); roofline over all decoder passes of the job",
+        }
+    if world == 1 and not args.no_extras and args.workload == "d4_b1":
+        # per-pass time across the decoder-step sweep (1 to 1024 rows per pass)
+        line["sweep"] = {
+            "note": "d_global 4096, BLT-D alpha 0.7, two blocks per sequence; per point one warm-up job and one timed job; "
+            "roofline over the timed job's decoder passes (weights + K/V per pass)",
+            "points": sweep_timing(barrier, generate, B, Engine, persistent, peak, pk_kind),
         }
     if world == 1 and not (args.no_extras or args.no_ar_baseline) and args.workload == "d4_b1":
         # the N_enc term of the pages' proxy, timed: one global-model step at the 1B size
